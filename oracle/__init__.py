@@ -1,0 +1,109 @@
+"""fp64 CPU oracle for the selective-scan forward (TEST INFRASTRUCTURE).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package.  The product path (the CUDA library and
+its Python binding) never does, and shares no code with it.
+
+``selective_scan`` widens every input exactly to float64 (bf16 and fp32 values
+are exactly representable) and runs the sequential loop of ``ss_oracle.c``.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_libs = {}
+
+
+def _load(path=None):
+    """The oracle library at ``path`` (default: the built ``liboracle.so``)."""
+    if path is None:
+        path = _build.build()
+    if path not in _libs:
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.ss_oracle_fwd.restype = ctypes.c_int
+        lib.ss_oracle_fwd.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P, P,
+                                      ctypes.c_int, P, P, ctypes.c_int]
+        lib.ss_oracle_threads.restype = ctypes.c_int
+        lib.ss_oracle_threads.argtypes = []
+        _libs[path] = lib
+    return _libs[path]
+
+
+def max_threads() -> int:
+    """Threads the oracle's OpenMP loop uses when asked for "all"."""
+    return int(_load().ss_oracle_threads())
+
+
+def _f64(x):
+    """Exact widening to a C-contiguous float64 numpy array (None stays None)."""
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float64).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                   delta_softplus=False, return_last_state=False, nthreads=0, lib=None):
+    """y[b,d,l] (and the state after the last step) in float64.
+
+    Shapes: u, delta, z (batch, dim, L); A (dim, N); B, C (batch, N, L);
+    D, delta_bias (dim,).  Returns y, or (y, last_state (batch, dim, N)).
+    ``lib`` selects another build of the oracle library by path (the pin tests
+    use it to show that planted mistakes are caught).
+    """
+    u, delta, A, B, C =(_f64(t) for t in (u, delta, A, B, C))
+    D, z, delta_bias = _f64(D), _f64(z), _f64(delta_bias)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    if delta.shape != u.shape:
+        raise ValueError("u and delta must have the same shape")
+    if A.shape != (dim, N) or B.shape != (batch, N, L) or C.shape != (batch, N, L):
+        raise ValueError("bad A/B/C shape")
+    if z is not None and z.shape != u.shape:
+        raise ValueError("bad z shape")
+    for v in (D, delta_bias):
+        if v is not None and v.shape != (dim,):
+            raise ValueError("bad D/delta_bias shape")
+    y = np.zeros((batch, dim, L), dtype=np.float64)
+    last = np.zeros((batch, dim, N), dtype=np.float64) if return_last_state else None
+    rc = _load(lib).ss_oracle_fwd(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                               _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                               1 if delta_softplus else 0, _ptr(y), _ptr(last), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle rejected its arguments")
+    return (y, last) if return_last_state else y
+
+
+def selective_scan_rows(inputs, rows, nthreads=0):
+    """Oracle outputs for selected (b, d) rows of a problem held as host tensors.
+
+    ``inputs`` maps the names u, delta, A, B, C, D, z, delta_bias,
+    delta_softplus, return_last_state; ``rows`` is a list of (b, d).  Each row
+    is run as its own batch-1, dim-1 problem (rows are independent).
+    Returns (y_rows (R, L), last_rows (R, N) or None).
+    """
+    ys, lasts = [], []
+    for (b, d) in rows:
+        sl = lambda t: None if t is None else t[b:b + 1, d:d + 1]  # noqa: E731
+        pd = lambda t: None if t is None else t[d:d + 1]  # noqa: E731
+        out = selective_scan(sl(inputs["u"]), sl(inputs["delta"]), inputs["A"][d:d + 1],
+                             inputs["B"][b:b + 1], inputs["C"][b:b + 1], pd(inputs.get("D")),
+                             sl(inputs.get("z")), pd(inputs.get("delta_bias")),
+                             inputs["delta_softplus"], True, nthreads)
+        ys.append(out[0][0, 0])
+        lasts.append(out[1][0, 0])
+    return np.stack(ys), np.stack(lasts)
