@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-scan forward (libselscan) on B200.
+
+One step = one ss_fwd over the whole workload (every (b, d, l, n) state
+update).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+Metric: state updates per second, B*D*L*N / t.  Timing: CUDA events on the
+launching stream around each ss_fwd call; L2 is flushed (a write larger than
+L2) before every timed step, outside the events.  ``value`` sums all ranks'
+updates over the slowest rank's time (ranks run independent problems: weak
+scaling, no data-path collective).  ``e2e`` is the same metric through the
+host-buffer entry point ss_fwd_hostio: pinned host inputs copied in, the
+forward, y copied back, per step.  The roofline of the scan kernel is its
+exp count against the SFU rate (16 ex2 per clock per SM at the maximum SM
+clock); its HBM side (compulsory bytes over measured copy bandwidth) is
+reported beside it.  ``--impl reference`` times the fp64 CPU oracle on the
+host cores instead (a bounded sample of rows per step).
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_41_b200 import selscan, workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = W.MAMBA130M
+METRIC = "selective-scan state-updates/s (B·D·L·N) & HBM GB/s vs roofline, 1×B200"
+SFU_EX2_PER_CLK_PER_SM = 16  # MUFU.EX2 results per clock per SM (compute capability 10.0)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_SM_MHZ = 1965.0
+
+# NVML clock-event reason bits
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MHZ}, "fallback"
+
+
+def algorithmic_bytes(w: W.Workload) -> int:
+    """Compulsory HBM bytes of one forward: u, delta, (z) read and y written
+    once per (b, d, l); B and C read once per (b, n, l); A, D, bias per
+    channel; last_state written once per (b, d, n)."""
+    ein = 2 if w.dtype == torch.bfloat16 else 4
+    eout = 2 if (w.out_dtype or w.dtype) == torch.bfloat16 else 4
+    bdl = w.batch * w.dim * w.seqlen
+    per_bdl = (2 + (1 if w.has_z else 0)) * ein + eout
+    bc = 2 * w.batch * w.dstate * w.seqlen * ein
+    params = w.dim * w.dstate * 4 + w.dim * 4 * ((w.D_kind != "none") + (w.bias_kind != "none"))
+    last = w.batch * w.dim * w.dstate * 4 if w.return_last_state else 0
+    return bdl * per_bdl + bc + params + last
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, max clock, clock-event reasons) in a thread."""
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no clocks
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if self.nv is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        names = [n for bit, n in _REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w: W.Workload, rank: int) -> W.Workload:
+    """Each rank runs its own problem of the same shape (its own seed)."""
+    return W.with_shape(w, seed=w.seed + 1000003 * rank)
+
+
+def cpu_oracle_sample(w: W.Workload, target_s: float = 10.0):
+    """The oracle, as it stands, on all host cores over a bounded sample of the
+    workload's rows (rows of batch entry 0, all L steps): returns
+    (updates/s, threads, description)."""
+    import oracle
+    inp = W.make_inputs(W.with_shape(w, batch=1))
+    threads = oracle.max_threads()
+
+    def run(rows):
+        sl = lambda t: None if t is None else t[:, :rows]  # noqa: E731
+        pd = lambda t: None if t is None else t[:rows]  # noqa: E731
+        t0 = time.perf_counter()
+        oracle.selective_scan(sl(inp["u"]), sl(inp["delta"]), inp["A"][:rows], inp["B"], inp["C"],
+                              D=pd(inp["D"]), z=sl(inp["z"]), delta_bias=pd(inp["delta_bias"]),
+                              delta_softplus=w.delta_softplus,
+                              return_last_state=w.return_last_state, nthreads=threads)
+        return time.perf_counter() - t0
+
+    rows = min(w.dim, max(threads, 1))
+    dt = run(rows)
+    if dt < target_s / 4 and rows < w.dim:
+        rows = int(min(w.dim, max(rows, rows * target_s / max(dt, 1e-6))))
+        dt = run(rows)
+    updates = rows * w.seqlen * w.dstate
+    desc = (f"{rows} of {w.batch * w.dim} (b, d) rows (batch entry 0, channels 0..{rows - 1}), "
+            f"all {w.seqlen} steps, N={w.dstate}: {updates:.3e} updates in {dt:.2f} s")
+    return updates / dt, threads, desc
+
+
+def bench_reference(args, w, world, rank):
+    """--impl reference: the fp64 oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    inp = W.make_inputs(W.with_shape(w, batch=1))
+    threads = oracle.max_threads()
+    # rows per step so that warm-up + timed steps take about a minute
+    probe_rows = min(w.dim, threads)
+    t0 = time.perf_counter()
+    oracle.selective_scan(inp["u"][:, :probe_rows], inp["delta"][:, :probe_rows],
+                          inp["A"][:probe_rows], inp["B"], inp["C"], delta_softplus=True,
+                          nthreads=threads)
+    per_row = (time.perf_counter() - t0) / probe_rows
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(w.dim, budget / max(per_row, 1e-9))))
+    sl = lambda t: None if t is None else t[:, :rows]  # noqa: E731
+    pd = lambda t: None if t is None else t[:rows]  # noqa: E731
+
+    def step():
+        oracle.selective_scan(sl(inp["u"]), sl(inp["delta"]), inp["A"][:rows], inp["B"], inp["C"],
+                              D=pd(inp["D"]), z=sl(inp["z"]), delta_bias=pd(inp["delta_bias"]),
+                              delta_softplus=w.delta_softplus,
+                              return_last_state=w.return_last_state, nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    updates = rows * w.seqlen * w.dstate
+    value = updates / dt
+    sample = (f"each step: {rows} of {w.batch * w.dim} (b, d) rows (batch entry 0), all "
+              f"{w.seqlen} steps, N={w.dstate} ({updates:.3e} updates)")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "updates/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox4x32-10)",
+            "config": dict(w.describe(), sample=sample),
+            "cpu_baseline": {"value": value, "unit": "updates/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "updates/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def bench_ours(args, w, world, rank, local):
+    peaks, peak_src = measured_peaks()
+    dev = torch.device("cuda", local)
+    wr = rank_workload(w, rank)
+    host = W.make_inputs(wr, pin=True)
+    names_in = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    d = {k: (host[k].to(dev, non_blocking=True) if host[k] is not None else None) for k in names_in}
+    out_dtype = host["out_dtype"]
+    y = torch.empty(host["u"].shape, dtype=out_dtype, device=dev)
+    last = (torch.empty((wr.batch, wr.dim, wr.dstate), dtype=torch.float32, device=dev)
+            if wr.return_last_state else None)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def launch():
+        selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
+                       delta_bias=d["delta_bias"], delta_softplus=wr.delta_softplus,
+                       last_state=last, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize(dev)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            launch()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    my_ms = sum(kernel_ms) / len(kernel_ms)
+    ms = max_over_ranks(my_ms, world)
+    updates = w.updates * world
+    value = updates / (ms * 1e-3)
+
+    # end to end through the host-buffer entry point: pinned inputs in, y out
+    host["y"] = torch.empty(y.shape, dtype=out_dtype).pin_memory()
+    host["last_state"] = (torch.empty(last.shape, dtype=torch.float32).pin_memory()
+                          if last is not None else None)
+    dd = dict(d, y=y, last_state=last)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names_in if host[k] is not None)
+    d2h = host["y"].numel() * host["y"].element_size() + (
+        host["last_state"].numel() * 4 if last is not None else 0)
+    e2e_steps = max(1, min(args.steps, 20))
+    for _ in range(2):
+        selscan.ss_fwd_hostio(host, dd, delta_softplus=wr.delta_softplus, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        selscan.ss_fwd_hostio(host, dd, delta_softplus=wr.delta_softplus, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    barrier(world)
+
+    # roofline of the scan kernel: exps at the SFU rate; bytes at HBM bandwidth
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sm_max = float(peaks.get("sm_max_mhz") or FALLBACK_SM_MHZ)
+    sfu_peak = SFU_EX2_PER_CLK_PER_SM * sms * sm_max * 1e6           # ex2/s
+    achieved_ex2 = w.updates / (my_ms * 1e-3)
+    nbytes = algorithmic_bytes(w)
+    hbm_gbs = nbytes / (my_ms * 1e-3) / 1e9
+    hbm_peak = float(peaks.get("hbm_gbs") or FALLBACK_HBM_GBS)
+    t_sfu = w.updates / sfu_peak
+    t_hbm = nbytes / (hbm_peak * 1e9)
+    roofline_ms = max(t_sfu, t_hbm) * 1e3
+    traffic = None
+    prof = args.traffic_bytes
+    if prof:
+        traffic = prof
+
+    lanes, warps = selscan.ss_fwd_heuristic(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, out_dtype)
+    line = {
+        "metric": METRIC, "value": value, "unit": "updates/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == torch.float32 else "bf16 in/out, f32 arithmetic",
+        "data": "synthetic (seeded Philox4x32-10 + Box-Muller)",
+        "config": dict(w.describe(), parallelism=f"{world} independent problem(s), one per GPU",
+                       l2="flushed before every timed step (write of %d MB)" % (flush.numel() >> 20),
+                       lanes_per_row=lanes, warps_per_block=warps),
+        "roofline": {"bound": "alu", "achieved": achieved_ex2 / 1e12, "peak": sfu_peak / 1e12,
+                     "unit": "T ex2/s", "frac": achieved_ex2 / sfu_peak, "traffic": traffic,
+                     "peak_source": f"derived: {SFU_EX2_PER_CLK_PER_SM} ex2/clk/SM x {sms} SMs x "
+                                    f"{sm_max:.0f} MHz ({peak_src} max SM clock)",
+                     "roofline_ms": roofline_ms, "frac_of_roofline_time": roofline_ms / ms},
+        "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": hbm_peak, "frac": hbm_gbs / hbm_peak,
+                "algorithmic_bytes": nbytes, "peak_source": peak_src},
+        "e2e": {"value": updates / (e2e_ms * 1e-3), "unit": "updates/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "api": "ss_fwd_hostio (pinned host buffers)"},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+        "kernel_ms": {"min": min(kernel_ms), "median": statistics.median(kernel_ms),
+                      "max": max(kernel_ms)},
+    }
+    del flush
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_sample(w)
+        line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    return line if rank == 0 else None
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per launch of the scan kernel from an ncu capture")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        # The oracle runs on rank 0's host cores only; other ranks do no work.
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        line = bench_reference(args, w, 1, 0)
+        print(json.dumps(line), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl ours needs a CUDA device")
+    world, rank, local = dist_setup(args)
+    try:
+        line = bench_ours(args, w, world, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

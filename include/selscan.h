@@ -1,0 +1,149 @@
+/*
+ * libselscan -- selective-scan forward on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operation is the selective scan of Mamba as the selective_scan_ref
+ * walkthrough defines it ("Mamba代码实战：手把手教你用PyTorch复现选择性扫描核心逻辑
+ * （附避坑指南）"), for every batch b, channel d, step l and state n:
+ *
+ *   delta'[b,d,l] = softplus(delta[b,d,l] + delta_bias[d])   (delta_softplus != 0)
+ *                 = exp(delta[b,d,l] + delta_bias[d])        (delta_softplus == 0)
+ *                                                             -- §2.2 delta的预处理
+ *   h[b,d,n] <- exp(delta' * A[d,n]) * h[b,d,n] + delta' * B[b,n,l] * u[b,d,l],
+ *                                           h starting at 0   -- §3.1, §3.2
+ *   y[b,d,l] = sum_n C[b,n,l] * h[b,d,n] + D[d] * u[b,d,l]    -- §3.2, §3.3
+ *   y[b,d,l] *= z[b,d,l] * sigmoid(z[b,d,l])  when z is given  -- §3.3
+ *   last_state[b,d,n] = h[b,d,n] after step L-1               -- §6 完整实现与测试
+ *
+ * softplus is torch's default (linear above 20).  The sum over n pairs the
+ * state with C[b,n,l], as the mamba-minimal page writes it ("Mamba-minimal
+ * 项目解析", 关键技术点 §1).  The argument list mirrors the page's
+ * selective_scan_ref(u, delta, A, B, C, D, delta_bias, delta_softplus,
+ * return_last_state) plus the z gate, the output buffers and a stream.
+ *
+ * Layout (row-major, innermost index contiguous, no padding or strides):
+ *   u, delta, z, y : (batch, dim, seqlen)      -- §2.1 初始化参数
+ *   A              : (dim, dstate)   float32
+ *   B, C           : (batch, dstate, seqlen)
+ *   D, delta_bias  : (dim)           float32
+ *   last_state     : (batch, dim, dstate) float32
+ * u, delta, B, C and z share `in_dtype`; y has `out_dtype`.
+ *
+ * Ownership: every pointer is caller-owned; the library allocates nothing,
+ * keeps no state between calls and may be called from several threads.
+ *
+ * Errors: arguments are validated on the host before anything is launched;
+ * a rejected call returns a status other than SS_OK and touches no memory.
+ * Execution is asynchronous on `stream`; a launch failure returns
+ * SS_ERR_CUDA, and faults during execution surface at the caller's next
+ * synchronisation with that stream.
+ */
+#ifndef SELSCAN_H
+#define SELSCAN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SS_VERSION 100 /* 1.0.0 */
+
+typedef enum {
+    SS_OK = 0,
+    SS_ERR_NULL_POINTER = 1,       /* a required pointer is NULL */
+    SS_ERR_BAD_SHAPE = 2,          /* a size is negative or too large */
+    SS_ERR_UNSUPPORTED_DTYPE = 3,  /* dtype pair not in {f32->f32, bf16->bf16, bf16->f32} */
+    SS_ERR_UNSUPPORTED_DSTATE = 4, /* dstate outside 1..64 */
+    SS_ERR_MISALIGNED = 5,         /* a pointer is not aligned to its element size */
+    SS_ERR_CUDA = 6,               /* the CUDA runtime reported an error */
+    SS_ERR_BAD_CONFIG = 7          /* ss_fwd_with_config: unsupported launch shape */
+} ss_status;
+
+typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
+
+/* A CUDA stream handle; the same object as cudaStream_t / CUstream.  NULL is
+ * the legacy default stream. */
+typedef struct CUstream_st *ss_stream_t;
+
+typedef struct {
+    int64_t batch;     /* B >= 0 */
+    int64_t dim;       /* D >= 0 (channels) */
+    int64_t seqlen;    /* L >= 0 (steps) */
+    int64_t dstate;    /* N in 1..64 (states per channel) */
+    ss_dtype in_dtype;  /* u, delta, B, C, z */
+    ss_dtype out_dtype; /* y: in_dtype, or SS_F32 for bf16 inputs */
+} ss_desc;
+
+/*
+ * Selective-scan forward on the device.
+ *   u, delta      device, (B, D, L) in_dtype, required
+ *   A             device, (D, N) float32, required (the caller applies
+ *                 A = -exp(A_log) if that is its parameterisation)
+ *   B, C          device, (B, N, L) in_dtype, required
+ *   D             device, (D,) float32, or NULL for no skip term
+ *   z             device, (B, D, L) in_dtype, or NULL for no gate
+ *   delta_bias    device, (D,) float32, or NULL for no bias
+ *   delta_softplus  non-zero: softplus; zero: exp
+ *   y             device, (B, D, L) out_dtype, required (may not alias inputs)
+ *   last_state    device, (B, D, N) float32, or NULL (= return_last_state off)
+ *   stream        the stream the work is queued on
+ * Every pointer must be aligned to its element size.  Sizes with B*D == 0 or
+ * L == 0 are valid: with L == 0 the last state (if asked for) is all zeros.
+ * Arithmetic: float32 throughout (state, products and sums), whatever the
+ * input dtype; results are bitwise reproducible run to run for a given
+ * device, shape and pointer alignment.
+ */
+ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                 const void *B, const void *C, const float *D, const void *z,
+                 const float *delta_bias, int delta_softplus, void *y, float *last_state,
+                 ss_stream_t stream);
+
+/*
+ * As ss_fwd, with the launch shape chosen by the caller instead of by the
+ * library's heuristic (for autotuning).  lanes_per_row in {1,2,4,8,16,32}
+ * is how many lanes of a warp share one (b, d) row, each lane taking 8
+ * consecutive steps of every chunk; warps_per_block in {1,2,4,8}.  Values of
+ * 0 pick the heuristic's choice.  Results are identical for every shape up
+ * to float32 rounding order.  Returns SS_ERR_BAD_CONFIG for other values.
+ */
+ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
+                             const float *A, const void *B, const void *C, const float *D,
+                             const void *z, const float *delta_bias, int delta_softplus,
+                             void *y, float *last_state, int lanes_per_row,
+                             int warps_per_block, ss_stream_t stream);
+
+/*
+ * Launch shape ss_fwd would use for `desc` (lanes per row, warps per block).
+ * Returns SS_OK, or the status ss_fwd would return for a bad descriptor.
+ */
+ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *warps_per_block);
+
+/*
+ * Host-buffer form: copies the inputs from host memory into caller-owned
+ * device staging buffers, runs ss_fwd, and copies y (and last_state) back to
+ * host memory, all queued on `stream` (one cudaMemcpyAsync per buffer).  The
+ * host buffers should be page-locked for the copies to be asynchronous; the
+ * caller synchronises `stream` before reading the results.
+ *   h_*  host pointers with the shapes and dtypes of ss_fwd (h_D, h_z,
+ *        h_delta_bias, h_last_state may be NULL exactly when the matching
+ *        device buffer is NULL)
+ *   d_*  device buffers of the same sizes, used as ss_fwd's arguments
+ */
+ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delta,
+                        const float *h_A, const void *h_B, const void *h_C, const float *h_D,
+                        const void *h_z, const float *h_delta_bias, int delta_softplus,
+                        void *h_y, float *h_last_state, void *d_u, void *d_delta, float *d_A,
+                        void *d_B, void *d_C, float *d_D, void *d_z, float *d_delta_bias,
+                        void *d_y, float *d_last_state, ss_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *ss_status_string(ss_status status);
+
+/* SS_VERSION of the built library. */
+int ss_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SELSCAN_H */

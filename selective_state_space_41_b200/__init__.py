@@ -1,0 +1,15 @@
+"""libselscan: the Mamba selective-scan forward as hand-written sm_100a CUDA
+kernels behind a C ABI (``include/selscan.h``), with a thin Python binding.
+
+    from selective_state_space_41_b200 import selective_scan_fwd
+    y, last = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias,
+                                 delta_softplus=True, return_last_state=True)
+
+``workloads`` and ``gen`` hold the synthetic workloads and their seeded input
+generator.
+"""
+from .selscan import (SS_BF16, SS_F32, SelscanError, lib, selective_scan_fwd, ss_fwd,  # noqa: F401
+                      ss_fwd_heuristic, ss_fwd_hostio, ss_status_string, ss_version)
+
+__all__ = ["selective_scan_fwd", "ss_fwd", "ss_fwd_heuristic", "ss_fwd_hostio",
+           "ss_status_string", "ss_version", "SelscanError", "SS_F32", "SS_BF16", "lib"]

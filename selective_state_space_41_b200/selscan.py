@@ -1,0 +1,178 @@
+"""Python binding of libselscan (argument marshalling only).
+
+Every function here maps torch tensors to the pointers, sizes and stream of
+the C entry points of ``include/selscan.h`` and calls them; the computation
+runs in the library's CUDA kernels.  PyTorch supplies device memory and the
+current stream.  There is no fallback: if ``libselscan.so`` is missing or
+fails to load, every call raises.
+
+The Python names match the C entry points (``ss_fwd``, ``ss_fwd_with_config``,
+``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_status_string``,
+``ss_version``); ``selective_scan_fwd`` is the allocate-and-call convenience
+form with the argument order of the walkthrough's selective_scan_ref
+("Mamba代码实战：手把手教你用PyTorch复现选择性扫描核心逻辑（附避坑指南）", §6).
+"""
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libselscan.so")
+
+SS_F32, SS_BF16 = 0, 1
+_DTYPE_CODE = {torch.float32: SS_F32, torch.bfloat16: SS_BF16}
+STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL_POINTER", 2: "SS_ERR_BAD_SHAPE",
+                3: "SS_ERR_UNSUPPORTED_DTYPE", 4: "SS_ERR_UNSUPPORTED_DSTATE",
+                5: "SS_ERR_MISALIGNED", 6: "SS_ERR_CUDA", 7: "SS_ERR_BAD_CONFIG"}
+
+# Names the header declares; the ABI test checks each is exported.
+EXPORTS = ("ss_fwd", "ss_fwd_with_config", "ss_fwd_heuristic", "ss_fwd_hostio",
+           "ss_status_string", "ss_version")
+
+
+class SelscanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({ss_status_string(status)})")
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded ``libselscan.so`` (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libselscan.so not built ({LIB_PATH}); run "
+                               "`python -m selective_state_space_41_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        DP = ctypes.POINTER(Desc)
+        L.ss_fwd.restype = I
+        L.ss_fwd.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
+        L.ss_fwd_with_config.restype = I
+        L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, I, I, P]
+        L.ss_fwd_heuristic.restype = I
+        L.ss_fwd_heuristic.argtypes = [DP, ctypes.POINTER(I), ctypes.POINTER(I)]
+        L.ss_fwd_hostio.restype = I
+        L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P]
+        L.ss_status_string.restype = ctypes.c_char_p
+        L.ss_status_string.argtypes = [I]
+        L.ss_version.restype = I
+        L.ss_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def ss_status_string(status: int) -> str:
+    return lib().ss_status_string(int(status)).decode()
+
+
+def ss_version() -> int:
+    return int(lib().ss_version())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype=None) -> Desc:
+    """A descriptor from sizes and torch dtypes (or SS_F32 / SS_BF16 codes)."""
+    code = lambda t: _DTYPE_CODE[t] if isinstance(t, torch.dtype) else int(t)  # noqa: E731
+    return Desc(int(batch), int(dim), int(seqlen), int(dstate), code(in_dtype),
+                code(out_dtype if out_dtype is not None else in_dtype))
+
+
+def _contig(t):
+    """The C ABI takes dense row-major tensors; make them so (as the
+    walkthrough's §4.1 does before its kernel call)."""
+    return None if t is None else (t if t.is_contiguous() else t.contiguous())
+
+
+def _check(status, where):
+    if status != 0:
+        raise SelscanError(status, where)
+
+
+def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
+           last_state=None, stream=None, lanes_per_row=None, warps_per_block=None):
+    """Queue the forward on ``stream`` (default: the current stream).
+
+    u, delta, z, y: (batch, dim, L); A: (dim, N) float32; B, C: (batch, N, L);
+    D, delta_bias: (dim,) float32; last_state: (batch, dim, N) float32.
+    ``lanes_per_row`` / ``warps_per_block`` select ``ss_fwd_with_config``.
+    Raises SelscanError on a rejected call.
+    """
+    u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
+    if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
+        raise ValueError("outputs must be contiguous")
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    desc = make_desc(batch, dim, L, N, u.dtype, y.dtype)
+    args = (ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+            _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(y), _ptr(last_state))
+    s = _stream_handle(stream, u.device)
+    if lanes_per_row is None and warps_per_block is None:
+        _check(lib().ss_fwd(*args, s), "ss_fwd")
+    else:
+        _check(lib().ss_fwd_with_config(*args, int(lanes_per_row or 0), int(warps_per_block or 0), s),
+               "ss_fwd_with_config")
+
+
+def ss_fwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None):
+    """(lanes_per_row, warps_per_block) the library picks for these sizes."""
+    desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
+    lanes, warps = ctypes.c_int(), ctypes.c_int()
+    _check(lib().ss_fwd_heuristic(ctypes.byref(desc), ctypes.byref(lanes), ctypes.byref(warps)),
+           "ss_fwd_heuristic")
+    return lanes.value, warps.value
+
+
+def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None):
+    """Host-buffer form: ``host`` and ``dev`` map u, delta, A, B, C, D, z,
+    delta_bias, y, last_state to host (ideally pinned) and device tensors of
+    the same shapes (optional entries None in both).  Queues copies in, the
+    forward, and copies of y / last_state out on ``stream``."""
+    g = lambda m, k: m.get(k)  # noqa: E731
+    batch, dim, L = host["u"].shape
+    N = host["A"].shape[-1]
+    desc = make_desc(batch, dim, L, N, host["u"].dtype, host["y"].dtype)
+    names_in = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    h_in = [_ptr(g(host, k)) for k in names_in]
+    d_all = [_ptr(g(dev, k)) for k in names_in + ("y", "last_state")]
+    s = _stream_handle(stream, dev["u"].device)
+    _check(lib().ss_fwd_hostio(ctypes.byref(desc), *h_in, 1 if delta_softplus else 0,
+                               _ptr(host["y"]), _ptr(g(host, "last_state")), *d_all, s),
+           "ss_fwd_hostio")
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+                       return_last_state=False, out_dtype=None, stream=None):
+    """y (and the last state) of the selective scan, computed by libselscan.
+
+    Same arguments as the walkthrough's selective_scan_ref, plus the z gate.
+    Inputs must be CUDA tensors; y is allocated in ``out_dtype`` (default:
+    u's dtype), last_state in float32.
+    """
+    if not u.is_cuda:
+        raise ValueError("selective_scan_fwd runs on CUDA tensors only")
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    y = torch.empty((batch, dim, L), dtype=out_dtype or u.dtype, device=u.device)
+    last = (torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
+            if return_last_state else None)
+    ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
+           last_state=last, stream=stream)
+    return (y, last) if return_last_state else y

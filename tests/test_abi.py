@@ -1,0 +1,94 @@
+"""The C-ABI library: it loads, exports every entry point the header declares,
+and rejects bad arguments on the host, before any CUDA call (so these run
+without a GPU: no pointer given here is ever dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_41_b200 import build, selscan
+
+HEADER = os.path.join(build.INCLUDE, "selscan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_selscan()
+    return selscan.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(ss_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert sorted(selscan.EXPORTS) == declared_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+def test_version_and_strings(lib):
+    assert selscan.ss_version() == 100
+    for code, name in selscan.STATUS_NAMES.items():
+        assert selscan.ss_status_string(code) and selscan.ss_status_string(code) != "unknown status"
+    assert selscan.ss_status_string(99) == "unknown status"
+
+
+def _desc(**kw):
+    d = dict(batch=2, dim=3, seqlen=16, dstate=4, in_dtype=0, out_dtype=0)
+    d.update(kw)
+    return selscan.Desc(**d)
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 64 KiB-aligned, never dereferenced
+ODD = ctypes.c_void_p(0x10001)       # not aligned to any element size
+
+
+def _call(lib, desc, u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None, bias=None,
+          y=FAKE, last=None):
+    return lib.ss_fwd(ctypes.byref(desc) if desc is not None else None, u, delta, A, B, C, D, z,
+                      bias, 1, y, last, None)
+
+
+def test_rejections_before_any_launch(lib):
+    assert _call(lib, None) == 1                                   # NULL descriptor
+    assert _call(lib, _desc(seqlen=-1)) == 2                       # negative size
+    assert _call(lib, _desc(batch=1 << 40, dim=1 << 40)) == 2      # overflow
+    assert _call(lib, _desc(dstate=0)) == 4
+    assert _call(lib, _desc(dstate=65)) == 4
+    assert _call(lib, _desc(in_dtype=0, out_dtype=1)) == 3         # f32 -> bf16 not offered
+    assert _call(lib, _desc(in_dtype=2)) == 3
+    assert _call(lib, _desc(), u=None) == 1
+    assert _call(lib, _desc(), A=None) == 1
+    assert _call(lib, _desc(), y=None) == 1
+    assert _call(lib, _desc(), u=ODD) == 5
+    assert _call(lib, _desc(), D=ODD) == 5
+    assert _call(lib, _desc(in_dtype=1, out_dtype=1), z=ctypes.c_void_p(0x10003)) == 5
+    # empty problems need no pointers at all
+    assert _call(lib, _desc(batch=0), u=None, delta=None, A=None, B=None, C=None, y=None) == 0
+    assert _call(lib, _desc(seqlen=0), u=None, delta=None, B=None, C=None, y=None) == 0
+
+
+def test_bad_launch_shapes_rejected(lib):
+    d = _desc()
+    args = (ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE, None)
+    assert lib.ss_fwd_with_config(*args, 3, 4, None) == 7
+    assert lib.ss_fwd_with_config(*args, 64, 4, None) == 7
+    assert lib.ss_fwd_with_config(*args, 4, 3, None) == 7
+
+
+def test_hostio_rejections(lib):
+    d = _desc()
+    P = FAKE
+    base = [P, P, P, P, P, None, None, None]   # h_u h_delta h_A h_B h_C h_D h_z h_bias
+    dev = [P, P, P, P, P, None, None, None, P, None]
+    # D given on the host but not on the device
+    base_d = [P, P, P, P, P, P, None, None]
+    assert lib.ss_fwd_hostio(ctypes.byref(d), *base_d, 1, P, None, *dev, None) == 1
+    assert lib.ss_fwd_hostio(None, *base, 1, P, None, *dev, None) == 1
