@@ -70,37 +70,46 @@ int sm_count() {
     return v;
 }
 
+// Dynamic shared memory of one block: B and C of one chunk for the state
+// bucket as fp32, plus a raw copy in the input dtype (see the kernel).
+size_t smem_for(const ss_desc *desc, int lanes, int warps) {
+    return selscan::smem_bytes(dtype_size(desc->in_dtype), selscan::state_bucket((int)desc->dstate),
+                               lanes, warps);
+}
+
 // Lanes per row: enough (row, lane) pairs for about 1024 threads per SM, but
-// no more lanes than the sequence can feed with 8 steps each.
+// no more lanes than the sequence can feed with 8 steps each, and a chunk
+// whose B and C fit in a quarter of an SM's shared memory.
 void heuristic(const ss_desc *desc, int64_t rows, int sms, int *lanes, int *warps) {
     int w = 1;
     const int64_t target = (int64_t)sms * 1024;
     while (w < 32 && rows * w < target) w *= 2;
     while (w > 1 && (int64_t)w * kItems / 2 >= desc->seqlen) w /= 2;
+    while (w > 1 && smem_for(desc, w, 4) > selscan::kMaxSmemBytes / 4) w /= 2;
     *lanes = w;
     *warps = 4;
 }
 
 // The launcher for the state bucket that holds n (4, 8, 16, 32 or 64).
 #define SS_PICK_BUCKET(PREFIX)                                            \
-    cudaError_t (*fn)(int, dim3, dim3, cudaStream_t, const FwdParams &) = \
+    cudaError_t (*fn)(int, dim3, dim3, size_t, cudaStream_t, const FwdParams &) = \
         n <= 4 ? selscan::PREFIX##_n4                                     \
         : n <= 8 ? selscan::PREFIX##_n8                                   \
         : n <= 16 ? selscan::PREFIX##_n16                                 \
         : n <= 32 ? selscan::PREFIX##_n32                                 \
                   : selscan::PREFIX##_n64;                                \
-    return fn(lanes, grid, block, s, p);
+    return fn(lanes, grid, block, smem, s, p);
 
-cudaError_t launch_f32_f32(int n, int lanes, dim3 grid, dim3 block, cudaStream_t s,
+cudaError_t launch_f32_f32(int n, int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                            const FwdParams &p) {
     SS_PICK_BUCKET(launch_f32_f32)
 }
-cudaError_t launch_bf16_bf16(int n, int lanes, dim3 grid, dim3 block, cudaStream_t s,
-                             const FwdParams &p) {
+cudaError_t launch_bf16_bf16(int n, int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           const FwdParams &p) {
     SS_PICK_BUCKET(launch_bf16_bf16)
 }
-cudaError_t launch_bf16_f32(int n, int lanes, dim3 grid, dim3 block, cudaStream_t s,
-                            const FwdParams &p) {
+cudaError_t launch_bf16_f32(int n, int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           const FwdParams &p) {
     SS_PICK_BUCKET(launch_bf16_f32)
 }
 
@@ -141,6 +150,8 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     if (lanes == 0) lanes = h_lanes;
     if (warps == 0) warps = h_warps;
 
+    const size_t smem = smem_for(desc, lanes, warps);
+    if (smem > selscan::kMaxSmemBytes) return SS_ERR_BAD_CONFIG;
     const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
     const int64_t dtiles = (desc->dim + rows_per_block - 1) / rows_per_block;
     const int64_t blocks = dtiles * desc->batch;
@@ -170,11 +181,11 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     const int n = p.dstate;
     cudaError_t err;
     if (desc->in_dtype == SS_F32)
-        err = launch_f32_f32(n, lanes, grid, block, s, p);
+        err = launch_f32_f32(n, lanes, grid, block, smem, s, p);
     else if (desc->out_dtype == SS_BF16)
-        err = launch_bf16_bf16(n, lanes, grid, block, s, p);
+        err = launch_bf16_bf16(n, lanes, grid, block, smem, s, p);
     else
-        err = launch_bf16_f32(n, lanes, grid, block, s, p);
+        err = launch_bf16_f32(n, lanes, grid, block, smem, s, p);
     return err == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 

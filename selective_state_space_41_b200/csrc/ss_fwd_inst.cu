@@ -8,20 +8,44 @@
 
 namespace selscan {
 
-cudaError_t SS_INST_NAME(int lanes, dim3 grid, dim3 block, cudaStream_t s, const FwdParams &p) {
-    using Tin = SS_INST_TIN;
-    using Tout = SS_INST_TOUT;
-    constexpr int kN = SS_INST_NMAX;
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Launch one instance; above the 48 KB default the kernel must opt in to
+// more dynamic shared memory, once per device.
+template <int kW>
+cudaError_t launch_one(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p) {
+    auto kernel = ss_fwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kW>;
+    if (smem > 48 * 1024) {
+        static bool opted_in[kMaxDevices];
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices || !opted_in[dev]) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kMaxSmemBytes);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < kMaxDevices) opted_in[dev] = true;
+        }
+    }
+    kernel<<<grid, block, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t SS_INST_NAME(int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                         const FwdParams &p) {
     switch (lanes) {
-        case 1: ss_fwd_kernel<Tin, Tout, kN, 1><<<grid, block, 0, s>>>(p); break;
-        case 2: ss_fwd_kernel<Tin, Tout, kN, 2><<<grid, block, 0, s>>>(p); break;
-        case 4: ss_fwd_kernel<Tin, Tout, kN, 4><<<grid, block, 0, s>>>(p); break;
-        case 8: ss_fwd_kernel<Tin, Tout, kN, 8><<<grid, block, 0, s>>>(p); break;
-        case 16: ss_fwd_kernel<Tin, Tout, kN, 16><<<grid, block, 0, s>>>(p); break;
-        case 32: ss_fwd_kernel<Tin, Tout, kN, 32><<<grid, block, 0, s>>>(p); break;
+        case 1: return launch_one<1>(grid, block, smem, s, p);
+        case 2: return launch_one<2>(grid, block, smem, s, p);
+        case 4: return launch_one<4>(grid, block, smem, s, p);
+        case 8: return launch_one<8>(grid, block, smem, s, p);
+        case 16: return launch_one<16>(grid, block, smem, s, p);
+        case 32: return launch_one<32>(grid, block, smem, s, p);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace selscan

@@ -10,7 +10,7 @@
 namespace selscan {
 
 #define SS_DECLARE_LAUNCHER(NAME) \
-    cudaError_t NAME(int lanes, dim3 grid, dim3 block, cudaStream_t s, const FwdParams &p);
+    cudaError_t NAME(int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p);
 
 #define SS_FOR_EACH_NBUCKET(X, PREFIX) X(PREFIX##_n4) X(PREFIX##_n8) X(PREFIX##_n16) X(PREFIX##_n32) X(PREFIX##_n64)
 
