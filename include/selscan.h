@@ -102,9 +102,11 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
  * As ss_fwd, with the launch shape chosen by the caller instead of by the
  * library's heuristic (for autotuning).  lanes_per_row in {1,2,4,8,16,32}
  * is how many lanes of a warp share one (b, d) row, each lane taking 8
- * consecutive steps of every chunk; warps_per_block in {1,2,4,8}.  Values of
- * 0 pick the heuristic's choice.  Results are identical for every shape up
- * to float32 rounding order.  Returns SS_ERR_BAD_CONFIG for other values.
+ * (up to 4 lanes) or 16 (8 lanes and more) consecutive steps of every chunk;
+ * warps_per_block in {1,2,4,8}.  Values of 0 pick the heuristic's choice.
+ * Results are identical for every shape up to float32 rounding order.
+ * Returns SS_ERR_BAD_CONFIG for other values, or when the block's shared
+ * memory for that shape would exceed 227 KB.
  */
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
                              const float *A, const void *B, const void *C, const float *D,

@@ -17,7 +17,6 @@
 namespace {
 
 using selscan::FwdParams;
-using selscan::kItems;
 
 constexpr int kMaxState = 64;
 constexpr int kMaxDevices = 64;
@@ -73,18 +72,19 @@ int sm_count() {
 // Dynamic shared memory of one block: B and C of one chunk for the state
 // bucket as fp32, plus a raw copy in the input dtype (see the kernel).
 size_t smem_for(const ss_desc *desc, int lanes, int warps) {
-    return selscan::smem_bytes(dtype_size(desc->in_dtype), selscan::state_bucket((int)desc->dstate),
-                               lanes, warps);
+    const int nmax = selscan::state_bucket((int)desc->dstate);
+    if (lanes == 1) return selscan::direct_smem_bytes(dtype_size(desc->in_dtype), nmax);
+    return selscan::smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
 }
 
 // Lanes per row: enough (row, lane) pairs for about 1024 threads per SM, but
-// no more lanes than the sequence can feed with 8 steps each, and a chunk
-// whose B and C fit in a quarter of an SM's shared memory.
+// no more lanes than the sequence can feed, and a block whose shared memory
+// fits in a quarter of an SM's.
 void heuristic(const ss_desc *desc, int64_t rows, int sms, int *lanes, int *warps) {
     int w = 1;
     const int64_t target = (int64_t)sms * 1024;
     while (w < 32 && rows * w < target) w *= 2;
-    while (w > 1 && (int64_t)w * kItems / 2 >= desc->seqlen) w /= 2;
+    while (w > 1 && (int64_t)selscan::chunk_len(w) / 2 >= desc->seqlen) w /= 2;
     while (w > 1 && smem_for(desc, w, 4) > selscan::kMaxSmemBytes / 4) w /= 2;
     *lanes = w;
     *warps = 4;

@@ -15,8 +15,14 @@ constexpr int kMaxDevices = 64;
 // Launch one instance; above the 48 KB default the kernel must opt in to
 // more dynamic shared memory, once per device.
 template <int kW>
+auto kernel_for() {
+    if constexpr (kW == 1) return ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX>;
+    else return ss_fwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kW>;
+}
+
+template <int kW>
 cudaError_t launch_one(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p) {
-    auto kernel = ss_fwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kW>;
+    auto kernel = kernel_for<kW>();
     if (smem > 48 * 1024) {
         static bool opted_in[kMaxDevices];
         int dev = 0;

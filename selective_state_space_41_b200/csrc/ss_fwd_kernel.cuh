@@ -10,20 +10,23 @@
 // reference builds (§3.1): every exp and product lives in registers.
 //
 // Work mapping.  A warp holds 32/W rows; the W lanes of a row split each
-// chunk of W*8 consecutive steps, 8 steps per lane.  For every state n a lane
-// runs its 8 steps from a zero state, recording the decays a_i and inputs b_i,
-// then the W lanes combine their (prod a, h) pairs with a shuffle scan under
-// the associative operator (a1, h1) . (a2, h2) = (a2 a1, a2 h1 + h2) (the
-// operator of "手把手用PyTorch实现Mamba的SSM层" §3.2), restricted to diagonal A.
-// The scan gives each lane its true incoming state; a second pass over the
-// recorded (a_i, b_i) then yields the states and y.  The chunk's outgoing
-// state per n stays in registers (`carry`) for the next chunk.  With W = 1 the
-// lane owns the whole row and runs the plain sequential recurrence.
+// chunk of W*K consecutive steps, K (8 or 16) steps per lane.  For every
+// state n a lane runs its K steps from a zero state, recording the decays a_i
+// and inputs b_i, then the W lanes combine their (prod a, h) pairs with a
+// shuffle scan under the associative operator
+// (a1, h1) . (a2, h2) = (a2 a1, a2 h1 + h2) (the operator of
+// "手把手用PyTorch实现Mamba的SSM层" §3.2, for diagonal A).  The scan gives each
+// lane its true incoming state; a second pass over the recorded (a_i, b_i)
+// yields the states and y.  The state leaving the chunk goes to a per-row
+// shared table for the next chunk.  With W = 1 the lane owns its row and runs
+// the plain sequential recurrence, the states in registers.
 //
-// exp(delta' A) is computed as ex2(delta' * (A log2 e)) on the SFU.  Streams
-// u, delta and z are prefetched one chunk ahead into registers; B and C rows
-// are shared by all rows of a batch and read through L1 (the lanes of a warp
-// that sit at the same steps read the same addresses).
+// exp(delta' A) is ex2(delta' * (A log2 e)) on the SFU.  Two consecutive steps
+// of one state share one packed sm_100 instruction (mul/fma .f32x2) for the
+// exponent arguments, delta' u B, the chunk decay product and y; the state
+// recurrence itself is sequential and stays scalar.  Every streamed operand
+// (u, delta, z, B, C) reaches shared memory by cp.async one chunk ahead; B and
+// C, shared by all rows of a batch entry, are converted once per block to fp32.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,7 +35,6 @@
 
 namespace selscan {
 
-constexpr int kItems = 8;  // consecutive steps per lane per chunk
 constexpr size_t kMaxSmemBytes = 227 * 1024;  // opt-in dynamic shared memory per block (sm_100)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -48,75 +50,39 @@ struct FwdParams {
     int64_t dtiles;   // row tiles per batch entry
 };
 
-// ---------------------------------------------------------------- element I/O
+// ------------------------------------------------------------ element I/O
 template <typename T>
 struct Io;
 
 template <>
 struct Io<float> {
-    static constexpr int kWords = kItems;  // one 32-bit word per element
-    __device__ __forceinline__ static void widen(const uint32_t (&w)[kWords], float (&f)[kItems]) {
-#pragma unroll
-        for (int i = 0; i < kItems; ++i) f[i] = __uint_as_float(w[i]);
-    }
-    __device__ __forceinline__ static uint32_t bits(const float *p, int64_t i) {
-        return __float_as_uint(p[i]);
-    }
-    __device__ __forceinline__ static void place(uint32_t (&w)[kWords], int i, uint32_t v) { w[i] = v; }
+    static constexpr int kUnit = 4;  // elements per 16-byte unit
+    __device__ __forceinline__ static float widen(const uint32_t *w, int i) { return __uint_as_float(w[i]); }
+    __device__ __forceinline__ static uint32_t bits(const float *p, int64_t i) { return __float_as_uint(p[i]); }
 };
 
 template <>
 struct Io<__nv_bfloat16> {
-    static constexpr int kWords = kItems / 2;  // two bf16 per word, element 2j in the low half
-    __device__ __forceinline__ static void widen(const uint32_t (&w)[kWords], float (&f)[kItems]) {
-#pragma unroll
-        for (int j = 0; j < kWords; ++j) {
-            f[2 * j] = __uint_as_float(w[j] << 16);
-            f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-        }
+    static constexpr int kUnit = 8;  // two bf16 per 32-bit word, element 2j in the low half
+    __device__ __forceinline__ static float widen(const uint32_t *w, int i) {
+        return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
     }
     __device__ __forceinline__ static uint32_t bits(const __nv_bfloat16 *p, int64_t i) {
         return reinterpret_cast<const unsigned short *>(p)[i];
     }
-    __device__ __forceinline__ static void place(uint32_t (&w)[kWords], int i, uint32_t v) {
-        w[i >> 1] |= v << (16 * (i & 1));
-    }
 };
 
-// Load steps [l0, l0 + 8) of one row as raw words; steps at or past L read 0.
-// kStream: the data is read once (u, delta, z), so keep it out of L1.
-template <typename T, bool kStream>
-__device__ __forceinline__ void load_run(uint32_t (&w)[Io<T>::kWords], const T *row, int64_t l0,
-                                         int64_t L, bool vec) {
-    constexpr int kWords = Io<T>::kWords;
-    if (vec && l0 + kItems <= L) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(row + l0);
-#pragma unroll
-        for (int j = 0; j < kWords / 4; ++j) {
-            const uint4 v = kStream ? __ldcs(p + j) : __ldg(p + j);
-            w[4 * j + 0] = v.x;
-            w[4 * j + 1] = v.y;
-            w[4 * j + 2] = v.z;
-            w[4 * j + 3] = v.w;
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < kWords; ++j) w[j] = 0u;
-#pragma unroll
-        for (int i = 0; i < kItems; ++i)
-            if (l0 + i < L) Io<T>::place(w, i, Io<T>::bits(row, l0 + i));
-    }
-}
-
-__device__ __forceinline__ void store_run(float *row, int64_t l0, int64_t L, bool vec,
-                                          const float (&v)[kItems]) {
-    if (vec && l0 + kItems <= L) {
+// Scalar (element) stores of y for steps [l0, l0 + K), guarded by L, or
+// 16-byte streaming stores when the run is complete and aligned.
+template <int K>
+__device__ __forceinline__ void store_run(float *row, int64_t l0, int64_t L, bool vec, const float (&v)[K]) {
+    if (vec && l0 + K <= L) {
         float4 *p = reinterpret_cast<float4 *>(row + l0);
-        __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
-        __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
+#pragma unroll
+        for (int j = 0; j < K / 4; ++j) __stcs(p + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
     } else {
 #pragma unroll
-        for (int i = 0; i < kItems; ++i)
+        for (int i = 0; i < K; ++i)
             if (l0 + i < L) row[l0 + i] = v[i];
     }
 }
@@ -126,18 +92,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+template <int K>
 __device__ __forceinline__ void store_run(__nv_bfloat16 *row, int64_t l0, int64_t L, bool vec,
-                                          const float (&v)[kItems]) {
-    if (vec && l0 + kItems <= L) {
-        uint4 q;
-        q.x = pack_bf16x2(v[0], v[1]);
-        q.y = pack_bf16x2(v[2], v[3]);
-        q.z = pack_bf16x2(v[4], v[5]);
-        q.w = pack_bf16x2(v[6], v[7]);
-        __stcs(reinterpret_cast<uint4 *>(row + l0), q);
+                                          const float (&v)[K]) {
+    if (vec && l0 + K <= L) {
+        uint4 *p = reinterpret_cast<uint4 *>(row + l0);
+#pragma unroll
+        for (int j = 0; j < K / 8; ++j) {
+            uint4 q;
+            q.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+            q.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+            q.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+            q.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+            __stcs(p + j, q);
+        }
     } else {
 #pragma unroll
-        for (int i = 0; i < kItems; ++i)
+        for (int i = 0; i < K; ++i)
             if (l0 + i < L) row[l0 + i] = __float2bfloat16_rn(v[i]);
     }
 }
@@ -241,40 +212,6 @@ __device__ __forceinline__ void scan_stage2(float &P0, float &h0, float &P1, flo
         : "r"(off), "n"(kSeg));
 }
 
-// float2 <-> one 64-bit register pair, for packed (f32x2) PTX operands.
-__device__ __forceinline__ unsigned long long as_u64(float2 v) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
-    return r;
-}
-__device__ __forceinline__ float2 as_f2(unsigned long long r) {
-    float2 v;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
-    return v;
-}
-
-// Scan stage for a state pair held as packed (P, h): shuffle both halves of
-// P and h `off` lanes up, then (only where the partner exists, shfl.up's
-// predicate) h = P hu + h and P = P Pu as two f32x2 instructions.
-template <int kW>
-__device__ __forceinline__ void scan_stage_x2(unsigned long long &P, unsigned long long &h, int off) {
-    constexpr int kSeg = (32 - kW) << 8;
-    asm("{\n\t.reg .pred p;\n\t.reg .b32 p0, p1, h0, h1, u0, u1, v0, v1;\n\t"
-        ".reg .b64 pu, hu;\n\t"
-        "mov.b64 {p0, p1}, %0;\n\t"
-        "mov.b64 {h0, h1}, %1;\n\t"
-        "shfl.sync.up.b32 u0|p, p0, %2, %3, -1;\n\t"
-        "shfl.sync.up.b32 u1, p1, %2, %3, -1;\n\t"
-        "shfl.sync.up.b32 v0, h0, %2, %3, -1;\n\t"
-        "shfl.sync.up.b32 v1, h1, %2, %3, -1;\n\t"
-        "mov.b64 pu, {u0, u1};\n\t"
-        "mov.b64 hu, {v0, v1};\n\t"
-        "@p fma.rn.f32x2 %1, %0, hu, %1;\n\t"
-        "@p mul.rn.f32x2 %0, %0, pu;\n\t}"
-        : "+l"(P), "+l"(h)
-        : "r"(off), "n"(kSeg));
-}
-
 // Store v to a shared-memory float2 only on the lanes where `pred` holds,
 // without a branch.
 __device__ __forceinline__ void st_shared_f2_if(float *dst, float2 v, bool pred) {
@@ -284,31 +221,45 @@ __device__ __forceinline__ void st_shared_f2_if(float *dst, float2 v, bool pred)
                  : "memory");
 }
 
-// ------------------------------------------------------------------- kernel
-// States are processed in pairs (n, n+1) held in float2 registers, so the
-// per-step arithmetic of two states is one packed sm_100 instruction
-// (fma/mul .f32x2): exponent arguments, delta' u B, the state update and the
-// output accumulation.  The two exps stay two MUFU.EX2.
-//
-// Shared memory of one block, for a chunk of Lc = 8 W steps and the state
-// bucket kNmax (states n >= N are zero rows, so they add nothing):
-//   F: float, B and C of the chunk in a pair-interleaved order: for state pair
-//      p and lane slot s, float4 number ((t kPairs + p) 4 + g) W + s holds
-//      (X[2p][i], X[2p+1][i], X[2p][i+1], X[2p+1][i+1]) for steps i = 8s + 2g
-//      and i + 1 of the chunk, X = B (t = 0) or C (t = 1).  The W slots of a
-//      row read consecutive float4s (no bank conflicts); rows that share a
-//      slot read the same address (broadcast).
-//   R: Tin, [2][kNmax][Lc], raw copy of the chunk in global order, filled by
-//      cp.async one chunk ahead (16-byte path only).
-//   With W > 1 lanes per row, two per-row tables of kNmax + 2 floats (the
-//      padding spreads rows over banks): A[d, n] log2(e), and the state that
-//      enters the next chunk.  (With W = 1 a lane owns its row and keeps both
-//      in registers.)
-__host__ __device__ constexpr int chunk_len(int w) { return w * kItems; }
+// Store v to a shared float only on the lanes where `pred` holds, without a branch.
+__device__ __forceinline__ void st_shared_f1_if(float *dst, float v, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t"
+                 "@p st.shared.f32 [%0], %1;\n\t}" ::"r"(smem_addr(dst)),
+                 "f"(v), "r"((unsigned)pred)
+                 : "memory");
+}
 
+// ------------------------------------------------------------------- kernel
+// Steps per lane per chunk for a lane count W: 8 for W <= 4 (two states per
+// iteration of the state loop), 16 for W >= 8 (one state per iteration; the
+// scan's cost is spread over twice the steps).
+#ifndef SS_K_SMALL_W
+#define SS_K_SMALL_W 8
+#endif
+#ifndef SS_K_LARGE_W
+#define SS_K_LARGE_W 16
+#endif
+__host__ __device__ constexpr int items_for(int w) { return w <= 4 ? SS_K_SMALL_W : SS_K_LARGE_W; }
+__host__ __device__ constexpr int chunk_len(int w) { return w * items_for(w); }
+
+// Shared memory of one block, for a chunk of Lc = W K steps, the state bucket
+// kNmax (states n >= N are zero rows, so they add nothing) and R rows:
+//   F : float4, B and C of the chunk as fp32: float4 number
+//       ((t kNmax + n) K/4 + q) W + s holds steps 4q..4q+3 of lane slot s for
+//       state n of X = B (t = 0) or C (t = 1).  The W slots of a row read
+//       consecutive float4s (no bank conflicts); rows that share a slot read
+//       the same address (broadcast).
+//   RB: Tin [2][kNmax][Lc], raw B and C in global order (cp.async target).
+//   RU: Tin [2 buffers][3 (u, delta, z)][R][Lc], raw streams; within a row,
+//       16-byte unit g of lane slot s sits at unit number g W + s, so each
+//       lane reads its K steps without bank conflicts.  Double-buffered: the
+//       next chunk lands while this one is read.
+//   With W > 1: two per-row tables of kNmax + 2 floats (padding spreads the
+//       rows over banks): A[d, n] log2(e), and the state entering the chunk.
 __host__ __device__ constexpr size_t smem_bytes(size_t in_size, int nmax, int w, int warps) {
-    return (2 * sizeof(float) + 2 * in_size) * (size_t)nmax * (size_t)chunk_len(w) +
-           (w > 1 ? 2 * sizeof(float) * (size_t)(nmax + 2) * (size_t)(warps * (32 / w)) : 0);
+    const size_t rows = (size_t)warps * (size_t)(32 / w), lc = (size_t)chunk_len(w);
+    return 2 * sizeof(float) * nmax * lc + 2 * in_size * nmax * lc + 6 * in_size * rows * lc +
+           (w > 1 ? 2 * sizeof(float) * (size_t)(nmax + 2) * rows : 0);
 }
 
 // State bucket (compile-time state count) for a runtime state count.
@@ -316,10 +267,14 @@ __host__ __device__ constexpr int state_bucket(int n) {
     return n <= 4 ? 4 : n <= 8 ? 8 : n <= 16 ? 16 : n <= 32 ? 32 : 64;
 }
 
-#ifndef SS_PAIR_UNROLL
-#define SS_PAIR_UNROLL 1
+#ifndef SS_Y_SCALAR
+#define SS_Y_SCALAR 0
 #endif
-constexpr int kPairUnroll = SS_PAIR_UNROLL;  // unroll of the W > 1 state-pair loop
+#ifndef SS_P_EXP
+#define SS_P_EXP 0
+#endif
+constexpr bool kYScalar = SS_Y_SCALAR != 0;  // y accumulated with scalar FMAs
+constexpr bool kPExp = SS_P_EXP != 0;        // chunk decay as 2^(A log2e sum delta')
 #ifndef SS_MIN_BLOCKS_SMALL_N
 #define SS_MIN_BLOCKS_SMALL_N 2
 #endif
@@ -331,30 +286,22 @@ struct Occupancy {
     static constexpr int kMinBlocks = kNmax <= 32 ? SS_MIN_BLOCKS_SMALL_N : 1;
 };
 
-__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
-
 template <typename Tin, typename Tout, int kNmax, int kW>
 __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kernel(const FwdParams p) {
     static_assert(kW >= 1 && kW <= 32 && (32 % kW) == 0, "lanes per row must divide 32");
-    static_assert(kItems == 8, "the F layout assumes 8 steps per lane");
+    constexpr int kK = items_for(kW);                    // steps per lane per chunk
+    static_assert(kK == 8 || kK == 16, "8 or 16 steps per lane");
+    constexpr int kJ = kK / 2;                           // step pairs per lane
     constexpr int kRowsPerWarp = 32 / kW;
-    constexpr int kChunk = chunk_len(kW);
-    constexpr int kPairs = kNmax / 2;
-    constexpr int kG = kItems / 2;                      // float4s per lane per (tensor, pair)
-    constexpr int kPairRow = kG * kW;                   // float4s per (tensor, pair) of F
-    constexpr int kUnit = 16 / (int)sizeof(Tin);        // elements per 16-byte unit
-    constexpr int kUnitsPerRow = kChunk / kUnit;        // a power of two
-    constexpr int kUnits = 2 * kNmax * kUnitsPerRow;    // 16-byte units of B and C per chunk
-    constexpr int kPairUnits = kUnits / 2;              // (unit, state pair) fill jobs
-    constexpr int kWords = Io<Tin>::kWords;
-    constexpr bool kFast = sizeof(Tin) == 2;            // bf16 inputs: SFU transforms
-    constexpr int kRowStride = kNmax + 2;               // per-row tables (W > 1)
+    constexpr int kChunk = kW * kK;
+    constexpr int kUnit = Io<Tin>::kUnit;                // elements per 16-byte unit
+    constexpr int kUnitsPerRow = kChunk / kUnit;         // a power of two
+    constexpr int kLaneUnits = kK / kUnit;               // 16-byte units per lane per stream
+    constexpr int kLaneWords = kK * (int)sizeof(Tin) / 4;
+    constexpr int kS = (kW == 1 || kK == 16) ? 1 : 2;    // states per scan iteration
+    constexpr bool kFast = sizeof(Tin) == 2;             // bf16 inputs: SFU transforms
+    constexpr int kRowStride = kNmax + 2;                // per-row tables (W > 1)
     constexpr unsigned kFull = 0xffffffffu;
-
-    extern __shared__ float4 smem[];
-    float4 *F = smem;                                                  // [2][kPairs][kPairRow]
-    Tin *R = reinterpret_cast<Tin *>(smem + 2 * kPairs * kPairRow);     // [2][kNmax][kChunk]
-    float *sA2 = reinterpret_cast<float *>(R + 2 * kNmax * kChunk);     // [rows][kRowStride]
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
@@ -362,10 +309,11 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
     const int warp = tid >> 5;
     const int seg = lane % kW;  // this lane's slot among the row's W lanes
     const int N = p.dstate;
-    const int64_t rows_per_block = (int64_t)(nthreads >> 5) * kRowsPerWarp;
+    const int rows = (nthreads >> 5) * kRowsPerWarp;
+    const int rloc = warp * kRowsPerWarp + lane / kW;    // row within the block
     const int64_t b = blockIdx.x / p.dtiles;
-    const int64_t tile = blockIdx.x % p.dtiles;
-    const int64_t d_raw = tile * rows_per_block + warp * kRowsPerWarp + lane / kW;
+    const int64_t d0 = (blockIdx.x % p.dtiles) * rows;
+    const int64_t d_raw = d0 + rloc;
     // Rows past the end mirror the last row (valid addresses) and store nothing;
     // they must still run so that every lane takes part in the shuffles.
     const bool row_ok = d_raw < p.dim;
@@ -376,36 +324,36 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
     const bool softplus = p.softplus != 0;
     const bool has_z = p.z != nullptr;
 
-    const Tin *u_row = static_cast<const Tin *>(p.u) + row * L;
-    const Tin *d_row = static_cast<const Tin *>(p.delta) + row * L;
-    const Tin *z_row = has_z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
-    const Tin *B_b = static_cast<const Tin *>(p.B) + b * N * L;
-    const Tin *C_b = static_cast<const Tin *>(p.C) + b * N * L;
+    extern __shared__ float4 smem[];
+    float4 *F = smem;                                                       // 2 kNmax kChunk / 4
+    Tin *RB = reinterpret_cast<Tin *>(smem + 2 * kNmax * (kChunk / 4));      // [2][kNmax][kChunk]
+    Tin *RU = RB + 2 * kNmax * kChunk;                                       // [2][3][rows][kChunk]
+    float *sA2 = reinterpret_cast<float *>(RU + 6 * rows * kChunk);          // [rows][kRowStride]
+    float *sCarry = sA2 + rows * kRowStride;
+    const float *rowA2 = sA2 + rloc * kRowStride;
+    float *rowCarry = sCarry + rloc * kRowStride;
+
+    const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * N * L,
+                          static_cast<const Tin *>(p.C) + b * N * L};
+    const Tin *Usrc[3] = {static_cast<const Tin *>(p.u), static_cast<const Tin *>(p.delta),
+                          static_cast<const Tin *>(p.z)};
     Tout *y_row = static_cast<Tout *>(p.y) + row * L;
 
-    // A[d, n] * log2(e) (0 for the padding states n >= N) and the state
-    // entering the chunk.  W = 1: registers (A in registers for up to 16
-    // states; more states re-read it, an L1 hit, once per chunk).  W > 1: the
-    // per-row shared tables, read by all W lanes of the row.
+    // A[d, n] log2(e) (0 for the padding states) and the state entering the
+    // chunk: registers when a lane owns its row (W = 1; A re-read per chunk,
+    // an L1 hit, above 16 states), per-row shared tables when W lanes share it.
     constexpr bool kRowInRegs = kW == 1;
     constexpr bool kA2InRegs = kRowInRegs && kNmax <= 16;
     const float *A_d = p.A + d * N;
-    float2 A2[kA2InRegs ? kPairs : 1], carry[kRowInRegs ? kPairs : 1];
-    const int rloc = warp * kRowsPerWarp + lane / kW;  // row within the block
-    float *sCarry = sA2 + rows_per_block * kRowStride;
-    const float *rowA2 = sA2 + rloc * kRowStride;
-    float *rowCarry = sCarry + rloc * kRowStride;
+    float A2[kA2InRegs ? kNmax : 1], carry[kRowInRegs ? kNmax : 1];
     if constexpr (kRowInRegs) {
 #pragma unroll
-        for (int q = 0; q < kPairs; ++q) {
-            if constexpr (kA2InRegs)
-                A2[q] = make_float2(2 * q < N ? A_d[2 * q] * kLog2e : 0.f,
-                                    2 * q + 1 < N ? A_d[2 * q + 1] * kLog2e : 0.f);
-            carry[q] = make_float2(0.f, 0.f);
+        for (int n = 0; n < kNmax; ++n) {
+            if constexpr (kA2InRegs) A2[n] = n < N ? A_d[n] * kLog2e : 0.f;
+            carry[n] = 0.f;
         }
     } else {
-        const int64_t d0 = tile * rows_per_block;
-        for (int idx = tid; idx < rows_per_block * kNmax; idx += nthreads) {
+        for (int idx = tid; idx < rows * kNmax; idx += nthreads) {
             const int r = idx / kNmax, n = idx % kNmax;
             const int64_t dr = d0 + r < p.dim ? d0 + r : p.dim - 1;
             sA2[r * kRowStride + n] = n < N ? p.A[dr * N + n] * kLog2e : 0.f;
@@ -417,214 +365,472 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
 
-    // The block's B and C for steps [c0, c0 + kChunk): 16-byte async copies
-    // into R when the whole chunk is in range and rows are aligned.
+    // Global row of block row r (mirrored past the end).
+    auto grow = [&](int r) -> int64_t {
+        const int64_t dr = d0 + r < p.dim ? d0 + r : p.dim - 1;
+        return b * p.dim + dr;
+    };
+    // Position, in elements, of chunk step e within a row of RU.
+    auto ru_pos = [&](int e) {
+        const int s = e / kK, i = e % kK;
+        return ((i / kUnit) * kW + s) * kUnit + (i % kUnit);
+    };
+    const int nstreams = has_z ? 3 : 2;
     auto chunk_async = [&](int64_t c0) { return vec && c0 + kChunk <= L; };
-    auto issue_copies = [&](int64_t c0) {
-        for (int u = tid; u < kUnits; u += nthreads) {
+    // Queue the 16-byte copies of chunk c0 into RB and RU[buf].
+    auto issue_copies = [&](int64_t c0, int buf) {
+        constexpr int kBCUnits = 2 * kNmax * kUnitsPerRow;
+        for (int u = tid; u < kBCUnits; u += nthreads) {
             const int j = u % kUnitsPerRow, rowid = u / kUnitsPerRow;
             const int t = rowid / kNmax, n = rowid % kNmax;
             if (n < N)
-                cp_async16(R + (rowid * kChunk + j * kUnit),
-                           (t ? C_b : B_b) + (int64_t)n * L + c0 + j * kUnit);
+                cp_async16(RB + (rowid * kChunk + j * kUnit), Bsrc[t] + (int64_t)n * L + c0 + j * kUnit);
+        }
+        Tin *dst = RU + buf * 3 * rows * kChunk;
+        const int uunits = nstreams * rows * kUnitsPerRow;
+        for (int u = tid; u < uunits; u += nthreads) {
+            const int j = u % kUnitsPerRow, sr = u / kUnitsPerRow;
+            const int t = sr / rows, r = sr % rows;
+            cp_async16(dst + (t * rows + r) * kChunk + ru_pos(j * kUnit),
+                       Usrc[t] + grow(r) * L + c0 + j * kUnit);
         }
         cp_async_commit();
     };
-    // One 16-byte unit (kUnit steps) of state n's row, as floats: from R, or
-    // element by element from global memory (partial or unaligned chunk);
-    // padding states read zeros.
-    auto read_unit = [&](int64_t c0, bool from_R, int t, int n, int j, float (&v)[kUnit]) {
-        if (n >= N) {
+    // B and C of chunk c0 into F as fp32: from RB, or element by element from
+    // global memory (partial or unaligned chunk); padding states get zeros.
+    auto fill_F = [&](int64_t c0, bool from_RB) {
+        constexpr int kBCUnits = 2 * kNmax * kUnitsPerRow;
+        for (int u = tid; u < kBCUnits; u += nthreads) {
+            const int j = u % kUnitsPerRow, rowid = u / kUnitsPerRow;
+            const int t = rowid / kNmax, n = rowid % kNmax;
+            float v[kUnit];
+            if (n >= N) {
 #pragma unroll
-            for (int m = 0; m < kUnit; ++m) v[m] = 0.f;
-        } else if (from_R) {
-            const uint4 raw =
-                *reinterpret_cast<const uint4 *>(R + ((t * kNmax + n) * kChunk + j * kUnit));
-            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                for (int m = 0; m < kUnit; ++m) v[m] = 0.f;
+            } else if (from_RB) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(RB + (rowid * kChunk + j * kUnit));
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-            for (int m = 0; m < kUnit; ++m) {
-                if constexpr (sizeof(Tin) == 2)
-                    v[m] = __uint_as_float((m & 1) ? (w[m >> 1] & 0xffff0000u) : (w[m >> 1] << 16));
-                else
-                    v[m] = __uint_as_float(w[m]);
+                for (int m = 0; m < kUnit; ++m) v[m] = Io<Tin>::widen(w, m);
+            } else {
+                const Tin *src = Bsrc[t] + (int64_t)n * L;
+#pragma unroll
+                for (int m = 0; m < kUnit; ++m) {
+                    const int64_t l = c0 + j * kUnit + m;
+                    uint32_t bits = 0u;
+                    if (l < L) bits = Io<Tin>::bits(src, l);
+                    if constexpr (sizeof(Tin) == 2) bits <<= 16;
+                    v[m] = __uint_as_float(bits);
+                }
             }
-        } else {
-            const Tin *src = (t ? C_b : B_b) + (int64_t)n * L;
 #pragma unroll
-            for (int m = 0; m < kUnit; ++m) {
-                const int64_t l = c0 + j * kUnit + m;
-                uint32_t bits = 0u;
-                if (l < L) bits = Io<Tin>::bits(src, l);
-                if constexpr (sizeof(Tin) == 2) bits <<= 16;
-                v[m] = __uint_as_float(bits);
-            }
-        }
-    };
-    // R (or global memory) -> F in the pair-interleaved order.
-    auto fill_F = [&](int64_t c0, bool from_R) {
-        for (int u = tid; u < kPairUnits; u += nthreads) {
-            const int j = u % kUnitsPerRow, pr = u / kUnitsPerRow;  // pr = t * kPairs + pair
-            const int t = pr / kPairs, q = pr % kPairs;
-            float v0[kUnit], v1[kUnit];
-            read_unit(c0, from_R, t, 2 * q, j, v0);
-            read_unit(c0, from_R, t, 2 * q + 1, j, v1);
-#pragma unroll
-            for (int m = 0; m < kUnit; m += 2) {
-                const int e = j * kUnit + m;  // step within the chunk (even)
-                const int sl = e / kItems, g = (e % kItems) / 2;
-                F[(pr * kG + g) * kW + sl] = make_float4(v0[m], v1[m], v0[m + 1], v1[m + 1]);
+            for (int m = 0; m < kUnit; m += 4) {
+                const int e = j * kUnit + m;  // step within the chunk
+                const int s = e / kK, q = (e % kK) / 4;
+                F[(rowid * (kK / 4) + q) * kW + s] = make_float4(v[m], v[m + 1], v[m + 2], v[m + 3]);
             }
         }
     };
+    // Streams of chunk c0 into RU[buf] element by element (partial or
+    // unaligned chunk); steps past L read 0.
+    auto fill_RU_scalar = [&](int64_t c0, int buf) {
+        Tin *dst = RU + buf * 3 * rows * kChunk;
+        const int elems = nstreams * rows * kChunk;
+        for (int e = tid; e < elems; e += nthreads) {
+            const int i = e % kChunk, sr = e / kChunk;
+            const int t = sr / rows, r = sr % rows;
+            const int64_t l = c0 + i;
+            Tin v;
+            if (l < L) v = Usrc[t][grow(r) * L + l];
+            else v = Tin(0.f);
+            dst[(t * rows + r) * kChunk + ru_pos(i)] = v;
+        }
+    };
+    // This lane's K steps of stream t, as raw words.
+    auto lane_words = [&](int buf, int t, uint32_t (&w)[kLaneWords]) {
+        const Tin *src = RU + (buf * 3 + t) * rows * kChunk + rloc * kChunk;
+#pragma unroll
+        for (int g = 0; g < kLaneUnits; ++g) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(src + (g * kW + seg) * kUnit);
+            w[4 * g] = x.x, w[4 * g + 1] = x.y, w[4 * g + 2] = x.z, w[4 * g + 3] = x.w;
+        }
+    };
+    // B or C of state n for this lane's steps, as step pairs (X[2j], X[2j+1]).
+    auto load_pairs = [&](int t, int n, float2 (&X)[kJ]) {
+        const float4 *src = F + (t * kNmax + n) * (kK / 4) * kW + seg;
+#pragma unroll
+        for (int q = 0; q < kK / 4; ++q) {
+            const float4 x = src[q * kW];
+            X[2 * q] = make_float2(x.x, x.y);
+            X[2 * q + 1] = make_float2(x.z, x.w);
+        }
+    };
 
-    uint32_t wu[kWords], wd[kWords], wz[kWords];
-    {
-        const int64_t l0 = (int64_t)seg * kItems;
-        load_run<Tin, true>(wu, u_row, l0, L, vec);
-        load_run<Tin, true>(wd, d_row, l0, L, vec);
-        if (has_z) load_run<Tin, true>(wz, z_row, l0, L, vec);
-    }
-    if (L > 0 && chunk_async(0)) issue_copies(0);
+    if (L > 0 && chunk_async(0)) issue_copies(0, 0);
 
-    for (int64_t c0 = 0; c0 < L; c0 += kChunk) {
+    int buf = 0;
+    for (int64_t c0 = 0; c0 < L; c0 += kChunk, buf ^= 1) {
         const bool async_here = chunk_async(c0);
         if (async_here) cp_async_wait_all();
-        __syncthreads();  // R holds this chunk; every warp is done with F
+        __syncthreads();  // this chunk's copies have landed; every warp is done with F
         fill_F(c0, async_here);
-        __syncthreads();  // F holds this chunk; R is free
-        const bool more = c0 + kChunk < L;
-        if (more && chunk_async(c0 + kChunk)) issue_copies(c0 + kChunk);
+        if (!async_here) fill_RU_scalar(c0, buf);
+        __syncthreads();  // F and RU[buf] hold this chunk; RB is free
+        if (c0 + kChunk < L && chunk_async(c0 + kChunk)) issue_copies(c0 + kChunk, buf ^ 1);
 
-        const int64_t l0 = c0 + (int64_t)seg * kItems;
-        float uf[kItems], df[kItems];
-        Io<Tin>::widen(wu, uf);
-        Io<Tin>::widen(wd, df);
-        uint32_t wzc[kWords];
+        const int64_t l0 = c0 + (int64_t)seg * kK;
+        // delta' and delta' u per step, as step pairs; y starts at D u (§3.3).
+        float2 dlp[kJ], dup[kJ], y[kJ];
+        float dsum = 0.f;
+        {
+            uint32_t wu[kLaneWords], wd[kLaneWords];
+            lane_words(buf, 0, wu);
+            lane_words(buf, 1, wd);
+            float dl[kK];
 #pragma unroll
-        for (int j = 0; j < kWords; ++j) wzc[j] = wz[j];
-        if (more) {  // prefetch the next chunk of this lane's steps
-            load_run<Tin, true>(wu, u_row, l0 + kChunk, L, vec);
-            load_run<Tin, true>(wd, d_row, l0 + kChunk, L, vec);
-            if (has_z) load_run<Tin, true>(wz, z_row, l0 + kChunk, L, vec);
-        }
-
-        // delta' and delta' * u, duplicated into both halves of a float2 to
-        // pair with two states; steps past L become the identity (a = 1, b = 0).
-        float dl[kItems];
+            for (int i = 0; i < kK; ++i) dl[i] = delta_transform<kFast>(Io<Tin>::widen(wd, i) + bias, softplus);
+            if (c0 + kChunk > L) {  // steps past L become the identity (a = 1, b = 0)
 #pragma unroll
-        for (int i = 0; i < kItems; ++i) dl[i] = delta_transform<kFast>(df[i] + bias, softplus);
-        if (c0 + kChunk > L) {
-#pragma unroll
-            for (int i = 0; i < kItems; ++i)
-                if (l0 + i >= L) dl[i] = 0.f;
-        }
-        float2 dl2[kItems], du2[kItems], y2[kItems];
-#pragma unroll
-        for (int i = 0; i < kItems; ++i) {
-            dl2[i] = f2(dl[i]);
-            du2[i] = f2(dl[i] * uf[i]);
-            y2[i] = make_float2(Dd * uf[i], 0.f);  // skip term D u (§3.3)
-        }
-
-        const float4 *FB = F + seg, *FC = F + kPairs * kPairRow + seg;
-        // B (or C) of state pair q for this lane's 8 steps: Xp[i] = (X[2q][i], X[2q+1][i]).
-        auto load_pair = [&](const float4 *base, int q, float2 (&Xp)[kItems]) {
-#pragma unroll
-            for (int g = 0; g < kG; ++g) {
-                const float4 x = base[(q * kG + g) * kW];
-                Xp[2 * g] = make_float2(x.x, x.y);
-                Xp[2 * g + 1] = make_float2(x.z, x.w);
+                for (int i = 0; i < kK; ++i)
+                    if (l0 + i >= L) dl[i] = 0.f;
             }
-        };
+            if constexpr (kPExp) {
+#pragma unroll
+                for (int i = 0; i < kK; ++i) dsum += dl[i];
+            }
+#pragma unroll
+            for (int j = 0; j < kJ; ++j) {
+                const float u0 = Io<Tin>::widen(wu, 2 * j), u1 = Io<Tin>::widen(wu, 2 * j + 1);
+                dlp[j] = make_float2(dl[2 * j], dl[2 * j + 1]);
+                dup[j] = make_float2(dl[2 * j] * u0, dl[2 * j + 1] * u1);
+                y[j] = make_float2(Dd * u0, Dd * u1);
+            }
+        }
+
         if constexpr (kW == 1) {
 #pragma unroll
-            for (int q = 0; q < kPairs; ++q) {
-                float2 A2q;
-                if constexpr (kA2InRegs) A2q = A2[q];
-                else A2q = make_float2(2 * q < N ? __ldg(A_d + 2 * q) * kLog2e : 0.f,
-                                       2 * q + 1 < N ? __ldg(A_d + 2 * q + 1) * kLog2e : 0.f);
-                float2 Bp[kItems], Cp[kItems];
-                load_pair(FB, q, Bp);
-                load_pair(FC, q, Cp);
-                float2 h = carry[q];
+            for (int n = 0; n < kNmax; ++n) {
+                float A2n;
+                if constexpr (kA2InRegs) A2n = A2[n];
+                else A2n = n < N ? __ldg(A_d + n) * kLog2e : 0.f;
+                const float2 A2d = make_float2(A2n, A2n);
+                float2 Bp[kJ], Cp[kJ];
+                load_pairs(0, n, Bp);
+                load_pairs(1, n, Cp);
+                float h = carry[n];
 #pragma unroll
-                for (int i = 0; i < kItems; ++i) {
-                    const float2 t = __fmul2_rn(dl2[i], A2q);
-                    const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
-                    h = __ffma2_rn(a, h, __fmul2_rn(du2[i], Bp[i]));
-                    y2[i] = __ffma2_rn(Cp[i], h, y2[i]);
+                for (int j = 0; j < kJ; ++j) {
+                    const float2 t = __fmul2_rn(dlp[j], A2d);
+                    const float2 bb = __fmul2_rn(dup[j], Bp[j]);
+                    float2 hp;
+                    hp.x = fmaf(sfu_exp2(t.x), h, bb.x);
+                    hp.y = fmaf(sfu_exp2(t.y), hp.x, bb.y);
+                    h = hp.y;
+                    if constexpr (kYScalar) {
+                        y[j].x = fmaf(Cp[j].x, hp.x, y[j].x);
+                        y[j].y = fmaf(Cp[j].y, hp.y, y[j].y);
+                    } else {
+                        y[j] = __ffma2_rn(Cp[j], hp, y[j]);
+                    }
                 }
-                carry[q] = h;
+                carry[n] = h;
             }
         } else {
-#pragma unroll kPairUnroll
-            for (int q = 0; q < kPairs; ++q) {
-                const float2 A2q = *reinterpret_cast<const float2 *>(rowA2 + 2 * q);
-                const float2 cin = *reinterpret_cast<const float2 *>(rowCarry + 2 * q);
-                float2 Bp[kItems];
-                load_pair(FB, q, Bp);
-                // Pass 1: this lane's steps from a zero state; keep a and delta' u B.
-                float2 a[kItems], bb[kItems];
-                float2 h = make_float2(0.f, 0.f), P = make_float2(1.f, 1.f);
+#pragma unroll 1
+            for (int n0 = 0; n0 < kNmax; n0 += kS) {
+                float A2s[kS], cin[kS];
 #pragma unroll
-                for (int i = 0; i < kItems; ++i) {
-                    const float2 t = __fmul2_rn(dl2[i], A2q);
-                    a[i] = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
-                    bb[i] = __fmul2_rn(du2[i], Bp[i]);
-                    h = __ffma2_rn(a[i], h, bb[i]);
-                    P = __fmul2_rn(P, a[i]);
+                for (int s = 0; s < kS; ++s) A2s[s] = rowA2[n0 + s], cin[s] = rowCarry[n0 + s];
+                // Pass 1: this lane's steps from a zero state; keep a and delta' u B.
+                float2 a[kS][kJ], bb[kS][kJ];
+                float h[kS], P[kS];
+#pragma unroll
+                for (int s = 0; s < kS; ++s) {
+                    float2 Bp[kJ];
+                    load_pairs(0, n0 + s, Bp);
+                    const float2 A2d = make_float2(A2s[s], A2s[s]);
+                    float hs = 0.f;
+                    float2 Pp = make_float2(1.f, 1.f);
+#pragma unroll
+                    for (int j = 0; j < kJ; ++j) {
+                        const float2 t = __fmul2_rn(dlp[j], A2d);
+                        a[s][j] = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
+                        bb[s][j] = __fmul2_rn(dup[j], Bp[j]);
+                        hs = fmaf(a[s][j].x, hs, bb[s][j].x);
+                        hs = fmaf(a[s][j].y, hs, bb[s][j].y);
+                        if constexpr (!kPExp) Pp = __fmul2_rn(Pp, a[s][j]);
+                    }
+                    h[s] = hs;
+                    if constexpr (kPExp) P[s] = sfu_exp2(A2s[s] * dsum);
+                    else P[s] = Pp.x * Pp.y;
                 }
                 // Scan of (P, h) over the row's W lanes.
-                {
-                    unsigned long long P64 = as_u64(P), h64 = as_u64(h);
 #pragma unroll
-                    for (int off = 1; off < kW; off <<= 1) scan_stage_x2<kW>(P64, h64, off);
-                    P = as_f2(P64);
-                    h = as_f2(h64);
+                for (int off = 1; off < kW; off <<= 1) {
+                    if constexpr (kS == 2) scan_stage2<kW>(P[0], h[0], P[1], h[1], off);
+                    else scan_stage<kW>(P[0], h[0], off);
                 }
-                // States after this lane's steps, given the chunk's incoming states.
-                const float2 X = __ffma2_rn(P, cin, h);
-                const float2 up = make_float2(__shfl_up_sync(kFull, X.x, 1, kW),
-                                              __shfl_up_sync(kFull, X.y, 1, kW));
-                const float2 hin0 = seg == 0 ? cin : up;
-                st_shared_f2_if(rowCarry + 2 * q, X, seg == kW - 1);
-                float2 hin = hin0;
-                // Pass 2: the true states and y.
-                float2 Cp[kItems];
-                load_pair(FC, q, Cp);
+                // States after this lane's steps; the lane before's is this one's start.
+                float hin[kS];
 #pragma unroll
-                for (int i = 0; i < kItems; ++i) {
-                    hin = __ffma2_rn(a[i], hin, bb[i]);
-                    y2[i] = __ffma2_rn(Cp[i], hin, y2[i]);
+                for (int s = 0; s < kS; ++s) {
+                    const float X = fmaf(P[s], cin[s], h[s]);
+                    const float up = __shfl_up_sync(kFull, X, 1, kW);
+                    hin[s] = seg == 0 ? cin[s] : up;
+                    st_shared_f1_if(rowCarry + n0 + s, X, seg == kW - 1);
+                }
+                // Pass 2: the true states and y.
+#pragma unroll
+                for (int s = 0; s < kS; ++s) {
+                    float2 Cp[kJ];
+                    load_pairs(1, n0 + s, Cp);
+                    float hs = hin[s];
+#pragma unroll
+                    for (int j = 0; j < kJ; ++j) {
+                        float2 hp;
+                        hp.x = fmaf(a[s][j].x, hs, bb[s][j].x);
+                        hp.y = fmaf(a[s][j].y, hp.x, bb[s][j].y);
+                        hs = hp.y;
+                        if constexpr (kYScalar) {
+                            y[j].x = fmaf(Cp[j].x, hp.x, y[j].x);
+                            y[j].y = fmaf(Cp[j].y, hp.y, y[j].y);
+                        } else {
+                            y[j] = __ffma2_rn(Cp[j], hp, y[j]);
+                        }
+                    }
                 }
             }
         }
 
-        float y[kItems];
+        float yv[kK];
 #pragma unroll
-        for (int i = 0; i < kItems; ++i) y[i] = y2[i].x + y2[i].y;
+        for (int j = 0; j < kJ; ++j) yv[2 * j] = y[j].x, yv[2 * j + 1] = y[j].y;
         if (has_z) {
-            float zf[kItems];
-            Io<Tin>::widen(wzc, zf);
+            uint32_t wz[kLaneWords];
+            lane_words(buf, 2, wz);
 #pragma unroll
-            for (int i = 0; i < kItems; ++i) y[i] *= silu<kFast>(zf[i]);
+            for (int i = 0; i < kK; ++i) yv[i] *= silu<kFast>(Io<Tin>::widen(wz, i));
         }
-        if (row_ok) store_run(y_row, l0, L, vec, y);
+        if (row_ok) store_run<kK>(y_row, l0, L, vec, yv);
     }
 
     if (p.last_state != nullptr) {
         if constexpr (kRowInRegs) {
             if (row_ok) {
 #pragma unroll
-                for (int q = 0; q < kPairs; ++q) {
-                    if (2 * q < N) p.last_state[row * N + 2 * q] = carry[q].x;
-                    if (2 * q + 1 < N) p.last_state[row * N + 2 * q + 1] = carry[q].y;
-                }
+                for (int n = 0; n < kNmax; ++n)
+                    if (n < N) p.last_state[row * N + n] = carry[n];
             }
         } else {
             __syncthreads();  // the row tables are written (also when L == 0)
             if (row_ok)
                 for (int n = seg; n < N; n += kW) p.last_state[row * N + n] = rowCarry[n];
+        }
+    }
+}
+
+// ------------------------------------------------------------ direct kernel
+// One lane per row (b, d), every state of the row in registers: the plain
+// sequential recurrence of §3.2, no scan.  Used when there are enough rows
+// to fill the GPU.  Steps are the outer loop and state pairs the inner one,
+// so each step has kNmax/2 independent packed updates
+//   t = delta' (A_n, A_n+1) log2e,  a = 2^t (two MUFU.EX2),
+//   h = a h + delta' u (B_n, B_n+1),  acc += (C_n, C_n+1) h      (f32x2)
+// and only h, A and a few per-step values stay live.
+//
+// B and C (shared by all rows of a batch entry) are staged per block for
+// kDirectStage steps: cp.async copies the raw rows into RB one stage ahead,
+// then the block converts them to fp32 in F, where float4 number
+// i (kNmax/2) + q holds (B[2q][i], B[2q+1][i], C[2q][i], C[2q+1][i]); every
+// lane reads the same address (broadcast).  u, delta and z are read by each
+// lane from its own row, 8 steps at a time, one sub-chunk ahead.
+#ifndef SS_DIRECT_MIN_BLOCKS
+#define SS_DIRECT_MIN_BLOCKS 2
+#endif
+constexpr int kDirectStage = 64;  // steps per shared-memory stage
+constexpr int kDirectSub = 8;     // steps per register sub-chunk
+
+__host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax) {
+    return 4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage;
+}
+
+template <typename Tin, typename Tout, int kNmax>
+__global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) ss_fwd_direct_kernel(const FwdParams p) {
+    constexpr int kPairs = kNmax / 2;
+    constexpr int kUnit = Io<Tin>::kUnit;
+    constexpr int kSubWords = kDirectSub * (int)sizeof(Tin) / 4;
+    constexpr int kStageUnits = kDirectStage / kUnit;       // 16-byte units per (tensor, n) row
+    constexpr bool kFast = sizeof(Tin) == 2;
+    constexpr bool kA2InRegs = kNmax <= 32;
+
+    const int tid = threadIdx.x;
+    const int nthreads = blockDim.x;
+    const int N = p.dstate;
+    const int64_t b = blockIdx.x / p.dtiles;
+    const int64_t d_raw = (blockIdx.x % p.dtiles) * nthreads + tid;
+    const bool row_ok = d_raw < p.dim;
+    const int64_t d = row_ok ? d_raw : p.dim - 1;
+    const int64_t L = p.seqlen;
+    const int64_t row = b * p.dim + d;
+    const bool vec = p.vec != 0;
+    const bool softplus = p.softplus != 0;
+    const bool has_z = p.z != nullptr;
+
+    extern __shared__ float4 smem[];
+    float4 *F = smem;                                                   // [kDirectStage][kPairs]
+    Tin *RB = reinterpret_cast<Tin *>(smem + kDirectStage * kPairs);     // [2][kNmax][kDirectStage]
+
+    const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * N * L,
+                          static_cast<const Tin *>(p.C) + b * N * L};
+    const Tin *u_row = static_cast<const Tin *>(p.u) + row * L;
+    const Tin *d_row = static_cast<const Tin *>(p.delta) + row * L;
+    const Tin *z_row = has_z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
+    Tout *y_row = static_cast<Tout *>(p.y) + row * L;
+
+    const float *A_d = p.A + d * N;
+    float2 A2[kA2InRegs ? kPairs : 1], h[kPairs];
+#pragma unroll
+    for (int q = 0; q < kPairs; ++q) {
+        if constexpr (kA2InRegs)
+            A2[q] = make_float2(2 * q < N ? A_d[2 * q] * kLog2e : 0.f,
+                                2 * q + 1 < N ? A_d[2 * q + 1] * kLog2e : 0.f);
+        h[q] = make_float2(0.f, 0.f);
+    }
+    const float Dd = p.D ? p.D[d] : 0.f;
+    const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
+
+    auto stage_async = [&](int64_t c0) { return vec && c0 + kDirectStage <= L; };
+    auto issue_copies = [&](int64_t c0) {
+        for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
+            const int j = u % kStageUnits, rowid = u / kStageUnits;
+            const int t = rowid / kNmax, n = rowid % kNmax;
+            if (n < N)
+                cp_async16(RB + (rowid * kDirectStage + j * kUnit), Bsrc[t] + (int64_t)n * L + c0 + j * kUnit);
+        }
+        cp_async_commit();
+    };
+    // RB (or global memory, element by element) -> F: job (q, step block of 8).
+    auto fill_F = [&](int64_t c0, bool from_RB) {
+        for (int jb = tid; jb < kPairs * (kDirectStage / 8); jb += nthreads) {
+            const int q = jb % kPairs, i0 = (jb / kPairs) * 8;
+            float v[4][8];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {  // c: B[2q], B[2q+1], C[2q], C[2q+1]
+                const int t = c >> 1, n = 2 * q + (c & 1);
+                if (n >= N) {
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) v[c][m] = 0.f;
+                } else if (from_RB) {
+                    const Tin *src = RB + (t * kNmax + n) * kDirectStage + i0;
+#pragma unroll
+                    for (int g = 0; g < 8 / kUnit; ++g) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(src + g * kUnit);
+                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int m = 0; m < kUnit; ++m) v[c][g * kUnit + m] = Io<Tin>::widen(w, m);
+                    }
+                } else {
+                    const Tin *src = Bsrc[t] + (int64_t)n * L;
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        const int64_t l = c0 + i0 + m;
+                        uint32_t bits = 0u;
+                        if (l < L) bits = Io<Tin>::bits(src, l);
+                        if constexpr (sizeof(Tin) == 2) bits <<= 16;
+                        v[c][m] = __uint_as_float(bits);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) F[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
+        }
+    };
+    // 8 steps of one row as raw words (16-byte loads kept in L1, or element loads).
+    auto load_sub = [&](const Tin *rowp, int64_t l0, uint32_t (&w)[kSubWords]) {
+        if (vec && l0 + kDirectSub <= L) {
+            const uint4 *q4 = reinterpret_cast<const uint4 *>(rowp + l0);
+#pragma unroll
+            for (int g = 0; g < kSubWords / 4; ++g) {
+                const uint4 x = __ldg(q4 + g);
+                w[4 * g] = x.x, w[4 * g + 1] = x.y, w[4 * g + 2] = x.z, w[4 * g + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kSubWords; ++j) w[j] = 0u;
+#pragma unroll
+            for (int i = 0; i < kDirectSub; ++i) {
+                if (l0 + i < L) {
+                    const uint32_t bits = Io<Tin>::bits(rowp, l0 + i);
+                    if constexpr (sizeof(Tin) == 2) w[i >> 1] |= bits << (16 * (i & 1));
+                    else w[i] = bits;
+                }
+            }
+        }
+    };
+
+    uint32_t wu[kSubWords], wd[kSubWords], wz[kSubWords];
+    load_sub(u_row, 0, wu);
+    load_sub(d_row, 0, wd);
+    if (has_z) load_sub(z_row, 0, wz);
+    if (L > 0 && stage_async(0)) issue_copies(0);
+
+    for (int64_t c0 = 0; c0 < L; c0 += kDirectStage) {
+        const bool async_here = stage_async(c0);
+        if (async_here) cp_async_wait_all();
+        __syncthreads();  // RB holds this stage; every warp is done with F
+        fill_F(c0, async_here);
+        __syncthreads();  // F holds this stage; RB is free
+        if (c0 + kDirectStage < L && stage_async(c0 + kDirectStage)) issue_copies(c0 + kDirectStage);
+
+        const int nsub = (int)((L - c0 < kDirectStage ? L - c0 : kDirectStage) + kDirectSub - 1) / kDirectSub;
+#pragma unroll 1
+        for (int m = 0; m < nsub; ++m) {
+            const int64_t l0 = c0 + m * kDirectSub;
+            uint32_t cu[kSubWords], cd[kSubWords], cz[kSubWords];
+#pragma unroll
+            for (int j = 0; j < kSubWords; ++j) cu[j] = wu[j], cd[j] = wd[j], cz[j] = wz[j];
+            if (l0 + kDirectSub < L) {  // next sub-chunk of this row
+                load_sub(u_row, l0 + kDirectSub, wu);
+                load_sub(d_row, l0 + kDirectSub, wd);
+                if (has_z) load_sub(z_row, l0 + kDirectSub, wz);
+            }
+            float yv[kDirectSub];
+            const float4 *Fm = F + (m * kDirectSub) * kPairs;
+#pragma unroll
+            for (int i = 0; i < kDirectSub; ++i) {
+                const float uf = Io<Tin>::widen(cu, i);
+                float dl = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
+                if (l0 + i >= L) dl = 0.f;  // past the end: identity step
+                const float2 d2 = make_float2(dl, dl), u2 = make_float2(dl * uf, dl * uf);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < kPairs; ++q) {
+                    const float4 bc = Fm[i * kPairs + q];
+                    float2 A2q;
+                    if constexpr (kA2InRegs) A2q = A2[q];
+                    else A2q = make_float2(2 * q < N ? __ldg(A_d + 2 * q) * kLog2e : 0.f,
+                                           2 * q + 1 < N ? __ldg(A_d + 2 * q + 1) * kLog2e : 0.f);
+                    const float2 t = __fmul2_rn(d2, A2q);
+                    const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
+                    h[q] = __ffma2_rn(a, h[q], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
+                    if (q & 1) acc1 = __ffma2_rn(make_float2(bc.z, bc.w), h[q], acc1);
+                    else acc0 = __ffma2_rn(make_float2(bc.z, bc.w), h[q], acc0);
+                }
+                yv[i] = fmaf(Dd, uf, (acc0.x + acc0.y) + (acc1.x + acc1.y));  // + D u (§3.3)
+            }
+            if (has_z) {
+#pragma unroll
+                for (int i = 0; i < kDirectSub; ++i) yv[i] *= silu<kFast>(Io<Tin>::widen(cz, i));
+            }
+            if (row_ok) store_run<kDirectSub>(y_row, l0, L, vec, yv);
+        }
+    }
+
+    if (p.last_state != nullptr && row_ok) {
+#pragma unroll
+        for (int q = 0; q < kPairs; ++q) {
+            if (2 * q < N) p.last_state[row * N + 2 * q] = h[q].x;
+            if (2 * q + 1 < N) p.last_state[row * N + 2 * q + 1] = h[q].y;
         }
     }
 }
