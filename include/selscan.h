@@ -100,25 +100,33 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
 
 /*
  * As ss_fwd, with the launch shape chosen by the caller instead of by the
- * library's heuristic (for autotuning).  lanes_per_row in {1,2,4,8,16,32}
- * is how many lanes of a warp share one (b, d) row, each lane taking 8
- * (up to 4 lanes) or 16 (8 lanes and more) consecutive steps of every chunk;
- * warps_per_block in {1,2,4,8}.  Values of 0 pick the heuristic's choice.
- * Results are identical for every shape up to float32 rounding order.
- * Returns SS_ERR_BAD_CONFIG for other values, or when the block's shared
- * memory for that shape would exceed 227 KB.
+ * library's heuristic (for autotuning).  lanes_per_row in {1,2,4,8,16,32} is
+ * how many lanes of a warp share one (b, d) row:
+ *   split_states = 0: the lanes split the row's steps (each takes 8 steps per
+ *     chunk up to 4 lanes, 16 from 8 lanes) and combine their states with a
+ *     scan over the lanes;
+ *   split_states = 1: the lanes (1, 2 or 4, at most half the state bucket
+ *     4/8/16/32/64 that holds dstate) split the row's states and each runs
+ *     every step;
+ *   one lane: the row's sequential recurrence in one lane, either way.
+ * warps_per_block in {1,2,4,8}.  lanes_per_row 0 (or warps 0) picks the
+ * heuristic's choice.  Results are identical for every shape up to float32
+ * rounding order.  Returns SS_ERR_BAD_CONFIG for other values, or when the
+ * block's shared memory for that shape would exceed 227 KB.
  */
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
                              const float *A, const void *B, const void *C, const float *D,
                              const void *z, const float *delta_bias, int delta_softplus,
-                             void *y, float *last_state, int lanes_per_row,
+                             void *y, float *last_state, int lanes_per_row, int split_states,
                              int warps_per_block, ss_stream_t stream);
 
 /*
- * Launch shape ss_fwd would use for `desc` (lanes per row, warps per block).
- * Returns SS_OK, or the status ss_fwd would return for a bad descriptor.
+ * Launch shape ss_fwd would use for `desc` (lanes per row, state split flag,
+ * warps per block).  Returns SS_OK, or the status ss_fwd would return for a
+ * bad descriptor.
  */
-ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *warps_per_block);
+ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *split_states,
+                           int *warps_per_block);
 
 /*
  * Host-buffer form: copies the inputs from host memory into caller-owned

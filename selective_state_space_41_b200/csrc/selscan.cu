@@ -71,57 +71,73 @@ int sm_count() {
 
 // Dynamic shared memory of one block: B and C of one chunk for the state
 // bucket as fp32, plus a raw copy in the input dtype (see the kernel).
-size_t smem_for(const ss_desc *desc, int lanes, int warps) {
+size_t smem_for(const ss_desc *desc, int lanes, int split, int warps) {
     const int nmax = selscan::state_bucket((int)desc->dstate);
-    if (lanes == 1) return selscan::direct_smem_bytes(dtype_size(desc->in_dtype), nmax);
+    if (lanes == 1 || split) return selscan::direct_smem_bytes(dtype_size(desc->in_dtype), nmax);
     return selscan::smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
 }
 
-// Lanes per row: enough (row, lane) pairs for about 1024 threads per SM, but
-// no more lanes than the sequence can feed, and a block whose shared memory
-// fits in a quarter of an SM's.
-void heuristic(const ss_desc *desc, int64_t rows, int sms, int *lanes, int *warps) {
-    int w = 1;
-    const int64_t target = (int64_t)sms * 1024;
-    while (w < 32 && rows * w < target) w *= 2;
-    while (w > 1 && (int64_t)selscan::chunk_len(w) / 2 >= desc->seqlen) w /= 2;
-    while (w > 1 && smem_for(desc, w, 4) > selscan::kMaxSmemBytes / 4) w /= 2;
+// Launch shape.  The direct kernel (lanes split a row's states, no scan) has
+// the least work per state update, so it is used whenever the rows alone
+// can give each SM sub-partition (4 per SM) enough warps: the smallest split
+// G in {1, 2, 4} (at most half the state bucket) with at least 4 warps per
+// sub-partition, or G = 4 down to 1.5 warps.  With fewer rows the steps are
+// split instead (scan kernel): the smallest W giving 3 warps per
+// sub-partition, no more lanes than the sequence can feed, and a block
+// within half of an SM's shared memory.
+void heuristic(const ss_desc *desc, int64_t rows, int sms, int *lanes, int *split, int *warps) {
+    const int64_t slots = (int64_t)sms * 4 * 32;  // lanes per "one warp per sub-partition"
+    const int gmax = selscan::state_bucket((int)desc->dstate) / 2 >= 4 ? 4 : 2;
+    int g = 1;
+    while (g < gmax && rows * g < 4 * slots) g *= 2;
+    if (rows * g >= 4 * slots || rows * gmax * 2 >= 3 * slots) {
+        *lanes = g;
+        *split = g > 1 ? 1 : 0;
+        *warps = 4;
+        return;
+    }
+    int w = 2;
+    while (w < 32 && rows * w < 3 * slots) w *= 2;
+    while (w > 2 && (int64_t)selscan::chunk_len(w) / 2 >= desc->seqlen) w /= 2;
+    while (w > 2 && smem_for(desc, w, 0, 8) > selscan::kMaxSmemBytes / 2) w /= 2;
     *lanes = w;
-    *warps = 4;
+    *split = 0;
+    *warps = 8;
 }
 
 // The launcher for the state bucket that holds n (4, 8, 16, 32 or 64).
-#define SS_PICK_BUCKET(PREFIX)                                            \
-    cudaError_t (*fn)(int, dim3, dim3, size_t, cudaStream_t, const FwdParams &) = \
+#define SS_PICK_BUCKET(PREFIX)                                                 \
+    cudaError_t (*fn)(int, int, dim3, dim3, size_t, cudaStream_t, const FwdParams &) = \
         n <= 4 ? selscan::PREFIX##_n4                                     \
         : n <= 8 ? selscan::PREFIX##_n8                                   \
         : n <= 16 ? selscan::PREFIX##_n16                                 \
         : n <= 32 ? selscan::PREFIX##_n32                                 \
                   : selscan::PREFIX##_n64;                                \
-    return fn(lanes, grid, block, smem, s, p);
+    return fn(lanes, split, grid, block, smem, s, p);
 
-cudaError_t launch_f32_f32(int n, int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                           const FwdParams &p) {
+cudaError_t launch_f32_f32(int n, int lanes, int split, dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t s, const FwdParams &p) {
     SS_PICK_BUCKET(launch_f32_f32)
 }
-cudaError_t launch_bf16_bf16(int n, int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                           const FwdParams &p) {
+cudaError_t launch_bf16_bf16(int n, int lanes, int split, dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t s, const FwdParams &p) {
     SS_PICK_BUCKET(launch_bf16_bf16)
 }
-cudaError_t launch_bf16_f32(int n, int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                           const FwdParams &p) {
+cudaError_t launch_bf16_f32(int n, int lanes, int split, dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t s, const FwdParams &p) {
     SS_PICK_BUCKET(launch_bf16_f32)
 }
 
 ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D, const void *z,
                    const float *delta_bias, int delta_softplus, void *y, float *last_state,
-                   int lanes, int warps, ss_stream_t stream) {
+                   int lanes, int split, int warps, ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
     if (lanes != 0 && (lanes < 1 || lanes > 32 || (lanes & (lanes - 1)) != 0))
         return SS_ERR_BAD_CONFIG;
+    if (split != 0 && split != 1) return SS_ERR_BAD_CONFIG;
     if (warps != 0 && warps != 1 && warps != 2 && warps != 4 && warps != 8)
         return SS_ERR_BAD_CONFIG;
     if (sz.rows == 0) return SS_OK;  // no rows: nothing to read or write
@@ -145,12 +161,19 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     if (y && !aligned(y, 16)) vec = false;
 
     int sms = sm_count();
-    int h_lanes, h_warps;
-    heuristic(desc, sz.rows, sms, &h_lanes, &h_warps);
-    if (lanes == 0) lanes = h_lanes;
+    int h_lanes, h_split, h_warps;
+    heuristic(desc, sz.rows, sms, &h_lanes, &h_split, &h_warps);
+    if (lanes == 0) {
+        lanes = h_lanes;
+        split = h_split;
+    }
     if (warps == 0) warps = h_warps;
+    // The direct kernel splits the state pairs of the state bucket over 1, 2 or 4 lanes.
+    if ((lanes == 1 || split) &&
+        (lanes > 4 || selscan::state_bucket((int)desc->dstate) / 2 < lanes))
+        return SS_ERR_BAD_CONFIG;
 
-    const size_t smem = smem_for(desc, lanes, warps);
+    const size_t smem = smem_for(desc, lanes, split, warps);
     if (smem > selscan::kMaxSmemBytes) return SS_ERR_BAD_CONFIG;
     const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
     const int64_t dtiles = (desc->dim + rows_per_block - 1) / rows_per_block;
@@ -181,11 +204,11 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     const int n = p.dstate;
     cudaError_t err;
     if (desc->in_dtype == SS_F32)
-        err = launch_f32_f32(n, lanes, grid, block, smem, s, p);
+        err = launch_f32_f32(n, lanes, split, grid, block, smem, s, p);
     else if (desc->out_dtype == SS_BF16)
-        err = launch_bf16_bf16(n, lanes, grid, block, smem, s, p);
+        err = launch_bf16_bf16(n, lanes, split, grid, block, smem, s, p);
     else
-        err = launch_bf16_f32(n, lanes, grid, block, smem, s, p);
+        err = launch_bf16_f32(n, lanes, split, grid, block, smem, s, p);
     return err == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
@@ -197,25 +220,26 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  const void *B, const void *C, const float *D, const void *z,
                  const float *delta_bias, int delta_softplus, void *y, float *last_state,
                  ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, 0, 0,
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, 0, 0, 0,
                     stream);
 }
 
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
                              const float *A, const void *B, const void *C, const float *D,
                              const void *z, const float *delta_bias, int delta_softplus,
-                             void *y, float *last_state, int lanes_per_row,
+                             void *y, float *last_state, int lanes_per_row, int split_states,
                              int warps_per_block, ss_stream_t stream) {
     return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state,
-                    lanes_per_row, warps_per_block, stream);
+                    lanes_per_row, split_states, warps_per_block, stream);
 }
 
-ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *warps_per_block) {
+ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *split_states,
+                           int *warps_per_block) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
-    if (!lanes_per_row || !warps_per_block) return SS_ERR_NULL_POINTER;
-    heuristic(desc, sz.rows, sm_count(), lanes_per_row, warps_per_block);
+    if (!lanes_per_row || !split_states || !warps_per_block) return SS_ERR_NULL_POINTER;
+    heuristic(desc, sz.rows, sm_count(), lanes_per_row, split_states, warps_per_block);
     return SS_OK;
 }
 
@@ -256,7 +280,7 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
         if (c.dst && c.bytes && cudaMemcpyAsync(c.dst, c.src, c.bytes, h2d, s) != cudaSuccess)
             return SS_ERR_CUDA;
     st = fwd_impl(desc, d_u, d_delta, d_A, d_B, d_C, d_D, d_z, d_delta_bias, delta_softplus, d_y,
-                  d_last_state, 0, 0, stream);
+                  d_last_state, 0, 0, 0, stream);
     if (st != SS_OK) return st;
     if (n_y && cudaMemcpyAsync(h_y, d_y, n_y, d2h, s) != cudaSuccess) return SS_ERR_CUDA;
     if (d_last_state && cudaMemcpyAsync(h_last_state, d_last_state, n_last, d2h, s) != cudaSuccess)

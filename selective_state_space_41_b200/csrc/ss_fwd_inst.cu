@@ -12,19 +12,12 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// Launch one instance; above the 48 KB default the kernel must opt in to
-// more dynamic shared memory, once per device.
-template <int kW>
-auto kernel_for() {
-    if constexpr (kW == 1) return ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX>;
-    else return ss_fwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kW>;
-}
-
-template <int kW>
-cudaError_t launch_one(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p) {
-    auto kernel = kernel_for<kW>();
+// Launch one kernel instance; above the 48 KB default a kernel must opt in
+// to more dynamic shared memory, once per device.
+template <typename Kernel>
+cudaError_t launch_kernel(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          const FwdParams &p, bool (&opted_in)[kMaxDevices]) {
     if (smem > 48 * 1024) {
-        static bool opted_in[kMaxDevices];
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
@@ -39,17 +32,42 @@ cudaError_t launch_one(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const
     return cudaGetLastError();
 }
 
+template <int kW>
+cudaError_t launch_scan(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p) {
+    static bool opted_in[kMaxDevices];
+    return launch_kernel(ss_fwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kW>, grid, block, smem,
+                         s, p, opted_in);
+}
+
+template <int kG>
+cudaError_t launch_direct(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p) {
+    if constexpr (SS_INST_NMAX / 2 / kG < 1) {
+        return cudaErrorInvalidValue;  // fewer state pairs than lanes
+    } else {
+        static bool opted_in[kMaxDevices];
+        return launch_kernel(ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kG>, grid,
+                             block, smem, s, p, opted_in);
+    }
+}
+
 }  // namespace
 
-cudaError_t SS_INST_NAME(int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                         const FwdParams &p) {
+cudaError_t SS_INST_NAME(int lanes, int split_states, dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t s, const FwdParams &p) {
+    if (lanes == 1 || split_states) {
+        switch (lanes) {
+            case 1: return launch_direct<1>(grid, block, smem, s, p);
+            case 2: return launch_direct<2>(grid, block, smem, s, p);
+            case 4: return launch_direct<4>(grid, block, smem, s, p);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (lanes) {
-        case 1: return launch_one<1>(grid, block, smem, s, p);
-        case 2: return launch_one<2>(grid, block, smem, s, p);
-        case 4: return launch_one<4>(grid, block, smem, s, p);
-        case 8: return launch_one<8>(grid, block, smem, s, p);
-        case 16: return launch_one<16>(grid, block, smem, s, p);
-        case 32: return launch_one<32>(grid, block, smem, s, p);
+        case 2: return launch_scan<2>(grid, block, smem, s, p);
+        case 4: return launch_scan<4>(grid, block, smem, s, p);
+        case 8: return launch_scan<8>(grid, block, smem, s, p);
+        case 16: return launch_scan<16>(grid, block, smem, s, p);
+        case 32: return launch_scan<32>(grid, block, smem, s, p);
         default: return cudaErrorInvalidValue;
     }
 }

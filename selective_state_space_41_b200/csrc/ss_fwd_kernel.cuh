@@ -72,14 +72,22 @@ struct Io<__nv_bfloat16> {
     }
 };
 
-// Scalar (element) stores of y for steps [l0, l0 + K), guarded by L, or
-// 16-byte streaming stores when the run is complete and aligned.
+// Stores of y for steps [l0, l0 + K): streaming vector stores (16, 8 or 4
+// bytes) when the run is complete and aligned, else element stores guarded
+// by L.
 template <int K>
 __device__ __forceinline__ void store_run(float *row, int64_t l0, int64_t L, bool vec, const float (&v)[K]) {
     if (vec && l0 + K <= L) {
-        float4 *p = reinterpret_cast<float4 *>(row + l0);
+        if constexpr (K % 4 == 0) {
+            float4 *p = reinterpret_cast<float4 *>(row + l0);
 #pragma unroll
-        for (int j = 0; j < K / 4; ++j) __stcs(p + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+            for (int j = 0; j < K / 4; ++j) __stcs(p + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        } else if constexpr (K == 2) {
+            __stcs(reinterpret_cast<float2 *>(row + l0), make_float2(v[0], v[1]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < K; ++i) row[l0 + i] = v[i];
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < K; ++i)
@@ -96,15 +104,25 @@ template <int K>
 __device__ __forceinline__ void store_run(__nv_bfloat16 *row, int64_t l0, int64_t L, bool vec,
                                           const float (&v)[K]) {
     if (vec && l0 + K <= L) {
-        uint4 *p = reinterpret_cast<uint4 *>(row + l0);
+        if constexpr (K % 8 == 0) {
+            uint4 *p = reinterpret_cast<uint4 *>(row + l0);
 #pragma unroll
-        for (int j = 0; j < K / 8; ++j) {
-            uint4 q;
-            q.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-            q.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-            q.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-            q.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-            __stcs(p + j, q);
+            for (int j = 0; j < K / 8; ++j) {
+                uint4 q;
+                q.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+                q.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+                q.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+                q.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+                __stcs(p + j, q);
+            }
+        } else if constexpr (K == 4) {
+            __stcs(reinterpret_cast<uint2 *>(row + l0),
+                   make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3])));
+        } else if constexpr (K == 2) {
+            __stcs(reinterpret_cast<unsigned int *>(row + l0), pack_bf16x2(v[0], v[1]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < K; ++i) row[l0 + i] = __float2bfloat16_rn(v[i]);
         }
     } else {
 #pragma unroll
@@ -630,20 +648,27 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
 }
 
 // ------------------------------------------------------------ direct kernel
-// One lane per row (b, d), every state of the row in registers: the plain
-// sequential recurrence of §3.2, no scan.  Used when there are enough rows
-// to fill the GPU.  Steps are the outer loop and state pairs the inner one,
-// so each step has kNmax/2 independent packed updates
+// No scan: the G lanes of a row (G = 1, 2 or 4) each own N/G of its states
+// and run the plain sequential recurrence of §3.2 over every step, states in
+// registers.  Used when there are enough rows to fill the GPU.  Steps are the
+// outer loop and state pairs the inner one, so each step has independent
+// packed updates per state pair (n, n+1)
 //   t = delta' (A_n, A_n+1) log2e,  a = 2^t (two MUFU.EX2),
 //   h = a h + delta' u (B_n, B_n+1),  acc += (C_n, C_n+1) h      (f32x2)
-// and only h, A and a few per-step values stay live.
+// with only h, A and a few per-step values live.
+//
+// Steps come in sub-chunks of 8.  Lane g of a row computes delta' and
+// delta' u for steps 8/G g .. 8/G (g+1) - 1 of the sub-chunk and the G lanes
+// all-gather them with shuffles; after the state loop each lane holds partial
+// sums of y over its states for all 8 steps, and a recursive-halving
+// exchange (shfl.xor) leaves lane g the totals of its own 8/G steps, which it
+// finishes (D u, silu(z)) and stores.
 //
 // B and C (shared by all rows of a batch entry) are staged per block for
 // kDirectStage steps: cp.async copies the raw rows into RB one stage ahead,
 // then the block converts them to fp32 in F, where float4 number
-// i (kNmax/2) + q holds (B[2q][i], B[2q+1][i], C[2q][i], C[2q+1][i]); every
-// lane reads the same address (broadcast).  u, delta and z are read by each
-// lane from its own row, 8 steps at a time, one sub-chunk ahead.
+// i (kNmax/2) + q holds (B[2q][i], B[2q+1][i], C[2q][i], C[2q+1][i]); the
+// lanes that own the same states read the same address (broadcast).
 #ifndef SS_DIRECT_MIN_BLOCKS
 #define SS_DIRECT_MIN_BLOCKS 2
 #endif
@@ -654,20 +679,47 @@ __host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax)
     return 4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage;
 }
 
-template <typename Tin, typename Tout, int kNmax>
-__global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) ss_fwd_direct_kernel(const FwdParams p) {
+// Load `bytes` (4, 8, 16 or 32) of one row starting at element l0 into words.
+template <int kBytes>
+__device__ __forceinline__ void ld_words(const void *src, uint32_t *w) {
+    if constexpr (kBytes >= 16) {
+#pragma unroll
+        for (int g = 0; g < kBytes / 16; ++g) {
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src) + g);
+            w[4 * g] = x.x, w[4 * g + 1] = x.y, w[4 * g + 2] = x.z, w[4 * g + 3] = x.w;
+        }
+    } else if constexpr (kBytes == 8) {
+        const uint2 x = __ldg(reinterpret_cast<const uint2 *>(src));
+        w[0] = x.x, w[1] = x.y;
+    } else {
+        w[0] = __ldg(reinterpret_cast<const unsigned int *>(src));
+    }
+}
+
+template <typename Tin, typename Tout, int kNmax, int kG>
+__global__ void __launch_bounds__(256, kNmax / kG <= 32 ? SS_DIRECT_MIN_BLOCKS : 1)
+    ss_fwd_direct_kernel(const FwdParams p) {
     constexpr int kPairs = kNmax / 2;
+    constexpr int kPL = kPairs / kG;                        // state pairs per lane
+    static_assert(kG == 1 || kG == 2 || kG == 4, "1, 2 or 4 lanes per row");
+    static_assert(kPL >= 1, "at least one state pair per lane");
+    constexpr int kOwn = kDirectSub / kG;                   // steps owned per lane per sub-chunk
+    constexpr int kOwnBytes = kOwn * (int)sizeof(Tin);
+    constexpr int kOwnWords = (kOwnBytes + 3) / 4;
     constexpr int kUnit = Io<Tin>::kUnit;
-    constexpr int kSubWords = kDirectSub * (int)sizeof(Tin) / 4;
     constexpr int kStageUnits = kDirectStage / kUnit;       // 16-byte units per (tensor, n) row
     constexpr bool kFast = sizeof(Tin) == 2;
-    constexpr bool kA2InRegs = kNmax <= 32;
+    constexpr bool kA2InRegs = kNmax / kG <= 32;
+    constexpr unsigned kFull = 0xffffffffu;
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
+    const int lane = tid & 31;
+    const int g = lane % kG;                                // state group of this lane
+    const int rows = nthreads / kG;
     const int N = p.dstate;
     const int64_t b = blockIdx.x / p.dtiles;
-    const int64_t d_raw = (blockIdx.x % p.dtiles) * nthreads + tid;
+    const int64_t d_raw = (blockIdx.x % p.dtiles) * rows + tid / kG;
     const bool row_ok = d_raw < p.dim;
     const int64_t d = row_ok ? d_raw : p.dim - 1;
     const int64_t L = p.seqlen;
@@ -687,14 +739,15 @@ __global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) s
     const Tin *z_row = has_z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
     Tout *y_row = static_cast<Tout *>(p.y) + row * L;
 
+    const int q0 = g * kPL;                                 // this lane's first state pair
     const float *A_d = p.A + d * N;
-    float2 A2[kA2InRegs ? kPairs : 1], h[kPairs];
+    float2 A2[kA2InRegs ? kPL : 1], h[kPL];
 #pragma unroll
-    for (int q = 0; q < kPairs; ++q) {
+    for (int qq = 0; qq < kPL; ++qq) {
+        const int n = 2 * (q0 + qq);
         if constexpr (kA2InRegs)
-            A2[q] = make_float2(2 * q < N ? A_d[2 * q] * kLog2e : 0.f,
-                                2 * q + 1 < N ? A_d[2 * q + 1] * kLog2e : 0.f);
-        h[q] = make_float2(0.f, 0.f);
+            A2[qq] = make_float2(n < N ? A_d[n] * kLog2e : 0.f, n + 1 < N ? A_d[n + 1] * kLog2e : 0.f);
+        h[qq] = make_float2(0.f, 0.f);
     }
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
@@ -723,11 +776,11 @@ __global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) s
                 } else if (from_RB) {
                     const Tin *src = RB + (t * kNmax + n) * kDirectStage + i0;
 #pragma unroll
-                    for (int g = 0; g < 8 / kUnit; ++g) {
-                        const uint4 raw = *reinterpret_cast<const uint4 *>(src + g * kUnit);
+                    for (int gg = 0; gg < 8 / kUnit; ++gg) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(src + gg * kUnit);
                         const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                        for (int m = 0; m < kUnit; ++m) v[c][g * kUnit + m] = Io<Tin>::widen(w, m);
+                        for (int m = 0; m < kUnit; ++m) v[c][gg * kUnit + m] = Io<Tin>::widen(w, m);
                     }
                 } else {
                     const Tin *src = Bsrc[t] + (int64_t)n * L;
@@ -745,22 +798,18 @@ __global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) s
             for (int m = 0; m < 8; ++m) F[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
         }
     };
-    // 8 steps of one row as raw words (16-byte loads kept in L1, or element loads).
-    auto load_sub = [&](const Tin *rowp, int64_t l0, uint32_t (&w)[kSubWords]) {
-        if (vec && l0 + kDirectSub <= L) {
-            const uint4 *q4 = reinterpret_cast<const uint4 *>(rowp + l0);
-#pragma unroll
-            for (int g = 0; g < kSubWords / 4; ++g) {
-                const uint4 x = __ldg(q4 + g);
-                w[4 * g] = x.x, w[4 * g + 1] = x.y, w[4 * g + 2] = x.z, w[4 * g + 3] = x.w;
-            }
+    // This lane's kOwn steps of one row from step l0 of the sub-chunk.
+    auto load_own = [&](const Tin *rowp, int64_t l0, uint32_t (&w)[kOwnWords]) {
+        const int64_t s0 = l0 + g * kOwn;
+        if (vec && s0 + kOwn <= L) {
+            ld_words<kOwnBytes>(rowp + s0, w);
         } else {
 #pragma unroll
-            for (int j = 0; j < kSubWords; ++j) w[j] = 0u;
+            for (int j = 0; j < kOwnWords; ++j) w[j] = 0u;
 #pragma unroll
-            for (int i = 0; i < kDirectSub; ++i) {
-                if (l0 + i < L) {
-                    const uint32_t bits = Io<Tin>::bits(rowp, l0 + i);
+            for (int i = 0; i < kOwn; ++i) {
+                if (s0 + i < L) {
+                    const uint32_t bits = Io<Tin>::bits(rowp, s0 + i);
                     if constexpr (sizeof(Tin) == 2) w[i >> 1] |= bits << (16 * (i & 1));
                     else w[i] = bits;
                 }
@@ -768,10 +817,10 @@ __global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) s
         }
     };
 
-    uint32_t wu[kSubWords], wd[kSubWords], wz[kSubWords];
-    load_sub(u_row, 0, wu);
-    load_sub(d_row, 0, wd);
-    if (has_z) load_sub(z_row, 0, wz);
+    uint32_t wu[kOwnWords], wd[kOwnWords], wz[kOwnWords];
+    load_own(u_row, 0, wu);
+    load_own(d_row, 0, wd);
+    if (has_z) load_own(z_row, 0, wz);
     if (L > 0 && stage_async(0)) issue_copies(0);
 
     for (int64_t c0 = 0; c0 < L; c0 += kDirectStage) {
@@ -786,51 +835,91 @@ __global__ void __launch_bounds__(256, kNmax <= 32 ? SS_DIRECT_MIN_BLOCKS : 1) s
 #pragma unroll 1
         for (int m = 0; m < nsub; ++m) {
             const int64_t l0 = c0 + m * kDirectSub;
-            uint32_t cu[kSubWords], cd[kSubWords], cz[kSubWords];
+            uint32_t cu[kOwnWords], cd[kOwnWords], cz[kOwnWords];
 #pragma unroll
-            for (int j = 0; j < kSubWords; ++j) cu[j] = wu[j], cd[j] = wd[j], cz[j] = wz[j];
-            if (l0 + kDirectSub < L) {  // next sub-chunk of this row
-                load_sub(u_row, l0 + kDirectSub, wu);
-                load_sub(d_row, l0 + kDirectSub, wd);
-                if (has_z) load_sub(z_row, l0 + kDirectSub, wz);
+            for (int j = 0; j < kOwnWords; ++j) cu[j] = wu[j], cd[j] = wd[j], cz[j] = wz[j];
+            if (l0 + kDirectSub < L) {  // next sub-chunk of this lane's steps
+                load_own(u_row, l0 + kDirectSub, wu);
+                load_own(d_row, l0 + kDirectSub, wd);
+                if (has_z) load_own(z_row, l0 + kDirectSub, wz);
             }
-            float yv[kDirectSub];
-            const float4 *Fm = F + (m * kDirectSub) * kPairs;
+            // delta' and delta' u of the owned steps (past L: the identity step).
+            float dl_own[kOwn], du_own[kOwn], u_own[kOwn];
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) {
+                u_own[i] = Io<Tin>::widen(cu, i);
+                dl_own[i] = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
+            }
+            if (l0 + kDirectSub > L) {
+#pragma unroll
+                for (int i = 0; i < kOwn; ++i)
+                    if (l0 + g * kOwn + i >= L) dl_own[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) du_own[i] = dl_own[i] * u_own[i];
+            // All 8 steps' values, gathered from the row's G lanes.
+            float dl[kDirectSub], du[kDirectSub];
 #pragma unroll
             for (int i = 0; i < kDirectSub; ++i) {
-                const float uf = Io<Tin>::widen(cu, i);
-                float dl = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
-                if (l0 + i >= L) dl = 0.f;  // past the end: identity step
-                const float2 d2 = make_float2(dl, dl), u2 = make_float2(dl * uf, dl * uf);
+                if constexpr (kG == 1) {
+                    dl[i] = dl_own[i], du[i] = du_own[i];
+                } else {
+                    dl[i] = __shfl_sync(kFull, dl_own[i % kOwn], i / kOwn, kG);
+                    du[i] = __shfl_sync(kFull, du_own[i % kOwn], i / kOwn, kG);
+                }
+            }
+            float part[kDirectSub];
+            const float4 *Fm = F + (m * kDirectSub) * kPairs + q0;
+#pragma unroll
+            for (int i = 0; i < kDirectSub; ++i) {
+                const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
                 float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int q = 0; q < kPairs; ++q) {
-                    const float4 bc = Fm[i * kPairs + q];
+                for (int qq = 0; qq < kPL; ++qq) {
+                    const float4 bc = Fm[i * kPairs + qq];
                     float2 A2q;
-                    if constexpr (kA2InRegs) A2q = A2[q];
-                    else A2q = make_float2(2 * q < N ? __ldg(A_d + 2 * q) * kLog2e : 0.f,
-                                           2 * q + 1 < N ? __ldg(A_d + 2 * q + 1) * kLog2e : 0.f);
+                    if constexpr (kA2InRegs) A2q = A2[qq];
+                    else {
+                        const int n = 2 * (q0 + qq);
+                        A2q = make_float2(n < N ? __ldg(A_d + n) * kLog2e : 0.f,
+                                          n + 1 < N ? __ldg(A_d + n + 1) * kLog2e : 0.f);
+                    }
                     const float2 t = __fmul2_rn(d2, A2q);
                     const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
-                    h[q] = __ffma2_rn(a, h[q], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
-                    if (q & 1) acc1 = __ffma2_rn(make_float2(bc.z, bc.w), h[q], acc1);
-                    else acc0 = __ffma2_rn(make_float2(bc.z, bc.w), h[q], acc0);
+                    h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
+                    if (qq & 1) acc1 = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc1);
+                    else acc0 = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc0);
                 }
-                yv[i] = fmaf(Dd, uf, (acc0.x + acc0.y) + (acc1.x + acc1.y));  // + D u (§3.3)
+                part[i] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
             }
+            // Recursive halving: lane g ends with the totals of its own steps in part[0..kOwn).
+#pragma unroll
+            for (int sdist = kG / 2, cnt = kDirectSub; sdist >= 1; sdist /= 2, cnt /= 2) {
+                const bool upper = (g & sdist) != 0;
+#pragma unroll
+                for (int k = 0; k < cnt / 2; ++k) {
+                    const float send = upper ? part[k] : part[k + cnt / 2];
+                    const float keep = upper ? part[k + cnt / 2] : part[k];
+                    part[k] = keep + __shfl_xor_sync(kFull, send, sdist, kG);
+                }
+            }
+            float yv[kOwn];
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) yv[i] = fmaf(Dd, u_own[i], part[i]);  // + D u (§3.3)
             if (has_z) {
 #pragma unroll
-                for (int i = 0; i < kDirectSub; ++i) yv[i] *= silu<kFast>(Io<Tin>::widen(cz, i));
+                for (int i = 0; i < kOwn; ++i) yv[i] *= silu<kFast>(Io<Tin>::widen(cz, i));
             }
-            if (row_ok) store_run<kDirectSub>(y_row, l0, L, vec, yv);
+            if (row_ok) store_run<kOwn>(y_row, l0 + g * kOwn, L, vec, yv);
         }
     }
 
     if (p.last_state != nullptr && row_ok) {
 #pragma unroll
-        for (int q = 0; q < kPairs; ++q) {
-            if (2 * q < N) p.last_state[row * N + 2 * q] = h[q].x;
-            if (2 * q + 1 < N) p.last_state[row * N + 2 * q + 1] = h[q].y;
+        for (int qq = 0; qq < kPL; ++qq) {
+            const int n = 2 * (q0 + qq);
+            if (n < N) p.last_state[row * N + n] = h[qq].x;
+            if (n + 1 < N) p.last_state[row * N + n + 1] = h[qq].y;
         }
     }
 }

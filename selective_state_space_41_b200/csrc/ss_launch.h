@@ -9,8 +9,12 @@
 
 namespace selscan {
 
-#define SS_DECLARE_LAUNCHER(NAME) \
-    cudaError_t NAME(int lanes, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const FwdParams &p);
+// lanes: lanes per row; split_states: the lanes split the row's states (direct
+// kernel, 1/2/4 lanes) rather than its steps (scan kernel, 2..32 lanes); one
+// lane is the direct kernel either way.
+#define SS_DECLARE_LAUNCHER(NAME)                                                            \
+    cudaError_t NAME(int lanes, int split_states, dim3 grid, dim3 block, size_t smem, cudaStream_t s, \
+                     const FwdParams &p);
 
 #define SS_FOR_EACH_NBUCKET(X, PREFIX) X(PREFIX##_n4) X(PREFIX##_n8) X(PREFIX##_n16) X(PREFIX##_n32) X(PREFIX##_n64)
 

@@ -57,9 +57,9 @@ def lib():
         L.ss_fwd.restype = I
         L.ss_fwd.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
         L.ss_fwd_with_config.restype = I
-        L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, I, I, P]
+        L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, I, I, I, P]
         L.ss_fwd_heuristic.restype = I
-        L.ss_fwd_heuristic.argtypes = [DP, ctypes.POINTER(I), ctypes.POINTER(I)]
+        L.ss_fwd_heuristic.argtypes = [DP, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]
         L.ss_fwd_hostio.restype = I
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P]
         L.ss_status_string.restype = ctypes.c_char_p
@@ -107,13 +107,14 @@ def _check(status, where):
 
 
 def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
-           last_state=None, stream=None, lanes_per_row=None, warps_per_block=None):
+           last_state=None, stream=None, lanes_per_row=None, warps_per_block=None,
+           split_states=False):
     """Queue the forward on ``stream`` (default: the current stream).
 
     u, delta, z, y: (batch, dim, L); A: (dim, N) float32; B, C: (batch, N, L);
     D, delta_bias: (dim,) float32; last_state: (batch, dim, N) float32.
-    ``lanes_per_row`` / ``warps_per_block`` select ``ss_fwd_with_config``.
-    Raises SelscanError on a rejected call.
+    ``lanes_per_row`` / ``split_states`` / ``warps_per_block`` select
+    ``ss_fwd_with_config``.  Raises SelscanError on a rejected call.
     """
     u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
     if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
@@ -127,17 +128,17 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
     if lanes_per_row is None and warps_per_block is None:
         _check(lib().ss_fwd(*args, s), "ss_fwd")
     else:
-        _check(lib().ss_fwd_with_config(*args, int(lanes_per_row or 0), int(warps_per_block or 0), s),
-               "ss_fwd_with_config")
+        _check(lib().ss_fwd_with_config(*args, int(lanes_per_row or 0), 1 if split_states else 0,
+                                        int(warps_per_block or 0), s), "ss_fwd_with_config")
 
 
 def ss_fwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None):
-    """(lanes_per_row, warps_per_block) the library picks for these sizes."""
+    """(lanes_per_row, split_states, warps_per_block) the library picks."""
     desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
-    lanes, warps = ctypes.c_int(), ctypes.c_int()
-    _check(lib().ss_fwd_heuristic(ctypes.byref(desc), ctypes.byref(lanes), ctypes.byref(warps)),
-           "ss_fwd_heuristic")
-    return lanes.value, warps.value
+    lanes, split, warps = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().ss_fwd_heuristic(ctypes.byref(desc), ctypes.byref(lanes), ctypes.byref(split),
+                                  ctypes.byref(warps)), "ss_fwd_heuristic")
+    return lanes.value, bool(split.value), warps.value
 
 
 def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None):

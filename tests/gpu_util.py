@@ -18,7 +18,7 @@ def to_dev(inp, device="cuda"):
     return out
 
 
-def run_gpu(inp, out_dtype=None, lanes=None, warps=None, device="cuda"):
+def run_gpu(inp, out_dtype=None, lanes=None, warps=None, split=False, device="cuda"):
     """(y, last_state) from libselscan for host inputs ``inp``."""
     d = to_dev(inp, device)
     u = d["u"]
@@ -30,7 +30,8 @@ def run_gpu(inp, out_dtype=None, lanes=None, warps=None, device="cuda"):
             if inp.get("return_last_state") else None)
     selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d.get("D"), z=d.get("z"),
                    delta_bias=d.get("delta_bias"), delta_softplus=inp["delta_softplus"],
-                   last_state=last, lanes_per_row=lanes, warps_per_block=warps)
+                   last_state=last, lanes_per_row=lanes, warps_per_block=warps,
+                   split_states=split)
     torch.cuda.synchronize()
     return y, last
 

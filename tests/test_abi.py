@@ -78,9 +78,10 @@ def test_rejections_before_any_launch(lib):
 def test_bad_launch_shapes_rejected(lib):
     d = _desc()
     args = (ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE, None)
-    assert lib.ss_fwd_with_config(*args, 3, 4, None) == 7
-    assert lib.ss_fwd_with_config(*args, 64, 4, None) == 7
-    assert lib.ss_fwd_with_config(*args, 4, 3, None) == 7
+    assert lib.ss_fwd_with_config(*args, 3, 0, 4, None) == 7
+    assert lib.ss_fwd_with_config(*args, 64, 0, 4, None) == 7
+    assert lib.ss_fwd_with_config(*args, 4, 0, 3, None) == 7
+    assert lib.ss_fwd_with_config(*args, 4, 2, 4, None) == 7
 
 
 def test_hostio_rejections(lib):

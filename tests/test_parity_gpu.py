@@ -119,14 +119,31 @@ def test_bf16_in_f32_out():
     assert_parity(y, last, y_ref, last_ref, 1e-4, "bf16->f32")
 
 
-@pytest.mark.parametrize("lanes", [1, 2, 4, 8, 16, 32])
+SHAPES = ([(w, False) for w in (1, 2, 4, 8, 16, 32)] + [(2, True), (4, True)])
+
+
+@pytest.mark.parametrize("lanes,split", SHAPES)
 @pytest.mark.parametrize("warps", [1, 2, 4, 8])
-def test_every_launch_shape(lanes, warps):
+def test_every_launch_shape(lanes, split, warps):
     inp = _case(2, 37, 517, 16, torch.float32, seed=lanes * 10 + warps, has_z=True,
                 return_last_state=True)
-    y, last = run_gpu(inp, lanes=lanes, warps=warps)
+    y, last = run_gpu(inp, lanes=lanes, warps=warps, split=split)
     y_ref, last_ref = run_oracle(inp)
-    assert_parity(y, last, y_ref, last_ref, TOL[torch.float32], f"lanes={lanes} warps={warps}")
+    assert_parity(y, last, y_ref, last_ref, TOL[torch.float32],
+                  f"lanes={lanes} split={split} warps={warps}")
+
+
+@pytest.mark.parametrize("N", [4, 8, 9, 16, 33, 64])
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_state_split_shapes(N, lanes):
+    """The state split over 2 or 4 lanes, bf16, ragged length and channels."""
+    if lanes == 4 and N <= 4:
+        pytest.skip("bucket 4 has two state pairs")
+    inp = _case(2, 19, 203, N, torch.bfloat16, seed=N * 7 + lanes, has_z=True,
+                return_last_state=True)
+    y, last = run_gpu(inp, lanes=lanes, warps=2, split=True)
+    y_ref, last_ref = run_oracle(inp)
+    assert_parity(y, last, y_ref, last_ref, TOL[torch.bfloat16], f"N={N} lanes={lanes} split")
 
 
 def test_unaligned_rows_take_the_scalar_path():
