@@ -105,9 +105,9 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
  *   split_states = 0: the lanes split the row's steps (each takes 8 steps per
  *     chunk up to 4 lanes, 16 from 8 lanes) and combine their states with a
  *     scan over the lanes;
- *   split_states = 1: the lanes (1, 2 or 4, at most half the state bucket
- *     4/8/16/32/64 that holds dstate) split the row's states and each runs
- *     every step;
+ *   split_states = 1: the lanes (1, 2, 4 or 8, at most half the state
+ *     bucket 4/8/16/32/64 that holds dstate) split the row's states and each
+ *     runs every step;
  *   one lane: the row's sequential recurrence in one lane, either way.
  * warps_per_block in {1,2,4,8}.  lanes_per_row 0 (or warps 0) picks the
  * heuristic's choice.  Results are identical for every shape up to float32

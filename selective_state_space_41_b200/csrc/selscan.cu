@@ -73,7 +73,7 @@ int sm_count() {
 // bucket as fp32, plus a raw copy in the input dtype (see the kernel).
 size_t smem_for(const ss_desc *desc, int lanes, int split, int warps) {
     const int nmax = selscan::state_bucket((int)desc->dstate);
-    if (lanes == 1 || split) return selscan::direct_smem_bytes(dtype_size(desc->in_dtype), nmax);
+    if (lanes == 1 || split) return selscan::direct_smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
     return selscan::smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
 }
 
@@ -81,16 +81,21 @@ size_t smem_for(const ss_desc *desc, int lanes, int split, int warps) {
 // the least work per state update, so it is used whenever the rows alone
 // can give each SM sub-partition (4 per SM) enough warps: the smallest split
 // G in {1, 2, 4} (at most half the state bucket) with at least 4 warps per
-// sub-partition, or G = 4 down to 1.5 warps.  With fewer rows the steps are
+// sub-partition (with 32 or 64 states, 32 states per lane once that gives 2
+// warps), or G = 4 down to 1.5 warps.  With fewer rows the steps are
 // split instead (scan kernel): the smallest W giving 3 warps per
 // sub-partition, no more lanes than the sequence can feed, and a block
 // within half of an SM's shared memory.
 void heuristic(const ss_desc *desc, int64_t rows, int sms, int *lanes, int *split, int *warps) {
     const int64_t slots = (int64_t)sms * 4 * 32;  // lanes per "one warp per sub-partition"
-    const int gmax = selscan::state_bucket((int)desc->dstate) / 2 >= 4 ? 4 : 2;
+    const int bucket = selscan::state_bucket((int)desc->dstate);
+    const int gmax = bucket / 2 >= 4 ? 4 : 2;
     int g = 1;
     while (g < gmax && rows * g < 4 * slots) g *= 2;
-    if (rows * g >= 4 * slots || rows * gmax * 2 >= 3 * slots) {
+    // Wide states: 32 states per lane (uncapped registers) once the rows alone
+    // give two warps per sub-partition.
+    if (bucket >= 32 && rows * (bucket / 32) >= 2 * slots) g = bucket / 32;
+    if (rows * g >= 2 * slots || rows * gmax * 2 >= 3 * slots) {
         *lanes = g;
         *split = g > 1 ? 1 : 0;
         *warps = 4;
@@ -168,9 +173,9 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
         split = h_split;
     }
     if (warps == 0) warps = h_warps;
-    // The direct kernel splits the state pairs of the state bucket over 1, 2 or 4 lanes.
+    // The direct kernel splits the state pairs of the state bucket over 1, 2, 4 or 8 lanes.
     if ((lanes == 1 || split) &&
-        (lanes > 4 || selscan::state_bucket((int)desc->dstate) / 2 < lanes))
+        (lanes > 8 || selscan::state_bucket((int)desc->dstate) / 2 < lanes))
         return SS_ERR_BAD_CONFIG;
 
     const size_t smem = smem_for(desc, lanes, split, warps);

@@ -59,6 +59,7 @@ cudaError_t SS_INST_NAME(int lanes, int split_states, dim3 grid, dim3 block, siz
             case 1: return launch_direct<1>(grid, block, smem, s, p);
             case 2: return launch_direct<2>(grid, block, smem, s, p);
             case 4: return launch_direct<4>(grid, block, smem, s, p);
+            case 8: return launch_direct<8>(grid, block, smem, s, p);
             default: return cudaErrorInvalidValue;
         }
     }

@@ -33,6 +33,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace selscan {
 
 constexpr size_t kMaxSmemBytes = 227 * 1024;  // opt-in dynamic shared memory per block (sm_100)
@@ -316,7 +318,10 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
     constexpr int kUnitsPerRow = kChunk / kUnit;         // a power of two
     constexpr int kLaneUnits = kK / kUnit;               // 16-byte units per lane per stream
     constexpr int kLaneWords = kK * (int)sizeof(Tin) / 4;
-    constexpr int kS = (kW == 1 || kK == 16) ? 1 : 2;    // states per scan iteration
+#ifndef SS_SCAN_STATES
+#define SS_SCAN_STATES 0
+#endif
+    constexpr int kS = SS_SCAN_STATES ? SS_SCAN_STATES : ((kW == 1 || kK == 16) ? 1 : 2);  // states per scan iteration
     constexpr bool kFast = sizeof(Tin) == 2;             // bf16 inputs: SFU transforms
     constexpr int kRowStride = kNmax + 2;                // per-row tables (W > 1)
     constexpr unsigned kFull = 0xffffffffu;
@@ -648,7 +653,7 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
 }
 
 // ------------------------------------------------------------ direct kernel
-// No scan: the G lanes of a row (G = 1, 2 or 4) each own N/G of its states
+// No scan: the G lanes of a row (G = 1, 2, 4 or 8) each own N/G of its states
 // and run the plain sequential recurrence of §3.2 over every step, states in
 // registers.  Used when there are enough rows to fill the GPU.  Steps are the
 // outer loop and state pairs the inner one, so each step has independent
@@ -658,28 +663,33 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
 // with only h, A and a few per-step values live.
 //
 // Steps come in sub-chunks of 8.  Lane g of a row computes delta' and
-// delta' u for steps 8/G g .. 8/G (g+1) - 1 of the sub-chunk and the G lanes
-// all-gather them with shuffles; after the state loop each lane holds partial
-// sums of y over its states for all 8 steps, and a recursive-halving
-// exchange (shfl.xor) leaves lane g the totals of its own 8/G steps, which it
-// finishes (D u, silu(z)) and stores.
+// delta' u for 8/G of them; with G > 1 the row's lanes all-gather them
+// through a small per-warp shared slab, and after the state loop each lane
+// writes its partial sums of y over its states for all 8 steps there and
+// reads back the G partials of its own 8/G steps, which it finishes (D u,
+// silu(z)) and stores.
 //
 // B and C (shared by all rows of a batch entry) are staged per block for
 // kDirectStage steps: cp.async copies the raw rows into RB one stage ahead,
 // then the block converts them to fp32 in F, where float4 number
 // i (kNmax/2) + q holds (B[2q][i], B[2q+1][i], C[2q][i], C[2q+1][i]); the
-// lanes that own the same states read the same address (broadcast).
+// lanes that own the same states read the same address (broadcast).  A stage
+// that lies wholly inside the sequence with aligned rows takes a path with no
+// bounds checks; the last, partial stage (or unaligned rows) a checked one.
 #ifndef SS_DIRECT_MIN_BLOCKS
 #define SS_DIRECT_MIN_BLOCKS 2
 #endif
 constexpr int kDirectStage = 64;  // steps per shared-memory stage
 constexpr int kDirectSub = 8;     // steps per register sub-chunk
+constexpr int kGatherStride = 20; // floats per row of the gather slab (16 used; spreads banks)
+constexpr int kReduceStride = 12; // floats per lane of the reduce slab (8 used)
 
-__host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax) {
-    return 4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage;
+__host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax, int g, int warps) {
+    return 4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage +
+           (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * kGatherStride + 32 * kReduceStride) : 0);
 }
 
-// Load `bytes` (4, 8, 16 or 32) of one row starting at element l0 into words.
+// Load `bytes` (4, 8, 16 or 32) from 16/8/4-byte aligned global memory into words.
 template <int kBytes>
 __device__ __forceinline__ void ld_words(const void *src, uint32_t *w) {
     if constexpr (kBytes >= 16) {
@@ -691,31 +701,45 @@ __device__ __forceinline__ void ld_words(const void *src, uint32_t *w) {
     } else if constexpr (kBytes == 8) {
         const uint2 x = __ldg(reinterpret_cast<const uint2 *>(src));
         w[0] = x.x, w[1] = x.y;
-    } else {
+    } else if constexpr (kBytes == 4) {
         w[0] = __ldg(reinterpret_cast<const unsigned int *>(src));
+    } else {
+        w[0] = __ldg(reinterpret_cast<const unsigned short *>(src));
     }
 }
 
+// Register budget: 128 per thread (two 256-thread blocks per SM) while a
+// lane holds up to 16 states; lanes holding 32 or more states (wide states,
+// few lanes per row) run better with up to 255 registers and fewer warps.
+template <int kStatesPerLane>
+struct DirectOccupancy {
+    static constexpr int kMinBlocks = kStatesPerLane <= 16 ? SS_DIRECT_MIN_BLOCKS : 1;
+};
+
 template <typename Tin, typename Tout, int kNmax, int kG>
-__global__ void __launch_bounds__(256, kNmax / kG <= 32 ? SS_DIRECT_MIN_BLOCKS : 1)
+__global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     ss_fwd_direct_kernel(const FwdParams p) {
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                        // state pairs per lane
-    static_assert(kG == 1 || kG == 2 || kG == 4, "1, 2 or 4 lanes per row");
+    static_assert(kG == 1 || kG == 2 || kG == 4 || kG == 8, "1, 2, 4 or 8 lanes per row");
     static_assert(kPL >= 1, "at least one state pair per lane");
     constexpr int kOwn = kDirectSub / kG;                   // steps owned per lane per sub-chunk
     constexpr int kOwnBytes = kOwn * (int)sizeof(Tin);
     constexpr int kOwnWords = (kOwnBytes + 3) / 4;
     constexpr int kUnit = Io<Tin>::kUnit;
     constexpr int kStageUnits = kDirectStage / kUnit;       // 16-byte units per (tensor, n) row
+    constexpr int kSubs = kDirectStage / kDirectSub;
+    constexpr int kRowsPerWarp = 32 / kG;
+    constexpr int kAccs = kPL >= 4 ? 2 : 1;                 // y accumulators per step
     constexpr bool kFast = sizeof(Tin) == 2;
     constexpr bool kA2InRegs = kNmax / kG <= 32;
-    constexpr unsigned kFull = 0xffffffffu;
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
     const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int g = lane % kG;                                // state group of this lane
+    const int r = lane / kG;                                // row within the warp
     const int rows = nthreads / kG;
     const int N = p.dstate;
     const int64_t b = blockIdx.x / p.dtiles;
@@ -731,13 +755,19 @@ __global__ void __launch_bounds__(256, kNmax / kG <= 32 ? SS_DIRECT_MIN_BLOCKS :
     extern __shared__ float4 smem[];
     float4 *F = smem;                                                   // [kDirectStage][kPairs]
     Tin *RB = reinterpret_cast<Tin *>(smem + kDirectStage * kPairs);     // [2][kNmax][kDirectStage]
+    float *slab = reinterpret_cast<float *>(RB + 2 * kNmax * kDirectStage) +
+                  warp * (kRowsPerWarp * kGatherStride + 32 * kReduceStride);
+    float *gat = slab + r * kGatherStride;                  // this row: 8 delta', 8 delta' u
+    float *red = slab + kRowsPerWarp * kGatherStride;       // per lane: 8 partial sums of y
 
     const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * N * L,
                           static_cast<const Tin *>(p.C) + b * N * L};
-    const Tin *u_row = static_cast<const Tin *>(p.u) + row * L;
-    const Tin *d_row = static_cast<const Tin *>(p.delta) + row * L;
-    const Tin *z_row = has_z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
-    Tout *y_row = static_cast<Tout *>(p.y) + row * L;
+    // This lane's first owned step of each stream (advanced per sub-chunk).
+    const Tin *u_own = static_cast<const Tin *>(p.u) + row * L + g * kOwn;
+    const Tin *d_own = static_cast<const Tin *>(p.delta) + row * L + g * kOwn;
+    const Tin *z_own = has_z ? static_cast<const Tin *>(p.z) + row * L + g * kOwn : nullptr;
+    Tout *const y_row = static_cast<Tout *>(p.y) + row * L;
+    Tout *y_own = y_row + g * kOwn;
 
     const int q0 = g * kPL;                                 // this lane's first state pair
     const float *A_d = p.A + d * N;
@@ -752,7 +782,7 @@ __global__ void __launch_bounds__(256, kNmax / kG <= 32 ? SS_DIRECT_MIN_BLOCKS :
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
 
-    auto stage_async = [&](int64_t c0) { return vec && c0 + kDirectStage <= L; };
+    auto stage_fast = [&](int64_t c0) { return vec && c0 + kDirectStage <= L; };
     auto issue_copies = [&](int64_t c0) {
         for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
             const int j = u % kStageUnits, rowid = u / kStageUnits;
@@ -798,18 +828,18 @@ __global__ void __launch_bounds__(256, kNmax / kG <= 32 ? SS_DIRECT_MIN_BLOCKS :
             for (int m = 0; m < 8; ++m) F[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
         }
     };
-    // This lane's kOwn steps of one row from step l0 of the sub-chunk.
-    auto load_own = [&](const Tin *rowp, int64_t l0, uint32_t (&w)[kOwnWords]) {
-        const int64_t s0 = l0 + g * kOwn;
-        if (vec && s0 + kOwn <= L) {
-            ld_words<kOwnBytes>(rowp + s0, w);
+    // This lane's kOwn steps of a stream starting `off` elements past `own`
+    // (0 past the end of the sequence), as raw words.
+    auto load_own_checked = [&](const Tin *own, int64_t s0, uint32_t (&w)[kOwnWords]) {
+        if (kOwnBytes >= 4 && vec && s0 + kOwn <= L) {
+            ld_words<kOwnBytes>(own, w);
         } else {
 #pragma unroll
             for (int j = 0; j < kOwnWords; ++j) w[j] = 0u;
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
                 if (s0 + i < L) {
-                    const uint32_t bits = Io<Tin>::bits(rowp, s0 + i);
+                    const uint32_t bits = Io<Tin>::bits(own, i);
                     if constexpr (sizeof(Tin) == 2) w[i >> 1] |= bits << (16 * (i & 1));
                     else w[i] = bits;
                 }
@@ -818,99 +848,133 @@ __global__ void __launch_bounds__(256, kNmax / kG <= 32 ? SS_DIRECT_MIN_BLOCKS :
     };
 
     uint32_t wu[kOwnWords], wd[kOwnWords], wz[kOwnWords];
-    load_own(u_row, 0, wu);
-    load_own(d_row, 0, wd);
-    if (has_z) load_own(z_row, 0, wz);
-    if (L > 0 && stage_async(0)) issue_copies(0);
+    load_own_checked(u_own, g * kOwn, wu);
+    load_own_checked(d_own, g * kOwn, wd);
+    if (has_z) load_own_checked(z_own, g * kOwn, wz);
+    if (L > 0 && stage_fast(0)) issue_copies(0);
+
+    // One sub-chunk of 8 steps from step l0; kChecked: guard the sequence end.
+    auto sub_chunk = [&](auto checked, int m, int64_t l0) {
+        constexpr bool kChecked = decltype(checked)::value;
+        uint32_t cu[kOwnWords], cd[kOwnWords], cz[kOwnWords];
+#pragma unroll
+        for (int j = 0; j < kOwnWords; ++j) cu[j] = wu[j], cd[j] = wd[j], cz[j] = wz[j];
+        const int64_t s_next = l0 + kDirectSub + g * kOwn;   // next owned step
+        u_own += kDirectSub, d_own += kDirectSub;
+        if (has_z) z_own += kDirectSub;
+        if (kOwnBytes >= 4 && !kChecked && m + 1 < kSubs) {  // next sub-chunk lies in this full stage
+            ld_words<kOwnBytes>(u_own, wu);
+            ld_words<kOwnBytes>(d_own, wd);
+            if (has_z) ld_words<kOwnBytes>(z_own, wz);
+        } else if (l0 + kDirectSub < L) {
+            load_own_checked(u_own, s_next, wu);
+            load_own_checked(d_own, s_next, wd);
+            if (has_z) load_own_checked(z_own, s_next, wz);
+        }
+        // delta' and delta' u of the owned steps (past L: the identity step).
+        float dl_own[kOwn], du_own[kOwn], uo[kOwn];
+#pragma unroll
+        for (int i = 0; i < kOwn; ++i) {
+            uo[i] = Io<Tin>::widen(cu, i);
+            dl_own[i] = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
+            if constexpr (kChecked) {
+                if (l0 + g * kOwn + i >= L) dl_own[i] = 0.f;
+            }
+            du_own[i] = dl_own[i] * uo[i];
+        }
+        // All 8 steps' values of the row.
+        float dl[kDirectSub], du[kDirectSub];
+        if constexpr (kG == 1) {
+#pragma unroll
+            for (int i = 0; i < kDirectSub; ++i) dl[i] = dl_own[i], du[i] = du_own[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) gat[g * kOwn + i] = dl_own[i], gat[8 + g * kOwn + i] = du_own[i];
+            __syncwarp();
+#pragma unroll
+            for (int q4 = 0; q4 < 2; ++q4) {
+                const float4 a4 = reinterpret_cast<const float4 *>(gat)[q4];
+                const float4 b4 = reinterpret_cast<const float4 *>(gat + 8)[q4];
+                dl[4 * q4] = a4.x, dl[4 * q4 + 1] = a4.y, dl[4 * q4 + 2] = a4.z, dl[4 * q4 + 3] = a4.w;
+                du[4 * q4] = b4.x, du[4 * q4 + 1] = b4.y, du[4 * q4 + 2] = b4.z, du[4 * q4 + 3] = b4.w;
+            }
+        }
+        float part[kDirectSub];
+        const float4 *Fm = F + (m * kDirectSub) * kPairs + q0;
+#pragma unroll
+        for (int i = 0; i < kDirectSub; ++i) {
+            const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
+            float2 acc[kAccs];
+#pragma unroll
+            for (int k = 0; k < kAccs; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int qq = 0; qq < kPL; ++qq) {
+                const float4 bc = Fm[i * kPairs + qq];
+                float2 A2q;
+                if constexpr (kA2InRegs) A2q = A2[qq];
+                else {
+                    const int n = 2 * (q0 + qq);
+                    A2q = make_float2(n < N ? __ldg(A_d + n) * kLog2e : 0.f,
+                                      n + 1 < N ? __ldg(A_d + n + 1) * kLog2e : 0.f);
+                }
+                const float2 t = __fmul2_rn(d2, A2q);
+                const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
+                h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
+                acc[qq % kAccs] = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc[qq % kAccs]);
+            }
+            if constexpr (kAccs == 2) acc[0] = __fadd2_rn(acc[0], acc[1]);
+            part[i] = acc[0].x + acc[0].y;
+        }
+        // Totals of the owned steps.
+        float yv[kOwn];
+        if constexpr (kG == 1) {
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) yv[i] = part[i];
+        } else {
+            float *mine = red + lane * kReduceStride;
+            reinterpret_cast<float4 *>(mine)[0] = make_float4(part[0], part[1], part[2], part[3]);
+            reinterpret_cast<float4 *>(mine)[1] = make_float4(part[4], part[5], part[6], part[7]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) yv[i] = 0.f;
+#pragma unroll
+            for (int gg = 0; gg < kG; ++gg) {
+                const float *src = red + (r * kG + gg) * kReduceStride + g * kOwn;
+#pragma unroll
+                for (int i = 0; i < kOwn; ++i) yv[i] += src[i];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kOwn; ++i) yv[i] = fmaf(Dd, uo[i], yv[i]);  // + D u (§3.3)
+        if (has_z) {
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) yv[i] *= silu<kFast>(Io<Tin>::widen(cz, i));
+        }
+        if (row_ok) {
+            if constexpr (kChecked) {
+                store_run<kOwn>(y_row, l0 + g * kOwn, L, vec, yv);
+            } else {
+                store_run<kOwn>(y_own, 0, kOwn, true, yv);
+            }
+        }
+        y_own += kDirectSub;
+    };
 
     for (int64_t c0 = 0; c0 < L; c0 += kDirectStage) {
-        const bool async_here = stage_async(c0);
-        if (async_here) cp_async_wait_all();
+        const bool fast = stage_fast(c0);
+        if (fast) cp_async_wait_all();
         __syncthreads();  // RB holds this stage; every warp is done with F
-        fill_F(c0, async_here);
+        fill_F(c0, fast);
         __syncthreads();  // F holds this stage; RB is free
-        if (c0 + kDirectStage < L && stage_async(c0 + kDirectStage)) issue_copies(c0 + kDirectStage);
+        if (c0 + kDirectStage < L && stage_fast(c0 + kDirectStage)) issue_copies(c0 + kDirectStage);
 
-        const int nsub = (int)((L - c0 < kDirectStage ? L - c0 : kDirectStage) + kDirectSub - 1) / kDirectSub;
+        if (fast) {
 #pragma unroll 1
-        for (int m = 0; m < nsub; ++m) {
-            const int64_t l0 = c0 + m * kDirectSub;
-            uint32_t cu[kOwnWords], cd[kOwnWords], cz[kOwnWords];
-#pragma unroll
-            for (int j = 0; j < kOwnWords; ++j) cu[j] = wu[j], cd[j] = wd[j], cz[j] = wz[j];
-            if (l0 + kDirectSub < L) {  // next sub-chunk of this lane's steps
-                load_own(u_row, l0 + kDirectSub, wu);
-                load_own(d_row, l0 + kDirectSub, wd);
-                if (has_z) load_own(z_row, l0 + kDirectSub, wz);
-            }
-            // delta' and delta' u of the owned steps (past L: the identity step).
-            float dl_own[kOwn], du_own[kOwn], u_own[kOwn];
-#pragma unroll
-            for (int i = 0; i < kOwn; ++i) {
-                u_own[i] = Io<Tin>::widen(cu, i);
-                dl_own[i] = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
-            }
-            if (l0 + kDirectSub > L) {
-#pragma unroll
-                for (int i = 0; i < kOwn; ++i)
-                    if (l0 + g * kOwn + i >= L) dl_own[i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < kOwn; ++i) du_own[i] = dl_own[i] * u_own[i];
-            // All 8 steps' values, gathered from the row's G lanes.
-            float dl[kDirectSub], du[kDirectSub];
-#pragma unroll
-            for (int i = 0; i < kDirectSub; ++i) {
-                if constexpr (kG == 1) {
-                    dl[i] = dl_own[i], du[i] = du_own[i];
-                } else {
-                    dl[i] = __shfl_sync(kFull, dl_own[i % kOwn], i / kOwn, kG);
-                    du[i] = __shfl_sync(kFull, du_own[i % kOwn], i / kOwn, kG);
-                }
-            }
-            float part[kDirectSub];
-            const float4 *Fm = F + (m * kDirectSub) * kPairs + q0;
-#pragma unroll
-            for (int i = 0; i < kDirectSub; ++i) {
-                const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
-                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int qq = 0; qq < kPL; ++qq) {
-                    const float4 bc = Fm[i * kPairs + qq];
-                    float2 A2q;
-                    if constexpr (kA2InRegs) A2q = A2[qq];
-                    else {
-                        const int n = 2 * (q0 + qq);
-                        A2q = make_float2(n < N ? __ldg(A_d + n) * kLog2e : 0.f,
-                                          n + 1 < N ? __ldg(A_d + n + 1) * kLog2e : 0.f);
-                    }
-                    const float2 t = __fmul2_rn(d2, A2q);
-                    const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
-                    h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
-                    if (qq & 1) acc1 = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc1);
-                    else acc0 = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc0);
-                }
-                part[i] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-            }
-            // Recursive halving: lane g ends with the totals of its own steps in part[0..kOwn).
-#pragma unroll
-            for (int sdist = kG / 2, cnt = kDirectSub; sdist >= 1; sdist /= 2, cnt /= 2) {
-                const bool upper = (g & sdist) != 0;
-#pragma unroll
-                for (int k = 0; k < cnt / 2; ++k) {
-                    const float send = upper ? part[k] : part[k + cnt / 2];
-                    const float keep = upper ? part[k + cnt / 2] : part[k];
-                    part[k] = keep + __shfl_xor_sync(kFull, send, sdist, kG);
-                }
-            }
-            float yv[kOwn];
-#pragma unroll
-            for (int i = 0; i < kOwn; ++i) yv[i] = fmaf(Dd, u_own[i], part[i]);  // + D u (§3.3)
-            if (has_z) {
-#pragma unroll
-                for (int i = 0; i < kOwn; ++i) yv[i] *= silu<kFast>(Io<Tin>::widen(cz, i));
-            }
-            if (row_ok) store_run<kOwn>(y_row, l0 + g * kOwn, L, vec, yv);
+            for (int m = 0; m < kSubs; ++m) sub_chunk(std::false_type{}, m, c0 + m * kDirectSub);
+        } else {
+            const int nsub = (int)((L - c0 < kDirectStage ? L - c0 : kDirectStage) + kDirectSub - 1) / kDirectSub;
+#pragma unroll 1
+            for (int m = 0; m < nsub; ++m) sub_chunk(std::true_type{}, m, c0 + m * kDirectSub);
         }
     }
 

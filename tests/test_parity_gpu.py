@@ -119,7 +119,7 @@ def test_bf16_in_f32_out():
     assert_parity(y, last, y_ref, last_ref, 1e-4, "bf16->f32")
 
 
-SHAPES = ([(w, False) for w in (1, 2, 4, 8, 16, 32)] + [(2, True), (4, True)])
+SHAPES = ([(w, False) for w in (1, 2, 4, 8, 16, 32)] + [(2, True), (4, True), (8, True)])
 
 
 @pytest.mark.parametrize("lanes,split", SHAPES)
@@ -134,11 +134,12 @@ def test_every_launch_shape(lanes, split, warps):
 
 
 @pytest.mark.parametrize("N", [4, 8, 9, 16, 33, 64])
-@pytest.mark.parametrize("lanes", [2, 4])
+@pytest.mark.parametrize("lanes", [2, 4, 8])
 def test_state_split_shapes(N, lanes):
-    """The state split over 2 or 4 lanes, bf16, ragged length and channels."""
-    if lanes == 4 and N <= 4:
-        pytest.skip("bucket 4 has two state pairs")
+    """The state split over 2, 4 or 8 lanes, bf16, ragged length and channels."""
+    bucket = 4 if N <= 4 else 8 if N <= 8 else 16 if N <= 16 else 32 if N <= 32 else 64
+    if bucket // 2 < lanes:
+        pytest.skip("fewer state pairs than lanes")
     inp = _case(2, 19, 203, N, torch.bfloat16, seed=N * 7 + lanes, has_z=True,
                 return_last_state=True)
     y, last = run_gpu(inp, lanes=lanes, warps=2, split=True)
