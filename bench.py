@@ -279,6 +279,8 @@ def bench_ours(args, w, world, rank, local):
     y = torch.empty(host["u"].shape, dtype=out_dtype, device=dev)
     last = (torch.empty((wr.batch, wr.dim, wr.dstate), dtype=torch.float32, device=dev)
             if wr.return_last_state else None)
+    ws = selscan.workspace_for(wr.batch, wr.dim, wr.seqlen, wr.dstate, wr.dtype, out_dtype,
+                               device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -286,7 +288,7 @@ def bench_ours(args, w, world, rank, local):
     def launch():
         selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
                        delta_bias=d["delta_bias"], delta_softplus=wr.delta_softplus,
-                       last_state=last, stream=stream)
+                       last_state=last, stream=stream, workspace=ws)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -321,14 +323,14 @@ def bench_ours(args, w, world, rank, local):
         host["last_state"].numel() * 4 if last is not None else 0)
     e2e_steps = max(1, min(args.steps, 20))
     for _ in range(2):
-        selscan.ss_fwd_hostio(host, dd, delta_softplus=wr.delta_softplus, stream=stream)
+        selscan.ss_fwd_hostio(host, dd, delta_softplus=wr.delta_softplus, stream=stream, workspace=ws)
     torch.cuda.synchronize(dev)
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        selscan.ss_fwd_hostio(host, dd, delta_softplus=wr.delta_softplus, stream=stream)
+        selscan.ss_fwd_hostio(host, dd, delta_softplus=wr.delta_softplus, stream=stream, workspace=ws)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
@@ -345,10 +347,11 @@ def bench_ours(args, w, world, rank, local):
     t_sfu = w.updates / sfu_peak
     t_hbm = nbytes / (hbm_peak * 1e9)
     roofline_ms = max(t_sfu, t_hbm) * 1e3
-    lanes, split, warps = selscan.ss_fwd_heuristic(w.batch, w.dim, w.seqlen, w.dstate, w.dtype,
-                                                   out_dtype)
+    shape = selscan.ss_fwd_heuristic(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, out_dtype,
+                                     workspace_bytes=ws.numel() if ws is not None else 0)
     traffic = (args.traffic_bytes if args.traffic_bytes
-               else recorded_traffic(w.name, [lanes, int(split), warps]))
+               else recorded_traffic(w.name, [shape["lanes_per_row"], int(shape["split_states"]),
+                                              shape["warps_per_block"], shape["segments"]]))
 
     line = {
         "metric": METRIC, "value": value, "unit": "updates/s", "n_gpus": world,
@@ -358,7 +361,7 @@ def bench_ours(args, w, world, rank, local):
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller)",
         "config": dict(w.describe(), parallelism=f"{world} independent problem(s), one per GPU",
                        l2="flushed before every timed step (write of %d MB)" % (flush.numel() >> 20),
-                       lanes_per_row=lanes, split_states=split, warps_per_block=warps),
+                       launch=shape),
         "roofline": {"bound": "alu", "achieved": achieved_ex2 / 1e12, "peak": sfu_peak / 1e12,
                      "unit": "T ex2/s", "frac": achieved_ex2 / sfu_peak, "traffic": traffic,
                      "peak_source": f"derived: {SFU_EX2_PER_CLK_PER_SM} ex2/clk/SM x {sms} SMs x "
@@ -369,7 +372,7 @@ def bench_ours(args, w, world, rank, local):
         "e2e": {"value": updates / (e2e_ms * 1e-3), "unit": "updates/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "api": "ss_fwd_hostio (pinned host buffers)"},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if shape["segments"] > 1 else 1),
         "clocks": clocks.summary(),
         "kernel_ms": {"min": min(kernel_ms), "median": statistics.median(kernel_ms),
                       "max": max(kernel_ms)},

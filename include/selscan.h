@@ -29,7 +29,9 @@
  * u, delta, B, C and z share `in_dtype`; y has `out_dtype`.
  *
  * Ownership: every pointer is caller-owned; the library allocates nothing,
- * keeps no state between calls and may be called from several threads.
+ * keeps no state between calls and may be called from several threads.  Some
+ * launch shapes need a device workspace, which the caller provides
+ * (ss_fwd_ws, ss_fwd_workspace_bytes).
  *
  * Errors: arguments are validated on the host before anything is launched;
  * a rejected call returns a status other than SS_OK and touches no memory.
@@ -40,6 +42,7 @@
 #ifndef SELSCAN_H
 #define SELSCAN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -56,7 +59,8 @@ typedef enum {
     SS_ERR_UNSUPPORTED_DSTATE = 4, /* dstate outside 1..64 */
     SS_ERR_MISALIGNED = 5,         /* a pointer is not aligned to its element size */
     SS_ERR_CUDA = 6,               /* the CUDA runtime reported an error */
-    SS_ERR_BAD_CONFIG = 7          /* ss_fwd_with_config: unsupported launch shape */
+    SS_ERR_BAD_CONFIG = 7,         /* ss_fwd_with_config: unsupported launch shape */
+    SS_ERR_WORKSPACE = 8           /* the launch shape needs a larger workspace */
 } ss_status;
 
 typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
@@ -99,38 +103,74 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  ss_stream_t stream);
 
 /*
- * As ss_fwd, with the launch shape chosen by the caller instead of by the
- * library's heuristic (for autotuning).  lanes_per_row in {1,2,4,8,16,32} is
- * how many lanes of a warp share one (b, d) row:
+ * Launch shape.  lanes_per_row in {1,2,4,8,16,32} is how many lanes of a warp
+ * share one (b, d) row:
  *   split_states = 0: the lanes split the row's steps (each takes 8 steps per
  *     chunk up to 4 lanes, 16 from 8 lanes) and combine their states with a
  *     scan over the lanes;
- *   split_states = 1: the lanes (1, 2, 4 or 8, at most half the state
- *     bucket 4/8/16/32/64 that holds dstate) split the row's states and each
- *     runs every step;
+ *   split_states = 1: the lanes (1, 2, 4 or 8, at most half the state bucket
+ *     4/8/16/32/64 that holds dstate) split the row's states and each runs
+ *     every step;
  *   one lane: the row's sequential recurrence in one lane, either way.
- * warps_per_block in {1,2,4,8}.  lanes_per_row 0 (or warps 0) picks the
- * heuristic's choice.  Results are identical for every shape up to float32
- * rounding order.  Returns SS_ERR_BAD_CONFIG for other values, or when the
- * block's shared memory for that shape would exceed 227 KB.
+ * warps_per_block in {1,2,4,8}.
+ * segments (states split or one lane only): 1 runs each row's whole sequence
+ *   in one pass; k > 1 cuts it into about k segments (a multiple of 64 steps
+ *   long) that run in parallel from a zero state, then a second kernel adds
+ *   the state carried into each segment to its outputs (exactly: it stops
+ *   once every state's decay of the carried state has underflowed to 0).  A
+ *   segmented launch needs ss_fwd_workspace_bytes() of device workspace.
+ * Zeros take the heuristic's choice for that field.
+ */
+typedef struct {
+    int lanes_per_row;
+    int split_states;
+    int warps_per_block;
+    int segments;
+} ss_launch_config;
+
+/*
+ * As ss_fwd, with a device workspace the library may use for a faster launch
+ * shape (sequence segments for long sequences with few rows).  workspace:
+ * caller-owned device memory, 16-byte aligned, of workspace_bytes bytes
+ * (NULL/0: none, then this is ss_fwd); its contents are scratch, overwritten,
+ * and must not be shared by calls that overlap on the GPU.
+ */
+ss_status ss_fwd_ws(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                    const void *B, const void *C, const float *D, const void *z,
+                    const float *delta_bias, int delta_softplus, void *y, float *last_state,
+                    void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
+/*
+ * Bytes of workspace the launch shape `config` (NULL: the heuristic's shape
+ * when a workspace is available) uses for `desc`; 0 if it uses none or the
+ * descriptor or config is invalid.
+ */
+size_t ss_fwd_workspace_bytes(const ss_desc *desc, const ss_launch_config *config);
+
+/*
+ * As ss_fwd_ws, with the launch shape chosen by the caller (for autotuning
+ * and tests).  Results agree for every shape up to float32 rounding order
+ * (and, for segmented bf16 outputs, one extra rounding of y in the steps the
+ * carried state still reaches).  Returns SS_ERR_BAD_CONFIG for unsupported
+ * values or a block needing more than 227 KB of shared memory, and
+ * SS_ERR_WORKSPACE when the shape needs more workspace than given.
  */
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
                              const float *A, const void *B, const void *C, const float *D,
                              const void *z, const float *delta_bias, int delta_softplus,
-                             void *y, float *last_state, int lanes_per_row, int split_states,
-                             int warps_per_block, ss_stream_t stream);
+                             void *y, float *last_state, const ss_launch_config *config,
+                             void *workspace, size_t workspace_bytes, ss_stream_t stream);
 
 /*
- * Launch shape ss_fwd would use for `desc` (lanes per row, state split flag,
- * warps per block).  Returns SS_OK, or the status ss_fwd would return for a
- * bad descriptor.
+ * The launch shape ss_fwd_ws would use for `desc` with `workspace_bytes` of
+ * workspace (0: as ss_fwd).  Returns SS_OK, or the status ss_fwd would return
+ * for a bad descriptor.
  */
-ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *split_states,
-                           int *warps_per_block);
+ss_status ss_fwd_heuristic(const ss_desc *desc, size_t workspace_bytes, ss_launch_config *config);
 
 /*
  * Host-buffer form: copies the inputs from host memory into caller-owned
- * device staging buffers, runs ss_fwd, and copies y (and last_state) back to
+ * device staging buffers, runs ss_fwd_ws, and copies y (and last_state) back to
  * host memory, all queued on `stream` (one cudaMemcpyAsync per buffer).  The
  * host buffers should be page-locked for the copies to be asynchronous; the
  * caller synchronises `stream` before reading the results.
@@ -138,13 +178,15 @@ ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *split_s
  *        h_delta_bias, h_last_state may be NULL exactly when the matching
  *        device buffer is NULL)
  *   d_*  device buffers of the same sizes, used as ss_fwd's arguments
+ *   d_workspace, workspace_bytes  as for ss_fwd_ws (NULL/0: none)
  */
 ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delta,
                         const float *h_A, const void *h_B, const void *h_C, const float *h_D,
                         const void *h_z, const float *h_delta_bias, int delta_softplus,
                         void *h_y, float *h_last_state, void *d_u, void *d_delta, float *d_A,
                         void *d_B, void *d_C, float *d_D, void *d_z, float *d_delta_bias,
-                        void *d_y, float *d_last_state, ss_stream_t stream);
+                        void *d_y, float *d_last_state, void *d_workspace, size_t workspace_bytes,
+                        ss_stream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char *ss_status_string(ss_status status);

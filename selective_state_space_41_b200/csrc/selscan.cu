@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <climits>
+#include <cstddef>
 #include <cstdint>
 
 #include "selscan.h"
@@ -77,37 +78,112 @@ size_t smem_for(const ss_desc *desc, int lanes, int split, int warps) {
     return selscan::smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
 }
 
+// A resolved launch: kernel shape plus sequence segmentation.
+struct Plan {
+    int lanes, split, warps;
+    int nseg;        // 1: no segmentation
+    int64_t seg_len;
+};
+
+constexpr int64_t kMinSegSteps = 2048;  // segments shorter than this are not worth a fix-up
+
+size_t workspace_for(const ss_desc *desc, int64_t rows, const Plan &pl) {
+    if (pl.nseg <= 1) return 0;
+    return (size_t)pl.nseg * (size_t)rows * (size_t)(desc->dstate + 1) * sizeof(float);
+}
+
+// Segment length for nseg segments: a multiple of the direct kernel's stage
+// (so segment starts keep 16-byte alignment); returns the segment count it gives.
+int segment(const ss_desc *desc, int nseg, int64_t *seg_len) {
+    const int64_t L = desc->seqlen;
+    if (L <= 0 || nseg <= 1) {
+        *seg_len = L;
+        return 1;
+    }
+    int64_t len = (L + nseg - 1) / nseg;
+    len = (len + selscan::kDirectStage - 1) / selscan::kDirectStage * selscan::kDirectStage;
+    *seg_len = len;
+    return (int)((L + len - 1) / len);
+}
+
 // Launch shape.  The direct kernel (lanes split a row's states, no scan) has
 // the least work per state update, so it is used whenever the rows alone
 // can give each SM sub-partition (4 per SM) enough warps: the smallest split
 // G in {1, 2, 4} (at most half the state bucket) with at least 4 warps per
 // sub-partition (with 32 or 64 states, 32 states per lane once that gives 2
-// warps), or G = 4 down to 1.5 warps.  With fewer rows the steps are
-// split instead (scan kernel): the smallest W giving 3 warps per
-// sub-partition, no more lanes than the sequence can feed, and a block
-// within half of an SM's shared memory.
-void heuristic(const ss_desc *desc, int64_t rows, int sms, int *lanes, int *split, int *warps) {
+// warps), or G = 4 down to 1.5 warps.  With fewer rows and a long sequence,
+// and a workspace, the sequence is cut into segments of at least
+// kMinSegSteps steps that the direct kernel runs as extra rows (2-way state
+// split, about 7 warps per sub-partition) and the fix-up kernel joins.
+// Otherwise the steps are split across lanes (scan kernel): the smallest W
+// giving 3 warps per sub-partition, no more lanes than the sequence can feed,
+// and a block within half of an SM's shared memory.
+Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_bytes) {
+    Plan pl{1, 0, 4, 1, desc->seqlen};
+    if (rows <= 0 || desc->seqlen <= 0) return pl;
     const int64_t slots = (int64_t)sms * 4 * 32;  // lanes per "one warp per sub-partition"
     const int bucket = selscan::state_bucket((int)desc->dstate);
     const int gmax = bucket / 2 >= 4 ? 4 : 2;
     int g = 1;
     while (g < gmax && rows * g < 4 * slots) g *= 2;
-    // Wide states: 32 states per lane (uncapped registers) once the rows alone
-    // give two warps per sub-partition.
     if (bucket >= 32 && rows * (bucket / 32) >= 2 * slots) g = bucket / 32;
     if (rows * g >= 2 * slots || rows * gmax * 2 >= 3 * slots) {
-        *lanes = g;
-        *split = g > 1 ? 1 : 0;
-        *warps = 4;
-        return;
+        pl.lanes = g;
+        pl.split = g > 1 ? 1 : 0;
+        return pl;
+    }
+    const int gs = bucket / 2 >= 2 ? 2 : 1;  // segmented: 2-way state split
+    int64_t want = (7 * slots + rows * gs - 1) / (rows * gs);
+    if (want > desc->seqlen / kMinSegSteps) want = desc->seqlen / kMinSegSteps;
+    if (want >= 2) {
+        Plan sp{gs, gs > 1 ? 1 : 0, 4, 1, 0};
+        sp.nseg = segment(desc, (int)want, &sp.seg_len);
+        if (sp.nseg >= 2 && workspace_for(desc, rows, sp) <= workspace_bytes) return sp;
     }
     int w = 2;
     while (w < 32 && rows * w < 3 * slots) w *= 2;
     while (w > 2 && (int64_t)selscan::chunk_len(w) / 2 >= desc->seqlen) w /= 2;
     while (w > 2 && smem_for(desc, w, 0, 8) > selscan::kMaxSmemBytes / 2) w /= 2;
-    *lanes = w;
-    *split = 0;
-    *warps = 8;
+    pl.lanes = w;
+    pl.split = 0;
+    pl.warps = 8;
+    return pl;
+}
+
+// The caller's launch config (zeros: the heuristic's choices) resolved into a
+// plan; SS_ERR_BAD_CONFIG for unsupported values.
+ss_status resolve(const ss_desc *desc, int64_t rows, const ss_launch_config *cfg,
+                  size_t workspace_bytes, Plan *out) {
+    Plan pl = heuristic(desc, rows, sm_count(), workspace_bytes);
+    if (cfg) {
+        const int lanes = cfg->lanes_per_row, warps = cfg->warps_per_block, split = cfg->split_states;
+        if (lanes != 0 && (lanes < 1 || lanes > 32 || (lanes & (lanes - 1)) != 0)) return SS_ERR_BAD_CONFIG;
+        if (split != 0 && split != 1) return SS_ERR_BAD_CONFIG;
+        if (warps != 0 && warps != 1 && warps != 2 && warps != 4 && warps != 8) return SS_ERR_BAD_CONFIG;
+        if (cfg->segments < 0) return SS_ERR_BAD_CONFIG;
+        if (lanes != 0) {
+            pl.lanes = lanes;
+            pl.split = split;
+            if (cfg->segments == 0) pl.nseg = 1, pl.seg_len = desc->seqlen;
+        }
+        if (warps != 0) pl.warps = warps;
+        if (cfg->segments == 1) {
+            pl.nseg = 1;
+            pl.seg_len = desc->seqlen;
+        } else if (cfg->segments > 1) {
+            pl.nseg = segment(desc, cfg->segments, &pl.seg_len);
+        }
+    }
+    const bool direct = pl.lanes == 1 || pl.split;
+    if (cfg && cfg->segments > 1 && !direct) return SS_ERR_BAD_CONFIG;  // segments need the direct kernel
+    // The direct kernel splits the state pairs of the state bucket over 1, 2, 4 or 8 lanes.
+    if (direct && (pl.lanes > 8 || selscan::state_bucket((int)desc->dstate) / 2 < pl.lanes))
+        return SS_ERR_BAD_CONFIG;
+    if (pl.nseg > 1 && !direct) return SS_ERR_BAD_CONFIG;  // segments run in the direct kernel
+    if (pl.nseg < 1) pl.nseg = 1;
+    if (pl.nseg == 1) pl.seg_len = desc->seqlen;
+    *out = pl;
+    return SS_OK;
 }
 
 // The launcher for the state bucket that holds n (4, 8, 16, 32 or 64).
@@ -125,31 +201,44 @@ cudaError_t launch_f32_f32(int n, int lanes, int split, dim3 grid, dim3 block, s
     SS_PICK_BUCKET(launch_f32_f32)
 }
 cudaError_t launch_bf16_bf16(int n, int lanes, int split, dim3 grid, dim3 block, size_t smem,
-                           cudaStream_t s, const FwdParams &p) {
+                             cudaStream_t s, const FwdParams &p) {
     SS_PICK_BUCKET(launch_bf16_bf16)
 }
 cudaError_t launch_bf16_f32(int n, int lanes, int split, dim3 grid, dim3 block, size_t smem,
-                           cudaStream_t s, const FwdParams &p) {
+                            cudaStream_t s, const FwdParams &p) {
     SS_PICK_BUCKET(launch_bf16_f32)
+}
+
+cudaError_t launch_fixup(const ss_desc *desc, int64_t rows, int nseg, cudaStream_t s, const FwdParams &p) {
+    const int64_t threads = rows * nseg;
+    const dim3 grid((unsigned)((threads + 255) / 256)), block(256);
+    if (desc->in_dtype == SS_F32)
+        selscan::ss_fwd_fixup_kernel<float, float><<<grid, block, 0, s>>>(p);
+    else if (desc->out_dtype == SS_BF16)
+        selscan::ss_fwd_fixup_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, block, 0, s>>>(p);
+    else
+        selscan::ss_fwd_fixup_kernel<__nv_bfloat16, float><<<grid, block, 0, s>>>(p);
+    return cudaGetLastError();
 }
 
 ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D, const void *z,
                    const float *delta_bias, int delta_softplus, void *y, float *last_state,
-                   int lanes, int split, int warps, ss_stream_t stream) {
+                   const ss_launch_config *cfg, void *workspace, size_t workspace_bytes,
+                   ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
-    if (lanes != 0 && (lanes < 1 || lanes > 32 || (lanes & (lanes - 1)) != 0))
-        return SS_ERR_BAD_CONFIG;
-    if (split != 0 && split != 1) return SS_ERR_BAD_CONFIG;
-    if (warps != 0 && warps != 1 && warps != 2 && warps != 4 && warps != 8)
-        return SS_ERR_BAD_CONFIG;
+    if (!workspace) workspace_bytes = 0;
+    Plan pl;
+    st = resolve(desc, sz.rows, cfg, workspace_bytes, &pl);
+    if (st != SS_OK) return st;
     if (sz.rows == 0) return SS_OK;  // no rows: nothing to read or write
     const bool need_seq = desc->seqlen > 0;
     if (!A) return SS_ERR_NULL_POINTER;
     if (need_seq && (!u || !delta || !B || !C || !y)) return SS_ERR_NULL_POINTER;
     if (!need_seq && !last_state) return SS_OK;  // nothing to write
+    if (!need_seq) pl.nseg = 1, pl.seg_len = 0;
 
     const size_t ein = dtype_size(desc->in_dtype), eout = dtype_size(desc->out_dtype);
     const void *in_ptrs[] = {u, delta, B, C, z};
@@ -158,6 +247,9 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     if ((y && !aligned(y, eout)) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
         (delta_bias && !aligned(delta_bias, 4)) || (last_state && !aligned(last_state, 4)))
         return SS_ERR_MISALIGNED;
+    const size_t ws_need = workspace_for(desc, sz.rows, pl);
+    if (ws_need > workspace_bytes) return SS_ERR_WORKSPACE;
+    if (ws_need && !aligned(workspace, 16)) return SS_ERR_MISALIGNED;
 
     // 16-byte vector path: every row of every streamed tensor starts aligned.
     bool vec = (desc->seqlen * (int64_t)ein) % 16 == 0 && (desc->seqlen * (int64_t)eout) % 16 == 0;
@@ -165,25 +257,12 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
         if (q && !aligned(q, 16)) vec = false;
     if (y && !aligned(y, 16)) vec = false;
 
-    int sms = sm_count();
-    int h_lanes, h_split, h_warps;
-    heuristic(desc, sz.rows, sms, &h_lanes, &h_split, &h_warps);
-    if (lanes == 0) {
-        lanes = h_lanes;
-        split = h_split;
-    }
-    if (warps == 0) warps = h_warps;
-    // The direct kernel splits the state pairs of the state bucket over 1, 2, 4 or 8 lanes.
-    if ((lanes == 1 || split) &&
-        (lanes > 8 || selscan::state_bucket((int)desc->dstate) / 2 < lanes))
-        return SS_ERR_BAD_CONFIG;
-
-    const size_t smem = smem_for(desc, lanes, split, warps);
+    const size_t smem = smem_for(desc, pl.lanes, pl.split, pl.warps);
     if (smem > selscan::kMaxSmemBytes) return SS_ERR_BAD_CONFIG;
-    const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
+    const int64_t rows_per_block = (int64_t)pl.warps * (32 / pl.lanes);
     const int64_t dtiles = (desc->dim + rows_per_block - 1) / rows_per_block;
-    const int64_t blocks = dtiles * desc->batch;
-    if (blocks > INT_MAX) return SS_ERR_BAD_SHAPE;
+    const int64_t blocks = dtiles * desc->batch * pl.nseg;
+    if (blocks > INT_MAX || sz.rows * pl.nseg > INT_MAX) return SS_ERR_BAD_SHAPE;
 
     FwdParams p;
     p.u = u;
@@ -203,10 +282,14 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.softplus = delta_softplus ? 1 : 0;
     p.vec = vec ? 1 : 0;
     p.dtiles = dtiles;
+    p.seg_len = pl.seg_len;
+    p.nseg = pl.nseg;
+    p.ws_hend = pl.nseg > 1 ? static_cast<float *>(workspace) : nullptr;
+    p.ws_dsum = pl.nseg > 1 ? p.ws_hend + (size_t)pl.nseg * sz.rows * desc->dstate : nullptr;
 
-    const dim3 grid((unsigned)blocks), block((unsigned)(warps * 32));
+    const dim3 grid((unsigned)blocks), block((unsigned)(pl.warps * 32));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int n = p.dstate;
+    const int n = p.dstate, lanes = pl.lanes, split = pl.split;
     cudaError_t err;
     if (desc->in_dtype == SS_F32)
         err = launch_f32_f32(n, lanes, split, grid, block, smem, s, p);
@@ -214,6 +297,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
         err = launch_bf16_bf16(n, lanes, split, grid, block, smem, s, p);
     else
         err = launch_bf16_f32(n, lanes, split, grid, block, smem, s, p);
+    if (err == cudaSuccess && pl.nseg > 1) err = launch_fixup(desc, sz.rows, pl.nseg, s, p);
     return err == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
@@ -225,27 +309,47 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  const void *B, const void *C, const float *D, const void *z,
                  const float *delta_bias, int delta_softplus, void *y, float *last_state,
                  ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, 0, 0, 0,
-                    stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, nullptr,
+                    nullptr, 0, stream);
+}
+
+ss_status ss_fwd_ws(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                    const void *B, const void *C, const float *D, const void *z,
+                    const float *delta_bias, int delta_softplus, void *y, float *last_state,
+                    void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, nullptr,
+                    workspace, workspace_bytes, stream);
 }
 
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
                              const float *A, const void *B, const void *C, const float *D,
                              const void *z, const float *delta_bias, int delta_softplus,
-                             void *y, float *last_state, int lanes_per_row, int split_states,
-                             int warps_per_block, ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state,
-                    lanes_per_row, split_states, warps_per_block, stream);
+                             void *y, float *last_state, const ss_launch_config *config,
+                             void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+    if (!config) return SS_ERR_NULL_POINTER;
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, config,
+                    workspace, workspace_bytes, stream);
 }
 
-ss_status ss_fwd_heuristic(const ss_desc *desc, int *lanes_per_row, int *split_states,
-                           int *warps_per_block) {
+ss_status ss_fwd_heuristic(const ss_desc *desc, size_t workspace_bytes, ss_launch_config *config) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
-    if (!lanes_per_row || !split_states || !warps_per_block) return SS_ERR_NULL_POINTER;
-    heuristic(desc, sz.rows, sm_count(), lanes_per_row, split_states, warps_per_block);
+    if (!config) return SS_ERR_NULL_POINTER;
+    const Plan pl = heuristic(desc, sz.rows, sm_count(), workspace_bytes);
+    config->lanes_per_row = pl.lanes;
+    config->split_states = pl.split;
+    config->warps_per_block = pl.warps;
+    config->segments = pl.nseg;
     return SS_OK;
+}
+
+size_t ss_fwd_workspace_bytes(const ss_desc *desc, const ss_launch_config *config) {
+    Sizes sz;
+    if (check_desc(desc, &sz) != SS_OK) return 0;
+    Plan pl;
+    if (resolve(desc, sz.rows, config, SIZE_MAX, &pl) != SS_OK) return 0;
+    return workspace_for(desc, sz.rows, pl);
 }
 
 ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delta,
@@ -253,7 +357,8 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
                         const void *h_z, const float *h_delta_bias, int delta_softplus,
                         void *h_y, float *h_last_state, void *d_u, void *d_delta, float *d_A,
                         void *d_B, void *d_C, float *d_D, void *d_z, float *d_delta_bias,
-                        void *d_y, float *d_last_state, ss_stream_t stream) {
+                        void *d_y, float *d_last_state, void *d_workspace, size_t workspace_bytes,
+                        ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
@@ -285,7 +390,7 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
         if (c.dst && c.bytes && cudaMemcpyAsync(c.dst, c.src, c.bytes, h2d, s) != cudaSuccess)
             return SS_ERR_CUDA;
     st = fwd_impl(desc, d_u, d_delta, d_A, d_B, d_C, d_D, d_z, d_delta_bias, delta_softplus, d_y,
-                  d_last_state, 0, 0, 0, stream);
+                  d_last_state, nullptr, d_workspace, workspace_bytes, stream);
     if (st != SS_OK) return st;
     if (n_y && cudaMemcpyAsync(h_y, d_y, n_y, d2h, s) != cudaSuccess) return SS_ERR_CUDA;
     if (d_last_state && cudaMemcpyAsync(h_last_state, d_last_state, n_last, d2h, s) != cudaSuccess)
@@ -303,6 +408,7 @@ const char *ss_status_string(ss_status status) {
         case SS_ERR_MISALIGNED: return "a pointer is not aligned to its element size";
         case SS_ERR_CUDA: return "CUDA runtime error";
         case SS_ERR_BAD_CONFIG: return "unsupported launch shape";
+        case SS_ERR_WORKSPACE: return "workspace missing or too small";
     }
     return "unknown status";
 }

@@ -50,6 +50,13 @@ struct FwdParams {
     int softplus;     // 1: softplus, 0: exp
     int vec;          // 1: every row of u/delta/z/B/C/y starts 16-byte aligned
     int64_t dtiles;   // row tiles per batch entry
+    // Sequence segments (direct kernel only): nseg > 1 runs each segment of
+    // seg_len steps from a zero state and records, per (segment, row), the
+    // end state (ws_hend, N floats) and the sum of delta' (ws_dsum) for the
+    // fix-up kernel, which adds the carried state's share of y.
+    int64_t seg_len;
+    int nseg;
+    float *ws_hend, *ws_dsum;
 };
 
 // ------------------------------------------------------------ element I/O
@@ -742,15 +749,21 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     const int r = lane / kG;                                // row within the warp
     const int rows = nthreads / kG;
     const int N = p.dstate;
-    const int64_t b = blockIdx.x / p.dtiles;
-    const int64_t d_raw = (blockIdx.x % p.dtiles) * rows + tid / kG;
+    const int64_t blocks_per_seg = p.batch * p.dtiles;
+    const int64_t seg = blockIdx.x / blocks_per_seg;
+    const int64_t bt = blockIdx.x % blocks_per_seg;
+    const int64_t b = bt / p.dtiles;
+    const int64_t d_raw = (bt % p.dtiles) * rows + tid / kG;
     const bool row_ok = d_raw < p.dim;
     const int64_t d = row_ok ? d_raw : p.dim - 1;
-    const int64_t L = p.seqlen;
+    const int64_t L = p.seqlen;  // row length (stride)
     const int64_t row = b * p.dim + d;
     const bool vec = p.vec != 0;
     const bool softplus = p.softplus != 0;
     const bool has_z = p.z != nullptr;
+    // This block's steps: [c_begin, Lend) (the whole row unless segmented).
+    const int64_t c_begin = seg * p.seg_len;
+    const int64_t Lend = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
 
     extern __shared__ float4 smem[];
     float4 *F = smem;                                                   // [kDirectStage][kPairs]
@@ -763,11 +776,11 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * N * L,
                           static_cast<const Tin *>(p.C) + b * N * L};
     // This lane's first owned step of each stream (advanced per sub-chunk).
-    const Tin *u_own = static_cast<const Tin *>(p.u) + row * L + g * kOwn;
-    const Tin *d_own = static_cast<const Tin *>(p.delta) + row * L + g * kOwn;
-    const Tin *z_own = has_z ? static_cast<const Tin *>(p.z) + row * L + g * kOwn : nullptr;
+    const Tin *u_own = static_cast<const Tin *>(p.u) + row * L + c_begin + g * kOwn;
+    const Tin *d_own = static_cast<const Tin *>(p.delta) + row * L + c_begin + g * kOwn;
+    const Tin *z_own = has_z ? static_cast<const Tin *>(p.z) + row * L + c_begin + g * kOwn : nullptr;
     Tout *const y_row = static_cast<Tout *>(p.y) + row * L;
-    Tout *y_own = y_row + g * kOwn;
+    Tout *y_own = y_row + c_begin + g * kOwn;
 
     const int q0 = g * kPL;                                 // this lane's first state pair
     const float *A_d = p.A + d * N;
@@ -782,7 +795,7 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
 
-    auto stage_fast = [&](int64_t c0) { return vec && c0 + kDirectStage <= L; };
+    auto stage_fast = [&](int64_t c0) { return vec && c0 + kDirectStage <= Lend; };
     auto issue_copies = [&](int64_t c0) {
         for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
             const int j = u % kStageUnits, rowid = u / kStageUnits;
@@ -818,7 +831,7 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
                     for (int m = 0; m < 8; ++m) {
                         const int64_t l = c0 + i0 + m;
                         uint32_t bits = 0u;
-                        if (l < L) bits = Io<Tin>::bits(src, l);
+                        if (l < Lend) bits = Io<Tin>::bits(src, l);
                         if constexpr (sizeof(Tin) == 2) bits <<= 16;
                         v[c][m] = __uint_as_float(bits);
                     }
@@ -831,14 +844,14 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     // This lane's kOwn steps of a stream starting `off` elements past `own`
     // (0 past the end of the sequence), as raw words.
     auto load_own_checked = [&](const Tin *own, int64_t s0, uint32_t (&w)[kOwnWords]) {
-        if (kOwnBytes >= 4 && vec && s0 + kOwn <= L) {
+        if (kOwnBytes >= 4 && vec && s0 + kOwn <= Lend) {
             ld_words<kOwnBytes>(own, w);
         } else {
 #pragma unroll
             for (int j = 0; j < kOwnWords; ++j) w[j] = 0u;
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
-                if (s0 + i < L) {
+                if (s0 + i < Lend) {
                     const uint32_t bits = Io<Tin>::bits(own, i);
                     if constexpr (sizeof(Tin) == 2) w[i >> 1] |= bits << (16 * (i & 1));
                     else w[i] = bits;
@@ -848,10 +861,11 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     };
 
     uint32_t wu[kOwnWords], wd[kOwnWords], wz[kOwnWords];
-    load_own_checked(u_own, g * kOwn, wu);
-    load_own_checked(d_own, g * kOwn, wd);
-    if (has_z) load_own_checked(z_own, g * kOwn, wz);
-    if (L > 0 && stage_fast(0)) issue_copies(0);
+    load_own_checked(u_own, c_begin + g * kOwn, wu);
+    load_own_checked(d_own, c_begin + g * kOwn, wd);
+    if (has_z) load_own_checked(z_own, c_begin + g * kOwn, wz);
+    if (c_begin < Lend && stage_fast(c_begin)) issue_copies(c_begin);
+    float dsum = 0.f;  // sum of this lane's delta' (segment record)
 
     // One sub-chunk of 8 steps from step l0; kChecked: guard the sequence end.
     auto sub_chunk = [&](auto checked, int m, int64_t l0) {
@@ -866,7 +880,7 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
             ld_words<kOwnBytes>(u_own, wu);
             ld_words<kOwnBytes>(d_own, wd);
             if (has_z) ld_words<kOwnBytes>(z_own, wz);
-        } else if (l0 + kDirectSub < L) {
+        } else if (l0 + kDirectSub < Lend) {
             load_own_checked(u_own, s_next, wu);
             load_own_checked(d_own, s_next, wd);
             if (has_z) load_own_checked(z_own, s_next, wz);
@@ -878,9 +892,10 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
             uo[i] = Io<Tin>::widen(cu, i);
             dl_own[i] = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
             if constexpr (kChecked) {
-                if (l0 + g * kOwn + i >= L) dl_own[i] = 0.f;
+                if (l0 + g * kOwn + i >= Lend) dl_own[i] = 0.f;
             }
             du_own[i] = dl_own[i] * uo[i];
+            dsum += dl_own[i];
         }
         // All 8 steps' values of the row.
         float dl[kDirectSub], du[kDirectSub];
@@ -952,7 +967,7 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
         }
         if (row_ok) {
             if constexpr (kChecked) {
-                store_run<kOwn>(y_row, l0 + g * kOwn, L, vec, yv);
+                store_run<kOwn>(y_row, l0 + g * kOwn, Lend, vec, yv);
             } else {
                 store_run<kOwn>(y_own, 0, kOwn, true, yv);
             }
@@ -960,31 +975,110 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
         y_own += kDirectSub;
     };
 
-    for (int64_t c0 = 0; c0 < L; c0 += kDirectStage) {
+    for (int64_t c0 = c_begin; c0 < Lend; c0 += kDirectStage) {
         const bool fast = stage_fast(c0);
         if (fast) cp_async_wait_all();
         __syncthreads();  // RB holds this stage; every warp is done with F
         fill_F(c0, fast);
         __syncthreads();  // F holds this stage; RB is free
-        if (c0 + kDirectStage < L && stage_fast(c0 + kDirectStage)) issue_copies(c0 + kDirectStage);
+        if (c0 + kDirectStage < Lend && stage_fast(c0 + kDirectStage)) issue_copies(c0 + kDirectStage);
 
         if (fast) {
 #pragma unroll 1
             for (int m = 0; m < kSubs; ++m) sub_chunk(std::false_type{}, m, c0 + m * kDirectSub);
         } else {
-            const int nsub = (int)((L - c0 < kDirectStage ? L - c0 : kDirectStage) + kDirectSub - 1) / kDirectSub;
+            const int nsub =
+                (int)((Lend - c0 < kDirectStage ? Lend - c0 : kDirectStage) + kDirectSub - 1) / kDirectSub;
 #pragma unroll 1
             for (int m = 0; m < nsub; ++m) sub_chunk(std::true_type{}, m, c0 + m * kDirectSub);
         }
     }
 
-    if (p.last_state != nullptr && row_ok) {
+    if (p.nseg > 1) {  // segment record for the fix-up kernel
+        const int64_t rec = seg * (p.batch * p.dim) + row;
+        if constexpr (kG > 1) {
+#pragma unroll
+            for (int sdist = 1; sdist < kG; sdist *= 2) dsum += __shfl_xor_sync(0xffffffffu, dsum, sdist, kG);
+        }
+        if (row_ok) {
+#pragma unroll
+            for (int qq = 0; qq < kPL; ++qq) {
+                const int n = 2 * (q0 + qq);
+                if (n < N) p.ws_hend[rec * N + n] = h[qq].x;
+                if (n + 1 < N) p.ws_hend[rec * N + n + 1] = h[qq].y;
+            }
+            if (g == 0) p.ws_dsum[rec] = dsum;
+        }
+    } else if (p.last_state != nullptr && row_ok) {
 #pragma unroll
         for (int qq = 0; qq < kPL; ++qq) {
             const int n = 2 * (q0 + qq);
             if (n < N) p.last_state[row * N + n] = h[qq].x;
             if (n + 1 < N) p.last_state[row * N + n + 1] = h[qq].y;
         }
+    }
+}
+
+// ------------------------------------------------------------ fix-up kernel
+// After the direct kernel ran every sequence segment from a zero state, the
+// true state entering segment s > 0 is the carry of segments 0..s-1:
+//   h_in(s) = P(s-1) h_in(s-1) + h_end(s-1),   P(j)_n = 2^(A_n log2e sum_j delta'),
+// and its share of y at step l of segment s is
+//   (sum_n C[b,n,l] 2^(A_n log2e S_l) h_in(s)_n) silu(z_l),   S_l = delta' summed
+// over the segment up to and including l (linearity of the recurrence in h).
+// One thread per (row, segment) adds that share to y step by step; it stops
+// once every state's exponent A_n log2e S_l is below -127, where ex2.ftz
+// returns exactly 0, so the remaining shares are exactly zero.  Thread
+// (row, segment 0) instead writes the last state h_in(nseg) when asked.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
+    constexpr bool kFast = sizeof(Tin) == 2;
+    constexpr int kMaxN = 64;
+    const int64_t rows_total = p.batch * p.dim;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= rows_total * p.nseg) return;
+    const int64_t row = t % rows_total;
+    const int s = (int)(t / rows_total);
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const int N = p.dstate;
+    const int64_t L = p.seqlen;
+    if (s == 0 && p.last_state == nullptr) return;
+
+    float A2[kMaxN], h[kMaxN];
+    float A2max = __int_as_float(0xff800000u);  // -inf
+    for (int n = 0; n < N; ++n) {
+        A2[n] = p.A[d * N + n] * kLog2e;
+        A2max = fmaxf(A2max, A2[n]);
+        h[n] = 0.f;
+    }
+    const int upto = s == 0 ? p.nseg : s;  // segments folded into the carry
+    for (int j = 0; j < upto; ++j) {
+        const int64_t rec = j * rows_total + row;
+        const float ds = p.ws_dsum[rec];
+        for (int n = 0; n < N; ++n) h[n] = fmaf(sfu_exp2(A2[n] * ds), h[n], p.ws_hend[rec * N + n]);
+    }
+    if (s == 0) {
+        for (int n = 0; n < N; ++n) p.last_state[row * N + n] = h[n];
+        return;
+    }
+
+    const Tin *dl_row = static_cast<const Tin *>(p.delta) + row * L;
+    const Tin *z_row = p.z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
+    const Tin *C_b = static_cast<const Tin *>(p.C) + b * N * L;
+    Tout *y_row = static_cast<Tout *>(p.y) + row * L;
+    const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
+    const bool softplus = p.softplus != 0;
+    const int64_t c_begin = (int64_t)s * p.seg_len;
+    const int64_t c_end = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
+    float S = 0.f;
+    for (int64_t l = c_begin; l < c_end; ++l) {
+        S += delta_transform<kFast>(static_cast<float>(dl_row[l]) + bias, softplus);
+        if (A2max * S < -127.f) break;  // every 2^(A2 S) is 0 from here on
+        float corr = 0.f;
+        for (int n = 0; n < N; ++n)
+            corr = fmaf(static_cast<float>(C_b[(int64_t)n * L + l]) * sfu_exp2(A2[n] * S), h[n], corr);
+        if (z_row) corr *= silu<kFast>(static_cast<float>(z_row[l]));
+        y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + corr);
     }
 }
 

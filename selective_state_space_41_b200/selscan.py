@@ -6,9 +6,11 @@ runs in the library's CUDA kernels.  PyTorch supplies device memory and the
 current stream.  There is no fallback: if ``libselscan.so`` is missing or
 fails to load, every call raises.
 
-The Python names match the C entry points (``ss_fwd``, ``ss_fwd_with_config``,
-``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_status_string``,
-``ss_version``); ``selective_scan_fwd`` is the allocate-and-call convenience
+The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
+``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_heuristic``,
+``ss_fwd_hostio``, ``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
+to the workspace and config forms by keyword); ``selective_scan_fwd`` is the
+allocate-and-call convenience
 form with the argument order of the walkthrough's selective_scan_ref
 ("Mamba代码实战：手把手教你用PyTorch复现选择性扫描核心逻辑（附避坑指南）", §6).
 """
@@ -23,11 +25,12 @@ SS_F32, SS_BF16 = 0, 1
 _DTYPE_CODE = {torch.float32: SS_F32, torch.bfloat16: SS_BF16}
 STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL_POINTER", 2: "SS_ERR_BAD_SHAPE",
                 3: "SS_ERR_UNSUPPORTED_DTYPE", 4: "SS_ERR_UNSUPPORTED_DSTATE",
-                5: "SS_ERR_MISALIGNED", 6: "SS_ERR_CUDA", 7: "SS_ERR_BAD_CONFIG"}
+                5: "SS_ERR_MISALIGNED", 6: "SS_ERR_CUDA", 7: "SS_ERR_BAD_CONFIG",
+                8: "SS_ERR_WORKSPACE"}
 
 # Names the header declares; the ABI test checks each is exported.
-EXPORTS = ("ss_fwd", "ss_fwd_with_config", "ss_fwd_heuristic", "ss_fwd_hostio",
-           "ss_status_string", "ss_version")
+EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config",
+           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_status_string", "ss_version")
 
 
 class SelscanError(RuntimeError):
@@ -39,6 +42,12 @@ class SelscanError(RuntimeError):
 class Desc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("seqlen", ctypes.c_int64),
                 ("dstate", ctypes.c_int64), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+class LaunchConfig(ctypes.Structure):
+    """ss_launch_config: zeros take the heuristic's choice."""
+    _fields_ = [("lanes_per_row", ctypes.c_int), ("split_states", ctypes.c_int),
+                ("warps_per_block", ctypes.c_int), ("segments", ctypes.c_int)]
 
 
 _lib = None
@@ -56,12 +65,18 @@ def lib():
         DP = ctypes.POINTER(Desc)
         L.ss_fwd.restype = I
         L.ss_fwd.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
+        SZ = ctypes.c_size_t
+        CP = ctypes.POINTER(LaunchConfig)
+        L.ss_fwd_ws.restype = I
+        L.ss_fwd_ws.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P, SZ, P]
+        L.ss_fwd_workspace_bytes.restype = SZ
+        L.ss_fwd_workspace_bytes.argtypes = [DP, CP]
         L.ss_fwd_with_config.restype = I
-        L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, I, I, I, P]
+        L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, CP, P, SZ, P]
         L.ss_fwd_heuristic.restype = I
-        L.ss_fwd_heuristic.argtypes = [DP, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]
+        L.ss_fwd_heuristic.argtypes = [DP, SZ, CP]
         L.ss_fwd_hostio.restype = I
-        L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P]
+        L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
         L.ss_status_string.restype = ctypes.c_char_p
         L.ss_status_string.argtypes = [I]
         L.ss_version.restype = I
@@ -106,15 +121,24 @@ def _check(status, where):
         raise SelscanError(status, where)
 
 
+def _config(lanes_per_row, split_states, warps_per_block, segments):
+    if lanes_per_row is None and warps_per_block is None and segments is None:
+        return None
+    return LaunchConfig(int(lanes_per_row or 0), 1 if split_states else 0, int(warps_per_block or 0),
+                        int(segments or 0))
+
+
 def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
-           last_state=None, stream=None, lanes_per_row=None, warps_per_block=None,
-           split_states=False):
+           last_state=None, stream=None, workspace=None, lanes_per_row=None, warps_per_block=None,
+           split_states=False, segments=None):
     """Queue the forward on ``stream`` (default: the current stream).
 
     u, delta, z, y: (batch, dim, L); A: (dim, N) float32; B, C: (batch, N, L);
     D, delta_bias: (dim,) float32; last_state: (batch, dim, N) float32.
-    ``lanes_per_row`` / ``split_states`` / ``warps_per_block`` select
-    ``ss_fwd_with_config``.  Raises SelscanError on a rejected call.
+    ``workspace`` (a CUDA tensor, e.g. uint8 of ss_fwd_workspace_bytes())
+    selects ``ss_fwd_ws``; ``lanes_per_row`` / ``split_states`` /
+    ``warps_per_block`` / ``segments`` select ``ss_fwd_with_config``.
+    Raises SelscanError on a rejected call.
     """
     u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
     if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
@@ -124,24 +148,47 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
     desc = make_desc(batch, dim, L, N, u.dtype, y.dtype)
     args = (ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
             _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(y), _ptr(last_state))
+    ws = _ptr(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     s = _stream_handle(stream, u.device)
-    if lanes_per_row is None and warps_per_block is None:
-        _check(lib().ss_fwd(*args, s), "ss_fwd")
+    cfg = _config(lanes_per_row, split_states, warps_per_block, segments)
+    if cfg is not None:
+        _check(lib().ss_fwd_with_config(*args, ctypes.byref(cfg), ws, ws_bytes, s),
+               "ss_fwd_with_config")
+    elif workspace is not None:
+        _check(lib().ss_fwd_ws(*args, ws, ws_bytes, s), "ss_fwd_ws")
     else:
-        _check(lib().ss_fwd_with_config(*args, int(lanes_per_row or 0), 1 if split_states else 0,
-                                        int(warps_per_block or 0), s), "ss_fwd_with_config")
+        _check(lib().ss_fwd(*args, s), "ss_fwd")
 
 
-def ss_fwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None):
-    """(lanes_per_row, split_states, warps_per_block) the library picks."""
+def ss_fwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None,
+                           lanes_per_row=None, split_states=False, warps_per_block=None,
+                           segments=None) -> int:
+    """Workspace bytes of the heuristic's shape (or the given one)."""
     desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
-    lanes, split, warps = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(lib().ss_fwd_heuristic(ctypes.byref(desc), ctypes.byref(lanes), ctypes.byref(split),
-                                  ctypes.byref(warps)), "ss_fwd_heuristic")
-    return lanes.value, bool(split.value), warps.value
+    cfg = _config(lanes_per_row, split_states, warps_per_block, segments)
+    return int(lib().ss_fwd_workspace_bytes(ctypes.byref(desc),
+                                            ctypes.byref(cfg) if cfg is not None else None))
 
 
-def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None):
+def workspace_for(batch, dim, seqlen, dstate, in_dtype, out_dtype=None, device="cuda", **config):
+    """A uint8 CUDA tensor large enough for the launch shape, or None if it needs none."""
+    n = ss_fwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype, out_dtype, **config)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def ss_fwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None,
+                     workspace_bytes=0):
+    """The launch shape the library picks, as a dict."""
+    desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
+    cfg = LaunchConfig()
+    _check(lib().ss_fwd_heuristic(ctypes.byref(desc), int(workspace_bytes), ctypes.byref(cfg)),
+           "ss_fwd_heuristic")
+    return {"lanes_per_row": cfg.lanes_per_row, "split_states": bool(cfg.split_states),
+            "warps_per_block": cfg.warps_per_block, "segments": cfg.segments}
+
+
+def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None, workspace=None):
     """Host-buffer form: ``host`` and ``dev`` map u, delta, A, B, C, D, z,
     delta_bias, y, last_state to host (ideally pinned) and device tensors of
     the same shapes (optional entries None in both).  Queues copies in, the
@@ -153,9 +200,11 @@ def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None):
     names_in = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
     h_in = [_ptr(g(host, k)) for k in names_in]
     d_all = [_ptr(g(dev, k)) for k in names_in + ("y", "last_state")]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     s = _stream_handle(stream, dev["u"].device)
     _check(lib().ss_fwd_hostio(ctypes.byref(desc), *h_in, 1 if delta_softplus else 0,
-                               _ptr(host["y"]), _ptr(g(host, "last_state")), *d_all, s),
+                               _ptr(host["y"]), _ptr(g(host, "last_state")), *d_all,
+                               _ptr(workspace), ws_bytes, s),
            "ss_fwd_hostio")
 
 
@@ -174,6 +223,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     y = torch.empty((batch, dim, L), dtype=out_dtype or u.dtype, device=u.device)
     last = (torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
             if return_last_state else None)
+    ws = workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=u.device)
     ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
-           last_state=last, stream=stream)
+           last_state=last, stream=stream, workspace=ws)
     return (y, last) if return_last_state else y

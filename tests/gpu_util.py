@@ -18,8 +18,11 @@ def to_dev(inp, device="cuda"):
     return out
 
 
-def run_gpu(inp, out_dtype=None, lanes=None, warps=None, split=False, device="cuda"):
-    """(y, last_state) from libselscan for host inputs ``inp``."""
+def run_gpu(inp, out_dtype=None, lanes=None, warps=None, split=False, segments=None,
+            workspace=True, device="cuda"):
+    """(y, last_state) from libselscan for host inputs ``inp``.  ``workspace``:
+    give the call the workspace its launch shape can use (as the benchmark and
+    selective_scan_fwd do); False: no workspace (plain ss_fwd)."""
     d = to_dev(inp, device)
     u = d["u"]
     batch, dim, L = u.shape
@@ -28,10 +31,14 @@ def run_gpu(inp, out_dtype=None, lanes=None, warps=None, split=False, device="cu
                     device=device)
     last = (torch.empty((batch, dim, N), dtype=torch.float32, device=device)
             if inp.get("return_last_state") else None)
+    cfg = {}
+    if lanes is not None or warps is not None or segments is not None:
+        cfg = dict(lanes_per_row=lanes, warps_per_block=warps, split_states=split, segments=segments)
+    ws = (selscan.workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=device, **cfg)
+          if workspace else None)
     selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d.get("D"), z=d.get("z"),
                    delta_bias=d.get("delta_bias"), delta_softplus=inp["delta_softplus"],
-                   last_state=last, lanes_per_row=lanes, warps_per_block=warps,
-                   split_states=split)
+                   last_state=last, workspace=ws, **cfg)
     torch.cuda.synchronize()
     return y, last
 

@@ -73,15 +73,44 @@ def test_rejections_before_any_launch(lib):
     # empty problems need no pointers at all
     assert _call(lib, _desc(batch=0), u=None, delta=None, A=None, B=None, C=None, y=None) == 0
     assert _call(lib, _desc(seqlen=0), u=None, delta=None, B=None, C=None, y=None) == 0
+    assert lib.ss_status_string(8) == b"workspace missing or too small"
+
+
+def _cfg(lanes=0, split=0, warps=0, segments=0):
+    return ctypes.byref(selscan.LaunchConfig(lanes, split, warps, segments))
 
 
 def test_bad_launch_shapes_rejected(lib):
-    d = _desc()
+    # Every call here must be rejected before any launch: the pointers are fake.
+    d = _desc(seqlen=4096)
     args = (ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE, None)
-    assert lib.ss_fwd_with_config(*args, 3, 0, 4, None) == 7
-    assert lib.ss_fwd_with_config(*args, 64, 0, 4, None) == 7
-    assert lib.ss_fwd_with_config(*args, 4, 0, 3, None) == 7
-    assert lib.ss_fwd_with_config(*args, 4, 2, 4, None) == 7
+    assert lib.ss_fwd_with_config(*args, _cfg(3, 0, 4), None, 0, None) == 7
+    assert lib.ss_fwd_with_config(*args, _cfg(64, 0, 4), None, 0, None) == 7
+    assert lib.ss_fwd_with_config(*args, _cfg(4, 0, 3), None, 0, None) == 7
+    assert lib.ss_fwd_with_config(*args, _cfg(4, 2, 4), None, 0, None) == 7
+    assert lib.ss_fwd_with_config(*args, _cfg(16, 1, 4), None, 0, None) == 7   # 16-way state split
+    assert lib.ss_fwd_with_config(*args, _cfg(4, 0, 4, 3), None, 0, None) == 7  # segments need split
+    assert lib.ss_fwd_with_config(*args, _cfg(segments=-1), None, 0, None) == 7
+    assert lib.ss_fwd_with_config(*args, None, None, 0, None) == 1
+
+
+def test_workspace_sizes(lib):
+    """Workspace query: segments need (segments x rows x (N + 1)) floats."""
+    d = _desc(batch=2, dim=3, seqlen=4096, dstate=4)
+    assert lib.ss_fwd_workspace_bytes(ctypes.byref(d), _cfg(2, 1, 4, 1)) == 0
+    # 4096 steps in about 4 segments of 1024 steps: 4 segments
+    assert lib.ss_fwd_workspace_bytes(ctypes.byref(d), _cfg(2, 1, 4, 4)) == 4 * 6 * 5 * 4
+    # 3 segments: 1366 rounded up to 1408 (a multiple of 64): 3 segments
+    assert lib.ss_fwd_workspace_bytes(ctypes.byref(d), _cfg(1, 0, 4, 3)) == 3 * 6 * 5 * 4
+    assert lib.ss_fwd_workspace_bytes(ctypes.byref(d), _cfg(4, 0, 4, 2)) == 0   # invalid: no split
+    assert lib.ss_fwd_workspace_bytes(None, None) == 0
+
+
+def test_segmented_call_without_workspace_rejected(lib):
+    d = _desc(batch=2, dim=3, seqlen=4096, dstate=4)
+    args = (ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE, None)
+    assert lib.ss_fwd_with_config(*args, _cfg(2, 1, 4, 4), None, 0, None) == 8
+    assert lib.ss_fwd_with_config(*args, _cfg(2, 1, 4, 4), FAKE, 100, None) == 8
 
 
 def test_hostio_rejections(lib):
@@ -91,5 +120,5 @@ def test_hostio_rejections(lib):
     dev = [P, P, P, P, P, None, None, None, P, None]
     # D given on the host but not on the device
     base_d = [P, P, P, P, P, P, None, None]
-    assert lib.ss_fwd_hostio(ctypes.byref(d), *base_d, 1, P, None, *dev, None) == 1
-    assert lib.ss_fwd_hostio(None, *base, 1, P, None, *dev, None) == 1
+    assert lib.ss_fwd_hostio(ctypes.byref(d), *base_d, 1, P, None, *dev, None, 0, None) == 1
+    assert lib.ss_fwd_hostio(None, *base, 1, P, None, *dev, None, 0, None) == 1

@@ -147,6 +147,40 @@ def test_state_split_shapes(N, lanes):
     assert_parity(y, last, y_ref, last_ref, TOL[torch.bfloat16], f"N={N} lanes={lanes} split")
 
 
+# ---------------------------------------------------------------- segments
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("L,segments", [(4096, 2), (3001, 3), (5000, 7), (640, 4), (129, 2)])
+@pytest.mark.parametrize("lanes,split", [(1, False), (2, True), (4, True)])
+def test_sequence_segments(dtype, L, segments, lanes, split):
+    """Segments run from a zero state plus the fix-up of the carried state."""
+    inp = _case(2, 5, L, 16, dtype, seed=L + segments + lanes, has_z=True, return_last_state=True)
+    y, last = run_gpu(inp, lanes=lanes, split=split, warps=2, segments=segments)
+    y_ref, last_ref = run_oracle(inp)
+    assert_parity(y, last, y_ref, last_ref, TOL[dtype], f"L={L} segments={segments} lanes={lanes}")
+
+
+def test_segments_long_memory():
+    """delta' tiny (long memory: the carried state never decays to 0, so the
+    fix-up runs through whole segments) and exp mode with large delta' (fast
+    decay), each segmented."""
+    inp = _case(1, 6, 2500, 8, torch.float32, seed=11, has_z=False, return_last_state=True)
+    slow = dict(inp, delta=inp["delta"] * 0.1 - 7.0)            # softplus(-7) ~ 1e-3
+    y, last = run_gpu(slow, lanes=2, split=True, warps=1, segments=5)
+    y_ref, last_ref = run_oracle(slow)
+    assert_parity(y, last, y_ref, last_ref, TOL[torch.float32], "slow decay")
+    fast = dict(inp, delta=inp["delta"] * 0.3 + 1.0, delta_softplus=False)
+    y, last = run_gpu(fast, lanes=2, split=True, warps=1, segments=5)
+    y_ref, last_ref = run_oracle(fast)
+    assert_parity(y, last, y_ref, last_ref, TOL[torch.float32], "fast decay")
+
+
+def test_heuristic_segments_genomic_shape():
+    """The genomic shape segments when given a workspace, and not without one."""
+    h_ws = selscan.ss_fwd_heuristic(4, 1024, 100000, 16, torch.bfloat16, workspace_bytes=1 << 30)
+    h_no = selscan.ss_fwd_heuristic(4, 1024, 100000, 16, torch.bfloat16)
+    assert h_ws["segments"] > 1 and h_no["segments"] == 1
+
+
 def test_unaligned_rows_take_the_scalar_path():
     """Pointers offset by one element (still element-aligned) and an odd L:
     the kernel must fall back from 16-byte vectors and still be exact."""
@@ -228,7 +262,8 @@ def test_hostio_matches_device_path():
     host["last_state"] = torch.empty(last_dev.shape, dtype=torch.float32).pin_memory()
     dev = {k: (torch.empty_like(v, device="cuda") if v is not None else None)
            for k, v in host.items()}
-    selscan.ss_fwd_hostio(host, dev, delta_softplus=True)
+    ws = selscan.workspace_for(w.batch, w.dim, w.seqlen, w.dstate, w.dtype)  # as run_gpu
+    selscan.ss_fwd_hostio(host, dev, delta_softplus=True, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(host["y"].view(torch.int16), y_dev.cpu().view(torch.int16))
     assert torch.equal(host["last_state"], last_dev.cpu())
