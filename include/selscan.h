@@ -31,7 +31,8 @@
  * Ownership: every pointer is caller-owned; the library allocates nothing,
  * keeps no state between calls and may be called from several threads.  Some
  * launch shapes need a device workspace, which the caller provides
- * (ss_fwd_ws, ss_fwd_workspace_bytes).
+ * (ss_fwd_ws, ss_fwd_workspace_bytes), or which ss_fwd_noalloc takes from a
+ * fixed static device array (the one piece of state: its cached address).
  *
  * Errors: arguments are validated on the host before anything is launched;
  * a rejected call returns a status other than SS_OK and touches no memory.
@@ -60,7 +61,8 @@ typedef enum {
     SS_ERR_MISALIGNED = 5,         /* a pointer is not aligned to its element size */
     SS_ERR_CUDA = 6,               /* the CUDA runtime reported an error */
     SS_ERR_BAD_CONFIG = 7,         /* ss_fwd_with_config: unsupported launch shape */
-    SS_ERR_WORKSPACE = 8           /* the launch shape needs a larger workspace */
+    SS_ERR_WORKSPACE = 8,          /* the launch shape needs a larger workspace */
+    SS_ERR_SCRATCH_LIMIT = 9       /* ss_fwd_noalloc: needs more than SS_NOALLOC_SCRATCH_BYTES */
 } ss_status;
 
 typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
@@ -187,6 +189,39 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
                         void *d_B, void *d_C, float *d_D, void *d_z, float *d_delta_bias,
                         void *d_y, float *d_last_state, void *d_workspace, size_t workspace_bytes,
                         ss_stream_t stream);
+
+/*
+ * Bytes of the device scratch array built into the library for
+ * ss_fwd_noalloc (8 MiB per device; 4.7 MB covers a 4 x 1024-channel,
+ * 16-state layer over 100000 steps).
+ */
+#define SS_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * As ss_fwd_ws given all the workspace its launch shape can use (same launch
+ * shape, bitwise the same results), but with the workspace taken from a
+ * static device array of SS_NOALLOC_SCRATCH_BYTES bytes inside the library,
+ * so the caller passes none and nothing is allocated.  This entry has no
+ * counterpart in the method's description; it exists for callers that may
+ * not allocate device memory when they call (a fixed memory budget, a host
+ * framework that owns all allocation, or a path where the device-wide
+ * synchronisation of cudaMalloc / cudaFree is not acceptable).
+ *   - Returns SS_ERR_SCRATCH_LIMIT, launching nothing, when that launch shape
+ *     needs more than SS_NOALLOC_SCRATCH_BYTES (ss_fwd_workspace_bytes(desc,
+ *     NULL) says how much it needs); other errors as ss_fwd_ws.
+ *   - The first call on each device (the device current at the call) looks
+ *     up the array's device address with cudaGetSymbolAddress and caches it;
+ *     make that first call before any stream capture on that device.
+ *   - All calls on one device share the one array: calls whose work overlaps
+ *     on the GPU (other streams, other host threads) race on it and give
+ *     wrong results.  Calls queued in order on one stream are safe.
+ *   - The array needs no initialisation: each call writes every scratch word
+ *     it reads before reading it.
+ */
+ss_status ss_fwd_noalloc(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D, const void *z,
+                         const float *delta_bias, int delta_softplus, void *y, float *last_state,
+                         ss_stream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char *ss_status_string(ss_status status);

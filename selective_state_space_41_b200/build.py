@@ -48,7 +48,9 @@ def _compile_jobs(verbose: bool):
     if verbose:
         base += ["-Xptxas", "-v"]
     jobs = [(base + [os.path.join(CSRC, "selscan.cu"), "-o",
-                     os.path.join(BUILD_DIR, "selscan.o")], "selscan")]
+                     os.path.join(BUILD_DIR, "selscan.o")], "selscan"),
+            (base + [os.path.join(CSRC, "ss_noalloc.cu"), "-o",
+                     os.path.join(BUILD_DIR, "ss_noalloc.o")], "ss_noalloc")]
     for tin, tout, tag in DTYPE_PAIRS:
         for n in STATE_BUCKETS:
             name = f"launch_{tag}_n{n}"

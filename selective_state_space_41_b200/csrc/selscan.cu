@@ -409,6 +409,7 @@ const char *ss_status_string(ss_status status) {
         case SS_ERR_CUDA: return "CUDA runtime error";
         case SS_ERR_BAD_CONFIG: return "unsupported launch shape";
         case SS_ERR_WORKSPACE: return "workspace missing or too small";
+        case SS_ERR_SCRATCH_LIMIT: return "needs more scratch than the no-alloc entry's static array";
     }
     return "unknown status";
 }

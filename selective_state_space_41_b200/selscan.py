@@ -8,7 +8,7 @@ fails to load, every call raises.
 
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_heuristic``,
-``ss_fwd_hostio``, ``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
+``ss_fwd_hostio``, ``ss_fwd_noalloc``, ``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
 to the workspace and config forms by keyword); ``selective_scan_fwd`` is the
 allocate-and-call convenience
 form with the argument order of the walkthrough's selective_scan_ref
@@ -26,11 +26,14 @@ _DTYPE_CODE = {torch.float32: SS_F32, torch.bfloat16: SS_BF16}
 STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL_POINTER", 2: "SS_ERR_BAD_SHAPE",
                 3: "SS_ERR_UNSUPPORTED_DTYPE", 4: "SS_ERR_UNSUPPORTED_DSTATE",
                 5: "SS_ERR_MISALIGNED", 6: "SS_ERR_CUDA", 7: "SS_ERR_BAD_CONFIG",
-                8: "SS_ERR_WORKSPACE"}
+                8: "SS_ERR_WORKSPACE", 9: "SS_ERR_SCRATCH_LIMIT"}
+
+# SS_NOALLOC_SCRATCH_BYTES: the static scratch array behind ss_fwd_noalloc.
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Names the header declares; the ABI test checks each is exported.
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config",
-           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_status_string", "ss_version")
+           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc", "ss_status_string", "ss_version")
 
 
 class SelscanError(RuntimeError):
@@ -77,6 +80,8 @@ def lib():
         L.ss_fwd_heuristic.argtypes = [DP, SZ, CP]
         L.ss_fwd_hostio.restype = I
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
+        L.ss_fwd_noalloc.restype = I
+        L.ss_fwd_noalloc.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
         L.ss_status_string.restype = ctypes.c_char_p
         L.ss_status_string.argtypes = [I]
         L.ss_version.restype = I
@@ -159,6 +164,24 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
         _check(lib().ss_fwd_ws(*args, ws, ws_bytes, s), "ss_fwd_ws")
     else:
         _check(lib().ss_fwd(*args, s), "ss_fwd")
+
+
+def ss_fwd_noalloc(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
+                   last_state=None, stream=None):
+    """Queue the forward with the library's static scratch array as the
+    workspace (no device memory is allocated).  Same tensors as ``ss_fwd``;
+    raises SelscanError (SS_ERR_SCRATCH_LIMIT) when the launch shape needs
+    more than NOALLOC_SCRATCH_BYTES.  Calls that overlap on the GPU share the
+    array and race."""
+    u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
+    if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
+        raise ValueError("outputs must be contiguous")
+    batch, dim, L = u.shape
+    desc = make_desc(batch, dim, L, A.shape[-1], u.dtype, y.dtype)
+    _check(lib().ss_fwd_noalloc(ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0,
+                                _ptr(y), _ptr(last_state), _stream_handle(stream, u.device)),
+           "ss_fwd_noalloc")
 
 
 def ss_fwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None,

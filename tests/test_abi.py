@@ -113,6 +113,20 @@ def test_segmented_call_without_workspace_rejected(lib):
     assert lib.ss_fwd_with_config(*args, _cfg(2, 1, 4, 4), FAKE, 100, None) == 8
 
 
+def test_noalloc_rejections_before_any_launch(lib):
+    """ss_fwd_noalloc rejects a bad descriptor, and a launch shape needing
+    more than the static scratch array, before any CUDA call."""
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE, None, None)
+    assert lib.ss_fwd_noalloc(None, *args) == 1
+    assert lib.ss_fwd_noalloc(ctypes.byref(_desc(dstate=0)), *args) == 4
+    assert lib.ss_fwd_noalloc(ctypes.byref(_desc(in_dtype=0, out_dtype=1)), *args) == 3
+    # 64 rows x 4M steps x 64 states: about 1025 segments, 17 MB of scratch
+    big = _desc(batch=1, dim=64, seqlen=4_000_000, dstate=64)
+    assert lib.ss_fwd_workspace_bytes(ctypes.byref(big), None) > selscan.NOALLOC_SCRATCH_BYTES
+    assert lib.ss_fwd_noalloc(ctypes.byref(big), *args) == 9
+    assert "scratch" in selscan.ss_status_string(9)
+
+
 def test_hostio_rejections(lib):
     d = _desc()
     P = FAKE
