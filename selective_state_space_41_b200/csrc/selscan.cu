@@ -133,7 +133,7 @@ Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_byte
         return pl;
     }
     const int gs = bucket / 2 >= 2 ? 2 : 1;  // segmented: 2-way state split
-    int64_t want = (7 * slots + rows * gs - 1) / (rows * gs);
+    int64_t want = (7 * slots) / (rows * gs);
     if (want > desc->seqlen / kMinSegSteps) want = desc->seqlen / kMinSegSteps;
     if (want >= 2) {
         Plan sp{gs, gs > 1 ? 1 : 0, 4, 1, 0};

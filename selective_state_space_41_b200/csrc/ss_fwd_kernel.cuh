@@ -687,13 +687,47 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
 #define SS_DIRECT_MIN_BLOCKS 2
 #endif
 constexpr int kDirectStage = 64;  // steps per shared-memory stage
-constexpr int kDirectSub = 8;     // steps per register sub-chunk
-constexpr int kGatherStride = 20; // floats per row of the gather slab (16 used; spreads banks)
-constexpr int kReduceStride = 12; // floats per lane of the reduce slab (8 used)
+
+// Steps per register sub-chunk: 16 when 4 or 8 lanes share a row (few states
+// per lane, so the per-sub-chunk exchanges and their latency are amortised
+// over more steps), 8 otherwise (more states per lane: register pressure).
+__host__ __device__ constexpr int direct_sub(int g) { return g >= 4 ? 16 : 8; }
+// Floats per row of the gather slab: delta' and delta' u of each step, plus
+// 4 to spread the rows over the banks.
+__host__ __device__ constexpr int gather_stride(int g) { return 2 * direct_sub(g) + 4; }
+// Reduce slab: lane (r, g) writes its sub-chunk's partial sums of y at
+// lane * stride, then reads the partials of its own steps from the lanes of
+// its row, `vec` floats per access.  Stride and width are chosen so that both
+// the writes and the reads of a warp hit distinct banks in each 128-byte
+// phase (checked with a model of the 32 four-byte banks).
+__host__ __device__ constexpr int reduce_stride(int g) {
+    return g <= 1 ? 0 : g == 2 ? 12 : g == 4 ? 20 : 18;
+}
+__host__ __device__ constexpr int reduce_vec(int g) { return g == 8 ? 2 : 4; }
 
 __host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax, int g, int warps) {
     return 4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage +
-           (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * kGatherStride + 32 * kReduceStride) : 0);
+           (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * gather_stride(g) + 32 * reduce_stride(g)) : 0);
+}
+
+// kW consecutive floats to / from shared memory as one access (kW in {1, 2, 4}).
+template <int kW>
+__device__ __forceinline__ void st_vec(float *p, const float *v) {
+    if constexpr (kW == 4) *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else if constexpr (kW == 2) *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    else p[0] = v[0];
+}
+template <int kW>
+__device__ __forceinline__ void ld_vec(const float *p, float *v) {
+    if constexpr (kW == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        v[0] = x.x, v[1] = x.y, v[2] = x.z, v[3] = x.w;
+    } else if constexpr (kW == 2) {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x, v[1] = x.y;
+    } else {
+        v[0] = p[0];
+    }
 }
 
 // Load `bytes` (4, 8, 16 or 32) from 16/8/4-byte aligned global memory into words.
@@ -723,13 +757,20 @@ struct DirectOccupancy {
     static constexpr int kMinBlocks = kStatesPerLane <= 16 ? SS_DIRECT_MIN_BLOCKS : 1;
 };
 
+#ifdef SS_DIRECT_MAXNREG
+#define SS_DIRECT_BOUNDS(SPL) __maxnreg__(SS_DIRECT_MAXNREG)
+#else
+#define SS_DIRECT_BOUNDS(SPL) __launch_bounds__(256, DirectOccupancy<SPL>::kMinBlocks)
+#endif
+
 template <typename Tin, typename Tout, int kNmax, int kG>
-__global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
-    ss_fwd_direct_kernel(const FwdParams p) {
+__global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParams p) {
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                        // state pairs per lane
     static_assert(kG == 1 || kG == 2 || kG == 4 || kG == 8, "1, 2, 4 or 8 lanes per row");
     static_assert(kPL >= 1, "at least one state pair per lane");
+    constexpr int kDirectSub = direct_sub(kG);              // steps per sub-chunk
+    constexpr int kGatherStride = gather_stride(kG);
     constexpr int kOwn = kDirectSub / kG;                   // steps owned per lane per sub-chunk
     constexpr int kOwnBytes = kOwn * (int)sizeof(Tin);
     constexpr int kOwnWords = (kOwnBytes + 3) / 4;
@@ -768,8 +809,9 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
     extern __shared__ float4 smem[];
     float4 *F = smem;                                                   // [kDirectStage][kPairs]
     Tin *RB = reinterpret_cast<Tin *>(smem + kDirectStage * kPairs);     // [2][kNmax][kDirectStage]
+    constexpr int kRS = reduce_stride(kG), kRV = reduce_vec(kG);
     float *slab = reinterpret_cast<float *>(RB + 2 * kNmax * kDirectStage) +
-                  warp * (kRowsPerWarp * kGatherStride + 32 * kReduceStride);
+                  warp * (kRowsPerWarp * kGatherStride + 32 * kRS);
     float *gat = slab + r * kGatherStride;                  // this row: 8 delta', 8 delta' u
     float *red = slab + kRowsPerWarp * kGatherStride;       // per lane: 8 partial sums of y
 
@@ -904,18 +946,24 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
             for (int i = 0; i < kDirectSub; ++i) dl[i] = dl_own[i], du[i] = du_own[i];
         } else {
 #pragma unroll
-            for (int i = 0; i < kOwn; ++i) gat[g * kOwn + i] = dl_own[i], gat[8 + g * kOwn + i] = du_own[i];
+            for (int i = 0; i < kOwn; ++i)
+                gat[g * kOwn + i] = dl_own[i], gat[kDirectSub + g * kOwn + i] = du_own[i];
             __syncwarp();
 #pragma unroll
-            for (int q4 = 0; q4 < 2; ++q4) {
+            for (int q4 = 0; q4 < kDirectSub / 4; ++q4) {
                 const float4 a4 = reinterpret_cast<const float4 *>(gat)[q4];
-                const float4 b4 = reinterpret_cast<const float4 *>(gat + 8)[q4];
+                const float4 b4 = reinterpret_cast<const float4 *>(gat + kDirectSub)[q4];
                 dl[4 * q4] = a4.x, dl[4 * q4 + 1] = a4.y, dl[4 * q4 + 2] = a4.z, dl[4 * q4 + 3] = a4.w;
                 du[4 * q4] = b4.x, du[4 * q4 + 1] = b4.y, du[4 * q4 + 2] = b4.z, du[4 * q4 + 3] = b4.w;
             }
         }
         float part[kDirectSub];
         const float4 *Fm = F + (m * kDirectSub) * kPairs + q0;
+        auto A2_of = [&](int qq) {
+            if constexpr (kA2InRegs) return A2[qq];
+            const int n = 2 * (q0 + qq);
+            return make_float2(n < N ? __ldg(A_d + n) * kLog2e : 0.f, n + 1 < N ? __ldg(A_d + n + 1) * kLog2e : 0.f);
+        };
 #pragma unroll
         for (int i = 0; i < kDirectSub; ++i) {
             const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
@@ -925,14 +973,7 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
 #pragma unroll
             for (int qq = 0; qq < kPL; ++qq) {
                 const float4 bc = Fm[i * kPairs + qq];
-                float2 A2q;
-                if constexpr (kA2InRegs) A2q = A2[qq];
-                else {
-                    const int n = 2 * (q0 + qq);
-                    A2q = make_float2(n < N ? __ldg(A_d + n) * kLog2e : 0.f,
-                                      n + 1 < N ? __ldg(A_d + n + 1) * kLog2e : 0.f);
-                }
-                const float2 t = __fmul2_rn(d2, A2q);
+                const float2 t = __fmul2_rn(d2, A2_of(qq));
                 const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
                 h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
                 acc[qq % kAccs] = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc[qq % kAccs]);
@@ -946,17 +987,23 @@ __global__ void __launch_bounds__(256, DirectOccupancy<kNmax / kG>::kMinBlocks)
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) yv[i] = part[i];
         } else {
-            float *mine = red + lane * kReduceStride;
-            reinterpret_cast<float4 *>(mine)[0] = make_float4(part[0], part[1], part[2], part[3]);
-            reinterpret_cast<float4 *>(mine)[1] = make_float4(part[4], part[5], part[6], part[7]);
+            static_assert(kOwn % kRV == 0 && kRS % kRV == 0, "reduce slab accesses stay aligned");
+            float *mine = red + lane * kRS;
+#pragma unroll
+            for (int k = 0; k < kDirectSub; k += kRV) st_vec<kRV>(mine + k, part + k);
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) yv[i] = 0.f;
 #pragma unroll
             for (int gg = 0; gg < kG; ++gg) {
-                const float *src = red + (r * kG + gg) * kReduceStride + g * kOwn;
+                const float *src = red + (r * kG + gg) * kRS + g * kOwn;
 #pragma unroll
-                for (int i = 0; i < kOwn; ++i) yv[i] += src[i];
+                for (int k = 0; k < kOwn; k += kRV) {
+                    float v[kRV];
+                    ld_vec<kRV>(src + k, v);
+#pragma unroll
+                    for (int j = 0; j < kRV; ++j) yv[k + j] += v[j];
+                }
             }
         }
 #pragma unroll
