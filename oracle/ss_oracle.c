@@ -16,6 +16,11 @@
  *     page ("Mamba-minimal项目解析", 关键技术点 §1 选择性扫描算法);
  *   - §3.3 (加入跳跃连接): y += D[d] * u, then y *= silu(z) when z is given;
  *   - §6 (完整实现与测试): the optional last state is the state after step L.
+ * Extension (no counterpart in the walkthrough, whose state always starts at
+ * zero): an optional initial state replaces that zero, so that a sequence can
+ * be run in pieces, each piece starting from the last state of the one before
+ * (the streaming and single-step use of the recurrence that "告别‘炼丹’：从
+ * Mamba-minimal入手..." describes in §2.1).
  * The "parallel" body printed in §4.2 / §6 (cumprod then cumsum) is NOT what
  * this follows: it disagrees with the §3.2 loop, which is the definition.
  *
@@ -24,8 +29,8 @@
  *   A              : (dim, dstate)
  *   B, C           : (batch, dstate, seqlen)
  *   D, delta_bias  : (dim)
- *   last_state     : (batch, dim, dstate)
- * D, z, delta_bias and last_state may be NULL (absent).
+ *   last_state, initial_state : (batch, dim, dstate)
+ * D, z, delta_bias, last_state and initial_state may be NULL (absent).
  *
  * Rows (b, d) are independent; the only parallelism here is an OpenMP loop
  * over rows, each row running the plain sequential loop above.
@@ -62,11 +67,12 @@ int ss_oracle_threads(void)
 }
 
 /* Returns 0 on success, -1 on a bad argument. nthreads <= 0 means "all". */
-int ss_oracle_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
-                  const double *u, const double *delta, const double *A,
-                  const double *B, const double *C, const double *D,
-                  const double *z, const double *delta_bias, int delta_softplus,
-                  double *y, double *last_state, int nthreads)
+int ss_oracle_fwd_init(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                       const double *u, const double *delta, const double *A,
+                       const double *B, const double *C, const double *D,
+                       const double *z, const double *delta_bias, int delta_softplus,
+                       const double *initial_state, double *y, double *last_state,
+                       int nthreads)
 {
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1)
         return -1;
@@ -88,8 +94,8 @@ int ss_oracle_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
             ok |= 1;
             continue;
         }
-        for (int64_t n = 0; n < dstate; ++n)
-            h[n] = 0.0; /* the state starts at zero (§3.2) */
+        for (int64_t n = 0; n < dstate; ++n) /* zero (§3.2) unless an initial state is given */
+            h[n] = initial_state ? initial_state[row * dstate + n] : 0.0;
 
         for (int64_t l = 0; l < seqlen; ++l) {
             const int64_t idx = row * seqlen + l;
@@ -120,4 +126,15 @@ int ss_oracle_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
         free(h);
     }
     return ok ? -1 : 0;
+}
+
+/* The walkthrough's form: the state starts at zero. */
+int ss_oracle_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                  const double *u, const double *delta, const double *A,
+                  const double *B, const double *C, const double *D,
+                  const double *z, const double *delta_bias, int delta_softplus,
+                  double *y, double *last_state, int nthreads)
+{
+    return ss_oracle_fwd_init(batch, dim, seqlen, dstate, u, delta, A, B, C, D, z, delta_bias,
+                              delta_softplus, NULL, y, last_state, nthreads);
 }

@@ -292,6 +292,94 @@ def pin_last_state(scan):
     assert np.all(last0 == 0.0), "empty sequence must leave the zero state"
 
 
+# ---- initial state (extension: the walkthrough's state always starts at 0;
+# a given state before step 0 lets a sequence run in pieces).
+
+def pin_initial_state_closed_form(scan):
+    """Constant delta, A, B, u from a given state h0: each state is
+    h_t = a^t h0 + beta (1 - a^t) / (1 - a) (t = 1..L steps taken)."""
+    rng = np.random.default_rng(23)
+    Bt, Dm, L, N = 2, 3, 30, 4
+    raw = rng.uniform(-1.5, 0.5, size=(Bt, Dm))
+    uc = rng.standard_normal((Bt, Dm))
+    A = -0.15 * (np.arange(1, N + 1)[None, :] * rng.uniform(0.5, 1.5, size=(Dm, 1)))
+    Bc = rng.standard_normal((Bt, N))
+    C = rng.standard_normal((Bt, N, L))
+    Dv = rng.standard_normal(Dm)
+    h0 = rng.standard_normal((Bt, Dm, N)) * 3.0
+    delta = np.repeat(raw[:, :, None], L, axis=2)
+    u = np.repeat(uc[:, :, None], L, axis=2)
+    Bm = np.repeat(Bc[:, :, None], L, axis=2)
+    y, last = scan(u, delta, A, Bm, C, D=Dv, delta_softplus=True, return_last_state=True,
+                   initial_state=h0)
+    dl = _softplus_ref(raw)
+    t = np.arange(1, L + 1)
+    want = np.empty((Bt, Dm, L))
+    want_last = np.empty((Bt, Dm, N))
+    for b in range(Bt):
+        for d in range(Dm):
+            a = np.exp(dl[b, d] * A[d])
+            beta = dl[b, d] * Bc[b] * uc[b, d]
+            at = a[:, None] ** t[None, :]
+            h = at * h0[b, d][:, None] + beta[:, None] * (1 - at) / (1 - a[:, None])
+            want[b, d] = (C[b] * h).sum(0) + Dv[d] * uc[b, d]
+            want_last[b, d] = h[:, -1]
+    _assert_close(y, want, 1e-11, "closed form from h0: y")
+    _assert_close(last, want_last, 1e-11, "closed form from h0: last state")
+
+
+def pin_initial_state_brute_force(scan):
+    """Tiny random problems from a given state against the unrolled sum plus
+    the decayed initial state, prod_{r <= t} a[r, n] * h0[n]."""
+    rng = np.random.default_rng(29)
+    Bt, Dm, L, N = 2, 3, 6, 4
+    u = _rand(rng, Bt, Dm, L)
+    delta = _rand(rng, Bt, Dm, L)
+    A = -rng.uniform(0.2, 2.0, size=(Dm, N))
+    Bm = _rand(rng, Bt, N, L)
+    C = _rand(rng, Bt, N, L)
+    h0 = _rand(rng, Bt, Dm, N)
+    z = _rand(rng, Bt, Dm, L)
+    y, last = scan(u, delta, A, Bm, C, z=z, delta_softplus=True, return_last_state=True,
+                   initial_state=h0)
+    y0, last0 = brute_force(u, delta, A, Bm, C, None, None, None, True)
+    dl = _softplus_ref(delta)
+    for b in range(Bt):
+        for d in range(Dm):
+            for n in range(N):
+                decay = 1.0
+                for t in range(L):
+                    decay *= math.exp(dl[b, d, t] * A[d, n])
+                    y0[b, d, t] += C[b, n, t] * decay * h0[b, d, n]
+                last0[b, d, n] += decay * h0[b, d, n]
+    _assert_close(y, y0 * _silu_ref(z), 1e-12, "brute force from h0: y")
+    _assert_close(last, last0, 1e-12, "brute force from h0: last state")
+
+
+def pin_initial_state_continuity(scan):
+    """Running steps [0, k) and then [k, L) from the state the first piece
+    left equals running [0, L) in one piece, y and last state."""
+    rng = np.random.default_rng(31)
+    Bt, Dm, L, N = 2, 3, 50, 5
+    u = _rand(rng, Bt, Dm, L)
+    delta = _rand(rng, Bt, Dm, L)
+    A = -rng.uniform(0.05, 1.0, size=(Dm, N))
+    Bm = _rand(rng, Bt, N, L)
+    C = _rand(rng, Bt, N, L)
+    Dv = _rand(rng, Dm)
+    z = _rand(rng, Bt, Dm, L)
+    bias = _rand(rng, Dm) * 0.3
+    kw = dict(D=Dv, delta_bias=bias, delta_softplus=True, return_last_state=True)
+    y, last = scan(u, delta, A, Bm, C, z=z, **kw)
+    for k in (1, 17, 49):
+        y1, h1 = scan(u[..., :k], delta[..., :k], A, Bm[..., :k], C[..., :k], z=z[..., :k], **kw)
+        y2, h2 = scan(u[..., k:], delta[..., k:], A, Bm[..., k:], C[..., k:], z=z[..., k:],
+                      initial_state=h1, **kw)
+        _assert_close(np.concatenate([y1, y2], axis=-1), y, 1e-13, f"pieces at {k}: y")
+        _assert_close(h2, last, 1e-13, f"pieces at {k}: last state")
+
+
 ALL_PINS = [pin_hand_worked, pin_delta_transform, pin_closed_form, pin_brute_force,
             pin_lfilter, pin_delta_to_zero, pin_causality, pin_linearity,
-            pin_state_separability, pin_last_state]
+            pin_state_separability, pin_last_state, pin_initial_state_closed_form,
+            pin_initial_state_brute_force, pin_initial_state_continuity]

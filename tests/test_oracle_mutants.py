@@ -30,6 +30,9 @@ MUTANTS = {
     "silu_sign": ("z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
     "last_state_wrong_index": ("last_state[row * dstate + n] = h[n];",
                                "last_state[row * dstate + n] = h[0];"),
+    "initial_state_ignored": ("h[n] = initial_state ? initial_state[row * dstate + n] : 0.0;",
+                              "h[n] = 0.0;"),
+    "initial_state_transposed": ("initial_state[row * dstate + n]", "initial_state[n * dim * batch + row]"),
 }
 
 
