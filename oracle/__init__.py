@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for the selective-scan forward (TEST INFRASTRUCTURE).
+"""fp64 CPU oracle for the selective-scan forward and its gradients (TEST
+INFRASTRUCTURE).
 
 Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
 baseline leg may import this package.  The product path (the CUDA library and
@@ -31,6 +32,10 @@ def _load(path=None):
         lib.ss_oracle_fwd_init.restype = ctypes.c_int
         lib.ss_oracle_fwd_init.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P, P,
                                            ctypes.c_int, P, P, P, ctypes.c_int]
+        if hasattr(lib, "ss_oracle_bwd"):  # (a planted-mistake build of the forward alone has none)
+            lib.ss_oracle_bwd.restype = ctypes.c_int
+            lib.ss_oracle_bwd.argtypes = [i64, i64, i64, i64] + [P] * 8 + [ctypes.c_int] + [P] * 9 + \
+                [ctypes.c_int]
         lib.ss_oracle_threads.restype = ctypes.c_int
         lib.ss_oracle_threads.argtypes = []
         _libs[path] = lib
@@ -100,6 +105,35 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise RuntimeError("oracle rejected its arguments")
     return (y, last) if return_last_state else y
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                       delta_softplus=False, nthreads=0, lib=None):
+    """Gradients of sum(dy * y) for the forward of ``selective_scan`` (state
+    starting at zero), in float64, as a dict: du, ddelta, dz (batch, dim, L);
+    dA (dim, N); dB, dC (batch, N, L); dD, ddelta_bias (dim,).  The entries
+    of absent optional operands are None."""
+    u, delta, A, B, C, dy = (_f64(t) for t in (u, delta, A, B, C, dy))
+    D, z, delta_bias = _f64(D), _f64(z), _f64(delta_bias)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    if delta.shape != u.shape or dy.shape != u.shape:
+        raise ValueError("u, delta and dy must have the same shape")
+    if A.shape != (dim, N) or B.shape != (batch, N, L) or C.shape != (batch, N, L):
+        raise ValueError("bad A/B/C shape")
+    g = {"du": np.zeros_like(u), "ddelta": np.zeros_like(u), "dA": np.zeros((dim, N)),
+         "dB": np.zeros((batch, N, L)), "dC": np.zeros((batch, N, L)),
+         "dD": np.zeros(dim) if D is not None else None,
+         "dz": np.zeros_like(u) if z is not None else None,
+         "ddelta_bias": np.zeros(dim) if delta_bias is not None else None}
+    rc = _load(lib).ss_oracle_bwd(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                  _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0,
+                                  _ptr(dy), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]),
+                                  _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]),
+                                  _ptr(g["ddelta_bias"]), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle rejected its arguments")
+    return g
 
 
 def selective_scan_rows(inputs, rows, nthreads=0):

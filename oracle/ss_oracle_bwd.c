@@ -1,0 +1,165 @@
+/*
+ * Selective-scan backward: plain fp64 CPU oracle of the gradients.
+ *
+ * TEST INFRASTRUCTURE ONLY, like ss_oracle.c: only the test suite and the
+ * benchmark's CPU legs load it; it shares no code with the CUDA library.
+ *
+ * The forward it differentiates is the one of ss_oracle.c (the
+ * selective_scan_ref walkthrough, "Mamba代码实战：手把手教你用PyTorch复现选择性扫描核心逻辑
+ * （附避坑指南）", §2.2-§3.3, state starting at zero):
+ *   x_l = delta_l + bias,  d_l = softplus(x_l) (or exp(x_l)),
+ *   a_ln = exp(d_l A_n),   h_ln = a_ln h_(l-1)n + d_l B_nl u_l,
+ *   s_l = sum_n C_nl h_ln + D u_l,   y_l = s_l silu(z_l)  (y_l = s_l without z).
+ * The walkthrough trains it through autograd (§6 mentions the gradient only
+ * in passing); the gradients here are the chain rule of that loop, written
+ * out.  With g_l = dL/ds_l = dy_l silu(z_l) and the adjoint state
+ *   lam_ln = dL/dh_ln = g_l C_nl + a_(l+1)n lam_(l+1)n   (lam past the end = 0),
+ * per row (b, d):
+ *   dz_l     = dy_l s_l silu'(z_l),  silu'(z) = sig(z) (1 + z (1 - sig(z)))
+ *   dD      += g_l u_l
+ *   dC_nl   += g_l h_ln                         (summed over the rows d of batch b)
+ *   dB_nl   += lam_ln d_l u_l                   (summed over d)
+ *   du_l     = g_l D + sum_n lam_ln d_l B_nl
+ *   dd_l     = sum_n lam_ln (B_nl u_l + h_(l-1)n a_ln A_n)
+ *   dA_n    += sum_l lam_ln h_(l-1)n a_ln d_l   (summed over b and l)
+ *   ddelta_l = dd_l softplus'(x_l) = dd_l sig(x_l)  (1 above torch's threshold 20;
+ *              dd_l d_l in exp mode),   dbias += ddelta_l (summed over b and l).
+ * Sums over rows are done in a fixed order, so results do not depend on the
+ * thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* Returns 0 on success, -1 on a bad argument or allocation failure.
+ * Required: u, delta, A, B, C, dy, du, ddelta, dA, dB, dC.  dD is required
+ * when D is given, dz when z is, ddelta_bias when delta_bias is. */
+int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                  const double *u, const double *delta, const double *A,
+                  const double *B, const double *C, const double *D,
+                  const double *z, const double *delta_bias, int delta_softplus,
+                  const double *dy, double *du, double *ddelta, double *dA,
+                  double *dB, double *dC, double *dD, double *dz,
+                  double *ddelta_bias, int nthreads)
+{
+    if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1)
+        return -1;
+    if (!A || !dA || (batch * dim > 0 && seqlen > 0 &&
+                      (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)))
+        return -1;
+    if ((D && !dD) || (z && !dz) || (delta_bias && !ddelta_bias))
+        return -1;
+    const int64_t N = dstate, L = seqlen;
+    /* per-row partial sums over l, reduced over b afterwards in order */
+    double *pA = calloc((size_t)(batch * dim * N + 1), sizeof(double));
+    double *pD = calloc((size_t)(batch * dim + 1), sizeof(double));
+    double *pbias = calloc((size_t)(batch * dim + 1), sizeof(double));
+    if (!pA || !pD || !pbias) {
+        free(pA), free(pD), free(pbias);
+        return -1;
+    }
+    if (batch > 0 && L > 0) {
+        memset(dB, 0, sizeof(double) * (size_t)(batch * N * L));
+        memset(dC, 0, sizeof(double) * (size_t)(batch * N * L));
+    }
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : bad)
+#endif
+    for (int64_t b = 0; b < batch; ++b) {
+        double *h = malloc(sizeof(double) * (size_t)((L + 1) * N)); /* h[(l+1)N + n]: after step l */
+        double *dl = malloc(sizeof(double) * (size_t)(L + 1));
+        double *xs = malloc(sizeof(double) * (size_t)(L + 1));
+        double *s = malloc(sizeof(double) * (size_t)(L + 1));
+        double *carry = malloc(sizeof(double) * (size_t)N);
+        if (!h || !dl || !xs || !s || !carry) {
+            bad |= 1;
+            free(h), free(dl), free(xs), free(s), free(carry);
+            continue;
+        }
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            /* forward, keeping every state */
+            for (int64_t n = 0; n < N; ++n)
+                h[n] = 0.0;
+            for (int64_t l = 0; l < L; ++l) {
+                const int64_t idx = row * L + l;
+                double x = delta[idx];
+                if (delta_bias)
+                    x += delta_bias[d];
+                xs[l] = x;
+                dl[l] = delta_softplus ? (x > 20.0 ? x : log1p(exp(x))) : exp(x);
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const int64_t bn = (b * N + n) * L + l;
+                    const double a = exp(dl[l] * A[d * N + n]);
+                    h[(l + 1) * N + n] = a * h[l * N + n] + dl[l] * B[bn] * u[idx];
+                    acc += C[bn] * h[(l + 1) * N + n];
+                }
+                if (D)
+                    acc += D[d] * u[idx];
+                s[l] = acc;
+            }
+            /* reverse sweep with the adjoint state */
+            for (int64_t n = 0; n < N; ++n)
+                carry[n] = 0.0; /* a_(l+1) lam_(l+1), zero past the end */
+            for (int64_t l = L - 1; l >= 0; --l) {
+                const int64_t idx = row * L + l;
+                double g = dy[idx];
+                if (z) {
+                    const double sg = sigmoid(z[idx]);
+                    dz[idx] = dy[idx] * s[l] * sg * (1.0 + z[idx] * (1.0 - sg));
+                    g = dy[idx] * z[idx] * sg;
+                }
+                double dui = D ? g * D[d] : 0.0;
+                if (D)
+                    pD[row] += g * u[idx];
+                double ddl = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const int64_t bn = (b * N + n) * L + l;
+                    const double a = exp(dl[l] * A[d * N + n]);
+                    const double lam = g * C[bn] + carry[n];
+                    dC[bn] += g * h[(l + 1) * N + n];
+                    dB[bn] += lam * dl[l] * u[idx];
+                    dui += lam * dl[l] * B[bn];
+                    const double da = lam * h[l * N + n];
+                    ddl += lam * B[bn] * u[idx] + da * a * A[d * N + n];
+                    pA[row * N + n] += da * a * dl[l];
+                    carry[n] = a * lam;
+                }
+                du[idx] = dui;
+                const double dx = delta_softplus ? ddl * (xs[l] > 20.0 ? 1.0 : sigmoid(xs[l]))
+                                                 : ddl * dl[l];
+                ddelta[idx] = dx;
+                pbias[row] += dx;
+            }
+        }
+        free(h), free(dl), free(xs), free(s), free(carry);
+    }
+    for (int64_t d = 0; d < dim; ++d) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < batch; ++b)
+                acc += pA[(b * dim + d) * N + n];
+            dA[d * N + n] = acc;
+        }
+        double accD = 0.0, accb = 0.0;
+        for (int64_t b = 0; b < batch; ++b)
+            accD += pD[b * dim + d], accb += pbias[b * dim + d];
+        if (D)
+            dD[d] = accD;
+        if (delta_bias)
+            ddelta_bias[d] = accb;
+    }
+    free(pA), free(pD), free(pbias);
+    return bad ? -1 : 0;
+}

@@ -1,0 +1,97 @@
+"""Pins for the fp64 backward oracle (gradients of sum(dy * y)).
+
+Each ``pin_*`` takes ``grad`` (a callable with the signature of
+``oracle.selective_scan_bwd``) and ``scan`` (the forward oracle, pinned on its
+own in ``pins.py``) and raises AssertionError on a disagreement.  The
+reference for every gradient is a central finite difference of the forward:
+(F(x + eps v) - F(x - eps v)) / (2 eps) with F = sum(dy * y), which involves
+no gradient formula at all.
+"""
+import numpy as np
+
+NAMES = [("u", "du"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"), ("D", "dD"),
+         ("z", "dz"), ("delta_bias", "ddelta_bias")]
+
+
+def _problem(rng, Bt, Dm, L, N, with_D=True, with_z=True, with_bias=True, bias_shift=0.0):
+    p = {"u": rng.standard_normal((Bt, Dm, L)), "delta": rng.standard_normal((Bt, Dm, L)),
+         "A": -rng.uniform(0.2, 2.0, size=(Dm, N)), "B": rng.standard_normal((Bt, N, L)),
+         "C": rng.standard_normal((Bt, N, L)),
+         "D": rng.standard_normal(Dm) if with_D else None,
+         "z": rng.standard_normal((Bt, Dm, L)) if with_z else None,
+         "delta_bias": (rng.standard_normal(Dm) * 0.3 + bias_shift) if with_bias else None}
+    return p
+
+
+def _F(scan, p, dy, sp):
+    y = scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+             delta_bias=p["delta_bias"], delta_softplus=sp)
+    return float((np.asarray(y) * dy).sum())
+
+
+def _grads(grad, p, dy, sp):
+    return grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+                delta_bias=p["delta_bias"], delta_softplus=sp)
+
+
+def _fd_dir(scan, p, dy, sp, name, v, eps=1e-6):
+    hi = dict(p, **{name: p[name] + eps * v})
+    lo = dict(p, **{name: p[name] - eps * v})
+    return (_F(scan, hi, dy, sp) - _F(scan, lo, dy, sp)) / (2 * eps)
+
+
+def pin_bwd_directional(grad, scan):
+    """<gradient, v> against the central difference along a random v, for
+    every input, softplus and exp modes, every optional operand on and off."""
+    rng = np.random.default_rng(41)
+    for case, (sp, wD, wz, wb) in enumerate([(True, True, True, True), (False, True, False, True),
+                                             (True, False, True, False), (False, False, False, False)]):
+        p = _problem(rng, 2, 3, 9, 4, wD, wz, wb)
+        dy = rng.standard_normal((2, 3, 9))
+        g = _grads(grad, p, dy, sp)
+        for name, gname in NAMES:
+            if p[name] is None:
+                assert g[gname] is None, f"{gname} given for an absent operand"
+                continue
+            v = rng.standard_normal(p[name].shape)
+            fd = _fd_dir(scan, p, dy, sp, name, v)
+            an = float((g[gname] * v).sum())
+            assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), \
+                f"case {case} d/d{name}: analytic {an!r} vs finite difference {fd!r}"
+
+
+def pin_bwd_every_element(grad, scan):
+    """Every element of every gradient of a tiny problem against its own
+    central difference (unit directions)."""
+    rng = np.random.default_rng(43)
+    p = _problem(rng, 2, 2, 5, 3)
+    dy = rng.standard_normal((2, 2, 5))
+    for sp in (True, False):
+        g = _grads(grad, p, dy, sp)
+        for name, gname in NAMES:
+            arr = p[name]
+            for idx in np.ndindex(arr.shape):
+                v = np.zeros_like(arr)
+                v[idx] = 1.0
+                fd = _fd_dir(scan, p, dy, sp, name, v)
+                an = float(g[gname][idx])
+                assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), \
+                    f"{gname}{idx} (softplus={sp}): analytic {an!r} vs finite difference {fd!r}"
+
+
+def pin_bwd_softplus_linear_region(grad, scan):
+    """delta + bias above torch's softplus threshold (20), where softplus is
+    the identity and its derivative is 1."""
+    rng = np.random.default_rng(47)
+    p = _problem(rng, 1, 2, 6, 3, bias_shift=25.0)
+    p["A"] = p["A"] * 0.01  # keep exp(delta' A) away from underflow
+    dy = rng.standard_normal((1, 2, 6))
+    g = _grads(grad, p, dy, True)
+    for name, gname in [("delta", "ddelta"), ("delta_bias", "ddelta_bias")]:
+        v = rng.standard_normal(p[name].shape)
+        fd = _fd_dir(scan, p, dy, True, name, v)
+        an = float((g[gname] * v).sum())
+        assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), f"d/d{name} above the threshold: {an!r} vs {fd!r}"
+
+
+ALL_PINS = [pin_bwd_directional, pin_bwd_every_element, pin_bwd_softplus_linear_region]
