@@ -32,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from selective_state_space_41_b200 import selscan, workloads as W  # noqa: E402
+from selective_state_space_41_b200 import gen, selscan, workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = W.MAMBA130M
 METRIC = "selective-scan state-updates/s (B·D·L·N) & HBM GB/s vs roofline, 1×B200"
@@ -377,12 +377,58 @@ def bench_ours(args, w, world, rank, local):
         "kernel_ms": {"min": min(kernel_ms), "median": statistics.median(kernel_ms),
                       "max": max(kernel_ms)},
     }
+    if not args.no_bwd and w.dstate <= 32:
+        line["backward"] = bench_backward(args, wr, d, host, out_dtype, flush, stream, sfu_peak, world)
     del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_sample(w, host)
         line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     return line if rank == 0 else None
+
+
+def bench_backward(args, w, d, host, out_dtype, flush, stream, sfu_peak, world):
+    """Device time of ss_bwd (all gradients of sum(dy * y)) on the same inputs:
+    a forward-state pass plus the adjoint pass recomputing the states, about
+    two exps per state update (a seeded synthetic dy)."""
+    dev = d["u"].device
+    dy = gen.fill(tuple(host["u"].shape), out_dtype, w.seed, 9).to(dev)
+    grads = {"du": torch.empty_like(d["u"]), "ddelta": torch.empty_like(d["u"]),
+             "dA": torch.empty((w.dim, w.dstate), dtype=torch.float32, device=dev),
+             "dB": torch.empty((w.batch, w.dstate, w.seqlen), dtype=torch.float32, device=dev),
+             "dC": torch.empty((w.batch, w.dstate, w.seqlen), dtype=torch.float32, device=dev),
+             "dD": torch.empty(w.dim, dtype=torch.float32, device=dev) if d["D"] is not None else None,
+             "dz": torch.empty_like(d["u"]) if d["z"] is not None else None,
+             "ddelta_bias": (torch.empty(w.dim, dtype=torch.float32, device=dev)
+                             if d["delta_bias"] is not None else None)}
+    nws = selscan.ss_bwd_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, out_dtype)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+
+    def launch():
+        selscan.ss_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], dy, grads, D=d["D"], z=d["z"],
+                       delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, workspace=ws,
+                       stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        launch()
+    steps = max(3, min(args.steps, 30))
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        launch()
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = max_over_ranks(statistics.median(ts), world)
+    del ws
+    return {"ms_per_step": ms, "value": w.updates * world / (ms * 1e-3), "unit": "updates/s",
+            "steps": steps, "workspace_bytes": nws, "gpu_launches_per_step": 3,
+            "ex2_per_update": 2, "sfu_frac": 2 * w.updates / sfu_peak / (ms * 1e-3),
+            "note": "forward-state checkpoint pass + adjoint pass (recomputing the states) + "
+                    "fixed-order reductions; L2 flushed before each step"}
 
 
 def main(argv=None):
@@ -393,6 +439,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per launch of the scan kernel from an ncu capture")
     args = ap.parse_args(argv)

@@ -94,7 +94,8 @@ typedef struct {
  *   last_state    device, (B, D, N) float32, or NULL (= return_last_state off)
  *   stream        the stream the work is queued on
  * Every pointer must be aligned to its element size.  Sizes with B*D == 0 or
- * L == 0 are valid: with L == 0 the last state (if asked for) is all zeros.
+ * L == 0 are valid: with L == 0 the last state (if asked for) is all zeros
+ * (the initial state, for ss_fwd_state).
  * Arithmetic: float32 throughout (state, products and sums), whatever the
  * input dtype; results are bitwise reproducible run to run for a given
  * device, shape and pointer alignment.
@@ -164,6 +165,24 @@ ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *del
                              void *workspace, size_t workspace_bytes, ss_stream_t stream);
 
 /*
+ * As ss_fwd_with_config (config NULL: the heuristic's shape, as ss_fwd_ws),
+ * starting from a given state instead of zero.  The walkthrough's state
+ * always starts at zero (§3.2); this extension lets a sequence run in pieces,
+ * each piece starting from the last state of the one before, down to single
+ * steps (L = 1) for recurrent decoding:
+ *   initial_state  device, (B, D, N) float32: the state before step 0, or
+ *                  NULL for zero.  It may be the same buffer as last_state
+ *                  (the state is then updated in place); it may not overlap
+ *                  any other argument.
+ * Other arguments and errors as ss_fwd_with_config.
+ */
+ss_status ss_fwd_state(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const float *initial_state,
+                       void *y, float *last_state, const ss_launch_config *config, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream);
+
+/*
  * The launch shape ss_fwd_ws would use for `desc` with `workspace_bytes` of
  * workspace (0: as ss_fwd).  Returns SS_OK, or the status ss_fwd would return
  * for a bad descriptor.
@@ -222,6 +241,32 @@ ss_status ss_fwd_noalloc(const ss_desc *desc, const void *u, const void *delta, 
                          const void *B, const void *C, const float *D, const void *z,
                          const float *delta_bias, int delta_softplus, void *y, float *last_state,
                          ss_stream_t stream);
+
+/*
+ * Backward of ss_fwd (state starting at zero): the gradients of sum(dy * y)
+ * with respect to every input.  The walkthrough trains the forward through
+ * autograd (§6); this is its chain rule written out (an adjoint state run
+ * backwards over the steps from checkpoints of the forward state).
+ *   dy                 device, (B, D, L) out_dtype: the gradient of y
+ *   du, ddelta, dz     device, (B, D, L) in_dtype; dz required exactly when z is given
+ *   dA                 device, (D, N) float32
+ *   dB, dC             device, (B, N, L) float32
+ *   dD, ddelta_bias    device, (D,) float32, required exactly when D / delta_bias are given
+ *   workspace          device, 256-byte aligned, ss_bwd_workspace_bytes(desc)
+ *                      bytes (forward-state checkpoints every 8 steps and
+ *                      partial sums); scratch, not shared by overlapping calls
+ * Other arguments as ss_fwd.  N must be at most 32 (SS_ERR_UNSUPPORTED_DSTATE
+ * otherwise).  Sums over rows (dA, dB, dC, dD, ddelta_bias) are taken in a
+ * fixed order: results are bitwise reproducible.
+ */
+ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                 const void *C, const float *D, const void *z, const float *delta_bias,
+                 int delta_softplus, const void *dy, void *du, void *ddelta, float *dA, float *dB,
+                 float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
+                 size_t workspace_bytes, ss_stream_t stream);
+
+/* Bytes of workspace ss_bwd needs for `desc` (0 for an invalid descriptor or N > 32). */
+size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 
 /* Static description of a status code (never NULL). */
 const char *ss_status_string(ss_status status);

@@ -8,11 +8,12 @@ kernels behind a C ABI (``include/selscan.h``), with a thin Python binding.
 ``workloads`` and ``gen`` hold the synthetic workloads and their seeded input
 generator.
 """
-from .selscan import (SS_BF16, SS_F32, SelscanError, lib, selective_scan_fwd, ss_fwd,  # noqa: F401
+from .selscan import (SS_BF16, SS_F32, SelscanError, lib, selective_scan_bwd, selective_scan_fwd,  # noqa: F401
+                      ss_bwd, ss_bwd_workspace_bytes, ss_fwd,
                       ss_fwd_heuristic, ss_fwd_hostio, ss_fwd_noalloc, ss_fwd_workspace_bytes,
                       ss_status_string,
                       ss_version, workspace_for)
 
-__all__ = ["selective_scan_fwd", "ss_fwd", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc",
+__all__ = ["selective_scan_fwd", "selective_scan_bwd", "ss_bwd", "ss_bwd_workspace_bytes", "ss_fwd", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc",
            "ss_fwd_workspace_bytes", "workspace_for", "ss_status_string", "ss_version",
            "SelscanError", "SS_F32", "SS_BF16", "lib"]

@@ -29,6 +29,7 @@ NVCC_FLAGS = [
 DTYPE_PAIRS = [("float", "float", "f32_f32"), ("__nv_bfloat16", "__nv_bfloat16", "bf16_bf16"),
                ("__nv_bfloat16", "float", "bf16_f32")]
 STATE_BUCKETS = [4, 8, 16, 32, 64]
+BWD_STATE_BUCKETS = [4, 8, 16, 32]  # the backward holds 4 states per lane, at most 8 lanes per row
 
 
 def _nvcc() -> str:
@@ -40,7 +41,7 @@ def _nvcc() -> str:
 
 def _sources():
     return (glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-            glob.glob(os.path.join(INCLUDE, "*.h")))
+            glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def _compile_jobs(verbose: bool):
@@ -51,6 +52,13 @@ def _compile_jobs(verbose: bool):
                      os.path.join(BUILD_DIR, "selscan.o")], "selscan"),
             (base + [os.path.join(CSRC, "ss_noalloc.cu"), "-o",
                      os.path.join(BUILD_DIR, "ss_noalloc.o")], "ss_noalloc")]
+    for tin, tout, tag in DTYPE_PAIRS:
+        for n in BWD_STATE_BUCKETS:
+            name = f"bwd_{tag}_n{n}"
+            jobs.append((base + [f"-DSS_INST_TIN={tin}", f"-DSS_INST_TOUT={tout}",
+                                 f"-DSS_INST_NMAX={n}", f"-DSS_INST_NAME={name}",
+                                 os.path.join(CSRC, "ss_bwd_inst.cu"), "-o",
+                                 os.path.join(BUILD_DIR, name + ".o")], name))
     for tin, tout, tag in DTYPE_PAIRS:
         for n in STATE_BUCKETS:
             name = f"launch_{tag}_n{n}"

@@ -13,6 +13,7 @@
 #include <cstdint>
 
 #include "selscan.h"
+#include "ss_bwd_launch.h"
 #include "ss_launch.h"
 
 namespace {
@@ -223,9 +224,9 @@ cudaError_t launch_fixup(const ss_desc *desc, int64_t rows, int nseg, cudaStream
 
 ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D, const void *z,
-                   const float *delta_bias, int delta_softplus, void *y, float *last_state,
-                   const ss_launch_config *cfg, void *workspace, size_t workspace_bytes,
-                   ss_stream_t stream) {
+                   const float *delta_bias, int delta_softplus, const float *initial_state,
+                   void *y, float *last_state, const ss_launch_config *cfg, void *workspace,
+                   size_t workspace_bytes, ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
@@ -239,6 +240,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     if (need_seq && (!u || !delta || !B || !C || !y)) return SS_ERR_NULL_POINTER;
     if (!need_seq && !last_state) return SS_OK;  // nothing to write
     if (!need_seq) pl.nseg = 1, pl.seg_len = 0;
+    if (initial_state && !aligned(initial_state, 4)) return SS_ERR_MISALIGNED;
 
     const size_t ein = dtype_size(desc->in_dtype), eout = dtype_size(desc->out_dtype);
     const void *in_ptrs[] = {u, delta, B, C, z};
@@ -275,6 +277,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.delta_bias = delta_bias;
     p.y = y;
     p.last_state = last_state;
+    p.init_state = initial_state;
     p.batch = desc->batch;
     p.dim = desc->dim;
     p.seqlen = desc->seqlen;
@@ -301,6 +304,38 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     return err == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- backward
+constexpr int kBwdWarps = 4;
+
+struct BwdLayout {
+    int lanes, rows;        // lanes per row, rows per block
+    int64_t dtiles, nsub;
+    size_t off_ckpt, off_dbc, off_dA, off_dD, off_dbias, total;  // workspace byte offsets
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz) {
+    BwdLayout lo{};
+    const int nmax = selscan::state_bucket((int)desc->dstate);
+    lo.lanes = selscan::bwd_lanes(nmax);
+    lo.rows = kBwdWarps * 32 / lo.lanes;
+    lo.dtiles = (desc->dim + lo.rows - 1) / lo.rows;
+    lo.nsub = (desc->seqlen + selscan::kBwdSub - 1) / selscan::kBwdSub;
+    const size_t N = (size_t)desc->dstate, rows = (size_t)sz.rows, L = (size_t)desc->seqlen;
+    lo.off_ckpt = 0;
+    lo.off_dbc = align256(lo.off_ckpt + rows * (size_t)lo.nsub * N * 4);
+    lo.off_dA = align256(lo.off_dbc + (size_t)lo.dtiles * (size_t)desc->batch * 2 * N * L * 4);
+    lo.off_dD = align256(lo.off_dA + rows * N * 4);
+    lo.off_dbias = align256(lo.off_dD + rows * 4);
+    lo.total = align256(lo.off_dbias + rows * 4);
+    return lo;
+}
+
+#define SS_PICK_BWD(PREFIX)                                                                  \
+    n <= 4 ? selscan::PREFIX##_n4 : n <= 8 ? selscan::PREFIX##_n8 : n <= 16 ? selscan::PREFIX##_n16 \
+                                                                  : selscan::PREFIX##_n32
+
 }  // namespace
 
 extern "C" {
@@ -309,16 +344,16 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  const void *B, const void *C, const float *D, const void *z,
                  const float *delta_bias, int delta_softplus, void *y, float *last_state,
                  ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, nullptr,
-                    nullptr, 0, stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    nullptr, nullptr, 0, stream);
 }
 
 ss_status ss_fwd_ws(const ss_desc *desc, const void *u, const void *delta, const float *A,
                     const void *B, const void *C, const float *D, const void *z,
                     const float *delta_bias, int delta_softplus, void *y, float *last_state,
                     void *workspace, size_t workspace_bytes, ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, nullptr,
-                    workspace, workspace_bytes, stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    nullptr, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
@@ -327,8 +362,17 @@ ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *del
                              void *y, float *last_state, const ss_launch_config *config,
                              void *workspace, size_t workspace_bytes, ss_stream_t stream) {
     if (!config) return SS_ERR_NULL_POINTER;
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, config,
-                    workspace, workspace_bytes, stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    config, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_fwd_state(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const float *initial_state,
+                       void *y, float *last_state, const ss_launch_config *config, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream) {
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, y,
+                    last_state, config, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_fwd_heuristic(const ss_desc *desc, size_t workspace_bytes, ss_launch_config *config) {
@@ -389,12 +433,88 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
     for (const Copy &c : in_copies)
         if (c.dst && c.bytes && cudaMemcpyAsync(c.dst, c.src, c.bytes, h2d, s) != cudaSuccess)
             return SS_ERR_CUDA;
-    st = fwd_impl(desc, d_u, d_delta, d_A, d_B, d_C, d_D, d_z, d_delta_bias, delta_softplus, d_y,
-                  d_last_state, nullptr, d_workspace, workspace_bytes, stream);
+    st = fwd_impl(desc, d_u, d_delta, d_A, d_B, d_C, d_D, d_z, d_delta_bias, delta_softplus, nullptr,
+                  d_y, d_last_state, nullptr, d_workspace, workspace_bytes, stream);
     if (st != SS_OK) return st;
     if (n_y && cudaMemcpyAsync(h_y, d_y, n_y, d2h, s) != cudaSuccess) return SS_ERR_CUDA;
     if (d_last_state && cudaMemcpyAsync(h_last_state, d_last_state, n_last, d2h, s) != cudaSuccess)
         return SS_ERR_CUDA;
+    return SS_OK;
+}
+
+size_t ss_bwd_workspace_bytes(const ss_desc *desc) {
+    Sizes sz;
+    if (check_desc(desc, &sz) != SS_OK || desc->dstate > 32) return 0;
+    return bwd_layout(desc, sz).total;
+}
+
+ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                 const void *C, const float *D, const void *z, const float *delta_bias,
+                 int delta_softplus, const void *dy, void *du, void *ddelta, float *dA, float *dB,
+                 float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
+                 size_t workspace_bytes, ss_stream_t stream) {
+    Sizes sz;
+    ss_status st = check_desc(desc, &sz);
+    if (st != SS_OK) return st;
+    if (desc->dstate > 32) return SS_ERR_UNSUPPORTED_DSTATE;
+    if (!A || !dA) return SS_ERR_NULL_POINTER;
+    const bool work = sz.rows > 0 && desc->seqlen > 0;
+    if (work && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)) return SS_ERR_NULL_POINTER;
+    if ((D && !dD) || (z && !dz) || (delta_bias && !ddelta_bias)) return SS_ERR_NULL_POINTER;
+    const size_t ein = dtype_size(desc->in_dtype), eout = dtype_size(desc->out_dtype);
+    const void *in_ptrs[] = {u, delta, B, C, z, du, ddelta, dz};
+    for (const void *q : in_ptrs)
+        if (q && !aligned(q, ein)) return SS_ERR_MISALIGNED;
+    const void *f_ptrs[] = {A, D, delta_bias, dA, dB, dC, dD, ddelta_bias};
+    for (const void *q : f_ptrs)
+        if (q && !aligned(q, 4)) return SS_ERR_MISALIGNED;
+    if (dy && !aligned(dy, eout)) return SS_ERR_MISALIGNED;
+    const BwdLayout lo = bwd_layout(desc, sz);
+    if (!workspace || workspace_bytes < lo.total) return SS_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SS_ERR_MISALIGNED;
+    const int64_t blocks = lo.dtiles * desc->batch;
+    if (blocks > INT_MAX) return SS_ERR_BAD_SHAPE;
+
+    char *ws = static_cast<char *>(workspace);
+    selscan::BwdParams p;
+    p.u = u, p.delta = delta, p.B = B, p.C = C, p.z = z, p.dy = dy;
+    p.A = A, p.D = D, p.delta_bias = delta_bias;
+    p.du = du, p.ddelta = ddelta, p.dz = dz;
+    p.ckpt = reinterpret_cast<float *>(ws + lo.off_ckpt);
+    p.ws_dBC = reinterpret_cast<float *>(ws + lo.off_dbc);
+    p.ws_dA = reinterpret_cast<float *>(ws + lo.off_dA);
+    p.ws_dD = reinterpret_cast<float *>(ws + lo.off_dD);
+    p.ws_dbias = reinterpret_cast<float *>(ws + lo.off_dbias);
+    p.batch = desc->batch, p.dim = desc->dim, p.seqlen = desc->seqlen;
+    p.dstate = (int)desc->dstate;
+    p.softplus = delta_softplus ? 1 : 0;
+    p.vec = (desc->seqlen * (int64_t)ein) % 16 == 0 && (!B || aligned(B, 16)) && (!C || aligned(C, 16));
+    p.dtiles = lo.dtiles;
+    p.nsub = lo.nsub;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int nmax = selscan::state_bucket(p.dstate), n = nmax;
+    if (sz.rows > 0) {
+        const size_t smem = selscan::bwd_smem_bytes(ein, nmax, kBwdWarps);
+        cudaError_t (*fn)(dim3, dim3, size_t, cudaStream_t, const selscan::BwdParams &) =
+            desc->in_dtype == SS_F32 ? (SS_PICK_BWD(bwd_f32_f32))
+            : desc->out_dtype == SS_BF16 ? (SS_PICK_BWD(bwd_bf16_bf16))
+                                         : (SS_PICK_BWD(bwd_bf16_f32));
+        if (fn(dim3((unsigned)blocks), dim3(kBwdWarps * 32), smem, s, p) != cudaSuccess) return SS_ERR_CUDA;
+        const int64_t bc = desc->batch * 2 * desc->dstate * desc->seqlen;
+        if (bc > 0) {
+            const int64_t gb = (bc + 255) / 256;
+            selscan::ss_bwd_reduce_bc_kernel<<<(unsigned)(gb < 4 * 148 * 8 ? gb : 4 * 148 * 8), 256, 0, s>>>(p, dB, dC);
+            if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+        }
+    }
+    const int64_t rr = desc->dim * (desc->dstate + 2);
+    if (rr > 0) {
+        const int64_t gb = (rr + 255) / 256;
+        selscan::ss_bwd_reduce_rows_kernel<<<(unsigned)(gb < 4 * 148 ? gb : 4 * 148), 256, 0, s>>>(p, dA, dD,
+                                                                                                 ddelta_bias);
+        if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    }
     return SS_OK;
 }
 

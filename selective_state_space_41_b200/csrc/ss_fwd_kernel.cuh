@@ -45,13 +45,15 @@ struct FwdParams {
     const float *A, *D, *delta_bias;
     void *y;
     float *last_state;
+    const float *init_state;  // (batch, dim, dstate) state before step 0, or null (zero)
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;     // 1: softplus, 0: exp
     int vec;          // 1: every row of u/delta/z/B/C/y starts 16-byte aligned
     int64_t dtiles;   // row tiles per batch entry
     // Sequence segments (direct kernel only): nseg > 1 runs each segment of
-    // seg_len steps from a zero state and records, per (segment, row), the
+    // seg_len steps from a zero state (the first one from init_state, if
+    // given) and records, per (segment, row), the
     // end state (ws_hend, N floats) and the sum of delta' (ws_dsum) for the
     // fix-up kernel, which adds the carried state's share of y.
     int64_t seg_len;
@@ -380,14 +382,15 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
 #pragma unroll
         for (int n = 0; n < kNmax; ++n) {
             if constexpr (kA2InRegs) A2[n] = n < N ? A_d[n] * kLog2e : 0.f;
-            carry[n] = 0.f;
+            carry[n] = (p.init_state != nullptr && n < N) ? p.init_state[row * N + n] : 0.f;
         }
     } else {
         for (int idx = tid; idx < rows * kNmax; idx += nthreads) {
             const int r = idx / kNmax, n = idx % kNmax;
             const int64_t dr = d0 + r < p.dim ? d0 + r : p.dim - 1;
             sA2[r * kRowStride + n] = n < N ? p.A[dr * N + n] * kLog2e : 0.f;
-            sCarry[r * kRowStride + n] = 0.f;
+            sCarry[r * kRowStride + n] =
+                (p.init_state != nullptr && n < N) ? p.init_state[(b * p.dim + dr) * N + n] : 0.f;
         }
         // (visible after the first __syncthreads of the chunk loop, or the one
         // before the last-state store)
@@ -833,6 +836,10 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         if constexpr (kA2InRegs)
             A2[qq] = make_float2(n < N ? A_d[n] * kLog2e : 0.f, n + 1 < N ? A_d[n + 1] * kLog2e : 0.f);
         h[qq] = make_float2(0.f, 0.f);
+        if (p.init_state != nullptr && seg == 0) {  // the given state enters the first segment only
+            if (n < N) h[qq].x = p.init_state[row * N + n];
+            if (n + 1 < N) h[qq].y = p.init_state[row * N + n + 1];
+        }
     }
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;

@@ -7,8 +7,9 @@ current stream.  There is no fallback: if ``libselscan.so`` is missing or
 fails to load, every call raises.
 
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
-``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_heuristic``,
-``ss_fwd_hostio``, ``ss_fwd_noalloc``, ``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
+``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``, ``ss_fwd_heuristic``,
+``ss_fwd_hostio``, ``ss_fwd_noalloc``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
+``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
 to the workspace and config forms by keyword); ``selective_scan_fwd`` is the
 allocate-and-call convenience
 form with the argument order of the walkthrough's selective_scan_ref
@@ -32,8 +33,9 @@ STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL_POINTER", 2: "SS_ERR_BAD_SHAPE",
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Names the header declares; the ABI test checks each is exported.
-EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config",
-           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc", "ss_status_string", "ss_version")
+EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
+           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
+           "ss_status_string", "ss_version")
 
 
 class SelscanError(RuntimeError):
@@ -76,12 +78,18 @@ def lib():
         L.ss_fwd_workspace_bytes.argtypes = [DP, CP]
         L.ss_fwd_with_config.restype = I
         L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, CP, P, SZ, P]
+        L.ss_fwd_state.restype = I
+        L.ss_fwd_state.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P, CP, P, SZ, P]
         L.ss_fwd_heuristic.restype = I
         L.ss_fwd_heuristic.argtypes = [DP, SZ, CP]
         L.ss_fwd_hostio.restype = I
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
         L.ss_fwd_noalloc.restype = I
         L.ss_fwd_noalloc.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
+        L.ss_bwd.restype = I
+        L.ss_bwd.argtypes = [DP] + [P] * 8 + [I] + [P] * 9 + [P, SZ, P]
+        L.ss_bwd_workspace_bytes.restype = SZ
+        L.ss_bwd_workspace_bytes.argtypes = [DP]
         L.ss_status_string.restype = ctypes.c_char_p
         L.ss_status_string.argtypes = [I]
         L.ss_version.restype = I
@@ -135,14 +143,15 @@ def _config(lanes_per_row, split_states, warps_per_block, segments):
 
 def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
            last_state=None, stream=None, workspace=None, lanes_per_row=None, warps_per_block=None,
-           split_states=False, segments=None):
+           split_states=False, segments=None, initial_state=None):
     """Queue the forward on ``stream`` (default: the current stream).
 
     u, delta, z, y: (batch, dim, L); A: (dim, N) float32; B, C: (batch, N, L);
-    D, delta_bias: (dim,) float32; last_state: (batch, dim, N) float32.
-    ``workspace`` (a CUDA tensor, e.g. uint8 of ss_fwd_workspace_bytes())
-    selects ``ss_fwd_ws``; ``lanes_per_row`` / ``split_states`` /
-    ``warps_per_block`` / ``segments`` select ``ss_fwd_with_config``.
+    D, delta_bias: (dim,) float32; last_state, initial_state: (batch, dim, N)
+    float32.  ``workspace`` (a CUDA tensor, e.g. uint8 of
+    ss_fwd_workspace_bytes()) selects ``ss_fwd_ws``; ``lanes_per_row`` /
+    ``split_states`` / ``warps_per_block`` / ``segments`` select
+    ``ss_fwd_with_config``; ``initial_state`` selects ``ss_fwd_state``.
     Raises SelscanError on a rejected call.
     """
     u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
@@ -157,7 +166,13 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     s = _stream_handle(stream, u.device)
     cfg = _config(lanes_per_row, split_states, warps_per_block, segments)
-    if cfg is not None:
+    if initial_state is not None:
+        if not initial_state.is_contiguous():
+            raise ValueError("initial_state must be contiguous")
+        state_args = args[:10] + (_ptr(initial_state),) + args[10:]
+        _check(lib().ss_fwd_state(*state_args, ctypes.byref(cfg) if cfg is not None else None, ws,
+                                  ws_bytes, s), "ss_fwd_state")
+    elif cfg is not None:
         _check(lib().ss_fwd_with_config(*args, ctypes.byref(cfg), ws, ws_bytes, s),
                "ss_fwd_with_config")
     elif workspace is not None:
@@ -182,6 +197,51 @@ def ss_fwd_noalloc(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_
                                 _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0,
                                 _ptr(y), _ptr(last_state), _stream_handle(stream, u.device)),
            "ss_fwd_noalloc")
+
+
+def ss_bwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None) -> int:
+    desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
+    return int(lib().ss_bwd_workspace_bytes(ctypes.byref(desc)))
+
+
+def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_softplus=False,
+           workspace=None, stream=None):
+    """Queue the backward: ``grads`` maps du, ddelta, dA, dB, dC and (when the
+    operand is given) dD, dz, ddelta_bias to output tensors (du, ddelta, dz in
+    u's dtype; the others float32).  ``workspace``: a CUDA tensor of at least
+    ss_bwd_workspace_bytes() bytes (allocated here when None)."""
+    u, delta, A, B, C, dy, D, z, delta_bias = map(_contig, (u, delta, A, B, C, dy, D, z, delta_bias))
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    desc = make_desc(batch, dim, L, N, u.dtype, dy.dtype)
+    if workspace is None:
+        n = ss_bwd_workspace_bytes(batch, dim, L, N, u.dtype, dy.dtype)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=u.device)
+    g = lambda k: _ptr(grads.get(k))  # noqa: E731
+    _check(lib().ss_bwd(ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                        _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(dy), g("du"),
+                        g("ddelta"), g("dA"), g("dB"), g("dC"), g("dD"), g("dz"), g("ddelta_bias"),
+                        _ptr(workspace), workspace.numel() * workspace.element_size(),
+                        _stream_handle(stream, u.device)), "ss_bwd")
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=False,
+                       stream=None):
+    """Gradients of sum(dy * y) as a dict (see ss_bwd); allocates the outputs."""
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    dev = u.device
+    f32 = torch.float32
+    grads = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+             "dA": torch.empty((dim, N), dtype=f32, device=dev),
+             "dB": torch.empty((batch, N, L), dtype=f32, device=dev),
+             "dC": torch.empty((batch, N, L), dtype=f32, device=dev),
+             "dD": torch.empty(dim, dtype=f32, device=dev) if D is not None else None,
+             "dz": torch.empty_like(u) if z is not None else None,
+             "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None}
+    ss_bwd(u, delta, A, B, C, dy, grads, D=D, z=z, delta_bias=delta_bias,
+           delta_softplus=delta_softplus, stream=stream)
+    return grads
 
 
 def ss_fwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None,
@@ -232,12 +292,13 @@ def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None, work
 
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
-                       return_last_state=False, out_dtype=None, stream=None):
+                       return_last_state=False, out_dtype=None, stream=None, initial_state=None):
     """y (and the last state) of the selective scan, computed by libselscan.
 
-    Same arguments as the walkthrough's selective_scan_ref, plus the z gate.
-    Inputs must be CUDA tensors; y is allocated in ``out_dtype`` (default:
-    u's dtype), last_state in float32.
+    Same arguments as the walkthrough's selective_scan_ref, plus the z gate
+    and an optional float32 (batch, dim, N) state before step 0.  Inputs must
+    be CUDA tensors; y is allocated in ``out_dtype`` (default: u's dtype),
+    last_state in float32.
     """
     if not u.is_cuda:
         raise ValueError("selective_scan_fwd runs on CUDA tensors only")
@@ -248,5 +309,5 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
             if return_last_state else None)
     ws = workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=u.device)
     ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
-           last_state=last, stream=stream, workspace=ws)
+           last_state=last, stream=stream, workspace=ws, initial_state=initial_state)
     return (y, last) if return_last_state else y

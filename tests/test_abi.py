@@ -4,6 +4,7 @@ without a GPU: no pointer given here is ever dereferenced)."""
 import ctypes
 import os
 import re
+import types
 
 import pytest
 
@@ -125,6 +126,43 @@ def test_noalloc_rejections_before_any_launch(lib):
     assert lib.ss_fwd_workspace_bytes(ctypes.byref(big), None) > selscan.NOALLOC_SCRATCH_BYTES
     assert lib.ss_fwd_noalloc(ctypes.byref(big), *args) == 9
     assert "scratch" in selscan.ss_status_string(9)
+
+
+def test_state_entry_rejections(lib):
+    """ss_fwd_state: a misaligned initial state or a bad config is rejected
+    before any launch."""
+    d = _desc(seqlen=64, dstate=4)
+    head = (ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1)
+    assert lib.ss_fwd_state(*head, ODD, FAKE, None, None, None, 0, None) == 5
+    assert lib.ss_fwd_state(*head, FAKE, FAKE, None, _cfg(3, 0, 4), None, 0, None) == 7
+    assert lib.ss_fwd_state(None, *head[1:], FAKE, FAKE, None, None, None, 0, None) == 1
+
+
+def test_bwd_rejections(lib):
+    """ss_bwd rejects before any launch (the pointers are fake): no
+    descriptor, more than 32 states, a missing gradient output, no workspace.
+    Also goes through the binding's argument list once (its call is rejected
+    on the state count before any pointer is used)."""
+    P = FAKE
+    args = (P, P, P, P, P, None, None, None, 1, P, P, P, P, P, P, None, None, None)
+    assert lib.ss_bwd(None, *args, None, 0, None) == 1
+    assert lib.ss_bwd(ctypes.byref(_desc(dstate=33)), *args, None, 0, None) == 4
+    d = _desc(dstate=16)
+    missing = (P, P, P, P, P, None, None, None, 1, P, None, P, P, P, P, None, None, None)
+    assert lib.ss_bwd(ctypes.byref(d), *missing, None, 0, None) == 1
+    withD = (P, P, P, P, P, P, None, None, 1, P, P, P, P, P, P, None, None, None)   # D without dD
+    assert lib.ss_bwd(ctypes.byref(d), *withD, None, 0, None) == 1
+    assert lib.ss_bwd(ctypes.byref(d), *args, None, 0, None) == 8
+    assert lib.ss_bwd_workspace_bytes(ctypes.byref(d)) > 0
+    assert lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(dstate=64))) == 0
+    import torch
+    t = torch.zeros(1, 2, 4)
+    with pytest.raises(selscan.SelscanError) as e:
+        selscan.ss_bwd(t, t, torch.zeros(2, 64), torch.zeros(1, 64, 4), torch.zeros(1, 64, 4), t,
+                       {"du": t, "ddelta": t, "dA": t, "dB": t, "dC": t},
+                       workspace=torch.zeros(16, dtype=torch.uint8),
+                       stream=types.SimpleNamespace(cuda_stream=0))
+    assert e.value.status == 4
 
 
 def test_hostio_rejections(lib):

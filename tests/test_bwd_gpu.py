@@ -1,0 +1,112 @@
+"""Backward (ss_bwd) through the C ABI against the fp64 backward oracle,
+which finite differences of the pinned forward oracle pin.
+
+Tolerances (the pages state none for gradients; derived from the arithmetic):
+  per-element gradients du, ddelta, dz:  |err| <= tol (1 + |ref|), tol 1e-4
+    for fp32 inputs, 2e-2 for bf16 (outputs rounded to bf16, 2^-9, plus the
+    SFU forms of exp, softplus and sigmoid);
+  sums over rows dA, dB, dC, dD, ddelta_bias: max |err| <= tol max |ref|,
+    tol 1e-4 for fp32 inputs, 1e-3 for bf16 (fp32 sums of up to B*D*L terms).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import to_dev
+from selective_state_space_41_b200 import gen, selscan, workloads as W
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DY_STREAM = 9
+ELEM = {"du", "ddelta", "dz"}
+TOL_ELEM = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+TOL_SUM = {torch.float32: 1e-4, torch.bfloat16: 1e-3}
+
+
+def _case(batch, dim, L, N, dtype, seed, out_dtype=None, **kw):
+    w = W.custom("bwd", batch, dim, L, N, dtype, seed, **kw)
+    inp = W.make_inputs(w)
+    inp["dy"] = gen.fill((batch, dim, L), out_dtype or dtype, seed, DY_STREAM)
+    return inp
+
+
+def _check(inp, dtype, what):
+    d = to_dev(inp)
+    got = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], D=d.get("D"),
+                                     z=d.get("z"), delta_bias=d.get("delta_bias"),
+                                     delta_softplus=inp["delta_softplus"])
+    torch.cuda.synchronize()
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"],
+                                    D=inp.get("D"), z=inp.get("z"), delta_bias=inp.get("delta_bias"),
+                                    delta_softplus=inp["delta_softplus"])
+    for k, want in ref.items():
+        if want is None:
+            assert got[k] is None
+            continue
+        g = got[k].detach().to("cpu", torch.float64).numpy()
+        assert np.isfinite(g).all(), f"{what}: {k} not finite"
+        if want.size == 0:
+            continue
+        if k in ELEM:
+            e = float(np.max(np.abs(g - want) / (1.0 + np.abs(want))))
+            assert e <= TOL_ELEM[dtype], f"{what}: {k} max |err|/(1+|ref|) = {e:.3e}"
+        else:
+            e = float(np.max(np.abs(g - want)) / max(np.max(np.abs(want)), 1e-30))
+            assert e <= TOL_SUM[dtype], f"{what}: {k} max |err| / max |ref| = {e:.3e}"
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N", [4, 8, 9, 16, 32])
+def test_bwd_state_sizes(dtype, N):
+    """Every state bucket, ragged length (partial stage and sub-chunk) and
+    channels (mirrored rows in the last tile), every operand present."""
+    _check(_case(2, 45, 203, N, dtype, seed=N + 100, has_z=True, return_last_state=False), dtype, f"N={N}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("has_z,D_kind,bias_kind,softplus",
+                         [(False, "none", "none", True), (True, "ones", "zeros", False),
+                          (False, "normal", "uniform_dt", True), (True, "none", "normal", False)])
+def test_bwd_optional_operands(dtype, has_z, D_kind, bias_kind, softplus):
+    inp = _case(3, 33, 130, 16, dtype, seed=7, has_z=has_z, D_kind=D_kind, bias_kind=bias_kind,
+                delta_softplus=softplus)
+    _check(inp, dtype, f"z={has_z} D={D_kind} bias={bias_kind} softplus={softplus}")
+
+
+def test_bwd_bf16_in_f32_dy():
+    _check(_case(2, 40, 150, 16, torch.bfloat16, seed=11, out_dtype=torch.float32, has_z=True),
+           torch.bfloat16, "bf16 in, f32 dy")
+
+
+@pytest.mark.parametrize("L", [1, 7, 8, 64, 65])
+def test_bwd_short_sequences(L):
+    _check(_case(2, 20, L, 16, torch.float32, seed=L, has_z=True), torch.float32, f"L={L}")
+
+
+def test_bwd_mamba130m_one_batch():
+    """One batch entry of the mamba-130m-shaped layer (1536 channels x 2048 steps)."""
+    w = W.with_shape(W.WORKLOADS[W.MAMBA130M], batch=1)
+    inp = W.make_inputs(w)
+    inp["dy"] = gen.fill((1, w.dim, w.seqlen), w.dtype, w.seed, DY_STREAM)
+    _check(inp, w.dtype, "mamba130m batch 1")
+
+
+def test_bwd_deterministic():
+    inp = _case(2, 64, 300, 16, torch.bfloat16, seed=5, has_z=True)
+    d = to_dev(inp)
+    args = (d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"])
+    kw = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"], delta_softplus=True)
+    g1 = selscan.selective_scan_bwd(*args, **kw)
+    g2 = selscan.selective_scan_bwd(*args, **kw)
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_bwd_rejects_wide_state():
+    inp = _case(1, 4, 16, 64, torch.float32, seed=1)
+    d = to_dev(inp)
+    with pytest.raises(selscan.SelscanError):
+        selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"])
