@@ -489,6 +489,9 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
     p.dstate = (int)desc->dstate;
     p.softplus = delta_softplus ? 1 : 0;
     p.vec = (desc->seqlen * (int64_t)ein) % 16 == 0 && (!B || aligned(B, 16)) && (!C || aligned(C, 16));
+    p.vec_rows = (desc->seqlen * (int64_t)ein) % 16 == 0 && (desc->seqlen * (int64_t)eout) % 16 == 0 &&
+                 (!u || aligned(u, 16)) && (!delta || aligned(delta, 16)) && (!z || aligned(z, 16)) &&
+                 (!dy || aligned(dy, 16));
     p.dtiles = lo.dtiles;
     p.nsub = lo.nsub;
 

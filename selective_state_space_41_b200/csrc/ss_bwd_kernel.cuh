@@ -26,6 +26,8 @@
 //   a fixed order (with the per-row partials of dA, dD and dbias).
 #pragma once
 
+#include <type_traits>
+
 #include "ss_fwd_kernel.cuh"
 
 namespace selscan {
@@ -41,7 +43,8 @@ struct BwdParams {
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;
-    int vec;                                  // every row of u/delta/z/dy/du/ddelta/dz starts 16-byte aligned
+    int vec;                                  // every row of B and C starts 16-byte aligned
+    int vec_rows;                             // every row of u, delta, z and dy starts 16-byte aligned
     int64_t dtiles;                           // row tiles per batch entry
     int64_t nsub;                             // sub-chunks per row
 };
@@ -49,10 +52,19 @@ struct BwdParams {
 constexpr int kBwdSub = 8;                    // steps per sub-chunk
 constexpr int kBwdStage = 64;                 // steps per B/C stage in shared memory
 constexpr int kBwdGather = 3 * kBwdSub + 4;   // floats per row: delta', delta' u, g of 8 steps (+pad)
-constexpr int kBwdReduce = 3 * kBwdSub + 1;   // floats per lane: s, sum lam B, sum lam a h A of 8 steps (+pad)
+constexpr int kBwdReduce = 3 * kBwdSub + 4;   // floats per lane: s, sum lam B, sum lam a h A of 8 steps (+pad)
 
 // Lanes per row for the backward: 4 states per lane.
 __host__ __device__ constexpr int bwd_lanes(int nmax) { return nmax / 4 < 1 ? 1 : nmax / 4; }
+
+// The block's dB/dC terms of a sub-chunk: per (dB or dC, state n) a group of
+// 8 steps x (rows + 2) floats, groups `bwd_group_stride` floats apart.  The
+// padding puts the lanes of one store instruction (rows r, state groups g) on
+// distinct banks, and keeps every row of rows 8-byte aligned for the float2
+// reads of the row sums.
+__host__ __device__ constexpr int bwd_group_stride(int rows, int g) {
+    return kBwdSub * (rows + 2) + (g == 2 ? 4 : g >= 4 ? 2 : 0);
+}
 
 __host__ __device__ constexpr size_t bwd_smem_bytes(size_t in_size, int nmax, int warps) {
     const int g = bwd_lanes(nmax);
@@ -60,7 +72,7 @@ __host__ __device__ constexpr size_t bwd_smem_bytes(size_t in_size, int nmax, in
     return 4 * sizeof(float) * (size_t)(nmax / 2) * kBwdStage +        // F
            2 * in_size * (size_t)nmax * kBwdStage +                     // RB
            sizeof(float) * (size_t)warps * ((32 / g) * kBwdGather + 32 * kBwdReduce) +
-           sizeof(float) * (size_t)2 * kBwdSub * nmax * (rows + 2);     // dB/dC terms of the block's rows
+           sizeof(float) * (size_t)2 * nmax * bwd_group_stride(rows, g);  // dB/dC terms of the block's rows
 }
 
 // sigmoid(x) = 1 / (1 + exp(-x)); kFast on the SFU.
@@ -70,8 +82,16 @@ __device__ __forceinline__ float sigmoid_of(float x) {
     else return 1.f / (1.f + expf(-x));
 }
 
+// Three 128-thread blocks per SM (at most 168 registers a thread): with the
+// 4-warp blocks of the mamba-130m-shaped layer (384 blocks) that is one wave
+// on 148 SMs; measured 1.35 ms there against 1.77 ms at 255 registers.
+#ifndef SS_BWD_MIN_BLOCKS
+#define SS_BWD_MIN_BLOCKS 3
+#endif
+
+// Blocks of 128 threads (4 warps).
 template <typename Tin, typename Tout, int kNmax>
-__global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const BwdParams p) {
     constexpr int kG = bwd_lanes(kNmax);
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                  // state pairs per lane (2)
@@ -82,6 +102,8 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
     constexpr int kStageUnits = kBwdStage / kUnit;
     constexpr int kRowsPerWarp = 32 / kG;
     constexpr bool kFast = sizeof(Tin) == 2;
+    constexpr int kInWords = (kOwn * (int)sizeof(Tin) + 3) / 4;
+    constexpr int kDyWords = (kOwn * (int)sizeof(Tout) + 3) / 4;
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
@@ -91,7 +113,8 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
     const int r = lane / kG;
     const int rows = nthreads / kG;                   // rows of the block
     const int rib = tid / kG;                         // this lane's row within the block
-    const int RS = rows + 2;                          // stride of the block's dB/dC slab
+    const int RS = rows + 2;                          // floats per step in the block's dB/dC slab
+    const int GS = bwd_group_stride(rows, kG);        // floats per (dB or dC, state) group
     const int N = p.dstate;
     const int64_t b = blockIdx.x / p.dtiles;
     const int64_t dtile = blockIdx.x % p.dtiles;
@@ -101,6 +124,7 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
     const int64_t L = p.seqlen;
     const int64_t row = b * p.dim + d;
     const bool vec = p.vec != 0;
+    const bool vrows = p.vec_rows != 0;
     const bool softplus = p.softplus != 0;
     const bool has_z = p.z != nullptr;
 
@@ -112,7 +136,7 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
     float *gat = slab + r * kBwdGather;                                 // this row: delta', delta' u, g
     float *red = slab + kRowsPerWarp * kBwdGather;                      // per lane: 3 x 8 partial sums
     float *dbc = reinterpret_cast<float *>(RB + 2 * kNmax * kBwdStage) +
-                 (nthreads / 32) * (kRowsPerWarp * kBwdGather + 32 * kBwdReduce);  // [2][8][kNmax][RS]
+                 (nthreads / 32) * (kRowsPerWarp * kBwdGather + 32 * kBwdReduce);  // [2][kNmax] groups of [8][RS]
 
     const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * N * L,
                           static_cast<const Tin *>(p.C) + b * N * L};
@@ -137,21 +161,24 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
 
-    // B/C of the stage from c0 into F (fp32 float4 per step and state pair).
-    auto load_stage = [&](int64_t c0) {
-        const bool fast = vec && c0 + kBwdStage <= L;
-        __syncthreads();  // every warp is done with F (and RB)
-        if (fast) {
-            for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
-                const int j = u % kStageUnits, rowid = u / kStageUnits;
-                const int t = rowid / kNmax, n = rowid % kNmax;
-                if (n < N)
-                    cp_async16(RB + (rowid * kBwdStage + j * kUnit), Bsrc[t] + (int64_t)n * L + c0 + j * kUnit);
-            }
-            cp_async_commit();
-            cp_async_wait_all();
-            __syncthreads();
+    // B/C of a stage: raw copies into RB by cp.async (issued one stage ahead),
+    // converted into F (fp32 float4 per step and state pair) at the stage's start.
+    auto stage_fast = [&](int64_t c0) { return vec && c0 >= 0 && c0 + kBwdStage <= L; };
+    auto issue_copies = [&](int64_t c0) {
+        for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
+            const int j = u % kStageUnits, rowid = u / kStageUnits;
+            const int t = rowid / kNmax, n = rowid % kNmax;
+            if (n < N)
+                cp_async16(RB + (rowid * kBwdStage + j * kUnit), Bsrc[t] + (int64_t)n * L + c0 + j * kUnit);
         }
+        cp_async_commit();
+    };
+    // Make F hold the stage from c0 (its copies were issued earlier when it is
+    // fast), then start the copies of the stage from `next` (if any).
+    auto load_stage = [&](int64_t c0, int64_t next) {
+        const bool fast = stage_fast(c0);
+        if (fast) cp_async_wait_all();
+        __syncthreads();  // RB holds the stage; every warp is done with F
         for (int jb = tid; jb < kPairs * (kBwdStage / 8); jb += nthreads) {
             const int q = jb % kPairs, i0 = (jb / kPairs) * 8;
             float v[4][8];
@@ -185,29 +212,45 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
 #pragma unroll
             for (int m = 0; m < 8; ++m) F[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
         }
-        __syncthreads();  // F holds the stage
-    };
-    // One input element as float (0 past the end).
-    auto in_at = [&](const Tin *src, int64_t l) -> float {
-        if (l >= L) return 0.f;
-        uint32_t bits = Io<Tin>::bits(src, l);
-        if constexpr (sizeof(Tin) == 2) bits <<= 16;
-        return __uint_as_float(bits);
-    };
-    auto dy_at = [&](int64_t l) -> float {
-        if (l >= L) return 0.f;
-        return static_cast<float>(dy_row[l]);
+        __syncthreads();  // F holds the stage; RB is free
+        if (stage_fast(next)) issue_copies(next);
     };
     auto put = [&](Tin *dst, int64_t l, float v) {
         if (l < L) dst[l] = static_cast<Tin>(v);
+    };
+
+    // This lane's kOwn steps of a row stream from step `so` as raw words (0 past the end).
+    auto load_own = [&](const auto *src, int64_t so, uint32_t *w) {
+        using T = std::remove_cv_t<std::remove_pointer_t<decltype(src)>>;
+        constexpr int kBytes = kOwn * (int)sizeof(T), kWords = (kBytes + 3) / 4;
+        if (kBytes >= 4 && vrows && so + kOwn <= L) {
+            ld_words<kBytes>(src + so, w);
+        } else {
+#pragma unroll
+            for (int j = 0; j < kWords; ++j) w[j] = 0u;
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) {
+                if (so + i < L) {
+                    const uint32_t bits = Io<T>::bits(src, so + i);
+                    if constexpr (sizeof(T) == 2) w[i >> 1] |= bits << (16 * (i & 1));
+                    else w[i] = bits;
+                }
+            }
+        }
     };
 
     // ---------------------------------------------------------------- phase A
     float2 h[kPL];
 #pragma unroll
     for (int qq = 0; qq < kPL; ++qq) h[qq] = make_float2(0.f, 0.f);
+    uint32_t wu[kInWords], wd[kInWords];  // raw owned inputs of the next sub-chunk
+    if (L > 0) {
+        load_own(u_row, g * kOwn, wu);
+        load_own(d_row, g * kOwn, wd);
+        if (stage_fast(0)) issue_copies(0);
+    }
     for (int64_t c0 = 0; c0 < L; c0 += kBwdStage) {
-        load_stage(c0);
+        load_stage(c0, c0 + kBwdStage < L ? c0 + kBwdStage : -1);
         const int nsub = (int)(((L - c0 < kBwdStage ? L - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
 #pragma unroll 1
         for (int m = 0; m < nsub; ++m) {
@@ -222,14 +265,23 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
                 const int64_t l = l0 + g * kOwn + i;
-                const float dl = l < L ? delta_transform<kFast>(in_at(d_row, l) + bias, softplus) : 0.f;
+                const float dl = l < L ? delta_transform<kFast>(Io<Tin>::widen(wd, i) + bias, softplus) : 0.f;
                 gat[g * kOwn + i] = dl;
-                gat[kBwdSub + g * kOwn + i] = dl * in_at(u_row, l);
+                gat[kBwdSub + g * kOwn + i] = dl * Io<Tin>::widen(wu, i);
+            }
+            if (l0 + kBwdSub < L) {
+                load_own(u_row, l0 + kBwdSub + g * kOwn, wu);
+                load_own(d_row, l0 + kBwdSub + g * kOwn, wd);
             }
             __syncwarp();
             float dl[kBwdSub], du[kBwdSub];
 #pragma unroll
-            for (int i = 0; i < kBwdSub; ++i) dl[i] = gat[i], du[i] = gat[kBwdSub + i];
+            for (int q4 = 0; q4 < kBwdSub / 4; ++q4) {
+                const float4 x = reinterpret_cast<const float4 *>(gat)[q4];
+                const float4 y = reinterpret_cast<const float4 *>(gat + kBwdSub)[q4];
+                dl[4 * q4] = x.x, dl[4 * q4 + 1] = x.y, dl[4 * q4 + 2] = x.z, dl[4 * q4 + 3] = x.w;
+                du[4 * q4] = y.x, du[4 * q4 + 1] = y.y, du[4 * q4 + 2] = y.z, du[4 * q4 + 3] = y.w;
+            }
             __syncwarp();
             const float4 *Fm = F + (m * kBwdSub) * kPairs + q0;
 #pragma unroll
@@ -245,6 +297,7 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
             }
         }
     }
+    __syncthreads();  // every checkpoint is written (mirrored rows read other lanes' ones)
 
     // ---------------------------------------------------------------- phase B
     float2 carry[kPL], dA_acc[kPL];
@@ -252,42 +305,67 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
     for (int qq = 0; qq < kPL; ++qq) carry[qq] = make_float2(0.f, 0.f), dA_acc[qq] = make_float2(0.f, 0.f);
     float dD_acc = 0.f, dbias_acc = 0.f;
     const int64_t nstages = (L + kBwdStage - 1) / kBwdStage;
+    // Prefetched for the next sub-chunk (backwards): its checkpoint and raw owned inputs.
+    float2 h0n[kPL];
+    uint32_t wz[kInWords], wdy[kDyWords];
+    auto prefetch = [&](int64_t l0) {
+        const int64_t k = l0 / kBwdSub;
+#pragma unroll
+        for (int qq = 0; qq < kPL; ++qq) {
+            const int n = 2 * (q0 + qq);
+            h0n[qq] = make_float2(n < N ? ck_row[k * N + n] : 0.f, n + 1 < N ? ck_row[k * N + n + 1] : 0.f);
+        }
+        load_own(u_row, l0 + g * kOwn, wu);
+        load_own(d_row, l0 + g * kOwn, wd);
+        if (has_z) load_own(z_row, l0 + g * kOwn, wz);
+        load_own(dy_row, l0 + g * kOwn, wdy);
+    };
+    if (L > 0) prefetch(((L - 1) / kBwdSub) * kBwdSub);
     for (int64_t st = nstages - 1; st >= 0; --st) {
         const int64_t c0 = st * kBwdStage;
-        load_stage(c0);
+        if (st == nstages - 1) {  // F still holds the last stage from phase A
+            if (stage_fast(c0 - kBwdStage)) issue_copies(c0 - kBwdStage);
+        } else {
+            load_stage(c0, c0 - kBwdStage);
+        }
         const int nsub = (int)(((L - c0 < kBwdStage ? L - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
 #pragma unroll 1
         for (int m = nsub - 1; m >= 0; --m) {
             const int64_t l0 = c0 + m * kBwdSub;
-            const int64_t k = l0 / kBwdSub;
             // Owned steps: the per-row quantities, shared with the row's lanes.
-            float o_u[kOwn], o_x[kOwn], o_dl[kOwn], o_z[kOwn], o_dy[kOwn], o_sg[kOwn];
+            float o_u[kOwn], o_x[kOwn], o_dl[kOwn], o_z[kOwn], o_dy[kOwn], o_sg[kOwn], o_g[kOwn];
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
                 const int64_t l = l0 + g * kOwn + i;
-                o_u[i] = in_at(u_row, l);
-                o_x[i] = in_at(d_row, l) + bias;
+                o_u[i] = Io<Tin>::widen(wu, i);
+                o_x[i] = Io<Tin>::widen(wd, i) + bias;
                 o_dl[i] = l < L ? delta_transform<kFast>(o_x[i], softplus) : 0.f;
-                o_dy[i] = row_ok ? dy_at(l) : 0.f;
-                o_z[i] = has_z ? in_at(z_row, l) : 0.f;
+                o_dy[i] = row_ok ? Io<Tout>::widen(wdy, i) : 0.f;
+                o_z[i] = has_z ? Io<Tin>::widen(wz, i) : 0.f;
                 o_sg[i] = has_z ? sigmoid_of<kFast>(o_z[i]) : 1.f;
-                const float gl = has_z ? o_dy[i] * o_z[i] * o_sg[i] : o_dy[i];
+                o_g[i] = has_z ? o_dy[i] * o_z[i] * o_sg[i] : o_dy[i];
                 gat[g * kOwn + i] = o_dl[i];
                 gat[kBwdSub + g * kOwn + i] = o_dl[i] * o_u[i];
-                gat[2 * kBwdSub + g * kOwn + i] = gl;
+                gat[2 * kBwdSub + g * kOwn + i] = o_g[i];
             }
+            float2 h0[kPL];
+#pragma unroll
+            for (int qq = 0; qq < kPL; ++qq) h0[qq] = h0n[qq];
+            if (l0 > 0) prefetch(l0 - kBwdSub);
             __syncwarp();
             float dl[kBwdSub], du[kBwdSub], gg[kBwdSub];
 #pragma unroll
-            for (int i = 0; i < kBwdSub; ++i) dl[i] = gat[i], du[i] = gat[kBwdSub + i], gg[i] = gat[2 * kBwdSub + i];
+            for (int q4 = 0; q4 < kBwdSub / 4; ++q4) {
+                const float4 x = reinterpret_cast<const float4 *>(gat)[q4];
+                const float4 y = reinterpret_cast<const float4 *>(gat + kBwdSub)[q4];
+                const float4 w = reinterpret_cast<const float4 *>(gat + 2 * kBwdSub)[q4];
+                dl[4 * q4] = x.x, dl[4 * q4 + 1] = x.y, dl[4 * q4 + 2] = x.z, dl[4 * q4 + 3] = x.w;
+                du[4 * q4] = y.x, du[4 * q4 + 1] = y.y, du[4 * q4 + 2] = y.z, du[4 * q4 + 3] = y.w;
+                gg[4 * q4] = w.x, gg[4 * q4 + 1] = w.y, gg[4 * q4 + 2] = w.z, gg[4 * q4 + 3] = w.w;
+            }
 
             // Recompute the sub-chunk's decays and states from its checkpoint.
-            float2 h0[kPL], a[kBwdSub][kPL], hs[kBwdSub][kPL];
-#pragma unroll
-            for (int qq = 0; qq < kPL; ++qq) {
-                const int n = 2 * (q0 + qq);
-                h0[qq] = make_float2(n < N ? ck_row[k * N + n] : 0.f, n + 1 < N ? ck_row[k * N + n + 1] : 0.f);
-            }
+            float2 a[kBwdSub][kPL], hs[kBwdSub][kPL];
             float sp[kBwdSub];
             const float4 *Fm = F + (m * kBwdSub) * kPairs + q0;
 #pragma unroll
@@ -323,18 +401,23 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
                     dA_acc[qq] = __ffma2_rn(t, make_float2(dl[i], dl[i]), dA_acc[qq]);
                     carry[qq] = __fmul2_rn(a[i][qq], lam);
                     const int n = 2 * (q0 + qq);
-                    dbc[((0 * kBwdSub + i) * kNmax + n) * RS + rib] = dBp.x;
-                    dbc[((0 * kBwdSub + i) * kNmax + n + 1) * RS + rib] = dBp.y;
-                    dbc[((1 * kBwdSub + i) * kNmax + n) * RS + rib] = dCp.x;
-                    dbc[((1 * kBwdSub + i) * kNmax + n + 1) * RS + rib] = dCp.y;
+                    float *slot = dbc + i * RS + rib;
+                    slot[n * GS] = dBp.x;
+                    slot[(n + 1) * GS] = dBp.y;
+                    slot[(kNmax + n) * GS] = dCp.x;
+                    slot[(kNmax + n + 1) * GS] = dCp.y;
                 }
                 lb[i] = sLB.x + sLB.y;
                 lha[i] = sLHA.x + sLHA.y;
             }
             // Per-row sums over the row's lanes: s (minus D u), sum lam B, sum lam a h A.
-            float *mine = red + lane * kBwdReduce;
+            float4 *mine = reinterpret_cast<float4 *>(red + lane * kBwdReduce);
 #pragma unroll
-            for (int i = 0; i < kBwdSub; ++i) mine[i] = sp[i], mine[kBwdSub + i] = lb[i], mine[2 * kBwdSub + i] = lha[i];
+            for (int q4 = 0; q4 < kBwdSub / 4; ++q4) {
+                mine[q4] = make_float4(sp[4 * q4], sp[4 * q4 + 1], sp[4 * q4 + 2], sp[4 * q4 + 3]);
+                mine[kBwdSub / 4 + q4] = make_float4(lb[4 * q4], lb[4 * q4 + 1], lb[4 * q4 + 2], lb[4 * q4 + 3]);
+                mine[kBwdSub / 2 + q4] = make_float4(lha[4 * q4], lha[4 * q4 + 1], lha[4 * q4 + 2], lha[4 * q4 + 3]);
+            }
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
@@ -346,29 +429,29 @@ __global__ void __launch_bounds__(256) ss_bwd_kernel(const BwdParams p) {
                     s += src[j], LB += src[kBwdSub + j], LHA += src[2 * kBwdSub + j];
                 }
                 const int64_t l = l0 + j;
-                const float gl = gg[j];
                 s = fmaf(Dd, o_u[i], s);
                 const float ddl = fmaf(o_u[i], LB, LHA);
                 const float dx = softplus ? (o_x[i] > 20.f ? ddl : ddl * sigmoid_of<kFast>(o_x[i])) : ddl * o_dl[i];
                 if (row_ok && l < L) {
-                    put(du_row, l, fmaf(gl, Dd, o_dl[i] * LB));
+                    put(du_row, l, fmaf(o_g[i], Dd, o_dl[i] * LB));
                     put(dd_row, l, dx);
                     if (has_z) put(dz_row, l, o_dy[i] * s * o_sg[i] * fmaf(o_z[i], 1.f - o_sg[i], 1.f));
-                    dD_acc = fmaf(gl, o_u[i], dD_acc);
+                    dD_acc = fmaf(o_g[i], o_u[i], dD_acc);
                     dbias_acc += dx;
                 }
             }
-            // dB, dC of the sub-chunk summed over the block's rows.
+            // dB, dC of the sub-chunk summed over the block's rows (row pairs as float2).
             __syncthreads();
-            const int nout = 2 * kBwdSub * kNmax;
+            const int nout = 2 * kNmax * kBwdSub;
             for (int o = tid; o < nout; o += nthreads) {
-                const int n = o % kNmax, i = (o / kNmax) % kBwdSub, which = o / (kNmax * kBwdSub);
-                const float *src = dbc + o * RS;
-                float s = 0.f;
-                for (int q = 0; q < rows; ++q) s += src[q];
+                const int i = o % kBwdSub, grp = o / kBwdSub;          // grp = which * kNmax + n
+                const int which = grp / kNmax, n = grp % kNmax;
+                const float2 *src = reinterpret_cast<const float2 *>(dbc + grp * GS + i * RS);
+                float2 s2 = make_float2(0.f, 0.f);
+                for (int q = 0; q < rows / 2; ++q) s2 = __fadd2_rn(s2, src[q]);
                 const int64_t l = l0 + i;
                 if (n < N && l < L)
-                    p.ws_dBC[(((dtile * p.batch + b) * 2 + which) * N + n) * L + l] = s;
+                    p.ws_dBC[(((dtile * p.batch + b) * 2 + which) * N + n) * L + l] = s2.x + s2.y;
             }
             __syncthreads();  // the slabs are free for the next sub-chunk
         }
