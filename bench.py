@@ -377,6 +377,7 @@ def bench_ours(args, w, world, rank, local):
         "kernel_ms": {"min": min(kernel_ms), "median": statistics.median(kernel_ms),
                       "max": max(kernel_ms)},
     }
+    line["decode"] = bench_decode(wr, d, out_dtype, stream, world)
     if not args.no_bwd and w.dstate <= 32:
         line["backward"] = bench_backward(args, wr, d, host, out_dtype, flush, stream, sfu_peak, world)
     del flush
@@ -385,6 +386,61 @@ def bench_ours(args, w, world, rank, local):
         line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     return line if rank == 0 else None
+
+
+def bench_decode(w, d, out_dtype, stream, world, calls=200):
+    """Latency of one recurrent decoding step (ss_step: the whole (batch, dim)
+    layer advanced one token, state updated in place), averaged over
+    back-to-back calls timed by CUDA events; bytes = state read + written plus
+    the step's inputs and y."""
+    dev = d["u"].device
+    col = lambda x: None if x is None else x[..., 0].contiguous()  # noqa: E731
+    u, delta, Bm, Cm, z = (col(d[k]) for k in ("u", "delta", "B", "C", "z"))
+    state = torch.zeros((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+    y = torch.empty((w.batch, w.dim), dtype=out_dtype, device=dev)
+
+    def step():
+        selscan.ss_step(u, delta, d["A"], Bm, Cm, state, y, D=d["D"], z=z, delta_bias=d["delta_bias"],
+                        delta_softplus=w.delta_softplus, stream=stream)
+
+    for _ in range(10):
+        step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(calls):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    us_host = max_over_ranks(e0.elapsed_time(e1) * 1e3 / calls, world)
+    # The same steps captured in a CUDA graph and replayed: the device time of
+    # a step without the per-call host overhead of the Python binding.
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    per_graph = 50
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(per_graph):
+                selscan.ss_step(u, delta, d["A"], Bm, Cm, state, y, D=d["D"], z=z,
+                                delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, stream=side)
+    stream.wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    reps = max(1, calls // per_graph)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / (reps * per_graph), world)
+    del graph
+    nbytes = (2 * state.numel() * 4 + y.numel() * y.element_size() +
+              sum(t.numel() * t.element_size() for t in (u, delta, Bm, Cm, z) if t is not None))
+    return {"us_per_step": us, "tokens_per_s": w.batch * world / (us * 1e-6), "bytes_per_step": nbytes,
+            "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "us_per_step_python_calls": us_host,
+            "steps_timed": reps * per_graph, "gpu_launches_per_step": 1,
+            "note": "ss_step replayed from a CUDA graph of 50 steps (device time per step); "
+                    "us_per_step_python_calls: the same steps called one by one from Python"}
 
 
 def bench_backward(args, w, d, host, out_dtype, flush, stream, sfu_peak, world):

@@ -243,6 +243,23 @@ ss_status ss_fwd_noalloc(const ss_desc *desc, const void *u, const void *delta, 
                          ss_stream_t stream);
 
 /*
+ * One step of recurrent decoding with the state updated in place: the same
+ * arithmetic as ss_fwd_state with L = 1 and initial_state == last_state, by a
+ * kernel made for it (one thread per row and state pair; the work is one read
+ * and one write of the state).  desc->seqlen must be 1 (SS_ERR_BAD_SHAPE
+ * otherwise).
+ *   u, delta, z    device, (B, D) in_dtype (z NULL: no gate)
+ *   B, C           device, (B, N) in_dtype
+ *   A, D, delta_bias  as ss_fwd
+ *   state          device, (B, D, N) float32: the state before the step on
+ *                  entry, after it on return
+ *   y              device, (B, D) out_dtype
+ */
+ss_status ss_step(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                  const void *C, const float *D, const void *z, const float *delta_bias,
+                  int delta_softplus, float *state, void *y, ss_stream_t stream);
+
+/*
  * Backward of ss_fwd (state starting at zero): the gradients of sum(dy * y)
  * with respect to every input.  The walkthrough trains the forward through
  * autograd (§6); this is its chain rule written out (an adjoint state run

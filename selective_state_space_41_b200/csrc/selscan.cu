@@ -14,6 +14,7 @@
 
 #include "selscan.h"
 #include "ss_bwd_launch.h"
+#include "ss_step_kernel.cuh"
 #include "ss_launch.h"
 
 namespace {
@@ -332,6 +333,18 @@ BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz) {
     return lo;
 }
 
+template <typename Tin, typename Tout>
+cudaError_t launch_step(int T, dim3 grid, cudaStream_t s, const selscan::StepParams &p) {
+    switch (T) {
+        case 2: selscan::ss_step_kernel<Tin, Tout, 2><<<grid, 256, 0, s>>>(p); break;
+        case 4: selscan::ss_step_kernel<Tin, Tout, 4><<<grid, 256, 0, s>>>(p); break;
+        case 8: selscan::ss_step_kernel<Tin, Tout, 8><<<grid, 256, 0, s>>>(p); break;
+        case 16: selscan::ss_step_kernel<Tin, Tout, 16><<<grid, 256, 0, s>>>(p); break;
+        default: selscan::ss_step_kernel<Tin, Tout, 32><<<grid, 256, 0, s>>>(p); break;
+    }
+    return cudaGetLastError();
+}
+
 #define SS_PICK_BWD(PREFIX)                                                                  \
     n <= 4 ? selscan::PREFIX##_n4 : n <= 8 ? selscan::PREFIX##_n8 : n <= 16 ? selscan::PREFIX##_n16 \
                                                                   : selscan::PREFIX##_n32
@@ -519,6 +532,44 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
         if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
     }
     return SS_OK;
+}
+
+ss_status ss_step(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                  const void *C, const float *D, const void *z, const float *delta_bias,
+                  int delta_softplus, float *state, void *y, ss_stream_t stream) {
+    Sizes sz;
+    ss_status st = check_desc(desc, &sz);
+    if (st != SS_OK) return st;
+    if (desc->seqlen != 1) return SS_ERR_BAD_SHAPE;
+    if (sz.rows == 0) return SS_OK;
+    if (!u || !delta || !A || !B || !C || !state || !y) return SS_ERR_NULL_POINTER;
+    const size_t ein = dtype_size(desc->in_dtype), eout = dtype_size(desc->out_dtype);
+    const void *in_ptrs[] = {u, delta, B, C, z};
+    for (const void *q : in_ptrs)
+        if (q && !aligned(q, ein)) return SS_ERR_MISALIGNED;
+    if (!aligned(y, eout) || !aligned(A, 4) || !aligned(state, 4) || (D && !aligned(D, 4)) ||
+        (delta_bias && !aligned(delta_bias, 4)))
+        return SS_ERR_MISALIGNED;
+    const int T = selscan::state_bucket((int)desc->dstate) / 2;  // threads per row: one per state pair
+    const int64_t blocks = (sz.rows * T + 255) / 256;
+    if (blocks > INT_MAX) return SS_ERR_BAD_SHAPE;
+    selscan::StepParams p;
+    p.u = u, p.delta = delta, p.B = B, p.C = C, p.z = z;
+    p.A = A, p.D = D, p.delta_bias = delta_bias;
+    p.state = state, p.y = y;
+    p.batch = desc->batch, p.dim = desc->dim;
+    p.dstate = (int)desc->dstate;
+    p.softplus = delta_softplus ? 1 : 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)blocks);
+    cudaError_t err;
+    if (desc->in_dtype == SS_F32)
+        err = launch_step<float, float>(T, grid, s, p);
+    else if (desc->out_dtype == SS_BF16)
+        err = launch_step<__nv_bfloat16, __nv_bfloat16>(T, grid, s, p);
+    else
+        err = launch_step<__nv_bfloat16, float>(T, grid, s, p);
+    return err == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
 const char *ss_status_string(ss_status status) {

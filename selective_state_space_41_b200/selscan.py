@@ -8,7 +8,7 @@ fails to load, every call raises.
 
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``, ``ss_fwd_heuristic``,
-``ss_fwd_hostio``, ``ss_fwd_noalloc``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
+``ss_fwd_hostio``, ``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
 ``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
 to the workspace and config forms by keyword); ``selective_scan_fwd`` is the
 allocate-and-call convenience
@@ -34,7 +34,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Names the header declares; the ABI test checks each is exported.
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
-           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
+           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc", "ss_step", "ss_bwd", "ss_bwd_workspace_bytes",
            "ss_status_string", "ss_version")
 
 
@@ -86,6 +86,8 @@ def lib():
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
         L.ss_fwd_noalloc.restype = I
         L.ss_fwd_noalloc.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
+        L.ss_step.restype = I
+        L.ss_step.argtypes = [DP] + [P] * 8 + [I, P, P, P]
         L.ss_bwd.restype = I
         L.ss_bwd.argtypes = [DP] + [P] * 8 + [I] + [P] * 9 + [P, SZ, P]
         L.ss_bwd_workspace_bytes.restype = SZ
@@ -197,6 +199,20 @@ def ss_fwd_noalloc(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_
                                 _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0,
                                 _ptr(y), _ptr(last_state), _stream_handle(stream, u.device)),
            "ss_fwd_noalloc")
+
+
+def ss_step(u, delta, A, B, C, state, y, D=None, z=None, delta_bias=None, delta_softplus=False,
+            stream=None):
+    """One decoding step, the state updated in place.  u, delta, z, y: (batch,
+    dim); B, C: (batch, N); state: (batch, dim, N) float32."""
+    u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
+    if not (state.is_contiguous() and y.is_contiguous()):
+        raise ValueError("state and y must be contiguous")
+    batch, dim = u.shape[0], u.shape[1]
+    desc = make_desc(batch, dim, 1, A.shape[-1], u.dtype, y.dtype)
+    _check(lib().ss_step(ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                         _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(state), _ptr(y),
+                         _stream_handle(stream, u.device)), "ss_step")
 
 
 def ss_bwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None) -> int:

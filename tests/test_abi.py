@@ -165,6 +165,17 @@ def test_bwd_rejections(lib):
     assert e.value.status == 4
 
 
+def test_step_rejections(lib):
+    """ss_step: one step only, required pointers, alignment; before any launch."""
+    P = FAKE
+    d = _desc(seqlen=1, dstate=16)
+    args = (P, P, P, P, P, None, None, None, 1, P, P, None)
+    assert lib.ss_step(ctypes.byref(_desc(seqlen=2)), *args) == 2
+    assert lib.ss_step(ctypes.byref(d), P, P, P, P, P, None, None, None, 1, None, P, None) == 1
+    assert lib.ss_step(ctypes.byref(d), P, P, P, P, P, None, None, None, 1, ODD, P, None) == 5
+    assert lib.ss_step(ctypes.byref(_desc(seqlen=1, batch=0)), *args) == 0
+
+
 def test_hostio_rejections(lib):
     d = _desc()
     P = FAKE

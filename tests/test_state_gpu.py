@@ -116,3 +116,57 @@ def test_initial_state_zero_equals_no_state():
     y1, l1 = _run(d, torch.bfloat16, None)
     torch.cuda.synchronize()
     assert torch.equal(y0, y1) and torch.equal(l0, l1)
+
+
+# ---------------------------------------------------------------- ss_step
+def _step_loop(d, out_dtype, steps, state):
+    ys = []
+    for t in range(steps):
+        col = lambda x: None if x is None else x[..., t].contiguous()  # noqa: E731
+        y = torch.empty(d["u"].shape[:2], dtype=out_dtype, device="cuda")
+        selscan.ss_step(col(d["u"]), col(d["delta"]), d["A"], col(d["B"]), col(d["C"]), state, y,
+                        D=d.get("D"), z=col(d.get("z")), delta_bias=d.get("delta_bias"),
+                        delta_softplus=d["delta_softplus"])
+        ys.append(y)
+    return torch.stack(ys, dim=-1)
+
+
+@pytest.mark.parametrize("dtype,out_dtype", [(torch.float32, torch.float32), (torch.bfloat16, torch.bfloat16),
+                                             (torch.bfloat16, torch.float32)])
+@pytest.mark.parametrize("N", [4, 9, 16, 33, 64])
+def test_step_decode_against_oracle(dtype, out_dtype, N):
+    """ss_step (the decoding kernel) for 20 steps, state in place, against the
+    oracle's 20-step run from the same initial state; ragged row count."""
+    inp = _case(3, 37, 20, N, dtype, seed=N + 31, has_z=True, out_dtype=out_dtype)
+    d = to_dev(inp)
+    state = d["initial_state"].clone()
+    y = _step_loop(d, out_dtype, 20, state)
+    torch.cuda.synchronize()
+    y_ref, last_ref = _oracle(inp)
+    assert_parity(y, state, y_ref, last_ref, 1e-4 if out_dtype == torch.float32 and dtype == torch.bfloat16
+                  else TOL[dtype], f"step N={N}")
+
+
+@pytest.mark.parametrize("has_z,D_kind,bias_kind,softplus",
+                         [(False, "none", "none", True), (True, "ones", "zeros", False)])
+def test_step_optional_operands(has_z, D_kind, bias_kind, softplus):
+    inp = _case(2, 50, 6, 16, torch.float32, seed=3, has_z=has_z, D_kind=D_kind, bias_kind=bias_kind,
+                delta_softplus=softplus)
+    d = to_dev(inp)
+    state = d["initial_state"].clone()
+    y = _step_loop(d, torch.float32, 6, state)
+    torch.cuda.synchronize()
+    y_ref, last_ref = _oracle(inp)
+    assert_parity(y, state, y_ref, last_ref, TOL[torch.float32], "step operands")
+
+
+def test_step_matches_forward_from_state():
+    """One ss_step equals ss_fwd_state with L = 1 up to float32 summation order."""
+    inp = _case(4, 64, 1, 16, torch.bfloat16, seed=41, has_z=True, out_dtype=torch.float32)
+    d = to_dev(inp)
+    s1 = d["initial_state"].clone()
+    y1 = _step_loop(d, torch.float32, 1, s1)
+    y2, s2 = _run(d, torch.float32, d["initial_state"])
+    torch.cuda.synchronize()
+    assert torch.allclose(y1, y2, rtol=1e-5, atol=1e-5)
+    assert torch.allclose(s1, s2, rtol=1e-6, atol=1e-6)
