@@ -285,6 +285,28 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
 /* Bytes of workspace ss_bwd needs for `desc` (0 for an invalid descriptor or N > 32). */
 size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 
+/*
+ * As ss_fwd_hostio, pipelined over `nstreams` caller-owned streams (1..16):
+ * the batch is cut into `chunks` ranges of batch entries (0: min(batch,
+ * 2 * nstreams)); range c has its inputs copied in, its forward run and its
+ * outputs copied out on stream c mod nstreams, so the copies of one range
+ * overlap the copies in the other direction and the kernels of others.  A,
+ * D and delta_bias are copied once on streams[0], which the other streams
+ * wait for; the call first orders itself after all work already queued on
+ * any of the streams.  The workspace is split evenly over the streams (each
+ * range runs the launch shape its share allows).  The caller synchronises
+ * every stream before reading the results.  Returns SS_ERR_BAD_CONFIG for
+ * a bad stream count or chunk count; other errors as ss_fwd_hostio.
+ */
+ss_status ss_fwd_hostio_streams(const ss_desc *desc, const void *h_u, const void *h_delta,
+                                const float *h_A, const void *h_B, const void *h_C, const float *h_D,
+                                const void *h_z, const float *h_delta_bias, int delta_softplus,
+                                void *h_y, float *h_last_state, void *d_u, void *d_delta, float *d_A,
+                                void *d_B, void *d_C, float *d_D, void *d_z, float *d_delta_bias,
+                                void *d_y, float *d_last_state, void *d_workspace,
+                                size_t workspace_bytes, const ss_stream_t *streams, int nstreams,
+                                int chunks);
+
 /* Static description of a status code (never NULL). */
 const char *ss_status_string(ss_status status);
 

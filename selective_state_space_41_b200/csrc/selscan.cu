@@ -455,6 +455,104 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
     return SS_OK;
 }
 
+ss_status ss_fwd_hostio_streams(const ss_desc *desc, const void *h_u, const void *h_delta,
+                                const float *h_A, const void *h_B, const void *h_C, const float *h_D,
+                                const void *h_z, const float *h_delta_bias, int delta_softplus,
+                                void *h_y, float *h_last_state, void *d_u, void *d_delta, float *d_A,
+                                void *d_B, void *d_C, float *d_D, void *d_z, float *d_delta_bias,
+                                void *d_y, float *d_last_state, void *d_workspace,
+                                size_t workspace_bytes, const ss_stream_t *streams, int nstreams,
+                                int chunks) {
+    Sizes sz;
+    ss_status st = check_desc(desc, &sz);
+    if (st != SS_OK) return st;
+    if (!streams || nstreams < 1 || nstreams > 16 || chunks < 0) return SS_ERR_BAD_CONFIG;
+    if (sz.rows == 0) return SS_OK;
+    if ((!h_D) != (!d_D) || (!h_z) != (!d_z) || (!h_delta_bias) != (!d_delta_bias) ||
+        (!h_last_state) != (!d_last_state))
+        return SS_ERR_NULL_POINTER;
+    if (!h_A || !d_A) return SS_ERR_NULL_POINTER;
+    if (desc->seqlen > 0 && (!h_u || !h_delta || !h_B || !h_C || !h_y || !d_u || !d_delta ||
+                             !d_B || !d_C || !d_y))
+        return SS_ERR_NULL_POINTER;
+
+    const int64_t Bt = desc->batch, Dm = desc->dim, L = desc->seqlen, N = desc->dstate;
+    const size_t ein = dtype_size(desc->in_dtype), eout = dtype_size(desc->out_dtype);
+    const cudaMemcpyKind h2d = cudaMemcpyHostToDevice, d2h = cudaMemcpyDeviceToHost;
+    int nch = chunks > 0 ? chunks : (int)(Bt < 2 * nstreams ? Bt : 2 * nstreams);
+    if (nch > Bt) nch = (int)Bt;
+    cudaStream_t s0 = reinterpret_cast<cudaStream_t>(streams[0]);
+
+    // Order this call after everything queued on any of the streams, copy the
+    // per-channel operands on the first stream, and let every stream wait for them.
+    cudaEvent_t ev[16] = {};
+    auto cleanup = [&]() {
+        for (int k = 0; k < nstreams; ++k)
+            if (ev[k]) cudaEventDestroy(ev[k]);
+    };
+    for (int k = 0; k < nstreams; ++k)
+        if (cudaEventCreateWithFlags(&ev[k], cudaEventDisableTiming) != cudaSuccess) return cleanup(), SS_ERR_CUDA;
+    for (int k = 1; k < nstreams; ++k) {
+        cudaStream_t sk = reinterpret_cast<cudaStream_t>(streams[k]);
+        if (cudaEventRecord(ev[k], sk) != cudaSuccess || cudaStreamWaitEvent(s0, ev[k], 0) != cudaSuccess)
+            return cleanup(), SS_ERR_CUDA;
+    }
+    const size_t n_A = (size_t)Dm * N * 4, n_vec = (size_t)Dm * 4;
+    if (cudaMemcpyAsync(d_A, h_A, n_A, h2d, s0) != cudaSuccess ||
+        (d_D && cudaMemcpyAsync(d_D, h_D, n_vec, h2d, s0) != cudaSuccess) ||
+        (d_delta_bias && cudaMemcpyAsync(d_delta_bias, h_delta_bias, n_vec, h2d, s0) != cudaSuccess) ||
+        cudaEventRecord(ev[0], s0) != cudaSuccess)
+        return cleanup(), SS_ERR_CUDA;
+    for (int k = 1; k < nstreams; ++k)
+        if (cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(streams[k]), ev[0], 0) != cudaSuccess)
+            return cleanup(), SS_ERR_CUDA;
+
+    // Each chunk of batch entries: its inputs in, its forward, its outputs out,
+    // all on one stream (chunk c on stream c mod nstreams, with that stream's
+    // share of the workspace), so copies of one chunk overlap the work of others.
+    const size_t ws_share = nstreams > 0 ? (workspace_bytes / (size_t)nstreams) / 256 * 256 : 0;
+    for (int c = 0; c < nch; ++c) {
+        const int64_t b0 = Bt * c / nch, b1 = Bt * (c + 1) / nch, bc = b1 - b0;
+        if (bc <= 0) continue;
+        const int k = c % nstreams;
+        cudaStream_t sk = reinterpret_cast<cudaStream_t>(streams[k]);
+        const size_t seq0 = (size_t)(b0 * Dm * L), nseq = (size_t)(bc * Dm * L);
+        const size_t bc0 = (size_t)(b0 * N * L), nbc = (size_t)(bc * N * L);
+        const size_t st0 = (size_t)(b0 * Dm * N), nst = (size_t)(bc * Dm * N);
+        auto off = [](const void *p, size_t e) -> void * {
+            return p ? const_cast<char *>(static_cast<const char *>(p)) + e : nullptr;
+        };
+        struct Copy {
+            void *dst;
+            const void *src;
+            size_t bytes;
+        } in_copies[] = {{off(d_u, seq0 * ein), off(h_u, seq0 * ein), nseq * ein},
+                         {off(d_delta, seq0 * ein), off(h_delta, seq0 * ein), nseq * ein},
+                         {off(d_z, seq0 * ein), off(h_z, seq0 * ein), nseq * ein},
+                         {off(d_B, bc0 * ein), off(h_B, bc0 * ein), nbc * ein},
+                         {off(d_C, bc0 * ein), off(h_C, bc0 * ein), nbc * ein}};
+        for (const Copy &cp : in_copies)
+            if (cp.dst && cp.bytes && cudaMemcpyAsync(cp.dst, cp.src, cp.bytes, h2d, sk) != cudaSuccess)
+                return cleanup(), SS_ERR_CUDA;
+        ss_desc dc = *desc;
+        dc.batch = bc;
+        st = fwd_impl(&dc, off(d_u, seq0 * ein), off(d_delta, seq0 * ein), d_A, off(d_B, bc0 * ein),
+                      off(d_C, bc0 * ein), d_D, off(d_z, seq0 * ein), d_delta_bias, delta_softplus, nullptr,
+                      off(d_y, seq0 * eout), static_cast<float *>(off(d_last_state, st0 * 4)), nullptr,
+                      d_workspace ? off(d_workspace, (size_t)k * ws_share) : nullptr,
+                      d_workspace ? ws_share : 0, reinterpret_cast<ss_stream_t>(sk));
+        if (st != SS_OK) return cleanup(), st;
+        if (nseq && cudaMemcpyAsync(off(h_y, seq0 * eout), off(d_y, seq0 * eout), nseq * eout, d2h, sk) !=
+                        cudaSuccess)
+            return cleanup(), SS_ERR_CUDA;
+        if (d_last_state && cudaMemcpyAsync(off(h_last_state, st0 * 4), off(d_last_state, st0 * 4), nst * 4,
+                                            d2h, sk) != cudaSuccess)
+            return cleanup(), SS_ERR_CUDA;
+    }
+    cleanup();  // (events are released once their waits are done)
+    return SS_OK;
+}
+
 size_t ss_bwd_workspace_bytes(const ss_desc *desc) {
     Sizes sz;
     if (check_desc(desc, &sz) != SS_OK || desc->dstate > 32) return 0;

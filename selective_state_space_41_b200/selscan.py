@@ -8,7 +8,7 @@ fails to load, every call raises.
 
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``, ``ss_fwd_heuristic``,
-``ss_fwd_hostio``, ``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
+``ss_fwd_hostio``, ``ss_fwd_hostio_streams``, ``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
 ``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
 to the workspace and config forms by keyword); ``selective_scan_fwd`` is the
 allocate-and-call convenience
@@ -34,7 +34,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Names the header declares; the ABI test checks each is exported.
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
-           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc", "ss_step", "ss_bwd", "ss_bwd_workspace_bytes",
+           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc", "ss_step", "ss_bwd", "ss_bwd_workspace_bytes",
            "ss_status_string", "ss_version")
 
 
@@ -86,6 +86,8 @@ def lib():
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
         L.ss_fwd_noalloc.restype = I
         L.ss_fwd_noalloc.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
+        L.ss_fwd_hostio_streams.restype = I
+        L.ss_fwd_hostio_streams.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P, I, I]
         L.ss_step.restype = I
         L.ss_step.argtypes = [DP] + [P] * 8 + [I, P, P, P]
         L.ss_bwd.restype = I
@@ -287,11 +289,14 @@ def ss_fwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dt
             "warps_per_block": cfg.warps_per_block, "segments": cfg.segments}
 
 
-def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None, workspace=None):
+def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None, workspace=None,
+                  streams=None, chunks=0):
     """Host-buffer form: ``host`` and ``dev`` map u, delta, A, B, C, D, z,
     delta_bias, y, last_state to host (ideally pinned) and device tensors of
     the same shapes (optional entries None in both).  Queues copies in, the
-    forward, and copies of y / last_state out on ``stream``."""
+    forward, and copies of y / last_state out on ``stream``; with ``streams``
+    (a list of CUDA streams) the work is pipelined over them by batch ranges
+    (``ss_fwd_hostio_streams``) and the caller synchronises every stream."""
     g = lambda m, k: m.get(k)  # noqa: E731
     batch, dim, L = host["u"].shape
     N = host["A"].shape[-1]
@@ -300,6 +305,13 @@ def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None, work
     h_in = [_ptr(g(host, k)) for k in names_in]
     d_all = [_ptr(g(dev, k)) for k in names_in + ("y", "last_state")]
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if streams:
+        handles = (ctypes.c_void_p * len(streams))(*[st.cuda_stream for st in streams])
+        _check(lib().ss_fwd_hostio_streams(ctypes.byref(desc), *h_in, 1 if delta_softplus else 0,
+                                           _ptr(host["y"]), _ptr(g(host, "last_state")), *d_all,
+                                           _ptr(workspace), ws_bytes, handles, len(streams), int(chunks)),
+               "ss_fwd_hostio_streams")
+        return
     s = _stream_handle(stream, dev["u"].device)
     _check(lib().ss_fwd_hostio(ctypes.byref(desc), *h_in, 1 if delta_softplus else 0,
                                _ptr(host["y"]), _ptr(g(host, "last_state")), *d_all,

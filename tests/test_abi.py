@@ -176,6 +176,20 @@ def test_step_rejections(lib):
     assert lib.ss_step(ctypes.byref(_desc(seqlen=1, batch=0)), *args) == 0
 
 
+def test_hostio_streams_rejections(lib):
+    d = _desc()
+    P = FAKE
+    host = [P, P, P, P, P, None, None, None]
+    dev = [P, P, P, P, P, None, None, None, P, None]
+    streams = (ctypes.c_void_p * 2)(None, None)
+    args = (ctypes.byref(d), *host, 1, P, None, *dev, None, 0)
+    assert lib.ss_fwd_hostio_streams(*args, None, 2, 0) == 7
+    assert lib.ss_fwd_hostio_streams(*args, streams, 0, 0) == 7
+    assert lib.ss_fwd_hostio_streams(*args, streams, 17, 0) == 7
+    assert lib.ss_fwd_hostio_streams(*args, streams, 2, -1) == 7
+    assert lib.ss_fwd_hostio_streams(None, *args[1:], streams, 2, 0) == 1
+
+
 def test_hostio_rejections(lib):
     d = _desc()
     P = FAKE

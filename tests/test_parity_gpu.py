@@ -269,6 +269,27 @@ def test_hostio_matches_device_path():
     assert torch.equal(host["last_state"], last_dev.cpu())
 
 
+@pytest.mark.parametrize("nstreams,chunks", [(1, 0), (2, 0), (3, 5), (2, 1)])
+def test_hostio_streams_against_oracle(nstreams, chunks):
+    """The host-buffer form pipelined over streams by batch ranges (ragged
+    ranges: 5 batch entries), two calls in a row on different inputs."""
+    streams = [torch.cuda.Stream() for _ in range(nstreams)]
+    for seed in (61, 62):
+        inp = _case(5, 40, 700, 16, torch.bfloat16, seed=seed, has_z=True, return_last_state=True)
+        host = {k: (inp[k].pin_memory() if inp[k] is not None else None)
+                for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+        host["y"] = torch.empty((5, 40, 700), dtype=torch.bfloat16).pin_memory()
+        host["last_state"] = torch.empty((5, 40, 16), dtype=torch.float32).pin_memory()
+        dev = {k: (torch.empty_like(v, device="cuda") if v is not None else None) for k, v in host.items()}
+        ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+        selscan.ss_fwd_hostio(host, dev, delta_softplus=True, workspace=ws, streams=streams, chunks=chunks)
+        for st in streams:
+            st.synchronize()
+        y_ref, last_ref = run_oracle(inp)
+        assert_parity(host["y"], host["last_state"], y_ref, last_ref, TOL[torch.bfloat16],
+                      f"streams={nstreams} chunks={chunks} seed={seed}")
+
+
 def test_convenience_wrapper():
     inp = _case(2, 4, 33, 16, torch.bfloat16, seed=2, has_z=True, return_last_state=True)
     d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
