@@ -390,7 +390,7 @@ def bench_ours(args, w, world, rank, local):
                       "max": max(kernel_ms)},
     }
     line["decode"] = bench_decode(wr, d, out_dtype, stream, world)
-    if not args.no_bwd and w.dstate <= 32:
+    if not args.no_bwd:
         line["backward"] = bench_backward(args, wr, d, host, out_dtype, flush, stream, sfu_peak, world)
     del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -272,9 +272,8 @@ ss_status ss_step(const ss_desc *desc, const void *u, const void *delta, const f
  *   workspace          device, 256-byte aligned, ss_bwd_workspace_bytes(desc)
  *                      bytes (forward-state checkpoints every 8 steps and
  *                      partial sums); scratch, not shared by overlapping calls
- * Other arguments as ss_fwd.  N must be at most 32 (SS_ERR_UNSUPPORTED_DSTATE
- * otherwise).  Sums over rows (dA, dB, dC, dD, ddelta_bias) are taken in a
- * fixed order: results are bitwise reproducible.
+ * Other arguments as ss_fwd (N in 1..64).  Sums over rows (dA, dB, dC, dD,
+ * ddelta_bias) are taken in a fixed order: results are bitwise reproducible.
  */
 ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
                  const void *C, const float *D, const void *z, const float *delta_bias,
@@ -282,7 +281,7 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
                  size_t workspace_bytes, ss_stream_t stream);
 
-/* Bytes of workspace ss_bwd needs for `desc` (0 for an invalid descriptor or N > 32). */
+/* Bytes of workspace ss_bwd needs for `desc` (0 for an invalid descriptor). */
 size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 
 /*

@@ -29,7 +29,7 @@ NVCC_FLAGS = [
 DTYPE_PAIRS = [("float", "float", "f32_f32"), ("__nv_bfloat16", "__nv_bfloat16", "bf16_bf16"),
                ("__nv_bfloat16", "float", "bf16_f32")]
 STATE_BUCKETS = [4, 8, 16, 32, 64]
-BWD_STATE_BUCKETS = [4, 8, 16, 32]  # the backward holds 4 states per lane, at most 8 lanes per row
+BWD_STATE_BUCKETS = [4, 8, 16, 32, 64]  # the backward holds 4 states per lane
 
 
 def _nvcc() -> str:

@@ -306,7 +306,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
 }
 
 // ---------------------------------------------------------------- backward
-constexpr int kBwdWarps = 4;
+constexpr int kBwdWarps = selscan::kBwdThreads / 32;
 
 struct BwdLayout {
     int lanes, rows;        // lanes per row, rows per block
@@ -347,7 +347,7 @@ cudaError_t launch_step(int T, dim3 grid, cudaStream_t s, const selscan::StepPar
 
 #define SS_PICK_BWD(PREFIX)                                                                  \
     n <= 4 ? selscan::PREFIX##_n4 : n <= 8 ? selscan::PREFIX##_n8 : n <= 16 ? selscan::PREFIX##_n16 \
-                                                                  : selscan::PREFIX##_n32
+    : n <= 32 ? selscan::PREFIX##_n32 : selscan::PREFIX##_n64
 
 }  // namespace
 
@@ -555,7 +555,7 @@ ss_status ss_fwd_hostio_streams(const ss_desc *desc, const void *h_u, const void
 
 size_t ss_bwd_workspace_bytes(const ss_desc *desc) {
     Sizes sz;
-    if (check_desc(desc, &sz) != SS_OK || desc->dstate > 32) return 0;
+    if (check_desc(desc, &sz) != SS_OK) return 0;
     return bwd_layout(desc, sz).total;
 }
 
@@ -567,7 +567,6 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
-    if (desc->dstate > 32) return SS_ERR_UNSUPPORTED_DSTATE;
     if (!A || !dA) return SS_ERR_NULL_POINTER;
     const bool work = sz.rows > 0 && desc->seqlen > 0;
     if (work && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)) return SS_ERR_NULL_POINTER;

@@ -50,11 +50,12 @@ struct BwdParams {
 };
 
 constexpr int kBwdSub = 8;                    // steps per sub-chunk
+constexpr int kBwdThreads = 128;              // threads per block (4 warps)
 constexpr int kBwdStage = 64;                 // steps per B/C stage in shared memory
 constexpr int kBwdGather = 3 * kBwdSub + 4;   // floats per row: delta', delta' u, g of 8 steps (+pad)
 constexpr int kBwdReduce = 3 * kBwdSub + 4;   // floats per lane: s, sum lam B, sum lam a h A of 8 steps (+pad)
 
-// Lanes per row for the backward: 4 states per lane.
+// Lanes per row for the backward: 4 states per lane (16 lanes for 64 states).
 __host__ __device__ constexpr int bwd_lanes(int nmax) { return nmax / 4 < 1 ? 1 : nmax / 4; }
 
 // The block's dB/dC terms of a sub-chunk: per (dB or dC, state n) a group of
@@ -96,8 +97,11 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                  // state pairs per lane (2)
     static_assert(kPL * kG == kPairs && kPL >= 1, "whole state pairs per lane");
-    constexpr int kOwn = kBwdSub / kG;                // steps owned per lane per sub-chunk
-    static_assert(kOwn >= 1, "at most 8 lanes per row");
+    // Steps of a sub-chunk owned per lane (their per-row work: delta', the
+    // gate, the outputs); with more lanes than steps (16 lanes for 64 states),
+    // one lane in every kStride owns one step.
+    constexpr int kOwn = kG <= kBwdSub ? kBwdSub / kG : 1;
+    constexpr int kStride = kG <= kBwdSub ? 1 : kG / kBwdSub;
     constexpr int kUnit = Io<Tin>::kUnit;
     constexpr int kStageUnits = kBwdStage / kUnit;
     constexpr int kRowsPerWarp = 32 / kG;
@@ -106,15 +110,15 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     constexpr int kDyWords = (kOwn * (int)sizeof(Tout) + 3) / 4;
 
     const int tid = threadIdx.x;
-    const int nthreads = blockDim.x;
+    constexpr int nthreads = kBwdThreads;             // the launch uses exactly this block size
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int g = lane % kG;
     const int r = lane / kG;
-    const int rows = nthreads / kG;                   // rows of the block
+    constexpr int rows = nthreads / kG;               // rows of the block
     const int rib = tid / kG;                         // this lane's row within the block
-    const int RS = rows + 2;                          // floats per step in the block's dB/dC slab
-    const int GS = bwd_group_stride(rows, kG);        // floats per (dB or dC, state) group
+    constexpr int RS = rows + 2;                      // floats per step in the block's dB/dC slab
+    constexpr int GS = bwd_group_stride(rows, kG);    // floats per (dB or dC, state) group
     const int N = p.dstate;
     const int64_t b = blockIdx.x / p.dtiles;
     const int64_t dtile = blockIdx.x % p.dtiles;
@@ -150,6 +154,8 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     float *ck_row = p.ckpt + row * p.nsub * N;
 
     const int q0 = g * kPL;
+    const bool owner = g % kStride == 0;
+    const int j0 = (g / kStride) * kOwn;              // first owned step within a sub-chunk
     const float *A_d = p.A + d * N;
     float2 A2[kPL], Aln[kPL];                          // A log2(e) and A
 #pragma unroll
@@ -245,8 +251,8 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     for (int qq = 0; qq < kPL; ++qq) h[qq] = make_float2(0.f, 0.f);
     uint32_t wu[kInWords], wd[kInWords];  // raw owned inputs of the next sub-chunk
     if (L > 0) {
-        load_own(u_row, g * kOwn, wu);
-        load_own(d_row, g * kOwn, wd);
+        load_own(u_row, j0, wu);
+        load_own(d_row, j0, wd);
         if (stage_fast(0)) issue_copies(0);
     }
     for (int64_t c0 = 0; c0 < L; c0 += kBwdStage) {
@@ -264,14 +270,16 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
             }
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
-                const int64_t l = l0 + g * kOwn + i;
+                const int64_t l = l0 + j0 + i;
                 const float dl = l < L ? delta_transform<kFast>(Io<Tin>::widen(wd, i) + bias, softplus) : 0.f;
-                gat[g * kOwn + i] = dl;
-                gat[kBwdSub + g * kOwn + i] = dl * Io<Tin>::widen(wu, i);
+                if (owner) {
+                    gat[j0 + i] = dl;
+                    gat[kBwdSub + j0 + i] = dl * Io<Tin>::widen(wu, i);
+                }
             }
             if (l0 + kBwdSub < L) {
-                load_own(u_row, l0 + kBwdSub + g * kOwn, wu);
-                load_own(d_row, l0 + kBwdSub + g * kOwn, wd);
+                load_own(u_row, l0 + kBwdSub + j0, wu);
+                load_own(d_row, l0 + kBwdSub + j0, wd);
             }
             __syncwarp();
             float dl[kBwdSub], du[kBwdSub];
@@ -315,10 +323,10 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
             const int n = 2 * (q0 + qq);
             h0n[qq] = make_float2(n < N ? ck_row[k * N + n] : 0.f, n + 1 < N ? ck_row[k * N + n + 1] : 0.f);
         }
-        load_own(u_row, l0 + g * kOwn, wu);
-        load_own(d_row, l0 + g * kOwn, wd);
-        if (has_z) load_own(z_row, l0 + g * kOwn, wz);
-        load_own(dy_row, l0 + g * kOwn, wdy);
+        load_own(u_row, l0 + j0, wu);
+        load_own(d_row, l0 + j0, wd);
+        if (has_z) load_own(z_row, l0 + j0, wz);
+        load_own(dy_row, l0 + j0, wdy);
     };
     if (L > 0) prefetch(((L - 1) / kBwdSub) * kBwdSub);
     for (int64_t st = nstages - 1; st >= 0; --st) {
@@ -336,7 +344,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
             float o_u[kOwn], o_x[kOwn], o_dl[kOwn], o_z[kOwn], o_dy[kOwn], o_sg[kOwn], o_g[kOwn];
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
-                const int64_t l = l0 + g * kOwn + i;
+                const int64_t l = l0 + j0 + i;
                 o_u[i] = Io<Tin>::widen(wu, i);
                 o_x[i] = Io<Tin>::widen(wd, i) + bias;
                 o_dl[i] = l < L ? delta_transform<kFast>(o_x[i], softplus) : 0.f;
@@ -344,9 +352,11 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 o_z[i] = has_z ? Io<Tin>::widen(wz, i) : 0.f;
                 o_sg[i] = has_z ? sigmoid_of<kFast>(o_z[i]) : 1.f;
                 o_g[i] = has_z ? o_dy[i] * o_z[i] * o_sg[i] : o_dy[i];
-                gat[g * kOwn + i] = o_dl[i];
-                gat[kBwdSub + g * kOwn + i] = o_dl[i] * o_u[i];
-                gat[2 * kBwdSub + g * kOwn + i] = o_g[i];
+                if (owner) {
+                    gat[j0 + i] = o_dl[i];
+                    gat[kBwdSub + j0 + i] = o_dl[i] * o_u[i];
+                    gat[2 * kBwdSub + j0 + i] = o_g[i];
+                }
             }
             float2 h0[kPL];
 #pragma unroll
@@ -395,11 +405,12 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     const float2 dCp = __fmul2_rn(g2, hs[i][qq]);
                     const float2 dBp = __fmul2_rn(lam, u2);
                     const float2 hp = i ? hs[i - 1][qq] : h0[qq];
-                    const float2 t = __fmul2_rn(__fmul2_rn(lam, a[i][qq]), hp);  // lam a h_prev
+                    const float2 la = __fmul2_rn(lam, a[i][qq]);   // a lam: the carry to the step before
+                    const float2 t = __fmul2_rn(la, hp);             // lam a h_prev
                     sLB = __ffma2_rn(lam, make_float2(bc.x, bc.y), sLB);
                     sLHA = __ffma2_rn(t, Aln[qq], sLHA);
                     dA_acc[qq] = __ffma2_rn(t, make_float2(dl[i], dl[i]), dA_acc[qq]);
-                    carry[qq] = __fmul2_rn(a[i][qq], lam);
+                    carry[qq] = la;
                     const int n = 2 * (q0 + qq);
                     float *slot = dbc + i * RS + rib;
                     slot[n * GS] = dBp.x;
@@ -421,7 +432,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
-                const int j = g * kOwn + i;
+                const int j = j0 + i;
                 float s = 0.f, LB = 0.f, LHA = 0.f;
 #pragma unroll
                 for (int q = 0; q < kG; ++q) {
@@ -432,7 +443,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 s = fmaf(Dd, o_u[i], s);
                 const float ddl = fmaf(o_u[i], LB, LHA);
                 const float dx = softplus ? (o_x[i] > 20.f ? ddl : ddl * sigmoid_of<kFast>(o_x[i])) : ddl * o_dl[i];
-                if (row_ok && l < L) {
+                if (owner && row_ok && l < L) {
                     put(du_row, l, fmaf(o_g[i], Dd, o_dl[i] * LB));
                     put(dd_row, l, dx);
                     if (has_z) put(dz_row, l, o_dy[i] * s * o_sg[i] * fmaf(o_z[i], 1.f - o_sg[i], 1.f));
@@ -448,7 +459,13 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 const int which = grp / kNmax, n = grp % kNmax;
                 const float2 *src = reinterpret_cast<const float2 *>(dbc + grp * GS + i * RS);
                 float2 s2 = make_float2(0.f, 0.f);
-                for (int q = 0; q < rows / 2; ++q) s2 = __fadd2_rn(s2, src[q]);
+                float2 t2 = make_float2(0.f, 0.f);  // two partial sums in flight
+#pragma unroll
+                for (int q = 0; q < rows / 2; q += 2) {
+                    s2 = __fadd2_rn(s2, src[q]);
+                    if (q + 1 < rows / 2) t2 = __fadd2_rn(t2, src[q + 1]);
+                }
+                s2 = __fadd2_rn(s2, t2);
                 const int64_t l = l0 + i;
                 if (n < N && l < L)
                     p.ws_dBC[(((dtile * p.batch + b) * 2 + which) * N + n) * L + l] = s2.x + s2.y;

@@ -140,13 +140,13 @@ def test_state_entry_rejections(lib):
 
 def test_bwd_rejections(lib):
     """ss_bwd rejects before any launch (the pointers are fake): no
-    descriptor, more than 32 states, a missing gradient output, no workspace.
+    descriptor, more than 64 states, a missing gradient output, no workspace.
     Also goes through the binding's argument list once (its call is rejected
     on the state count before any pointer is used)."""
     P = FAKE
     args = (P, P, P, P, P, None, None, None, 1, P, P, P, P, P, P, None, None, None)
     assert lib.ss_bwd(None, *args, None, 0, None) == 1
-    assert lib.ss_bwd(ctypes.byref(_desc(dstate=33)), *args, None, 0, None) == 4
+    assert lib.ss_bwd(ctypes.byref(_desc(dstate=65)), *args, None, 0, None) == 4
     d = _desc(dstate=16)
     missing = (P, P, P, P, P, None, None, None, 1, P, None, P, P, P, P, None, None, None)
     assert lib.ss_bwd(ctypes.byref(d), *missing, None, 0, None) == 1
@@ -154,11 +154,12 @@ def test_bwd_rejections(lib):
     assert lib.ss_bwd(ctypes.byref(d), *withD, None, 0, None) == 1
     assert lib.ss_bwd(ctypes.byref(d), *args, None, 0, None) == 8
     assert lib.ss_bwd_workspace_bytes(ctypes.byref(d)) > 0
-    assert lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(dstate=64))) == 0
+    assert lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(dstate=64))) > 0
+    assert lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(dstate=65))) == 0
     import torch
     t = torch.zeros(1, 2, 4)
     with pytest.raises(selscan.SelscanError) as e:
-        selscan.ss_bwd(t, t, torch.zeros(2, 64), torch.zeros(1, 64, 4), torch.zeros(1, 64, 4), t,
+        selscan.ss_bwd(t, t, torch.zeros(2, 65), torch.zeros(1, 65, 4), torch.zeros(1, 65, 4), t,
                        {"du": t, "ddelta": t, "dA": t, "dB": t, "dC": t},
                        workspace=torch.zeros(16, dtype=torch.uint8),
                        stream=types.SimpleNamespace(cuda_stream=0))

@@ -58,7 +58,7 @@ def _check(inp, dtype, what):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("N", [4, 8, 9, 16, 32])
+@pytest.mark.parametrize("N", [4, 8, 9, 16, 32, 33, 64])
 def test_bwd_state_sizes(dtype, N):
     """Every state bucket, ragged length (partial stage and sub-chunk) and
     channels (mirrored rows in the last tile), every operand present."""
@@ -105,8 +105,10 @@ def test_bwd_deterministic():
         assert torch.equal(g1[k], g2[k]), k
 
 
-def test_bwd_rejects_wide_state():
-    inp = _case(1, 4, 16, 64, torch.float32, seed=1)
-    d = to_dev(inp)
-    with pytest.raises(selscan.SelscanError):
-        selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"])
+def test_bwd_wide_state_layer_rows():
+    """64 states (16 lanes per row, one lane in two owning a step), bf16,
+    a few rows of the wide-state layer shape."""
+    w = W.with_shape(W.WORKLOADS["wide_state_b16_d4096_l8192_n64"], batch=1, dim=48, seqlen=1000)
+    inp = W.make_inputs(w)
+    inp["dy"] = gen.fill((1, 48, 1000), w.dtype, w.seed, DY_STREAM)
+    _check(inp, w.dtype, "wide state N=64")
