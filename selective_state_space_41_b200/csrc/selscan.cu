@@ -211,15 +211,27 @@ cudaError_t launch_bf16_f32(int n, int lanes, int split, dim3 grid, dim3 block, 
     SS_PICK_BUCKET(launch_bf16_f32)
 }
 
+template <typename Tin, typename Tout>
+void launch_fixup_t(int nmax, dim3 grid, cudaStream_t s, const FwdParams &p) {
+    switch (nmax) {
+        case 4: selscan::ss_fwd_fixup_kernel<Tin, Tout, 4><<<grid, 256, 0, s>>>(p); break;
+        case 8: selscan::ss_fwd_fixup_kernel<Tin, Tout, 8><<<grid, 256, 0, s>>>(p); break;
+        case 16: selscan::ss_fwd_fixup_kernel<Tin, Tout, 16><<<grid, 256, 0, s>>>(p); break;
+        case 32: selscan::ss_fwd_fixup_kernel<Tin, Tout, 32><<<grid, 256, 0, s>>>(p); break;
+        default: selscan::ss_fwd_fixup_kernel<Tin, Tout, 64><<<grid, 256, 0, s>>>(p); break;
+    }
+}
+
 cudaError_t launch_fixup(const ss_desc *desc, int64_t rows, int nseg, cudaStream_t s, const FwdParams &p) {
     const int64_t threads = rows * nseg;
-    const dim3 grid((unsigned)((threads + 255) / 256)), block(256);
+    const dim3 grid((unsigned)((threads + 255) / 256));
+    const int nmax = selscan::state_bucket((int)desc->dstate);
     if (desc->in_dtype == SS_F32)
-        selscan::ss_fwd_fixup_kernel<float, float><<<grid, block, 0, s>>>(p);
+        launch_fixup_t<float, float>(nmax, grid, s, p);
     else if (desc->out_dtype == SS_BF16)
-        selscan::ss_fwd_fixup_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, block, 0, s>>>(p);
+        launch_fixup_t<__nv_bfloat16, __nv_bfloat16>(nmax, grid, s, p);
     else
-        selscan::ss_fwd_fixup_kernel<__nv_bfloat16, float><<<grid, block, 0, s>>>(p);
+        launch_fixup_t<__nv_bfloat16, float>(nmax, grid, s, p);
     return cudaGetLastError();
 }
 

@@ -1084,10 +1084,9 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 // once every state's exponent A_n log2e S_l is below -127, where ex2.ftz
 // returns exactly 0, so the remaining shares are exactly zero.  Thread
 // (row, segment 0) instead writes the last state h_in(nseg) when asked.
-template <typename Tin, typename Tout>
+template <typename Tin, typename Tout, int kNmax>
 __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
     constexpr bool kFast = sizeof(Tin) == 2;
-    constexpr int kMaxN = 64;
     const int64_t rows_total = p.batch * p.dim;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= rows_total * p.nseg) return;
@@ -1098,21 +1097,27 @@ __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
     const int64_t L = p.seqlen;
     if (s == 0 && p.last_state == nullptr) return;
 
-    float A2[kMaxN], h[kMaxN];
+    // Registers: the state bucket is a compile-time size (states past N stay 0).
+    float A2[kNmax], h[kNmax];
     float A2max = __int_as_float(0xff800000u);  // -inf
-    for (int n = 0; n < N; ++n) {
-        A2[n] = p.A[d * N + n] * kLog2e;
-        A2max = fmaxf(A2max, A2[n]);
+#pragma unroll
+    for (int n = 0; n < kNmax; ++n) {
+        A2[n] = n < N ? p.A[d * N + n] * kLog2e : 0.f;
+        if (n < N) A2max = fmaxf(A2max, A2[n]);
         h[n] = 0.f;
     }
     const int upto = s == 0 ? p.nseg : s;  // segments folded into the carry
     for (int j = 0; j < upto; ++j) {
         const int64_t rec = j * rows_total + row;
         const float ds = p.ws_dsum[rec];
-        for (int n = 0; n < N; ++n) h[n] = fmaf(sfu_exp2(A2[n] * ds), h[n], p.ws_hend[rec * N + n]);
+#pragma unroll
+        for (int n = 0; n < kNmax; ++n)
+            if (n < N) h[n] = fmaf(sfu_exp2(A2[n] * ds), h[n], p.ws_hend[rec * N + n]);
     }
     if (s == 0) {
-        for (int n = 0; n < N; ++n) p.last_state[row * N + n] = h[n];
+#pragma unroll
+        for (int n = 0; n < kNmax; ++n)
+            if (n < N) p.last_state[row * N + n] = h[n];
         return;
     }
 
@@ -1129,8 +1134,9 @@ __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
         S += delta_transform<kFast>(static_cast<float>(dl_row[l]) + bias, softplus);
         if (A2max * S < -127.f) break;  // every 2^(A2 S) is 0 from here on
         float corr = 0.f;
-        for (int n = 0; n < N; ++n)
-            corr = fmaf(static_cast<float>(C_b[(int64_t)n * L + l]) * sfu_exp2(A2[n] * S), h[n], corr);
+#pragma unroll
+        for (int n = 0; n < kNmax; ++n)
+            if (n < N) corr = fmaf(static_cast<float>(C_b[(int64_t)n * L + l]) * sfu_exp2(A2[n] * S), h[n], corr);
         if (z_row) corr *= silu<kFast>(static_cast<float>(z_row[l]));
         y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + corr);
     }
