@@ -430,15 +430,29 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 mine[kBwdSub / 2 + q4] = make_float4(lha[4 * q4], lha[4 * q4 + 1], lha[4 * q4 + 2], lha[4 * q4 + 3]);
             }
             __syncwarp();
+            // Sums over the row's lanes of this lane's owned steps (vector reads).
+            constexpr int kRV = kOwn >= 4 ? 4 : kOwn;
+            float sS[kOwn], sB[kOwn], sH[kOwn];
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) sS[i] = 0.f, sB[i] = 0.f, sH[i] = 0.f;
+#pragma unroll
+            for (int q = 0; q < kG; ++q) {
+                const float *src = red + (r * kG + q) * kBwdReduce + j0;
+#pragma unroll
+                for (int i = 0; i < kOwn; i += kRV) {
+                    float v0[kRV], v1[kRV], v2[kRV];
+                    ld_vec<kRV>(src + i, v0);
+                    ld_vec<kRV>(src + kBwdSub + i, v1);
+                    ld_vec<kRV>(src + 2 * kBwdSub + i, v2);
+#pragma unroll
+                    for (int e = 0; e < kRV; ++e) sS[i + e] += v0[e], sB[i + e] += v1[e], sH[i + e] += v2[e];
+                }
+            }
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
                 const int j = j0 + i;
-                float s = 0.f, LB = 0.f, LHA = 0.f;
-#pragma unroll
-                for (int q = 0; q < kG; ++q) {
-                    const float *src = red + (r * kG + q) * kBwdReduce;
-                    s += src[j], LB += src[kBwdSub + j], LHA += src[2 * kBwdSub + j];
-                }
+                float s = sS[i];
+                const float LB = sB[i], LHA = sH[i];
                 const int64_t l = l0 + j;
                 s = fmaf(Dd, o_u[i], s);
                 const float ddl = fmaf(o_u[i], LB, LHA);

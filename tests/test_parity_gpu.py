@@ -290,6 +290,25 @@ def test_hostio_streams_against_oracle(nstreams, chunks):
                       f"streams={nstreams} chunks={chunks} seed={seed}")
 
 
+def test_hostio_streams_segmented_ranges():
+    """Few rows and a long sequence: every batch range runs the segmented
+    shape inside its stream's share of the workspace."""
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    inp = _case(3, 16, 6000, 16, torch.float32, seed=71, has_z=True, return_last_state=True)
+    assert selscan.ss_fwd_heuristic(1, 16, 6000, 16, torch.float32, workspace_bytes=1 << 19)["segments"] > 1
+    host = {k: (inp[k].pin_memory() if inp[k] is not None else None)
+            for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    host["y"] = torch.empty((3, 16, 6000), dtype=torch.float32).pin_memory()
+    host["last_state"] = torch.empty((3, 16, 16), dtype=torch.float32).pin_memory()
+    dev = {k: (torch.empty_like(v, device="cuda") if v is not None else None) for k, v in host.items()}
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    selscan.ss_fwd_hostio(host, dev, delta_softplus=True, workspace=ws, streams=streams)
+    for st in streams:
+        st.synchronize()
+    y_ref, last_ref = run_oracle(inp)
+    assert_parity(host["y"], host["last_state"], y_ref, last_ref, TOL[torch.float32], "segmented ranges")
+
+
 def test_convenience_wrapper():
     inp = _case(2, 4, 33, 16, torch.bfloat16, seed=2, has_z=True, return_last_state=True)
     d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
