@@ -206,6 +206,8 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
+// Wait until at most one (the most recent) committed group is still in flight.
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;\n" ::); }
 
 // One stage of the inclusive scan of (P, h) pairs over the W lanes of a row,
 // under (P1, h1) . (P2, h2) = (P2 P1, P2 h1 + h2): take the pair `off` lanes
@@ -684,8 +686,16 @@ __host__ __device__ constexpr int reduce_stride(int g) {
 }
 __host__ __device__ constexpr int reduce_vec(int g) { return g == 8 ? 2 : 4; }
 
+// B/C stages are double-buffered (one block barrier per stage; the next
+// stage's conversion overlaps this one's recurrence) unless a lane holds 16
+// states: there the second buffer's shared memory would cost blocks per SM
+// (measured: 16 x 4096 x 8192 x 32 layer 6.94 ms double-buffered, 6.24 ms not).
+__host__ __device__ constexpr bool direct_double_buffer(int nmax, int g) { return nmax / g != 16; }
+
+// B/C stage buffers (F as fp32 float4s, RB raw), one or two of each, then the slabs.
 __host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax, int g, int warps) {
-    return 4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage +
+    return (direct_double_buffer(nmax, g) ? 2 : 1) *
+               (4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage) +
            (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * gather_stride(g) + 32 * reduce_stride(g)) : 0);
 }
 
@@ -786,10 +796,15 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     const int64_t Lend = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
 
     extern __shared__ float4 smem[];
-    float4 *F = smem;                                                   // [kDirectStage][kPairs]
-    Tin *RB = reinterpret_cast<Tin *>(smem + kDirectStage * kPairs);     // [2][kNmax][kDirectStage]
+    // Stage buffers, one or two of each: F [kDirectStage][kPairs] float4, RB [2][kNmax][kDirectStage] raw.
+    constexpr bool kDB = direct_double_buffer(kNmax, kG);
+    constexpr int kNB = kDB ? 2 : 1;
+    float4 *const F0 = smem, *const F1 = smem + (kNB - 1) * kDirectStage * kPairs;
+    Tin *const RB0 = reinterpret_cast<Tin *>(smem + kNB * kDirectStage * kPairs);
+    Tin *const RB1 = RB0 + (kNB - 1) * 2 * kNmax * kDirectStage;
+    float4 *F = F0;                                                     // the stage being computed
     constexpr int kRS = reduce_stride(kG), kRV = reduce_vec(kG);
-    float *slab = reinterpret_cast<float *>(RB + 2 * kNmax * kDirectStage) +
+    float *slab = reinterpret_cast<float *>(RB1 + 2 * kNmax * kDirectStage) +
                   warp * (kRowsPerWarp * kGatherStride + 32 * kRS);
     float *gat = slab + r * kGatherStride;                  // this row: 8 delta', 8 delta' u
     float *red = slab + kRowsPerWarp * kGatherStride;       // per lane: 8 partial sums of y
@@ -821,7 +836,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
 
     auto stage_fast = [&](int64_t c0) { return vec && c0 + kDirectStage <= Lend; };
-    auto issue_copies = [&](int64_t c0) {
+    auto issue_copies = [&](int64_t c0, Tin *RB) {
         for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
             const int j = u % kStageUnits, rowid = u / kStageUnits;
             const int t = rowid / kNmax, n = rowid % kNmax;
@@ -830,8 +845,8 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         }
         cp_async_commit();
     };
-    // RB (or global memory, element by element) -> F: job (q, step block of 8).
-    auto fill_F = [&](int64_t c0, bool from_RB) {
+    // RB (or global memory, element by element) -> Fs: job (q, step block of 8).
+    auto fill_F = [&](int64_t c0, bool from_RB, const Tin *RB, float4 *Fs) {
         for (int jb = tid; jb < kPairs * (kDirectStage / 8); jb += nthreads) {
             const int q = jb % kPairs, i0 = (jb / kPairs) * 8;
             float v[4][8];
@@ -863,7 +878,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
                 }
             }
 #pragma unroll
-            for (int m = 0; m < 8; ++m) F[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
+            for (int m = 0; m < 8; ++m) Fs[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
         }
     };
     // This lane's kOwn steps of a stream starting `off` elements past `own`
@@ -889,7 +904,23 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     load_own_checked(u_own, c_begin + g * kOwn, wu);
     load_own_checked(d_own, c_begin + g * kOwn, wd);
     if (has_z) load_own_checked(z_own, c_begin + g * kOwn, wz);
-    if (c_begin < Lend && stage_fast(c_begin)) issue_copies(c_begin);
+    // Stage k's B/C sit in F[k & 1]; the raw copies of stage k + 1 are in
+    // flight (into RB[(k + 1) & 1]) while stage k is computed.  The first
+    // stage is converted here.
+    if (!kDB) {
+        if (c_begin < Lend && stage_fast(c_begin)) issue_copies(c_begin, RB0);
+    } else if (c_begin < Lend) {
+        const int64_t c1 = c_begin + kDirectStage;
+        const bool f0 = stage_fast(c_begin), f1 = c1 < Lend && stage_fast(c1);
+        if (f0) issue_copies(c_begin, RB0);
+        if (f1) issue_copies(c1, RB1);
+        if (f0) {
+            if (f1) cp_async_wait_one();
+            else cp_async_wait_all();
+        }
+        __syncthreads();  // every thread's copies of the first stage have landed
+        fill_F(c_begin, f0, RB0, F0);
+    }
     float dsum = 0.f;  // sum of this lane's delta' (segment record)
 
     // One sub-chunk of 8 steps from step l0; kChecked: guard the sequence end.
@@ -1005,13 +1036,25 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         y_own += kDirectSub;
     };
 
-    for (int64_t c0 = c_begin; c0 < Lend; c0 += kDirectStage) {
+    int stage = 0;
+    for (int64_t c0 = c_begin; c0 < Lend; c0 += kDirectStage, ++stage) {
         const bool fast = stage_fast(c0);
-        if (fast) cp_async_wait_all();
-        __syncthreads();  // RB holds this stage; every warp is done with F
-        fill_F(c0, fast);
-        __syncthreads();  // F holds this stage; RB is free
-        if (c0 + kDirectStage < Lend && stage_fast(c0 + kDirectStage)) issue_copies(c0 + kDirectStage);
+        const int64_t cn = c0 + kDirectStage, cnn = cn + kDirectStage;
+        if constexpr (kDB) {
+            const bool odd = stage & 1;
+            F = odd ? F1 : F0;
+            if (cn < Lend && stage_fast(cn)) cp_async_wait_all();  // the next stage's copies (the only group in flight)
+            __syncthreads();  // F of this stage is complete; the next stage's raw copies have landed; the
+                              // other F (last stage's) and this stage's RB (converted before) are free
+            if (cn < Lend) fill_F(cn, stage_fast(cn), odd ? RB0 : RB1, odd ? F0 : F1);
+            if (cnn < Lend && stage_fast(cnn)) issue_copies(cnn, odd ? RB1 : RB0);
+        } else {
+            if (fast) cp_async_wait_all();
+            __syncthreads();  // RB holds this stage; every warp is done with F
+            fill_F(c0, fast, RB0, F0);
+            __syncthreads();  // F holds this stage; RB is free
+            if (cn < Lend && stage_fast(cn)) issue_copies(cn, RB0);
+        }
 
         if (fast) {
 #pragma unroll 1
