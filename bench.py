@@ -55,12 +55,16 @@ def measured_peaks():
 
 
 def kernel_source_digest() -> str:
-    """sha256 of the kernel source (csrc/ss_fwd_kernel.cuh): identifies the
-    kernel a recorded ncu traffic figure belongs to."""
+    """sha256 of the kernel source (csrc/ss_fwd_kernel.cuh) with its // comments
+    and blank lines removed: identifies the kernel code a recorded ncu traffic
+    figure belongs to (editing a comment does not change the kernel)."""
     import hashlib
+    import re
     path = os.path.join(ROOT, "selective_state_space_41_b200", "csrc", "ss_fwd_kernel.cuh")
-    with open(path, "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()
+    with open(path, encoding="utf-8") as fh:
+        lines = [re.sub(r"//.*$", "", line).rstrip() for line in fh.read().splitlines()]
+    code = "\n".join(line for line in lines if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()
 
 
 def recorded_traffic(workload: str, shape):

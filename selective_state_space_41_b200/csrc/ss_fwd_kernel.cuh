@@ -1,4 +1,7 @@
-// Selective-scan forward kernel for sm_100a.
+// Selective-scan forward kernels for sm_100a: the scan kernel (lanes split a
+// row's steps; described here), the direct kernel (lanes split a row's
+// states; used whenever the rows fill the GPU) and the fix-up kernel of
+// sequence segments, each with its own description further down.
 //
 // Computes, per row (b, d) of the (batch, dim) grid and per state n, the
 // recurrence of the selective_scan_ref walkthrough ("Mamba代码实战：手把手教你用
@@ -650,16 +653,18 @@ __global__ void __launch_bounds__(256, Occupancy<kNmax>::kMinBlocks) ss_fwd_kern
 //   h = a h + delta' u (B_n, B_n+1),  acc += (C_n, C_n+1) h      (f32x2)
 // with only h, A and a few per-step values live.
 //
-// Steps come in sub-chunks of 8.  Lane g of a row computes delta' and
-// delta' u for 8/G of them; with G > 1 the row's lanes all-gather them
-// through a small per-warp shared slab, and after the state loop each lane
-// writes its partial sums of y over its states for all 8 steps there and
-// reads back the G partials of its own 8/G steps, which it finishes (D u,
-// silu(z)) and stores.
+// Steps come in sub-chunks of S (8, or 16 when 4 or 8 lanes share a row).
+// Lane g of a row computes delta' and delta' u for S/G of them; with G > 1
+// the row's lanes all-gather them through a small per-warp shared slab, and
+// after the state loop each lane writes its partial sums of y over its states
+// for all S steps there and reads back the G partials of its own S/G steps,
+// which it finishes (D u, silu(z)) and stores.
 //
 // B and C (shared by all rows of a batch entry) are staged per block for
-// kDirectStage steps: cp.async copies the raw rows into RB one stage ahead,
-// then the block converts them to fp32 in F, where float4 number
+// kDirectStage steps: cp.async copies the raw rows into RB ahead of use, and
+// the block converts them to fp32 in F (both buffers doubled, so that the
+// next stage converts while this one runs: see direct_double_buffer), where
+// float4 number
 // i (kNmax/2) + q holds (B[2q][i], B[2q+1][i], C[2q][i], C[2q+1][i]); the
 // lanes that own the same states read the same address (broadcast).  A stage
 // that lies wholly inside the sequence with aligned rows takes a path with no

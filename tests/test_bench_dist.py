@@ -93,3 +93,4 @@ def test_two_ranks_gloo():
     res = sorted(q.get(timeout=10) for _ in range(world))
     assert [m for _, m, _ in res] == [3.0, 3.0]           # max over ranks
     assert res[0][2] != res[1][2]                          # independent problems per rank
+
