@@ -1,5 +1,6 @@
-// libselscan: C ABI of the selective-scan forward (declarations and the
-// meaning of every argument are in include/selscan.h).
+// libselscan: C ABI of the selective scan -- forward, host-buffer forms,
+// decoding step and backward (declarations and the meaning of every argument
+// are in include/selscan.h).
 //
 // Host side: validates the descriptor and pointers before touching CUDA,
 // picks a launch shape, and dispatches to the kernel instance for the dtype

@@ -7,12 +7,14 @@ current stream.  There is no fallback: if ``libselscan.so`` is missing or
 fails to load, every call raises.
 
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
-``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``, ``ss_fwd_heuristic``,
-``ss_fwd_hostio``, ``ss_fwd_hostio_streams``, ``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
-``ss_status_string``, ``ss_version``; ``ss_fwd`` dispatches
-to the workspace and config forms by keyword); ``selective_scan_fwd`` is the
-allocate-and-call convenience
-form with the argument order of the walkthrough's selective_scan_ref
+``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``,
+``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
+``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
+``ss_status_string``, ``ss_version``); ``ss_fwd`` dispatches to the
+workspace, config and initial-state forms by keyword, ``ss_fwd_hostio`` to
+the pipelined form when given streams.  ``selective_scan_fwd`` and
+``selective_scan_bwd`` are the allocate-and-call convenience forms, with the
+argument order of the walkthrough's selective_scan_ref
 ("Mamba代码实战：手把手教你用PyTorch复现选择性扫描核心逻辑（附避坑指南）", §6).
 """
 import ctypes
