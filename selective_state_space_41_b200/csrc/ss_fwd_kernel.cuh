@@ -697,10 +697,18 @@ __host__ __device__ constexpr int reduce_vec(int g) { return g == 8 ? 2 : 4; }
 // (measured: 16 x 4096 x 8192 x 32 layer 6.94 ms double-buffered, 6.24 ms not).
 __host__ __device__ constexpr bool direct_double_buffer(int nmax, int g) { return nmax / g != 16; }
 
-// B/C stage buffers (F as fp32 float4s, RB raw), one or two of each, then the slabs.
+// Bytes of F per (step, state pair): fp32 (B_n, B_n+1, C_n, C_n+1) for fp32
+// inputs; for bf16 inputs the two bf16 pairs as two 32-bit words, widened by
+// shifts when read.  Halving F halves the shared-memory traffic of the B/C
+// reads, the busiest part of that pipe (mamba-130m-shaped layer 221 -> 208 us,
+// 16 x 4096 x 8192 layers with 32 / 64 states 6.24 -> 5.61 / 10.98 -> 10.34 ms;
+// the 100k-step genomic layer 2.40 -> 2.47 ms).
+__host__ __device__ constexpr size_t direct_f_bytes(size_t in_size) { return in_size == 2 ? 8 : 16; }
+
+// B/C stage buffers (F, RB raw), one or two of each, then the slabs.
 __host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax, int g, int warps) {
     return (direct_double_buffer(nmax, g) ? 2 : 1) *
-               (4 * sizeof(float) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage) +
+               (direct_f_bytes(in_size) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage) +
            (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * gather_stride(g) + 32 * reduce_stride(g)) : 0);
 }
 
@@ -804,8 +812,10 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     // Stage buffers, one or two of each: F [kDirectStage][kPairs] float4, RB [2][kNmax][kDirectStage] raw.
     constexpr bool kDB = direct_double_buffer(kNmax, kG);
     constexpr int kNB = kDB ? 2 : 1;
-    float4 *const F0 = smem, *const F1 = smem + (kNB - 1) * kDirectStage * kPairs;
-    Tin *const RB0 = reinterpret_cast<Tin *>(smem + kNB * kDirectStage * kPairs);
+    constexpr bool kPack = direct_f_bytes(sizeof(Tin)) == 8;                  // F as packed bf16 pairs
+    constexpr int kFUnits = kDirectStage * kPairs / (kPack ? 2 : 1);         // float4 units per F buffer
+    float4 *const F0 = smem, *const F1 = smem + (kNB - 1) * kFUnits;
+    Tin *const RB0 = reinterpret_cast<Tin *>(smem + kNB * kFUnits);
     Tin *const RB1 = RB0 + (kNB - 1) * 2 * kNmax * kDirectStage;
     float4 *F = F0;                                                     // the stage being computed
     constexpr int kRS = reduce_stride(kG), kRV = reduce_vec(kG);
@@ -882,8 +892,17 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
                     }
                 }
             }
+            if constexpr (kPack) {
+                uint2 *Fp = reinterpret_cast<uint2 *>(Fs);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) Fs[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
+                for (int m = 0; m < 8; ++m)
+                    Fp[(i0 + m) * kPairs + q] =
+                        make_uint2((__float_as_uint(v[0][m]) >> 16) | (__float_as_uint(v[1][m]) & 0xffff0000u),
+                                   (__float_as_uint(v[2][m]) >> 16) | (__float_as_uint(v[3][m]) & 0xffff0000u));
+            } else {
+#pragma unroll
+                for (int m = 0; m < 8; ++m) Fs[(i0 + m) * kPairs + q] = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
+            }
         }
     };
     // This lane's kOwn steps of a stream starting `off` elements past `own`
@@ -978,6 +997,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         }
         float part[kDirectSub];
         const float4 *Fm = F + (m * kDirectSub) * kPairs + q0;
+        const uint2 *Fm2 = reinterpret_cast<const uint2 *>(F) + (m * kDirectSub) * kPairs + q0;
         auto A2_of = [&](int qq) {
             if constexpr (kA2InRegs) return A2[qq];
             const int n = 2 * (q0 + qq);
@@ -991,7 +1011,14 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
             for (int k = 0; k < kAccs; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int qq = 0; qq < kPL; ++qq) {
-                const float4 bc = Fm[i * kPairs + qq];
+                float4 bc;  // (B_n, B_n+1, C_n, C_n+1) of this step and state pair
+                if constexpr (kPack) {
+                    const uint2 w = Fm2[i * kPairs + qq];
+                    bc = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+                } else {
+                    bc = Fm[i * kPairs + qq];
+                }
                 const float2 t = __fmul2_rn(d2, A2_of(qq));
                 const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
                 h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
