@@ -224,9 +224,9 @@ void launch_fixup_t(int nmax, dim3 grid, cudaStream_t s, const FwdParams &p) {
 }
 
 cudaError_t launch_fixup(const ss_desc *desc, int64_t rows, int nseg, cudaStream_t s, const FwdParams &p) {
-    const int64_t threads = rows * nseg;
-    const dim3 grid((unsigned)((threads + 255) / 256));
     const int nmax = selscan::state_bucket((int)desc->dstate);
+    const int64_t threads = rows * nseg * (nmax / 4);  // 4 states per thread
+    const dim3 grid((unsigned)((threads + 255) / 256));
     if (desc->in_dtype == SS_F32)
         launch_fixup_t<float, float>(nmax, grid, s, p);
     else if (desc->out_dtype == SS_BF16)

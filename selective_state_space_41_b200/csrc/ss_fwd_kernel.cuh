@@ -1135,40 +1135,54 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 // once every state's exponent A_n log2e S_l is below -127, where ex2.ftz
 // returns exactly 0, so the remaining shares are exactly zero.  Thread
 // (row, segment 0) instead writes the last state h_in(nseg) when asked.
+// Threads: kT = kNmax/4 per (row, segment), 4 states each; they share the
+// step loop (each computes the same delta' sums, so they stop together) and
+// add their shares of the correction by shuffles within their group.
 template <typename Tin, typename Tout, int kNmax>
 __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
     constexpr bool kFast = sizeof(Tin) == 2;
+    constexpr int kT = kNmax / 4 < 1 ? 1 : kNmax / 4;  // threads per (row, segment)
+    constexpr int kS = kNmax / kT;                       // states per thread
     const int64_t rows_total = p.batch * p.dim;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= rows_total * p.nseg) return;
-    const int64_t row = t % rows_total;
-    const int s = (int)(t / rows_total);
+    const int64_t grp = t / kT;                          // (row, segment) of this thread's group
+    const int q = (int)(t % kT);
+    if (grp >= rows_total * p.nseg) return;              // whole groups leave together
+    const int64_t row = grp % rows_total;
+    const int s = (int)(grp / rows_total);
     const int64_t b = row / p.dim, d = row % p.dim;
     const int N = p.dstate;
     const int64_t L = p.seqlen;
     if (s == 0 && p.last_state == nullptr) return;
+    const int lane = threadIdx.x & 31;
+    const unsigned mask = (kT >= 32 ? 0xffffffffu : ((1u << kT) - 1u) << (lane / kT * kT));
 
-    // Registers: the state bucket is a compile-time size (states past N stay 0).
-    float A2[kNmax], h[kNmax];
-    float A2max = __int_as_float(0xff800000u);  // -inf
+    // Registers: this thread's 4 states of the bucket (states past N stay 0).
+    float A2[kS], h[kS];
+    float A2max = __int_as_float(0xff800000u);  // -inf, over all N states: the group stops together
+    for (int n = 0; n < N; ++n) A2max = fmaxf(A2max, p.A[d * N + n] * kLog2e);
 #pragma unroll
-    for (int n = 0; n < kNmax; ++n) {
-        A2[n] = n < N ? p.A[d * N + n] * kLog2e : 0.f;
-        if (n < N) A2max = fmaxf(A2max, A2[n]);
-        h[n] = 0.f;
+    for (int k = 0; k < kS; ++k) {
+        const int n = q * kS + k;
+        A2[k] = n < N ? p.A[d * N + n] * kLog2e : 0.f;
+        h[k] = 0.f;
     }
     const int upto = s == 0 ? p.nseg : s;  // segments folded into the carry
     for (int j = 0; j < upto; ++j) {
         const int64_t rec = j * rows_total + row;
         const float ds = p.ws_dsum[rec];
 #pragma unroll
-        for (int n = 0; n < kNmax; ++n)
-            if (n < N) h[n] = fmaf(sfu_exp2(A2[n] * ds), h[n], p.ws_hend[rec * N + n]);
+        for (int k = 0; k < kS; ++k) {
+            const int n = q * kS + k;
+            if (n < N) h[k] = fmaf(sfu_exp2(A2[k] * ds), h[k], p.ws_hend[rec * N + n]);
+        }
     }
     if (s == 0) {
 #pragma unroll
-        for (int n = 0; n < kNmax; ++n)
-            if (n < N) p.last_state[row * N + n] = h[n];
+        for (int k = 0; k < kS; ++k) {
+            const int n = q * kS + k;
+            if (n < N) p.last_state[row * N + n] = h[k];
+        }
         return;
     }
 
@@ -1186,10 +1200,16 @@ __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
         if (A2max * S < -127.f) break;  // every 2^(A2 S) is 0 from here on
         float corr = 0.f;
 #pragma unroll
-        for (int n = 0; n < kNmax; ++n)
-            if (n < N) corr = fmaf(static_cast<float>(C_b[(int64_t)n * L + l]) * sfu_exp2(A2[n] * S), h[n], corr);
-        if (z_row) corr *= silu<kFast>(static_cast<float>(z_row[l]));
-        y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + corr);
+        for (int k = 0; k < kS; ++k) {
+            const int n = q * kS + k;
+            if (n < N) corr = fmaf(static_cast<float>(C_b[(int64_t)n * L + l]) * sfu_exp2(A2[k] * S), h[k], corr);
+        }
+#pragma unroll
+        for (int off = kT / 2; off >= 1; off /= 2) corr += __shfl_xor_sync(mask, corr, off, kT);
+        if (q == 0) {
+            if (z_row) corr *= silu<kFast>(static_cast<float>(z_row[l]));
+            y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + corr);
+        }
     }
 }
 
