@@ -112,3 +112,12 @@ def test_bwd_wide_state_layer_rows():
     inp = W.make_inputs(w)
     inp["dy"] = gen.fill((1, 48, 1000), w.dtype, w.seed, DY_STREAM)
     _check(inp, w.dtype, "wide state N=64")
+
+
+def test_bwd_softplus_linear_region():
+    """delta + bias above torch's softplus threshold (20) on most steps: the
+    derivative there is 1, below it sigmoid (both paths of the kernel)."""
+    inp = _case(2, 24, 150, 16, torch.float32, seed=23, has_z=True)
+    inp["delta_bias"] = torch.full((24,), 20.0)          # delta ~ N(0, 1): both sides of 20
+    inp["A"] = (inp["A"] * 0.01).contiguous()            # keep exp(delta' A) away from underflow
+    _check(inp, torch.float32, "softplus threshold")
