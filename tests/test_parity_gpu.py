@@ -68,6 +68,37 @@ def test_full_size_sampled_rows(name):
     torch.cuda.empty_cache()
 
 
+def test_over_2g_elements_per_tensor():
+    """A layer with more than 2^31 elements per (batch, dim, L) tensor
+    (1 x 1024 x 2.1M steps, bf16, 16 states): 64-bit offsets throughout,
+    the segmented shape over a 2.1M-step sequence and its fix-up; rows at
+    both ends and the middle against the oracle.  Inputs are drawn on the
+    device from a seeded generator (no host copy of the whole layer)."""
+    D, L, N = 1024, 2_100_000, 16
+    assert D * L > 2**31
+    g = torch.Generator(device="cuda").manual_seed(4107)
+    u = torch.randn((1, D, L), generator=g, device="cuda").to(torch.bfloat16)
+    delta = torch.randn((1, D, L), generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn((1, N, L), generator=g, device="cuda").to(torch.bfloat16)
+    C = torch.randn((1, N, L), generator=g, device="cuda").to(torch.bfloat16)
+    A = -torch.arange(1, N + 1, dtype=torch.float32, device="cuda").repeat(D, 1).contiguous()
+    Dv = torch.ones(D, device="cuda")
+    y = torch.empty((1, D, L), dtype=torch.bfloat16, device="cuda")
+    last = torch.empty((1, D, N), dtype=torch.float32, device="cuda")
+    ws = selscan.workspace_for(1, D, L, N, torch.bfloat16)
+    assert ws is not None   # the segmented shape
+    selscan.ss_fwd(u, delta, A, B, C, y, D=Dv, delta_softplus=True, last_state=last, workspace=ws)
+    torch.cuda.synchronize()
+    rows = [0, 511, D - 1]
+    host = {"u": u[:, rows].cpu(), "delta": delta[:, rows].cpu(), "A": A[rows].cpu(), "B": B.cpu(),
+            "C": C.cpu(), "D": Dv[rows].cpu()}
+    y_ref, last_ref = oracle.selective_scan(host["u"], host["delta"], host["A"], host["B"], host["C"],
+                                            D=host["D"], delta_softplus=True, return_last_state=True)
+    assert_parity(y[:, rows], last[:, rows], y_ref, last_ref, TOL[torch.bfloat16], "2^31+ elements")
+    del u, delta, B, C, y, last, ws
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------- edge cases
 @pytest.mark.parametrize("L", [1, 2, 7, 8, 9, 63, 64, 65, 255, 257, 1000, 1003])
 def test_ragged_lengths(L):
