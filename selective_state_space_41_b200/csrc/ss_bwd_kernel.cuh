@@ -307,6 +307,24 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     }
     __syncthreads();  // every checkpoint is written (mirrored rows read other lanes' ones)
 
+    // This thread's slots of the block's dB/dC sums: output o = (which * kNmax
+    // + n) * 8 + i, the slab offset of its row group and the address of step
+    // i of its (which, n) row in the block partials (to be indexed by l0).
+    constexpr int kOut = 2 * kNmax * kBwdSub;
+    constexpr int kOutPer = (kOut + nthreads - 1) / nthreads;
+    int out_src[kOutPer], out_i[kOutPer];
+    float *out_dst[kOutPer];
+#pragma unroll
+    for (int k = 0; k < kOutPer; ++k) {
+        const int o = tid + k * nthreads;
+        const int i = o % kBwdSub, grp = o / kBwdSub;  // grp = which * kNmax + n
+        const int which = grp / kNmax, n = grp % kNmax;
+        const bool ok = o < kOut && n < N;
+        out_src[k] = ok ? grp * GS + i * RS : -1;
+        out_i[k] = i;
+        out_dst[k] = ok ? p.ws_dBC + (((dtile * p.batch + b) * 2 + which) * N + n) * L + i : nullptr;
+    }
+
     // ---------------------------------------------------------------- phase B
     float2 carry[kPL], dA_acc[kPL];
 #pragma unroll
@@ -465,13 +483,13 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     dbias_acc += dx;
                 }
             }
-            // dB, dC of the sub-chunk summed over the block's rows (row pairs as float2).
+            // dB, dC of the sub-chunk summed over the block's rows (row pairs as float2);
+            // this thread's output slots and their addresses are fixed (set up once).
             __syncthreads();
-            const int nout = 2 * kNmax * kBwdSub;
-            for (int o = tid; o < nout; o += nthreads) {
-                const int i = o % kBwdSub, grp = o / kBwdSub;          // grp = which * kNmax + n
-                const int which = grp / kNmax, n = grp % kNmax;
-                const float2 *src = reinterpret_cast<const float2 *>(dbc + grp * GS + i * RS);
+#pragma unroll
+            for (int k = 0; k < kOutPer; ++k) {
+                if (out_src[k] < 0) continue;
+                const float2 *src = reinterpret_cast<const float2 *>(dbc + out_src[k]);
                 float2 s2 = make_float2(0.f, 0.f);
                 float2 t2 = make_float2(0.f, 0.f);  // two partial sums in flight
 #pragma unroll
@@ -480,9 +498,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     if (q + 1 < rows / 2) t2 = __fadd2_rn(t2, src[q + 1]);
                 }
                 s2 = __fadd2_rn(s2, t2);
-                const int64_t l = l0 + i;
-                if (n < N && l < L)
-                    p.ws_dBC[(((dtile * p.batch + b) * 2 + which) * N + n) * L + l] = s2.x + s2.y;
+                if (l0 + out_i[k] < L) out_dst[k][l0] = s2.x + s2.y;
             }
             __syncthreads();  // the slabs are free for the next sub-chunk
         }
