@@ -698,17 +698,24 @@ __host__ __device__ constexpr int reduce_vec(int g) { return g == 8 ? 2 : 4; }
 __host__ __device__ constexpr bool direct_double_buffer(int nmax, int g) { return nmax / g != 16; }
 
 // Bytes of F per (step, state pair): fp32 (B_n, B_n+1, C_n, C_n+1) for fp32
-// inputs; for bf16 inputs the two bf16 pairs as two 32-bit words, widened by
-// shifts when read.  Halving F halves the shared-memory traffic of the B/C
-// reads, the busiest part of that pipe (mamba-130m-shaped layer 221 -> 208 us,
-// 16 x 4096 x 8192 layers with 32 / 64 states 6.24 -> 5.61 / 10.98 -> 10.34 ms;
-// the 100k-step genomic layer 2.40 -> 2.47 ms).
-__host__ __device__ constexpr size_t direct_f_bytes(size_t in_size) { return in_size == 2 ? 8 : 16; }
+// inputs.  For bf16 inputs F is narrower, which cuts the shared-memory
+// traffic of the B/C reads, the busiest part of that pipe, at the cost of
+// integer widening when read:
+//  - a lane with 4 states keeps both bf16 pairs as two 32-bit words (8 bytes),
+//    widened by shifts (mamba-130m-shaped layer 221 -> 205 us);
+//  - a lane with 8 or more states keeps B as fp32 and only C packed
+//    (12 bytes), half the widening: there the integer pipe, not shared
+//    memory, was the tighter limit (16 x 4096 x 8192 layers with 32 / 64
+//    states 5.74 -> 5.39 / 10.60 -> 10.14 ms, the 100k-step genomic layer
+//    2.46 -> 2.40 ms against both packed; 6.24 / 10.98 / 2.40 ms all fp32).
+__host__ __device__ constexpr size_t direct_f_bytes(size_t in_size, int nmax, int g) {
+    return in_size == 2 ? (nmax / g >= 8 ? 12 : 8) : 16;
+}
 
 // B/C stage buffers (F, RB raw), one or two of each, then the slabs.
 __host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax, int g, int warps) {
     return (direct_double_buffer(nmax, g) ? 2 : 1) *
-               (direct_f_bytes(in_size) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage) +
+               (direct_f_bytes(in_size, nmax, g) * (size_t)(nmax / 2) * kDirectStage + 2 * in_size * (size_t)nmax * kDirectStage) +
            (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * gather_stride(g) + 32 * reduce_stride(g)) : 0);
 }
 
@@ -812,8 +819,9 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     // Stage buffers, one or two of each: F [kDirectStage][kPairs] float4, RB [2][kNmax][kDirectStage] raw.
     constexpr bool kDB = direct_double_buffer(kNmax, kG);
     constexpr int kNB = kDB ? 2 : 1;
-    constexpr bool kPack = direct_f_bytes(sizeof(Tin)) == 8;                  // F as packed bf16 pairs
-    constexpr int kFUnits = kDirectStage * kPairs / (kPack ? 2 : 1);         // float4 units per F buffer
+    constexpr bool kPack = direct_f_bytes(sizeof(Tin), kNmax, kG) == 8;      // F as packed bf16 pairs
+    constexpr bool kHalf = direct_f_bytes(sizeof(Tin), kNmax, kG) == 12;     // B fp32, C packed
+    constexpr int kFUnits = (int)(kDirectStage * kPairs * direct_f_bytes(sizeof(Tin), kNmax, kG) / 16);  // float4 units per F buffer
     float4 *const F0 = smem, *const F1 = smem + (kNB - 1) * kFUnits;
     Tin *const RB0 = reinterpret_cast<Tin *>(smem + kNB * kFUnits);
     Tin *const RB1 = RB0 + (kNB - 1) * 2 * kNmax * kDirectStage;
@@ -892,7 +900,15 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
                     }
                 }
             }
-            if constexpr (kPack) {
+            if constexpr (kHalf) {
+                float2 *FB = reinterpret_cast<float2 *>(Fs);
+                uint32_t *FC = reinterpret_cast<uint32_t *>(FB + kDirectStage * kPairs);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    FB[(i0 + m) * kPairs + q] = make_float2(v[0][m], v[1][m]);
+                    FC[(i0 + m) * kPairs + q] = (__float_as_uint(v[2][m]) >> 16) | (__float_as_uint(v[3][m]) & 0xffff0000u);
+                }
+            } else if constexpr (kPack) {
                 uint2 *Fp = reinterpret_cast<uint2 *>(Fs);
 #pragma unroll
                 for (int m = 0; m < 8; ++m)
@@ -998,6 +1014,9 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         float part[kDirectSub];
         const float4 *Fm = F + (m * kDirectSub) * kPairs + q0;
         const uint2 *Fm2 = reinterpret_cast<const uint2 *>(F) + (m * kDirectSub) * kPairs + q0;
+        const float2 *FmB = reinterpret_cast<const float2 *>(F) + (m * kDirectSub) * kPairs + q0;
+        const uint32_t *FmC = reinterpret_cast<const uint32_t *>(reinterpret_cast<const float2 *>(F) + kDirectStage * kPairs) +
+                              (m * kDirectSub) * kPairs + q0;
         auto A2_of = [&](int qq) {
             if constexpr (kA2InRegs) return A2[qq];
             const int n = 2 * (q0 + qq);
@@ -1012,7 +1031,11 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 #pragma unroll
             for (int qq = 0; qq < kPL; ++qq) {
                 float4 bc;  // (B_n, B_n+1, C_n, C_n+1) of this step and state pair
-                if constexpr (kPack) {
+                if constexpr (kHalf) {
+                    const float2 bb = FmB[i * kPairs + qq];
+                    const uint32_t cw = FmC[i * kPairs + qq];
+                    bc = make_float4(bb.x, bb.y, __uint_as_float(cw << 16), __uint_as_float(cw & 0xffff0000u));
+                } else if constexpr (kPack) {
                     const uint2 w = Fm2[i * kPairs + qq];
                     bc = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
                                      __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
