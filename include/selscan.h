@@ -185,6 +185,31 @@ ss_status ss_fwd_state(const ss_desc *desc, const void *u, const void *delta, co
                        size_t workspace_bytes, ss_stream_t stream);
 
 /*
+ * As ss_fwd_state, for rows that hold several sequences one after another
+ * (packed or concatenated sequences, or a long sequence whose state is reset
+ * at chosen steps): the state is reset at each sequence start, so nothing of
+ * one sequence leaks into the next (the boundary reset of "Mamba实战：如何用
+ * 选择性状态空间模型提升你的长序列处理效率（附代码）" §2, and its periodic reset
+ * of very long sequences in §5).
+ *   reset   device, (B, L) bytes, required when B*D*L > 0 (SS_ERR_NULL_POINTER
+ *           otherwise); reset[b*L + l] != 0 means a new sequence starts at
+ *           step l of every row of batch entry b: the state entering step l
+ *           is zero, so h_l = delta'_l B_l u_l there, whatever came before
+ *           (a reset at l = 0 overrides initial_state).  Read only.
+ * The rows run in the direct kernel (the states split over the lanes; with a
+ * workspace, in sequence segments as ss_fwd_ws, a segment that holds a start
+ * passing no state on): a config asking for the scan kernel
+ * (split_states = 0 with lanes_per_row > 1) returns SS_ERR_BAD_CONFIG.
+ * Other arguments and errors as ss_fwd_state.
+ */
+ss_status ss_fwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const uint8_t *reset,
+                       const float *initial_state, void *y, float *last_state,
+                       const ss_launch_config *config, void *workspace, size_t workspace_bytes,
+                       ss_stream_t stream);
+
+/*
  * The launch shape ss_fwd_ws would use for `desc` with `workspace_bytes` of
  * workspace (0: as ss_fwd).  Returns SS_OK, or the status ss_fwd would return
  * for a bad descriptor.

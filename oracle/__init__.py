@@ -29,6 +29,9 @@ def _load(path=None):
         lib.ss_oracle_fwd.restype = ctypes.c_int
         lib.ss_oracle_fwd.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P, P,
                                       ctypes.c_int, P, P, ctypes.c_int]
+        lib.ss_oracle_fwd_reset.restype = ctypes.c_int
+        lib.ss_oracle_fwd_reset.argtypes = [i64, i64, i64, i64] + [P] * 8 + [ctypes.c_int] + [P] * 4 + \
+            [ctypes.c_int]
         lib.ss_oracle_fwd_init.restype = ctypes.c_int
         lib.ss_oracle_fwd_init.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P, P,
                                            ctypes.c_int, P, P, P, ctypes.c_int]
@@ -66,12 +69,13 @@ def _ptr(a):
 
 def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                    delta_softplus=False, return_last_state=False, nthreads=0, lib=None,
-                   initial_state=None):
+                   initial_state=None, reset=None):
     """y[b,d,l] (and the state after the last step) in float64.
 
     Shapes: u, delta, z (batch, dim, L); A (dim, N); B, C (batch, N, L);
     D, delta_bias (dim,); initial_state (batch, dim, N), the state before
-    step 0 (zero when None).  Returns y, or (y, last_state (batch, dim, N)).
+    step 0 (zero when None); reset (batch, L), nonzero where a new sequence
+    starts (the state entering that step is zero).  Returns y, or (y, last_state (batch, dim, N)).
     ``lib`` selects another build of the oracle library by path (the pin tests
     use it to show that planted mistakes are caught).
     """
@@ -91,9 +95,19 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     h0 = _f64(initial_state)
     if h0 is not None and h0.shape != (batch, dim, N):
         raise ValueError("bad initial_state shape")
+    rs = None
+    if reset is not None:
+        rs = np.ascontiguousarray(np.asarray(reset) != 0, dtype=np.uint8)
+        if rs.shape != (batch, L):
+            raise ValueError("bad reset shape")
     y = np.zeros((batch, dim, L), dtype=np.float64)
     last = np.zeros((batch, dim, N), dtype=np.float64) if return_last_state else None
-    if h0 is None:
+    if rs is not None:
+        rc = _load(lib).ss_oracle_fwd_reset(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                                            _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                                            1 if delta_softplus else 0, _ptr(rs), _ptr(h0), _ptr(y),
+                                            _ptr(last), int(nthreads))
+    elif h0 is None:
         rc = _load(lib).ss_oracle_fwd(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
                                       _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
                                       1 if delta_softplus else 0, _ptr(y), _ptr(last), int(nthreads))

@@ -21,6 +21,13 @@
  * be run in pieces, each piece starting from the last state of the one before
  * (the streaming and single-step use of the recurrence that "告别‘炼丹’：从
  * Mamba-minimal入手..." describes in §2.1).
+ * Extension: an optional (batch, seqlen) byte mask of sequence starts.  A
+ * nonzero reset[b][l] sets the state of every row of batch entry b to zero
+ * before step l, so that sequences laid end to end in one row do not leak
+ * into one another: the boundary reset that "Mamba实战：如何用选择性状态空间
+ * 模型提升你的长序列处理效率（附代码）" lists in §2 (and its periodic reset of
+ * very long sequences in §5).  The pages give no interface for it; a reset at
+ * step 0 overrides the initial state.
  * The "parallel" body printed in §4.2 / §6 (cumprod then cumsum) is NOT what
  * this follows: it disagrees with the §3.2 loop, which is the definition.
  *
@@ -67,12 +74,12 @@ int ss_oracle_threads(void)
 }
 
 /* Returns 0 on success, -1 on a bad argument. nthreads <= 0 means "all". */
-int ss_oracle_fwd_init(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
-                       const double *u, const double *delta, const double *A,
-                       const double *B, const double *C, const double *D,
-                       const double *z, const double *delta_bias, int delta_softplus,
-                       const double *initial_state, double *y, double *last_state,
-                       int nthreads)
+int ss_oracle_fwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                        const double *u, const double *delta, const double *A,
+                        const double *B, const double *C, const double *D,
+                        const double *z, const double *delta_bias, int delta_softplus,
+                        const uint8_t *reset, const double *initial_state, double *y,
+                        double *last_state, int nthreads)
 {
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1)
         return -1;
@@ -99,6 +106,9 @@ int ss_oracle_fwd_init(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
 
         for (int64_t l = 0; l < seqlen; ++l) {
             const int64_t idx = row * seqlen + l;
+            if (reset && reset[b * seqlen + l]) /* a sequence starts at l: no carried state */
+                for (int64_t n = 0; n < dstate; ++n)
+                    h[n] = 0.0;
             /* §2.2: add the per-channel bias, then make delta positive. */
             double x = delta[idx];
             if (delta_bias)
@@ -126,6 +136,17 @@ int ss_oracle_fwd_init(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
         free(h);
     }
     return ok ? -1 : 0;
+}
+
+int ss_oracle_fwd_init(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                       const double *u, const double *delta, const double *A,
+                       const double *B, const double *C, const double *D,
+                       const double *z, const double *delta_bias, int delta_softplus,
+                       const double *initial_state, double *y, double *last_state,
+                       int nthreads)
+{
+    return ss_oracle_fwd_reset(batch, dim, seqlen, dstate, u, delta, A, B, C, D, z, delta_bias,
+                               delta_softplus, NULL, initial_state, y, last_state, nthreads);
 }
 
 /* The walkthrough's form: the state starts at zero. */

@@ -120,8 +120,11 @@ int segment(const ss_desc *desc, int nseg, int64_t *seg_len) {
 // split, about 7 warps per sub-partition) and the fix-up kernel joins.
 // Otherwise the steps are split across lanes (scan kernel): the smallest W
 // giving 3 warps per sub-partition, no more lanes than the sequence can feed,
-// and a block within half of an SM's shared memory.
-Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_bytes) {
+// and a block within half of an SM's shared memory.  direct_only (sequence
+// starts given, which only the direct kernel reads): the direct kernel with
+// the widest state split instead of the scan kernel.
+Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_bytes,
+               bool direct_only = false) {
     Plan pl{1, 0, 4, 1, desc->seqlen};
     if (rows <= 0 || desc->seqlen <= 0) return pl;
     const int64_t slots = (int64_t)sms * 4 * 32;  // lanes per "one warp per sub-partition"
@@ -143,6 +146,11 @@ Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_byte
         sp.nseg = segment(desc, (int)want, &sp.seg_len);
         if (sp.nseg >= 2 && workspace_for(desc, rows, sp) <= workspace_bytes) return sp;
     }
+    if (direct_only) {
+        pl.lanes = gmax;
+        pl.split = 1;
+        return pl;
+    }
     int w = 2;
     while (w < 32 && rows * w < 3 * slots) w *= 2;
     while (w > 2 && (int64_t)selscan::chunk_len(w) / 2 >= desc->seqlen) w /= 2;
@@ -156,8 +164,8 @@ Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_byte
 // The caller's launch config (zeros: the heuristic's choices) resolved into a
 // plan; SS_ERR_BAD_CONFIG for unsupported values.
 ss_status resolve(const ss_desc *desc, int64_t rows, const ss_launch_config *cfg,
-                  size_t workspace_bytes, Plan *out) {
-    Plan pl = heuristic(desc, rows, sm_count(), workspace_bytes);
+                  size_t workspace_bytes, Plan *out, bool direct_only = false) {
+    Plan pl = heuristic(desc, rows, sm_count(), workspace_bytes, direct_only);
     if (cfg) {
         const int lanes = cfg->lanes_per_row, warps = cfg->warps_per_block, split = cfg->split_states;
         if (lanes != 0 && (lanes < 1 || lanes > 32 || (lanes & (lanes - 1)) != 0)) return SS_ERR_BAD_CONFIG;
@@ -183,6 +191,7 @@ ss_status resolve(const ss_desc *desc, int64_t rows, const ss_launch_config *cfg
     if (direct && (pl.lanes > 8 || selscan::state_bucket((int)desc->dstate) / 2 < pl.lanes))
         return SS_ERR_BAD_CONFIG;
     if (pl.nseg > 1 && !direct) return SS_ERR_BAD_CONFIG;  // segments run in the direct kernel
+    if (direct_only && !direct) return SS_ERR_BAD_CONFIG;  // sequence starts: direct kernel only
     if (pl.nseg < 1) pl.nseg = 1;
     if (pl.nseg == 1) pl.seg_len = desc->seqlen;
     *out = pl;
@@ -239,14 +248,14 @@ cudaError_t launch_fixup(const ss_desc *desc, int64_t rows, int nseg, cudaStream
 ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D, const void *z,
                    const float *delta_bias, int delta_softplus, const float *initial_state,
-                   void *y, float *last_state, const ss_launch_config *cfg, void *workspace,
-                   size_t workspace_bytes, ss_stream_t stream) {
+                   const uint8_t *reset, void *y, float *last_state, const ss_launch_config *cfg,
+                   void *workspace, size_t workspace_bytes, ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
     if (!workspace) workspace_bytes = 0;
     Plan pl;
-    st = resolve(desc, sz.rows, cfg, workspace_bytes, &pl);
+    st = resolve(desc, sz.rows, cfg, workspace_bytes, &pl, reset != nullptr);
     if (st != SS_OK) return st;
     if (sz.rows == 0) return SS_OK;  // no rows: nothing to read or write
     const bool need_seq = desc->seqlen > 0;
@@ -292,6 +301,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.y = y;
     p.last_state = last_state;
     p.init_state = initial_state;
+    p.reset = reset;
     p.batch = desc->batch;
     p.dim = desc->dim;
     p.seqlen = desc->seqlen;
@@ -370,16 +380,16 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  const void *B, const void *C, const float *D, const void *z,
                  const float *delta_bias, int delta_softplus, void *y, float *last_state,
                  ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
-                    nullptr, nullptr, 0, stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y,
+                    last_state, nullptr, nullptr, 0, stream);
 }
 
 ss_status ss_fwd_ws(const ss_desc *desc, const void *u, const void *delta, const float *A,
                     const void *B, const void *C, const float *D, const void *z,
                     const float *delta_bias, int delta_softplus, void *y, float *last_state,
                     void *workspace, size_t workspace_bytes, ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
-                    nullptr, workspace, workspace_bytes, stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y,
+                    last_state, nullptr, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *delta,
@@ -388,8 +398,8 @@ ss_status ss_fwd_with_config(const ss_desc *desc, const void *u, const void *del
                              void *y, float *last_state, const ss_launch_config *config,
                              void *workspace, size_t workspace_bytes, ss_stream_t stream) {
     if (!config) return SS_ERR_NULL_POINTER;
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
-                    config, workspace, workspace_bytes, stream);
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y,
+                    last_state, config, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_fwd_state(const ss_desc *desc, const void *u, const void *delta, const float *A,
@@ -397,7 +407,18 @@ ss_status ss_fwd_state(const ss_desc *desc, const void *u, const void *delta, co
                        const float *delta_bias, int delta_softplus, const float *initial_state,
                        void *y, float *last_state, const ss_launch_config *config, void *workspace,
                        size_t workspace_bytes, ss_stream_t stream) {
-    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, y,
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, nullptr,
+                    y, last_state, config, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_fwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const uint8_t *reset,
+                       const float *initial_state, void *y, float *last_state,
+                       const ss_launch_config *config, void *workspace, size_t workspace_bytes,
+                       ss_stream_t stream) {
+    if (!reset && desc && desc->batch > 0 && desc->dim > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, reset, y,
                     last_state, config, workspace, workspace_bytes, stream);
 }
 
@@ -460,7 +481,7 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
         if (c.dst && c.bytes && cudaMemcpyAsync(c.dst, c.src, c.bytes, h2d, s) != cudaSuccess)
             return SS_ERR_CUDA;
     st = fwd_impl(desc, d_u, d_delta, d_A, d_B, d_C, d_D, d_z, d_delta_bias, delta_softplus, nullptr,
-                  d_y, d_last_state, nullptr, d_workspace, workspace_bytes, stream);
+                  nullptr, d_y, d_last_state, nullptr, d_workspace, workspace_bytes, stream);
     if (st != SS_OK) return st;
     if (n_y && cudaMemcpyAsync(h_y, d_y, n_y, d2h, s) != cudaSuccess) return SS_ERR_CUDA;
     if (d_last_state && cudaMemcpyAsync(h_last_state, d_last_state, n_last, d2h, s) != cudaSuccess)
@@ -551,7 +572,7 @@ ss_status ss_fwd_hostio_streams(const ss_desc *desc, const void *h_u, const void
         dc.batch = bc;
         st = fwd_impl(&dc, off(d_u, seq0 * ein), off(d_delta, seq0 * ein), d_A, off(d_B, bc0 * ein),
                       off(d_C, bc0 * ein), d_D, off(d_z, seq0 * ein), d_delta_bias, delta_softplus, nullptr,
-                      off(d_y, seq0 * eout), static_cast<float *>(off(d_last_state, st0 * 4)), nullptr,
+                      nullptr, off(d_y, seq0 * eout), static_cast<float *>(off(d_last_state, st0 * 4)), nullptr,
                       d_workspace ? off(d_workspace, (size_t)k * ws_share) : nullptr,
                       d_workspace ? ws_share : 0, reinterpret_cast<ss_stream_t>(sk));
         if (st != SS_OK) return cleanup(), st;

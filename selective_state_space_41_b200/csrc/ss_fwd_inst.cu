@@ -44,6 +44,11 @@ cudaError_t launch_direct(dim3 grid, dim3 block, size_t smem, cudaStream_t s, co
     if constexpr (SS_INST_NMAX / 2 / kG < 1) {
         return cudaErrorInvalidValue;  // fewer state pairs than lanes
     } else {
+        if (p.reset) {  // the instance that reads the sequence starts
+            static bool opted_in_reset[kMaxDevices];
+            return launch_kernel(ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kG, true>,
+                                 grid, block, smem, s, p, opted_in_reset);
+        }
         static bool opted_in[kMaxDevices];
         return launch_kernel(ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kG>, grid,
                              block, smem, s, p, opted_in);
@@ -63,6 +68,7 @@ cudaError_t SS_INST_NAME(int lanes, int split_states, dim3 grid, dim3 block, siz
             default: return cudaErrorInvalidValue;
         }
     }
+    if (p.reset) return cudaErrorInvalidValue;  // the scan kernel does not read sequence starts
     switch (lanes) {
         case 2: return launch_scan<2>(grid, block, smem, s, p);
         case 4: return launch_scan<4>(grid, block, smem, s, p);

@@ -49,6 +49,10 @@ struct FwdParams {
     void *y;
     float *last_state;
     const float *init_state;  // (batch, dim, dstate) state before step 0, or null (zero)
+    // (batch, seqlen) bytes, or null: nonzero at (b, l) means a new sequence
+    // starts at step l, so the state entering step l is zero (direct kernel
+    // and fix-up only).
+    const uint8_t *reset;
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;     // 1: softplus, 0: exp
@@ -58,7 +62,8 @@ struct FwdParams {
     // seg_len steps from a zero state (the first one from init_state, if
     // given) and records, per (segment, row), the
     // end state (ws_hend, N floats) and the sum of delta' (ws_dsum) for the
-    // fix-up kernel, which adds the carried state's share of y.
+    // fix-up kernel, which adds the carried state's share of y.  A segment
+    // holding a reset records -1 as its delta' sum: it passes no state on.
     int64_t seg_len;
     int nseg;
     float *ws_hend, *ws_dsum;
@@ -772,7 +777,9 @@ struct DirectOccupancy {
 #define SS_DIRECT_BOUNDS(SPL) __launch_bounds__(256, DirectOccupancy<SPL>::kMinBlocks)
 #endif
 
-template <typename Tin, typename Tout, int kNmax, int kG>
+// kReset: the instance that reads p.reset (sequence starts inside the rows);
+// the other one has no code for it.
+template <typename Tin, typename Tout, int kNmax, int kG, bool kReset = false>
 __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParams p) {
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                        // state pairs per lane
@@ -857,6 +864,8 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     }
     const float Dd = p.D ? p.D[d] : 0.f;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
+    const uint8_t *const reset_b = kReset ? p.reset + b * L : nullptr;  // this batch entry's starts
+    bool seg_reset = false;  // a sequence starts inside this segment
 
     auto stage_fast = [&](int64_t c0) { return vec && c0 + kDirectStage <= Lend; };
     auto issue_copies = [&](int64_t c0, Tin *RB) {
@@ -981,6 +990,21 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
             load_own_checked(d_own, s_next, wd);
             if (has_z) load_own_checked(z_own, s_next, wz);
         }
+        // Bit i: a sequence starts at step l0 + i (the state entering it is
+        // zero).  Each lane reads its owned steps; the row's lanes (and so the
+        // warp, whose rows share the batch entry) end up with the same mask.
+        uint32_t rmask = 0u;
+        if constexpr (kReset) {
+            const int64_t s0 = l0 + g * kOwn;
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i)
+                if (s0 + i < Lend && reset_b[s0 + i] != 0) rmask |= 1u << (g * kOwn + i);
+            if constexpr (kG > 1) {
+#pragma unroll
+                for (int off = 1; off < kG; off *= 2) rmask |= __shfl_xor_sync(0xffffffffu, rmask, off, kG);
+            }
+            seg_reset |= rmask != 0u;
+        }
         // delta' and delta' u of the owned steps (past L: the identity step).
         float dl_own[kOwn], du_own[kOwn], uo[kOwn];
 #pragma unroll
@@ -1044,6 +1068,9 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
                 }
                 const float2 t = __fmul2_rn(d2, A2_of(qq));
                 const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
+                if constexpr (kReset) {
+                    if ((rmask >> i) & 1u) h[qq] = make_float2(0.f, 0.f);
+                }
                 h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
                 acc[qq % kAccs] = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc[qq % kAccs]);
             }
@@ -1135,7 +1162,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
                 if (n < N) p.ws_hend[rec * N + n] = h[qq].x;
                 if (n + 1 < N) p.ws_hend[rec * N + n + 1] = h[qq].y;
             }
-            if (g == 0) p.ws_dsum[rec] = dsum;
+            if (g == 0) p.ws_dsum[rec] = (kReset && seg_reset) ? -1.f : dsum;
         }
     } else if (p.last_state != nullptr && row_ok) {
 #pragma unroll
@@ -1156,8 +1183,11 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 // over the segment up to and including l (linearity of the recurrence in h).
 // One thread per (row, segment) adds that share to y step by step; it stops
 // once every state's exponent A_n log2e S_l is below -127, where ex2.ftz
-// returns exactly 0, so the remaining shares are exactly zero.  Thread
-// (row, segment 0) instead writes the last state h_in(nseg) when asked.
+// returns exactly 0, so the remaining shares are exactly zero, or at the
+// segment's first sequence start (p.reset), where the carried state is
+// dropped; a segment holding a start passes no state on (P = 0, recorded as
+// a delta' sum of -1).  Thread (row, segment 0) instead writes the last
+// state h_in(nseg) when asked.
 // Threads: kT = kNmax/4 per (row, segment), 4 states each; they share the
 // step loop (each computes the same delta' sums, so they stop together) and
 // add their shares of the correction by shuffles within their group.
@@ -1197,7 +1227,7 @@ __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
 #pragma unroll
         for (int k = 0; k < kS; ++k) {
             const int n = q * kS + k;
-            if (n < N) h[k] = fmaf(sfu_exp2(A2[k] * ds), h[k], p.ws_hend[rec * N + n]);
+            if (n < N) h[k] = fmaf(ds < 0.f ? 0.f : sfu_exp2(A2[k] * ds), h[k], p.ws_hend[rec * N + n]);
         }
     }
     if (s == 0) {
@@ -1215,10 +1245,12 @@ __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
     Tout *y_row = static_cast<Tout *>(p.y) + row * L;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
     const bool softplus = p.softplus != 0;
+    const uint8_t *const reset_b = p.reset ? p.reset + b * L : nullptr;
     const int64_t c_begin = (int64_t)s * p.seg_len;
     const int64_t c_end = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
     float S = 0.f;
     for (int64_t l = c_begin; l < c_end; ++l) {
+        if (reset_b && reset_b[l] != 0) break;  // a new sequence: the carried state ends here
         S += delta_transform<kFast>(static_cast<float>(dl_row[l]) + bias, softplus);
         if (A2max * S < -127.f) break;  // every 2^(A2 S) is 0 from here on
         float corr = 0.f;

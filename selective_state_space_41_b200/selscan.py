@@ -8,10 +8,10 @@ fails to load, every call raises.
 
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``,
-``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
+``ss_fwd_reset``, ``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
 ``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
 ``ss_status_string``, ``ss_version``); ``ss_fwd`` dispatches to the
-workspace, config and initial-state forms by keyword, ``ss_fwd_hostio`` to
+workspace, config, initial-state and sequence-start forms by keyword, ``ss_fwd_hostio`` to
 the pipelined form when given streams.  ``selective_scan_fwd`` and
 ``selective_scan_bwd`` are the allocate-and-call convenience forms, with the
 argument order of the walkthrough's selective_scan_ref
@@ -36,7 +36,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Names the header declares; the ABI test checks each is exported.
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
-           "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc", "ss_step", "ss_bwd", "ss_bwd_workspace_bytes",
+           "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc", "ss_step", "ss_bwd", "ss_bwd_workspace_bytes",
            "ss_status_string", "ss_version")
 
 
@@ -82,6 +82,8 @@ def lib():
         L.ss_fwd_with_config.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, CP, P, SZ, P]
         L.ss_fwd_state.restype = I
         L.ss_fwd_state.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P, CP, P, SZ, P]
+        L.ss_fwd_reset.restype = I
+        L.ss_fwd_reset.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P, P, CP, P, SZ, P]
         L.ss_fwd_heuristic.restype = I
         L.ss_fwd_heuristic.argtypes = [DP, SZ, CP]
         L.ss_fwd_hostio.restype = I
@@ -149,7 +151,7 @@ def _config(lanes_per_row, split_states, warps_per_block, segments):
 
 def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
            last_state=None, stream=None, workspace=None, lanes_per_row=None, warps_per_block=None,
-           split_states=False, segments=None, initial_state=None):
+           split_states=False, segments=None, initial_state=None, reset=None):
     """Queue the forward on ``stream`` (default: the current stream).
 
     u, delta, z, y: (batch, dim, L); A: (dim, N) float32; B, C: (batch, N, L);
@@ -157,8 +159,9 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
     float32.  ``workspace`` (a CUDA tensor, e.g. uint8 of
     ss_fwd_workspace_bytes()) selects ``ss_fwd_ws``; ``lanes_per_row`` /
     ``split_states`` / ``warps_per_block`` / ``segments`` select
-    ``ss_fwd_with_config``; ``initial_state`` selects ``ss_fwd_state``.
-    Raises SelscanError on a rejected call.
+    ``ss_fwd_with_config``; ``initial_state`` selects ``ss_fwd_state``;
+    ``reset`` ((batch, L) uint8 or bool, nonzero where a new sequence starts)
+    selects ``ss_fwd_reset``.  Raises SelscanError on a rejected call.
     """
     u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
     if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
@@ -172,7 +175,17 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     s = _stream_handle(stream, u.device)
     cfg = _config(lanes_per_row, split_states, warps_per_block, segments)
-    if initial_state is not None:
+    if initial_state is not None and not initial_state.is_contiguous():
+        raise ValueError("initial_state must be contiguous")
+    if reset is not None:
+        if reset.dtype == torch.bool:
+            reset = reset.view(torch.uint8)
+        if reset.dtype != torch.uint8 or tuple(reset.shape) != (batch, L) or not reset.is_contiguous():
+            raise ValueError("reset must be a contiguous (batch, L) uint8 or bool tensor")
+        reset_args = args[:10] + (_ptr(reset), _ptr(initial_state)) + args[10:]
+        _check(lib().ss_fwd_reset(*reset_args, ctypes.byref(cfg) if cfg is not None else None, ws,
+                                  ws_bytes, s), "ss_fwd_reset")
+    elif initial_state is not None:
         if not initial_state.is_contiguous():
             raise ValueError("initial_state must be contiguous")
         state_args = args[:10] + (_ptr(initial_state),) + args[10:]
@@ -322,11 +335,13 @@ def ss_fwd_hostio(host: dict, dev: dict, delta_softplus=False, stream=None, work
 
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
-                       return_last_state=False, out_dtype=None, stream=None, initial_state=None):
+                       return_last_state=False, out_dtype=None, stream=None, initial_state=None,
+                       reset=None):
     """y (and the last state) of the selective scan, computed by libselscan.
 
     Same arguments as the walkthrough's selective_scan_ref, plus the z gate
-    and an optional float32 (batch, dim, N) state before step 0.  Inputs must
+    and an optional float32 (batch, dim, N) state before step 0 and (batch, L)
+    mask of sequence starts (the state entering a start is zero).  Inputs must
     be CUDA tensors; y is allocated in ``out_dtype`` (default: u's dtype),
     last_state in float32.
     """
@@ -339,5 +354,5 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
             if return_last_state else None)
     ws = workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=u.device)
     ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
-           last_state=last, stream=stream, workspace=ws, initial_state=initial_state)
+           last_state=last, stream=stream, workspace=ws, initial_state=initial_state, reset=reset)
     return (y, last) if return_last_state else y

@@ -379,7 +379,88 @@ def pin_initial_state_continuity(scan):
         _assert_close(h2, last, 1e-13, f"pieces at {k}: last state")
 
 
+# ---- sequence starts (extension: the boundary reset of "Mamba实战：如何用选择性
+# 状态空间模型提升你的长序列处理效率（附代码）" §2; the state entering a start is zero).
+
+def pin_reset_pieces(scan):
+    """Rows holding several sequences: with starts marked, y over each piece
+    and the last state equal independent runs of the pieces (each from the
+    zero state, the first one from the given initial state unless a start
+    sits at step 0), batch entry by batch entry."""
+    rng = np.random.default_rng(37)
+    Bt, Dm, L, N = 2, 3, 40, 4
+    u = _rand(rng, Bt, Dm, L)
+    delta = _rand(rng, Bt, Dm, L)
+    A = -rng.uniform(0.05, 1.0, size=(Dm, N))
+    Bm = _rand(rng, Bt, N, L)
+    C = _rand(rng, Bt, N, L)
+    Dv = _rand(rng, Dm)
+    z = _rand(rng, Bt, Dm, L)
+    bias = _rand(rng, Dm) * 0.3
+    h0 = _rand(rng, Bt, Dm, N)
+    starts = {0: [7, 8, 23], 1: [0, 15, 39]}
+    reset = np.zeros((Bt, L), dtype=np.uint8)
+    for b, ls in starts.items():
+        reset[b, ls] = 1
+    kw = dict(D=Dv, delta_bias=bias, delta_softplus=True, return_last_state=True)
+    y, last = scan(u, delta, A, Bm, C, z=z, initial_state=h0, reset=reset, **kw)
+    for b, ls in starts.items():
+        cuts = [0] + [l for l in ls if l > 0] + [L]
+        for k in range(len(cuts) - 1):
+            lo, hi = cuts[k], cuts[k + 1]
+            first_from_h0 = lo == 0 and 0 not in ls
+            yp, hp = scan(u[b:b + 1, :, lo:hi], delta[b:b + 1, :, lo:hi], A, Bm[b:b + 1, :, lo:hi],
+                          C[b:b + 1, :, lo:hi], z=z[b:b + 1, :, lo:hi],
+                          initial_state=h0[b:b + 1] if first_from_h0 else None, **kw)
+            _assert_close(y[b:b + 1, :, lo:hi], yp, 1e-15, f"batch {b} piece [{lo}, {hi}): y")
+        _assert_close(last[b:b + 1], hp, 1e-15, f"batch {b}: last state")
+
+
+def pin_reset_every_step(scan):
+    """A start at every step leaves no memory: y_l = (sum_n C[n,l] delta'_l
+    B[n,l] u_l + D u_l) silu(z_l), and the last state is delta'_L B[:,L] u_L."""
+    rng = np.random.default_rng(41)
+    Bt, Dm, L, N = 2, 3, 12, 5
+    u = _rand(rng, Bt, Dm, L)
+    delta = _rand(rng, Bt, Dm, L)
+    A = -rng.uniform(0.05, 1.0, size=(Dm, N))
+    Bm = _rand(rng, Bt, N, L)
+    C = _rand(rng, Bt, N, L)
+    Dv = _rand(rng, Dm)
+    z = _rand(rng, Bt, Dm, L)
+    h0 = _rand(rng, Bt, Dm, N)
+    y, last = scan(u, delta, A, Bm, C, D=Dv, z=z, delta_softplus=True, return_last_state=True,
+                   initial_state=h0, reset=np.ones((Bt, L), dtype=np.uint8))
+    dl = _softplus_ref(delta)
+    h = dl[:, :, None, :] * Bm[:, None, :, :] * u[:, :, None, :]       # (b, d, n, l)
+    want = ((C[:, None, :, :] * h).sum(2) + Dv[None, :, None] * u) * _silu_ref(z)
+    _assert_close(y, want, 1e-13, "start at every step: y")
+    _assert_close(last, h[..., -1], 1e-13, "start at every step: last state")
+
+
+def pin_reset_none(scan):
+    """An all-zero start mask is no mask; a single start changes y from that
+    step on and not before it."""
+    rng = np.random.default_rng(43)
+    Bt, Dm, L, N = 2, 2, 20, 3
+    u = _rand(rng, Bt, Dm, L)
+    delta = _rand(rng, Bt, Dm, L)
+    A = -rng.uniform(0.05, 1.0, size=(Dm, N))
+    Bm = _rand(rng, Bt, N, L)
+    C = _rand(rng, Bt, N, L)
+    y = scan(u, delta, A, Bm, C, delta_softplus=True)
+    y0 = scan(u, delta, A, Bm, C, delta_softplus=True, reset=np.zeros((Bt, L), dtype=np.uint8))
+    assert np.array_equal(y, y0), "all-zero start mask must be no mask"
+    one = np.zeros((Bt, L), dtype=np.uint8)
+    one[1, 9] = 1
+    y1 = scan(u, delta, A, Bm, C, delta_softplus=True, reset=one)
+    assert np.array_equal(y1[0], y[0]) and np.array_equal(y1[1, :, :9], y[1, :, :9]), \
+        "a start must not change other batch entries or earlier steps"
+    assert np.all(y1[1, :, 9] != y[1, :, 9]), "a start must change its own step"
+
+
 ALL_PINS = [pin_hand_worked, pin_delta_transform, pin_closed_form, pin_brute_force,
             pin_lfilter, pin_delta_to_zero, pin_causality, pin_linearity,
             pin_state_separability, pin_last_state, pin_initial_state_closed_form,
-            pin_initial_state_brute_force, pin_initial_state_continuity]
+            pin_initial_state_brute_force, pin_initial_state_continuity, pin_reset_pieces,
+            pin_reset_every_step, pin_reset_none]

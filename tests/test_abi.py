@@ -138,6 +138,22 @@ def test_state_entry_rejections(lib):
     assert lib.ss_fwd_state(None, *head[1:], FAKE, FAKE, None, None, None, 0, None) == 1
 
 
+def test_reset_entry_rejections(lib):
+    """ss_fwd_reset: no mask for a non-empty problem, a config asking for the
+    scan kernel (which reads no sequence starts), a misaligned initial state
+    and no descriptor are rejected before any launch; an empty problem needs
+    no mask."""
+    d = _desc(seqlen=64, dstate=4)
+    head = (ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1)
+    assert lib.ss_fwd_reset(*head, None, None, FAKE, None, None, None, 0, None) == 1
+    assert lib.ss_fwd_reset(*head, FAKE, None, FAKE, None, _cfg(4, 0, 4), None, 0, None) == 7
+    assert lib.ss_fwd_reset(*head, FAKE, ODD, FAKE, None, None, None, 0, None) == 5
+    assert lib.ss_fwd_reset(None, *head[1:], FAKE, None, FAKE, None, None, None, 0, None) == 1
+    empty = _desc(batch=0, seqlen=64, dstate=4)
+    assert lib.ss_fwd_reset(ctypes.byref(empty), *head[1:], None, None, None, None, None, None, 0,
+                            None) == 0
+
+
 def test_bwd_rejections(lib):
     """ss_bwd rejects before any launch (the pointers are fake): no
     descriptor, more than 64 states, a missing gradient output, no workspace.

@@ -33,6 +33,11 @@ MUTANTS = {
     "initial_state_ignored": ("h[n] = initial_state ? initial_state[row * dstate + n] : 0.0;",
                               "h[n] = 0.0;"),
     "initial_state_transposed": ("initial_state[row * dstate + n]", "initial_state[n * dim * batch + row]"),
+    "reset_ignored": ("if (reset && reset[b * seqlen + l])", "if (0)"),
+    "reset_one_step_late": ("reset[b * seqlen + l])", "reset[b * seqlen + (l > 0 ? l - 1 : 0)])"),
+    "reset_wrong_batch_entry": ("reset[b * seqlen + l])", "reset[(batch - 1 - b) * seqlen + l])"),
+    "reset_keeps_one_state": ("                for (int64_t n = 0; n < dstate; ++n)\n                    h[n] = 0.0;",
+                              "                for (int64_t n = 1; n < dstate; ++n)\n                    h[n] = 0.0;"),
 }
 
 
