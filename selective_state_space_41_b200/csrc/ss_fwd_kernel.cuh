@@ -950,6 +950,16 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     };
 
     uint32_t wu[kOwnWords], wd[kOwnWords], wz[kOwnWords];
+    // Start flags of this lane's owned steps of the coming sub-chunk (loaded
+    // one sub-chunk ahead, like u, delta and z).
+    uint8_t rb[kReset ? kOwn : 1];
+    auto load_starts = [&](int64_t s0) {
+        if constexpr (kReset) {
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) rb[i] = s0 + i < Lend ? reset_b[s0 + i] : (uint8_t)0;
+        }
+    };
+    load_starts(c_begin + g * kOwn);
     load_own_checked(u_own, c_begin + g * kOwn, wu);
     load_own_checked(d_own, c_begin + g * kOwn, wd);
     if (has_z) load_own_checked(z_own, c_begin + g * kOwn, wz);
@@ -995,10 +1005,10 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         // warp, whose rows share the batch entry) end up with the same mask.
         uint32_t rmask = 0u;
         if constexpr (kReset) {
-            const int64_t s0 = l0 + g * kOwn;
 #pragma unroll
             for (int i = 0; i < kOwn; ++i)
-                if (s0 + i < Lend && reset_b[s0 + i] != 0) rmask |= 1u << (g * kOwn + i);
+                if (rb[i] != 0) rmask |= 1u << (g * kOwn + i);
+            load_starts(s_next);
             if constexpr (kG > 1) {
 #pragma unroll
                 for (int off = 1; off < kG; off *= 2) rmask |= __shfl_xor_sync(0xffffffffu, rmask, off, kG);
@@ -1046,36 +1056,48 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
             const int n = 2 * (q0 + qq);
             return make_float2(n < N ? __ldg(A_d + n) * kLog2e : 0.f, n + 1 < N ? __ldg(A_d + n + 1) * kLog2e : 0.f);
         };
+        // The state loop; with_starts: a start in this sub-chunk (zero the
+        // state entering it).  The mask is warp-uniform, so a sub-chunk
+        // without one takes the plain loop.
+        auto steps = [&](auto with_starts) {
+            constexpr bool kStarts = decltype(with_starts)::value;
 #pragma unroll
-        for (int i = 0; i < kDirectSub; ++i) {
-            const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
-            float2 acc[kAccs];
+            for (int i = 0; i < kDirectSub; ++i) {
+                const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
+                float2 acc[kAccs];
 #pragma unroll
-            for (int k = 0; k < kAccs; ++k) acc[k] = make_float2(0.f, 0.f);
+                for (int k = 0; k < kAccs; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int qq = 0; qq < kPL; ++qq) {
-                float4 bc;  // (B_n, B_n+1, C_n, C_n+1) of this step and state pair
-                if constexpr (kHalf) {
-                    const float2 bb = FmB[i * kPairs + qq];
-                    const uint32_t cw = FmC[i * kPairs + qq];
-                    bc = make_float4(bb.x, bb.y, __uint_as_float(cw << 16), __uint_as_float(cw & 0xffff0000u));
-                } else if constexpr (kPack) {
-                    const uint2 w = Fm2[i * kPairs + qq];
-                    bc = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
-                                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
-                } else {
-                    bc = Fm[i * kPairs + qq];
+                for (int qq = 0; qq < kPL; ++qq) {
+                    float4 bc;  // (B_n, B_n+1, C_n, C_n+1) of this step and state pair
+                    if constexpr (kHalf) {
+                        const float2 bb = FmB[i * kPairs + qq];
+                        const uint32_t cw = FmC[i * kPairs + qq];
+                        bc = make_float4(bb.x, bb.y, __uint_as_float(cw << 16), __uint_as_float(cw & 0xffff0000u));
+                    } else if constexpr (kPack) {
+                        const uint2 w = Fm2[i * kPairs + qq];
+                        bc = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                                         __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+                    } else {
+                        bc = Fm[i * kPairs + qq];
+                    }
+                    const float2 t = __fmul2_rn(d2, A2_of(qq));
+                    const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
+                    if constexpr (kStarts) {
+                        if ((rmask >> i) & 1u) h[qq] = make_float2(0.f, 0.f);
+                    }
+                    h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
+                    acc[qq % kAccs] = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc[qq % kAccs]);
                 }
-                const float2 t = __fmul2_rn(d2, A2_of(qq));
-                const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
-                if constexpr (kReset) {
-                    if ((rmask >> i) & 1u) h[qq] = make_float2(0.f, 0.f);
-                }
-                h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
-                acc[qq % kAccs] = __ffma2_rn(make_float2(bc.z, bc.w), h[qq], acc[qq % kAccs]);
+                if constexpr (kAccs == 2) acc[0] = __fadd2_rn(acc[0], acc[1]);
+                part[i] = acc[0].x + acc[0].y;
             }
-            if constexpr (kAccs == 2) acc[0] = __fadd2_rn(acc[0], acc[1]);
-            part[i] = acc[0].x + acc[0].y;
+        };
+        if constexpr (kReset) {
+            if (rmask != 0u) steps(std::true_type{});
+            else steps(std::false_type{});
+        } else {
+            steps(std::false_type{});
         }
         // Totals of the owned steps.
         float yv[kOwn];
