@@ -308,7 +308,22 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
                  size_t workspace_bytes, ss_stream_t stream);
 
-/* Bytes of workspace ss_bwd needs for `desc` (0 for an invalid descriptor). */
+/*
+ * ss_bwd for a forward run with sequence starts (ss_fwd_reset): the same
+ * gradients, with `reset` the forward's (B, L) byte mask (required when
+ * B*D*L > 0, SS_ERR_NULL_POINTER otherwise).  At a start l the state h_(l-1)
+ * has no part in h_l, so no adjoint passes from step l to l-1 and the
+ * h_(l-1) terms of ddelta and dA vanish there.  Workspace as ss_bwd
+ * (ss_bwd_workspace_bytes); other arguments and errors as ss_bwd.
+ */
+ss_status ss_bwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const uint8_t *reset,
+                       const void *dy, void *du, void *ddelta, float *dA, float *dB, float *dC,
+                       float *dD, void *dz, float *ddelta_bias, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream);
+
+/* Bytes of workspace ss_bwd and ss_bwd_reset need for `desc` (0 for an invalid descriptor). */
 size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 
 /*

@@ -36,6 +36,9 @@ def _load(path=None):
         lib.ss_oracle_fwd_init.argtypes = [i64, i64, i64, i64, P, P, P, P, P, P, P, P,
                                            ctypes.c_int, P, P, P, ctypes.c_int]
         if hasattr(lib, "ss_oracle_bwd"):  # (a planted-mistake build of the forward alone has none)
+            lib.ss_oracle_bwd_reset.restype = ctypes.c_int
+            lib.ss_oracle_bwd_reset.argtypes = [i64, i64, i64, i64] + [P] * 8 + [ctypes.c_int] + \
+                [P] * 10 + [ctypes.c_int]
             lib.ss_oracle_bwd.restype = ctypes.c_int
             lib.ss_oracle_bwd.argtypes = [i64, i64, i64, i64] + [P] * 8 + [ctypes.c_int] + [P] * 9 + \
                 [ctypes.c_int]
@@ -122,11 +125,11 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-                       delta_softplus=False, nthreads=0, lib=None):
+                       delta_softplus=False, nthreads=0, lib=None, reset=None):
     """Gradients of sum(dy * y) for the forward of ``selective_scan`` (state
-    starting at zero), in float64, as a dict: du, ddelta, dz (batch, dim, L);
-    dA (dim, N); dB, dC (batch, N, L); dD, ddelta_bias (dim,).  The entries
-    of absent optional operands are None."""
+    starting at zero; ``reset`` as there), in float64, as a dict: du, ddelta,
+    dz (batch, dim, L); dA (dim, N); dB, dC (batch, N, L); dD, ddelta_bias
+    (dim,).  The entries of absent optional operands are None."""
     u, delta, A, B, C, dy = (_f64(t) for t in (u, delta, A, B, C, dy))
     D, z, delta_bias = _f64(D), _f64(z), _f64(delta_bias)
     batch, dim, L = u.shape
@@ -140,11 +143,17 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
          "dD": np.zeros(dim) if D is not None else None,
          "dz": np.zeros_like(u) if z is not None else None,
          "ddelta_bias": np.zeros(dim) if delta_bias is not None else None}
-    rc = _load(lib).ss_oracle_bwd(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
-                                  _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0,
-                                  _ptr(dy), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]),
-                                  _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]),
-                                  _ptr(g["ddelta_bias"]), int(nthreads))
+    rs = None
+    if reset is not None:
+        rs = np.ascontiguousarray(np.asarray(reset) != 0, dtype=np.uint8)
+        if rs.shape != (batch, L):
+            raise ValueError("bad reset shape")
+    rc = _load(lib).ss_oracle_bwd_reset(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                                        _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                                        1 if delta_softplus else 0, _ptr(rs), _ptr(dy), _ptr(g["du"]),
+                                        _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+                                        _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]),
+                                        int(nthreads))
     if rc != 0:
         raise RuntimeError("oracle rejected its arguments")
     return g

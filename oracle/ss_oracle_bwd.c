@@ -26,6 +26,9 @@
  *              dd_l d_l in exp mode),   dbias += ddelta_l (summed over b and l).
  * Sums over rows are done in a fixed order, so results do not depend on the
  * thread count.
+ * With sequence starts (the reset mask of ss_oracle.c: the state entering a
+ * start is zero), h_(l-1) has no part in h_l at a start l, so there the
+ * h_(l-1) terms of dd_l and dA vanish and no adjoint passes from l to l-1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -41,13 +44,13 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 /* Returns 0 on success, -1 on a bad argument or allocation failure.
  * Required: u, delta, A, B, C, dy, du, ddelta, dA, dB, dC.  dD is required
  * when D is given, dz when z is, ddelta_bias when delta_bias is. */
-int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
-                  const double *u, const double *delta, const double *A,
-                  const double *B, const double *C, const double *D,
-                  const double *z, const double *delta_bias, int delta_softplus,
-                  const double *dy, double *du, double *ddelta, double *dA,
-                  double *dB, double *dC, double *dD, double *dz,
-                  double *ddelta_bias, int nthreads)
+int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                        const double *u, const double *delta, const double *A,
+                        const double *B, const double *C, const double *D,
+                        const double *z, const double *delta_bias, int delta_softplus,
+                        const uint8_t *reset, const double *dy, double *du, double *ddelta,
+                        double *dA, double *dB, double *dC, double *dD, double *dz,
+                        double *ddelta_bias, int nthreads)
 {
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1)
         return -1;
@@ -93,6 +96,7 @@ int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                 h[n] = 0.0;
             for (int64_t l = 0; l < L; ++l) {
                 const int64_t idx = row * L + l;
+                const int keep = !(reset && reset[b * L + l]); /* 0 at a sequence start */
                 double x = delta[idx];
                 if (delta_bias)
                     x += delta_bias[d];
@@ -102,7 +106,7 @@ int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                 for (int64_t n = 0; n < N; ++n) {
                     const int64_t bn = (b * N + n) * L + l;
                     const double a = exp(dl[l] * A[d * N + n]);
-                    h[(l + 1) * N + n] = a * h[l * N + n] + dl[l] * B[bn] * u[idx];
+                    h[(l + 1) * N + n] = a * (keep ? h[l * N + n] : 0.0) + dl[l] * B[bn] * u[idx];
                     acc += C[bn] * h[(l + 1) * N + n];
                 }
                 if (D)
@@ -114,6 +118,7 @@ int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                 carry[n] = 0.0; /* a_(l+1) lam_(l+1), zero past the end */
             for (int64_t l = L - 1; l >= 0; --l) {
                 const int64_t idx = row * L + l;
+                const int keep = !(reset && reset[b * L + l]);
                 double g = dy[idx];
                 if (z) {
                     const double sg = sigmoid(z[idx]);
@@ -131,10 +136,10 @@ int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                     dC[bn] += g * h[(l + 1) * N + n];
                     dB[bn] += lam * dl[l] * u[idx];
                     dui += lam * dl[l] * B[bn];
-                    const double da = lam * h[l * N + n];
+                    const double da = keep ? lam * h[l * N + n] : 0.0;
                     ddl += lam * B[bn] * u[idx] + da * a * A[d * N + n];
                     pA[row * N + n] += da * a * dl[l];
-                    carry[n] = a * lam;
+                    carry[n] = keep ? a * lam : 0.0;
                 }
                 du[idx] = dui;
                 const double dx = delta_softplus ? ddl * (xs[l] > 20.0 ? 1.0 : sigmoid(xs[l]))
@@ -162,4 +167,18 @@ int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
     }
     free(pA), free(pD), free(pbias);
     return bad ? -1 : 0;
+}
+
+/* The walkthrough's form: no sequence starts. */
+int ss_oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                  const double *u, const double *delta, const double *A,
+                  const double *B, const double *C, const double *D,
+                  const double *z, const double *delta_bias, int delta_softplus,
+                  const double *dy, double *du, double *ddelta, double *dA,
+                  double *dB, double *dC, double *dD, double *dz,
+                  double *ddelta_bias, int nthreads)
+{
+    return ss_oracle_bwd_reset(batch, dim, seqlen, dstate, u, delta, A, B, C, D, z, delta_bias,
+                               delta_softplus, NULL, dy, du, ddelta, dA, dB, dC, dD, dz,
+                               ddelta_bias, nthreads);
 }

@@ -593,11 +593,15 @@ size_t ss_bwd_workspace_bytes(const ss_desc *desc) {
     return bwd_layout(desc, sz).total;
 }
 
-ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
-                 const void *C, const float *D, const void *z, const float *delta_bias,
-                 int delta_softplus, const void *dy, void *du, void *ddelta, float *dA, float *dB,
-                 float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
-                 size_t workspace_bytes, ss_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                   const void *C, const float *D, const void *z, const float *delta_bias,
+                   int delta_softplus, const uint8_t *reset, const void *dy, void *du, void *ddelta,
+                   float *dA, float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                   void *workspace, size_t workspace_bytes, ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
@@ -638,6 +642,8 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  (!dy || aligned(dy, 16));
     p.dtiles = lo.dtiles;
     p.nsub = lo.nsub;
+    p.reset = reset;
+    p.reset_vec = reset && desc->seqlen % selscan::kBwdSub == 0 && aligned(reset, selscan::kBwdSub);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int nmax = selscan::state_bucket(p.dstate), n = nmax;
@@ -663,6 +669,30 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
         if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
     }
     return SS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                 const void *C, const float *D, const void *z, const float *delta_bias,
+                 int delta_softplus, const void *dy, void *du, void *ddelta, float *dA, float *dB,
+                 float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
+                 size_t workspace_bytes, ss_stream_t stream) {
+    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, dy, du, ddelta,
+                    dA, dB, dC, dD, dz, ddelta_bias, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_bwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const uint8_t *reset,
+                       const void *dy, void *du, void *ddelta, float *dA, float *dB, float *dC,
+                       float *dD, void *dz, float *ddelta_bias, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream) {
+    if (!reset && desc && desc->batch > 0 && desc->dim > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
+    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, reset, dy, du, ddelta,
+                    dA, dB, dC, dD, dz, ddelta_bias, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_step(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,

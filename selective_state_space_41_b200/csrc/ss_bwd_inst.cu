@@ -8,10 +8,13 @@
 
 namespace selscan {
 
-cudaError_t SS_INST_NAME(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const BwdParams &p) {
+namespace {
+
+template <bool kReset>
+cudaError_t launch(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const BwdParams &p) {
     constexpr int kMaxDevices = 64;
     static bool opted_in[kMaxDevices];
-    auto kernel = ss_bwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX>;
+    auto kernel = ss_bwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kReset>;
     if (smem > 48 * 1024) {  // above the default a kernel opts in to more dynamic shared memory, once per device
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
@@ -24,6 +27,13 @@ cudaError_t SS_INST_NAME(dim3 grid, dim3 block, size_t smem, cudaStream_t s, con
     }
     kernel<<<grid, block, smem, s>>>(p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// The instance that reads sequence starts when p.reset is given.
+cudaError_t SS_INST_NAME(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const BwdParams &p) {
+    return p.reset ? launch<true>(grid, block, smem, s, p) : launch<false>(grid, block, smem, s, p);
 }
 
 }  // namespace selscan

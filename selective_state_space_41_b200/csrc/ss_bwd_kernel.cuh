@@ -24,6 +24,10 @@
 //   lanes and the dB/dC terms over the block's rows in shared memory, and
 //   writes per-block partial sums of dB/dC, which a second kernel adds up in
 //   a fixed order (with the per-row partials of dA, dD and dbias).
+// With sequence starts (p.reset, the forward's (batch, L) mask: the state
+// entering a start is zero), h_(l-1) has no part in h_l at a start l: both
+// passes zero the state entering it, and the adjoint passes nothing from l to
+// l-1 and has no h_(l-1) term there (ddelta', dA).
 #pragma once
 
 #include <type_traits>
@@ -47,6 +51,8 @@ struct BwdParams {
     int vec_rows;                             // every row of u, delta, z and dy starts 16-byte aligned
     int64_t dtiles;                           // row tiles per batch entry
     int64_t nsub;                             // sub-chunks per row
+    const uint8_t *reset;                     // (batch, seqlen) sequence starts, or null
+    int reset_vec;                            // every 8-step group of reset is 8-byte aligned
 };
 
 constexpr int kBwdSub = 8;                    // steps per sub-chunk
@@ -90,8 +96,8 @@ __device__ __forceinline__ float sigmoid_of(float x) {
 #define SS_BWD_MIN_BLOCKS 3
 #endif
 
-// Blocks of 128 threads (4 warps).
-template <typename Tin, typename Tout, int kNmax>
+// Blocks of 128 threads (4 warps).  kReset: the instance that reads p.reset.
+template <typename Tin, typename Tout, int kNmax, bool kReset = false>
 __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const BwdParams p) {
     constexpr int kG = bwd_lanes(kNmax);
     constexpr int kPairs = kNmax / 2;
@@ -245,6 +251,31 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         }
     };
 
+    // Start flags of the 8 steps from l0 (one byte each, as two words), read
+    // one sub-chunk ahead; every lane of the block reads the same ones.
+    const uint8_t *const reset_b = kReset ? p.reset + b * L : nullptr;
+    auto load_flags = [&](int64_t l0, uint2 &w) {
+        if constexpr (kReset) {
+            if (p.reset_vec && l0 + kBwdSub <= L) {
+                w = __ldg(reinterpret_cast<const uint2 *>(reset_b + l0));
+            } else {
+                w = make_uint2(0u, 0u);
+#pragma unroll
+                for (int i = 0; i < kBwdSub; ++i)
+                    if (l0 + i < L && reset_b[l0 + i] != 0) (i < 4 ? w.x : w.y) |= 1u << (8 * (i & 3));
+            }
+        }
+    };
+    // Bit i: a sequence starts at step l0 + i.
+    auto flag_bits = [&](uint2 w) {
+        uint32_t mask = 0u;
+#pragma unroll
+        for (int i = 0; i < kBwdSub; ++i)
+            if (((i < 4 ? w.x : w.y) >> (8 * (i & 3))) & 0xffu) mask |= 1u << i;
+        return mask;
+    };
+    uint2 wfl = make_uint2(0u, 0u);  // flags of the next sub-chunk
+
     // ---------------------------------------------------------------- phase A
     float2 h[kPL];
 #pragma unroll
@@ -253,6 +284,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     if (L > 0) {
         load_own(u_row, j0, wu);
         load_own(d_row, j0, wd);
+        load_flags(0, wfl);
         if (stage_fast(0)) issue_copies(0);
     }
     for (int64_t c0 = 0; c0 < L; c0 += kBwdStage) {
@@ -277,9 +309,11 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     gat[kBwdSub + j0 + i] = dl * Io<Tin>::widen(wu, i);
                 }
             }
+            const uint32_t starts = kReset ? flag_bits(wfl) : 0u;
             if (l0 + kBwdSub < L) {
                 load_own(u_row, l0 + kBwdSub + j0, wu);
                 load_own(d_row, l0 + kBwdSub + j0, wd);
+                load_flags(l0 + kBwdSub, wfl);
             }
             __syncwarp();
             float dl[kBwdSub], du[kBwdSub];
@@ -300,6 +334,9 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     const float4 bc = Fm[i * kPairs + qq];
                     const float2 t = __fmul2_rn(d2, A2[qq]);
                     const float2 a = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
+                    if constexpr (kReset) {
+                        if ((starts >> i) & 1u) h[qq] = make_float2(0.f, 0.f);
+                    }
                     h[qq] = __ffma2_rn(a, h[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
                 }
             }
@@ -345,6 +382,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         load_own(d_row, l0 + j0, wd);
         if (has_z) load_own(z_row, l0 + j0, wz);
         load_own(dy_row, l0 + j0, wdy);
+        load_flags(l0, wfl);
     };
     if (L > 0) prefetch(((L - 1) / kBwdSub) * kBwdSub);
     for (int64_t st = nstages - 1; st >= 0; --st) {
@@ -379,6 +417,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
             float2 h0[kPL];
 #pragma unroll
             for (int qq = 0; qq < kPL; ++qq) h0[qq] = h0n[qq];
+            const uint32_t starts = kReset ? flag_bits(wfl) : 0u;
             if (l0 > 0) prefetch(l0 - kBwdSub);
             __syncwarp();
             float dl[kBwdSub], du[kBwdSub], gg[kBwdSub];
@@ -405,7 +444,11 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     const float4 bc = Fm[i * kPairs + qq];
                     const float2 t = __fmul2_rn(d2, A2[qq]);
                     a[i][qq] = make_float2(sfu_exp2(t.x), sfu_exp2(t.y));
-                    hs[i][qq] = __ffma2_rn(a[i][qq], i ? hs[i - 1][qq] : h0[qq], __fmul2_rn(u2, make_float2(bc.x, bc.y)));
+                    float2 prev = i ? hs[i - 1][qq] : h0[qq];
+                    if constexpr (kReset) {
+                        if ((starts >> i) & 1u) prev = make_float2(0.f, 0.f);
+                    }
+                    hs[i][qq] = __ffma2_rn(a[i][qq], prev, __fmul2_rn(u2, make_float2(bc.x, bc.y)));
                     acc = __ffma2_rn(make_float2(bc.z, bc.w), hs[i][qq], acc);
                 }
                 sp[i] = acc.x + acc.y;
@@ -422,8 +465,11 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     const float2 lam = __ffma2_rn(g2, make_float2(bc.z, bc.w), carry[qq]);
                     const float2 dCp = __fmul2_rn(g2, hs[i][qq]);
                     const float2 dBp = __fmul2_rn(lam, u2);
-                    const float2 hp = i ? hs[i - 1][qq] : h0[qq];
-                    const float2 la = __fmul2_rn(lam, a[i][qq]);   // a lam: the carry to the step before
+                    float2 hp = i ? hs[i - 1][qq] : h0[qq];
+                    float2 la = __fmul2_rn(lam, a[i][qq]);   // a lam: the carry to the step before
+                    if constexpr (kReset) {
+                        if ((starts >> i) & 1u) hp = make_float2(0.f, 0.f), la = make_float2(0.f, 0.f);
+                    }
                     const float2 t = __fmul2_rn(la, hp);             // lam a h_prev
                     sLB = __ffma2_rn(lam, make_float2(bc.x, bc.y), sLB);
                     sLHA = __ffma2_rn(t, Aln[qq], sLHA);

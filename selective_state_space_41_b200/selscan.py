@@ -9,7 +9,7 @@ fails to load, every call raises.
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``,
 ``ss_fwd_reset``, ``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
-``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_workspace_bytes``,
+``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_reset``, ``ss_bwd_workspace_bytes``,
 ``ss_status_string``, ``ss_version``); ``ss_fwd`` dispatches to the
 workspace, config, initial-state and sequence-start forms by keyword, ``ss_fwd_hostio`` to
 the pipelined form when given streams.  ``selective_scan_fwd`` and
@@ -36,8 +36,8 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # Names the header declares; the ABI test checks each is exported.
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
-           "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc", "ss_step", "ss_bwd", "ss_bwd_workspace_bytes",
-           "ss_status_string", "ss_version")
+           "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc",
+           "ss_step", "ss_bwd", "ss_bwd_reset", "ss_bwd_workspace_bytes", "ss_status_string", "ss_version")
 
 
 class SelscanError(RuntimeError):
@@ -96,6 +96,8 @@ def lib():
         L.ss_step.argtypes = [DP] + [P] * 8 + [I, P, P, P]
         L.ss_bwd.restype = I
         L.ss_bwd.argtypes = [DP] + [P] * 8 + [I] + [P] * 9 + [P, SZ, P]
+        L.ss_bwd_reset.restype = I
+        L.ss_bwd_reset.argtypes = [DP] + [P] * 8 + [I] + [P] * 10 + [P, SZ, P]
         L.ss_bwd_workspace_bytes.restype = SZ
         L.ss_bwd_workspace_bytes.argtypes = [DP]
         L.ss_status_string.restype = ctypes.c_char_p
@@ -238,11 +240,12 @@ def ss_bwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, 
 
 
 def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_softplus=False,
-           workspace=None, stream=None):
+           workspace=None, stream=None, reset=None):
     """Queue the backward: ``grads`` maps du, ddelta, dA, dB, dC and (when the
     operand is given) dD, dz, ddelta_bias to output tensors (du, ddelta, dz in
     u's dtype; the others float32).  ``workspace``: a CUDA tensor of at least
-    ss_bwd_workspace_bytes() bytes (allocated here when None)."""
+    ss_bwd_workspace_bytes() bytes (allocated here when None).  ``reset``: the
+    forward's (batch, L) mask of sequence starts (selects ``ss_bwd_reset``)."""
     u, delta, A, B, C, dy, D, z, delta_bias = map(_contig, (u, delta, A, B, C, dy, D, z, delta_bias))
     batch, dim, L = u.shape
     N = A.shape[-1]
@@ -251,15 +254,22 @@ def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_
         n = ss_bwd_workspace_bytes(batch, dim, L, N, u.dtype, dy.dtype)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=u.device)
     g = lambda k: _ptr(grads.get(k))  # noqa: E731
-    _check(lib().ss_bwd(ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                        _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(dy), g("du"),
-                        g("ddelta"), g("dA"), g("dB"), g("dC"), g("dD"), g("dz"), g("ddelta_bias"),
-                        _ptr(workspace), workspace.numel() * workspace.element_size(),
-                        _stream_handle(stream, u.device)), "ss_bwd")
+    head = (ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+            _ptr(delta_bias), 1 if delta_softplus else 0)
+    tail = (_ptr(dy), g("du"), g("ddelta"), g("dA"), g("dB"), g("dC"), g("dD"), g("dz"), g("ddelta_bias"),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream, u.device))
+    if reset is not None:
+        if reset.dtype == torch.bool:
+            reset = reset.view(torch.uint8)
+        if reset.dtype != torch.uint8 or tuple(reset.shape) != (batch, L) or not reset.is_contiguous():
+            raise ValueError("reset must be a contiguous (batch, L) uint8 or bool tensor")
+        _check(lib().ss_bwd_reset(*head, _ptr(reset), *tail), "ss_bwd_reset")
+    else:
+        _check(lib().ss_bwd(*head, *tail), "ss_bwd")
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=False,
-                       stream=None):
+                       stream=None, reset=None):
     """Gradients of sum(dy * y) as a dict (see ss_bwd); allocates the outputs."""
     batch, dim, L = u.shape
     N = A.shape[-1]
@@ -273,7 +283,7 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, d
              "dz": torch.empty_like(u) if z is not None else None,
              "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None}
     ss_bwd(u, delta, A, B, C, dy, grads, D=D, z=z, delta_bias=delta_bias,
-           delta_softplus=delta_softplus, stream=stream)
+           delta_softplus=delta_softplus, stream=stream, reset=reset)
     return grads
 
 

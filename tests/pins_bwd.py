@@ -94,4 +94,37 @@ def pin_bwd_softplus_linear_region(grad, scan):
         assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), f"d/d{name} above the threshold: {an!r} vs {fd!r}"
 
 
-ALL_PINS = [pin_bwd_directional, pin_bwd_every_element, pin_bwd_softplus_linear_region]
+def pin_bwd_sequence_starts(grad, scan):
+    """With sequence starts (the state entering a start is zero), every
+    gradient against central differences of the forward with the same starts:
+    directions for every input of a mid-sized problem, and every element of a
+    tiny one (starts at step 0, inside, on consecutive steps and at the end)."""
+    rng = np.random.default_rng(53)
+    cases = [((2, 3, 12, 4), {0: [4, 5, 11], 1: [0, 7]}), ((2, 2, 6, 3), {0: [2], 1: [0, 3, 4]})]
+    for k, ((Bt, Dm, L, N), starts) in enumerate(cases):
+        p = _problem(rng, Bt, Dm, L, N)
+        dy = rng.standard_normal((Bt, Dm, L))
+        reset = np.zeros((Bt, L), dtype=np.uint8)
+        for b, ls in starts.items():
+            reset[b, ls] = 1
+
+        def F(q):
+            y = scan(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                     delta_bias=q["delta_bias"], delta_softplus=True, reset=reset)
+            return float((np.asarray(y) * dy).sum())
+
+        g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+                 delta_bias=p["delta_bias"], delta_softplus=True, reset=reset)
+        for name, gname in NAMES:
+            dirs = ([rng.standard_normal(p[name].shape)] if k == 0 else
+                    [np.eye(p[name].size)[i].reshape(p[name].shape) for i in range(p[name].size)])
+            for v in dirs:
+                eps = 1e-6
+                fd = (F(dict(p, **{name: p[name] + eps * v})) - F(dict(p, **{name: p[name] - eps * v}))) / (2 * eps)
+                an = float((g[gname] * v).sum())
+                assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), \
+                    f"starts case {k} d/d{name}: analytic {an!r} vs finite difference {fd!r}"
+
+
+ALL_PINS = [pin_bwd_directional, pin_bwd_every_element, pin_bwd_softplus_linear_region,
+            pin_bwd_sequence_starts]

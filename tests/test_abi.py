@@ -182,6 +182,28 @@ def test_bwd_rejections(lib):
     assert e.value.status == 4
 
 
+def test_bwd_reset_rejections(lib):
+    """ss_bwd_reset: no mask for a non-empty problem, and the ss_bwd
+    rejections, before any launch; the binding passes its mask through (the
+    call is rejected on the state count before any pointer is used)."""
+    P = FAKE
+    head = (P, P, P, P, P, None, None, None, 1)
+    tail = (P, P, P, P, P, P, None, None, None)
+    d = _desc(dstate=16)
+    assert lib.ss_bwd_reset(ctypes.byref(d), *head, None, *tail, None, 0, None) == 1
+    assert lib.ss_bwd_reset(None, *head, P, *tail, None, 0, None) == 1
+    assert lib.ss_bwd_reset(ctypes.byref(_desc(dstate=65)), *head, P, *tail, None, 0, None) == 4
+    assert lib.ss_bwd_reset(ctypes.byref(d), *head, P, *tail, None, 0, None) == 8
+    import torch
+    t = torch.zeros(1, 2, 4)
+    with pytest.raises(selscan.SelscanError) as e:
+        selscan.ss_bwd(t, t, torch.zeros(2, 65), torch.zeros(1, 65, 4), torch.zeros(1, 65, 4), t,
+                       {"du": t, "ddelta": t, "dA": t, "dB": t, "dC": t},
+                       workspace=torch.zeros(16, dtype=torch.uint8),
+                       stream=types.SimpleNamespace(cuda_stream=0), reset=torch.zeros(1, 4, dtype=torch.uint8))
+    assert e.value.status == 4
+
+
 def test_step_rejections(lib):
     """ss_step: one step only, required pointers, alignment; before any launch."""
     P = FAKE

@@ -32,15 +32,16 @@ def _case(batch, dim, L, N, dtype, seed, out_dtype=None, **kw):
     return inp
 
 
-def _check(inp, dtype, what):
+def _check(inp, dtype, what, reset=None):
     d = to_dev(inp)
     got = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], D=d.get("D"),
                                      z=d.get("z"), delta_bias=d.get("delta_bias"),
-                                     delta_softplus=inp["delta_softplus"])
+                                     delta_softplus=inp["delta_softplus"],
+                                     reset=None if reset is None else torch.as_tensor(reset).cuda())
     torch.cuda.synchronize()
     ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"],
                                     D=inp.get("D"), z=inp.get("z"), delta_bias=inp.get("delta_bias"),
-                                    delta_softplus=inp["delta_softplus"])
+                                    delta_softplus=inp["delta_softplus"], reset=reset)
     for k, want in ref.items():
         if want is None:
             assert got[k] is None
@@ -121,3 +122,66 @@ def test_bwd_softplus_linear_region():
     inp["delta_bias"] = torch.full((24,), 20.0)          # delta ~ N(0, 1): both sides of 20
     inp["A"] = (inp["A"] * 0.01).contiguous()            # keep exp(delta' A) away from underflow
     _check(inp, torch.float32, "softplus threshold")
+
+
+# ---------------------------------------------------------------- sequence starts
+# (ss_bwd_reset: the backward of a forward whose state is zeroed entering each
+# start of the (batch, L) mask; the oracle's reset form is pinned by finite
+# differences of the forward with the same starts.)
+
+def _starts(batch, L, seed, fixed=(), p=0.0):
+    m = np.zeros((batch, L), dtype=np.uint8)
+    for l in fixed:
+        if 0 <= l < L:
+            m[:, l] = 1
+    if p > 0:
+        r = gen.fill((batch, L), torch.float32, seed, DY_STREAM + 1, gen.UNIFORM, 0.0, 1.0).numpy()
+        m |= (r < p).astype(np.uint8)
+    return m
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N", [4, 16, 33, 64])
+def test_bwd_starts_state_sizes(dtype, N):
+    """Every state bucket; 203 steps (flags read byte by byte), starts at
+    step 0, on and beside sub-chunk (8) and stage (64) boundaries, at the last
+    step, and seeded ones; batch entries with different starts."""
+    inp = _case(2, 45, 203, N, dtype, seed=N + 300, has_z=True, return_last_state=False)
+    reset = _starts(2, 203, seed=N, fixed=(7, 8, 9, 63, 64, 100, 202), p=0.02)
+    reset[0, 0] = 1
+    _check(inp, dtype, f"starts N={N}", reset=reset)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_bwd_starts_aligned_rows(dtype):
+    """256 steps (flags read as 8-byte words), starts every 32 steps plus
+    seeded ones, every optional operand."""
+    inp = _case(3, 40, 256, 16, dtype, seed=17, has_z=True, bias_kind="uniform_dt")
+    _check(inp, dtype, "starts, aligned rows", reset=_starts(3, 256, seed=17, fixed=range(0, 256, 32), p=0.03))
+
+
+def test_bwd_start_every_step():
+    inp = _case(2, 20, 65, 16, torch.float32, seed=19, has_z=True)
+    _check(inp, torch.float32, "a start at every step", reset=np.ones((2, 65), np.uint8))
+
+
+def test_bwd_all_zero_starts_bitwise_plain():
+    """The reset instance with no start set does the plain instance's arithmetic."""
+    inp = _case(2, 40, 256, 16, torch.bfloat16, seed=23, has_z=True)
+    d = to_dev(inp)
+    args = (d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"])
+    kw = dict(D=d.get("D"), z=d.get("z"), delta_bias=d.get("delta_bias"), delta_softplus=True)
+    g0 = selscan.selective_scan_bwd(*args, **kw)
+    g1 = selscan.selective_scan_bwd(*args, reset=torch.zeros(2, 256, dtype=torch.uint8, device="cuda"), **kw)
+    torch.cuda.synchronize()
+    for k, v in g0.items():
+        assert (v is None and g1[k] is None) or torch.equal(v, g1[k]), k
+
+
+def test_bwd_starts_mamba130m_one_batch():
+    """One batch entry of the mamba-130m-shaped layer cut into 512-step sequences."""
+    w = W.with_shape(W.WORKLOADS[W.MAMBA130M], batch=1)
+    inp = W.make_inputs(w)
+    inp["dy"] = gen.fill((1, w.dim, w.seqlen), torch.bfloat16, 77, DY_STREAM)
+    _check(inp, torch.bfloat16, "starts, mamba-130m-shaped batch entry",
+           reset=_starts(1, w.seqlen, seed=77, fixed=range(0, w.seqlen, 512), p=0.002))

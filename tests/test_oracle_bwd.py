@@ -36,7 +36,11 @@ def test_threads_do_not_change_results():
 
 
 MUTANTS = {
-    "carry_without_decay": ("carry[n] = a * lam;", "carry[n] = lam;"),
+    "carry_without_decay": ("carry[n] = keep ? a * lam : 0.0;", "carry[n] = keep ? lam : 0.0;"),
+    "start_passes_adjoint": ("carry[n] = keep ? a * lam : 0.0;", "carry[n] = a * lam;"),
+    "start_keeps_old_state": ("a * (keep ? h[l * N + n] : 0.0)", "a * h[l * N + n]"),
+    "start_keeps_dA_term": ("const double da = keep ? lam * h[l * N + n] : 0.0;",
+                            "const double da = lam * h[l * N + n];"),
     "silu_grad_sign": ("(1.0 + z[idx] * (1.0 - sg))", "(1.0 - z[idx] * (1.0 - sg))"),
     "softplus_grad_missing": ("ddl * (xs[l] > 20.0 ? 1.0 : sigmoid(xs[l]))", "ddl"),
     "dB_uses_B": ("dB[bn] += lam * dl[l] * u[idx];", "dB[bn] += lam * dl[l] * B[bn];"),
