@@ -1,7 +1,8 @@
 /*
  * libselscan -- the selective scan of Mamba on NVIDIA B200 (sm_100a), C ABI:
- * the forward (from a zero or a given state), one-step decoding, and the
- * backward (gradients of every input).
+ * the forward (from a zero or a given state, optionally with sequence starts
+ * inside the rows), one-step decoding, and the backward (gradients of every
+ * input, with or without sequence starts).
  *
  * The operation is the selective scan of Mamba as the selective_scan_ref
  * walkthrough defines it ("Mamba代码实战：手把手教你用PyTorch复现选择性扫描核心逻辑

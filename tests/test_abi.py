@@ -154,6 +154,22 @@ def test_reset_entry_rejections(lib):
                             None) == 0
 
 
+def test_reset_mask_checked_by_the_binding():
+    """The binding rejects a start mask of the wrong shape or dtype before it
+    calls the library (CPU tensors; nothing reaches a device)."""
+    import torch
+    t = torch.zeros(1, 2, 8)
+    A, BC = torch.zeros(2, 4), torch.zeros(1, 4, 8)
+    s0 = types.SimpleNamespace(cuda_stream=0)
+    for bad in (torch.zeros(1, 7, dtype=torch.uint8), torch.zeros(2, 8, dtype=torch.uint8),
+                torch.zeros(1, 8, dtype=torch.int32)):
+        with pytest.raises(ValueError):
+            selscan.ss_fwd(t, t, A, BC, BC, t, stream=s0, reset=bad)
+        with pytest.raises(ValueError):
+            selscan.ss_bwd(t, t, A, BC, BC, t, {"du": t, "ddelta": t, "dA": A, "dB": BC, "dC": BC},
+                           workspace=torch.zeros(16, dtype=torch.uint8), stream=s0, reset=bad)
+
+
 def test_bwd_rejections(lib):
     """ss_bwd rejects before any launch (the pointers are fake): no
     descriptor, more than 64 states, a missing gradient output, no workspace.
