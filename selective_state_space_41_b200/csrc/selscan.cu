@@ -113,8 +113,11 @@ int segment(const ss_desc *desc, int nseg, int64_t *seg_len) {
 // the least work per state update, so it is used whenever the rows alone
 // can give each SM sub-partition (4 per SM) enough warps: the smallest split
 // G in {1, 2, 4} (at most half the state bucket) with at least 4 warps per
-// sub-partition (with 32 or 64 states, 32 states per lane once that gives 2
-// warps), or G = 4 down to 1.5 warps.  With fewer rows and a long sequence,
+// sub-partition (with 64 states, 32 states per lane once that gives 2 warps:
+// 16 states per lane there measured 3x slower), or G = 4 down to 1.5 warps.
+// 32 states take 2 lanes of 16 rather than one of 32, whose 254 registers
+// leave 2 warps per sub-partition (16 x 4096 x 8192 x 32 layer: 6.0 against
+// 7.2 ms).  With fewer rows and a long sequence,
 // and a workspace, the sequence is cut into segments of at least
 // kMinSegSteps steps that the direct kernel runs as extra rows (2-way state
 // split, about 7 warps per sub-partition) and the fix-up kernel joins.
@@ -132,7 +135,7 @@ Plan heuristic(const ss_desc *desc, int64_t rows, int sms, size_t workspace_byte
     const int gmax = bucket / 2 >= 4 ? 4 : 2;
     int g = 1;
     while (g < gmax && rows * g < 4 * slots) g *= 2;
-    if (bucket >= 32 && rows * (bucket / 32) >= 2 * slots) g = bucket / 32;
+    if (bucket >= 64 && rows * (bucket / 32) >= 2 * slots) g = bucket / 32;
     if (rows * g >= 2 * slots || rows * gmax * 2 >= 3 * slots) {
         pl.lanes = g;
         pl.split = g > 1 ? 1 : 0;

@@ -170,6 +170,32 @@ def test_reset_mask_checked_by_the_binding():
                            workspace=torch.zeros(16, dtype=torch.uint8), stream=s0, reset=bad)
 
 
+@pytest.mark.parametrize("shape,ws,want", [
+    # (B, D, L, N), workspace bytes, (lanes_per_row, split_states, warps_per_block, segments)
+    ((8, 1536, 2048, 16), 0, (4, True, 4, 1)),          # mamba-130m-shaped layer: measured best 4s/4
+    ((4, 1024, 100000, 16), 1 << 30, (2, True, 4, 16)),  # 100k genomic, with workspace: 2s/4, 16 segments
+    ((16, 4096, 8192, 16), 0, (2, True, 4, 1)),          # wide layers: 2s/4 at 16, 32 and 64 states
+    ((16, 4096, 8192, 32), 0, (2, True, 4, 1)),
+    ((16, 4096, 8192, 64), 0, (2, True, 4, 1)),
+])
+def test_heuristic_picks_the_measured_shapes(shape, ws, want):
+    """The launch heuristic (host logic, 148 SMs when no device answers)
+    chooses, for the benchmark workloads, the shapes the sweeps measured
+    fastest on a B200."""
+    import torch
+    h = selscan.ss_fwd_heuristic(*shape, torch.bfloat16, workspace_bytes=ws)
+    assert (h["lanes_per_row"], h["split_states"], h["warps_per_block"], h["segments"]) == want
+
+
+def test_heuristic_genomic_without_workspace_and_its_workspace():
+    """Without a workspace the 100k-step genomic layer takes the scan kernel;
+    with one, 16 segments need nseg x rows x (N + 1) floats."""
+    import torch
+    h = selscan.ss_fwd_heuristic(4, 1024, 100000, 16, torch.bfloat16)
+    assert h["split_states"] is False and h["segments"] == 1
+    assert selscan.ss_fwd_workspace_bytes(4, 1024, 100000, 16, torch.bfloat16) == 16 * 4096 * 17 * 4
+
+
 def test_bwd_rejections(lib):
     """ss_bwd rejects before any launch (the pointers are fake): no
     descriptor, more than 64 states, a missing gradient output, no workspace.
