@@ -382,6 +382,30 @@ def pin_initial_state_continuity(scan):
 # ---- sequence starts (extension: the boundary reset of "Mamba实战：如何用选择性
 # 状态空间模型提升你的长序列处理效率（附代码）" §2; the state entering a start is zero).
 
+def pin_reset_hand_worked(scan):
+    """The golden example of tests/golden/hand_worked.json with a sequence
+    start at step 1 and at step 2 (values derived by hand there), both delta
+    modes; a start at step 0 changes nothing."""
+    g = json.load(open(os.path.join(GOLDEN, "hand_worked.json")))
+    inp, exp_ = g["inputs"], g["expected"]
+    ln2 = math.log(2.0)
+    u = np.array(inp["u"])
+    A = np.array(inp["A"])
+    B = np.array(inp["B_times_ln2"]) / ln2
+    C = np.array(inp["C"])
+    D = np.array(inp["D"])
+    tol = g["tolerance_rel"]
+    L = u.shape[-1]
+    for delta, sp in [(np.full(u.shape, math.log(ln2)), False), (np.array(inp["delta_softplus_mode"]), True)]:
+        for at, key in ((1, "start_at_1"), (2, "start_at_2"), (0, None)):
+            reset = np.zeros((u.shape[0], L), dtype=np.uint8)
+            reset[:, at] = 1
+            y, last = scan(u, delta, A, B, C, D=D, delta_softplus=sp, return_last_state=True, reset=reset)
+            want = g["expected_reset"][key] if key else exp_
+            _assert_close(y, want["y"], tol, f"hand-worked start at {at} y (softplus={sp})")
+            _assert_close(last, want["last_state"], tol, f"hand-worked start at {at} last state (softplus={sp})")
+
+
 def pin_reset_pieces(scan):
     """Rows holding several sequences: with starts marked, y over each piece
     and the last state equal independent runs of the pieces (each from the
@@ -462,5 +486,5 @@ def pin_reset_none(scan):
 ALL_PINS = [pin_hand_worked, pin_delta_transform, pin_closed_form, pin_brute_force,
             pin_lfilter, pin_delta_to_zero, pin_causality, pin_linearity,
             pin_state_separability, pin_last_state, pin_initial_state_closed_form,
-            pin_initial_state_brute_force, pin_initial_state_continuity, pin_reset_pieces,
+            pin_initial_state_brute_force, pin_initial_state_continuity, pin_reset_hand_worked, pin_reset_pieces,
             pin_reset_every_step, pin_reset_none]
