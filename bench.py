@@ -372,7 +372,7 @@ def bench_ours(args, w, world, rank, local):
         "metric": METRIC, "value": value, "unit": "updates/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32" if w.dtype == torch.float32 else "bf16 in/out, f32 arithmetic",
+        "dtype": "f32",  # the arithmetic; the inputs' and outputs' dtype is in config
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller)",
         "config": dict(w.describe(), parallelism=f"{world} independent problem(s), one per GPU",
                        l2="flushed before every timed step (write of %d MB)" % (flush.numel() >> 20),
