@@ -34,6 +34,34 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), f"{name} not exported"
 
 
+def test_header_is_c_and_links(lib, tmp_path):
+    """The header compiles as C99 with every warning an error, every function
+    it declares resolves when a C program links the library, and the
+    host-only calls answer from C."""
+    import subprocess
+    funcs = declared_functions()
+    src = tmp_path / "uses_header.c"
+    src.write_text(
+        "#include <stdio.h>\n#include <string.h>\n#include \"selscan.h\"\n"
+        "typedef void (*any_fn)(void);\n"
+        "int main(void) {\n"
+        "    any_fn fns[] = {" + ", ".join(f"(any_fn)&{f}" for f in funcs) + "};\n"
+        "    for (size_t i = 0; i < sizeof fns / sizeof fns[0]; ++i)\n"
+        "        if (!fns[i]) return 2;\n"
+        "    if (ss_version() != SS_VERSION) return 3;\n"
+        "    if (strlen(ss_status_string(SS_ERR_NULL_POINTER)) == 0) return 4;\n"
+        "    printf(\"%d\\n\", ss_version());\n"
+        "    return 0;\n"
+        "}\n")
+    exe = tmp_path / "uses_header"
+    libdir = os.path.dirname(selscan.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", build.INCLUDE,
+                    str(src), "-o", str(exe), "-L", libdir, "-lselscan", "-Wl,-rpath," + libdir],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    assert int(out) == lib.ss_version()
+
+
 def test_version_and_strings(lib):
     assert selscan.ss_version() == 100
     for code, name in selscan.STATUS_NAMES.items():
