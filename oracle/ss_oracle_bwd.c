@@ -29,6 +29,14 @@
  * With sequence starts (the reset mask of ss_oracle.c: the state entering a
  * start is zero), h_(l-1) has no part in h_l at a start l, so there the
  * h_(l-1) terms of dd_l and dA vanish and no adjoint passes from l to l-1.
+ * With a given state h0 before step 0 (the initial state of ss_oracle.c),
+ * h_(-1) = h0 in the loop above and its gradient is the adjoint carried past
+ * step 0:  dh0_n = a_0n lam_0n  (0 when a sequence starts at step 0).
+ *
+ * Optionally, for every gradient that is a sum over rows or steps (dA, dB,
+ * dC, dD, ddelta_bias), the sum of the absolute values of its terms (the
+ * same terms, each taken with |.|).  These scale the tolerance of a finite
+ * precision sum per element; they are not gradients.
  */
 #include <math.h>
 #include <stdint.h>
@@ -43,34 +51,45 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 /* Returns 0 on success, -1 on a bad argument or allocation failure.
  * Required: u, delta, A, B, C, dy, du, ddelta, dA, dB, dC.  dD is required
- * when D is given, dz when z is, ddelta_bias when delta_bias is. */
-int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
-                        const double *u, const double *delta, const double *A,
-                        const double *B, const double *C, const double *D,
-                        const double *z, const double *delta_bias, int delta_softplus,
-                        const uint8_t *reset, const double *dy, double *du, double *ddelta,
-                        double *dA, double *dB, double *dC, double *dD, double *dz,
-                        double *ddelta_bias, int nthreads)
+ * when D is given, dz when z is, ddelta_bias when delta_bias is, dh0 when h0
+ * is.  h0 (batch, dim, N): the state before step 0 (NULL: zero).  mA, mB, mC,
+ * mD, mbias: NULL, or the sums of |terms| of dA, dB, dC, dD, ddelta_bias
+ * (shapes of those). */
+int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                       const double *u, const double *delta, const double *A,
+                       const double *B, const double *C, const double *D,
+                       const double *z, const double *delta_bias, int delta_softplus,
+                       const uint8_t *reset, const double *h0, const double *dy, double *du,
+                       double *ddelta, double *dA, double *dB, double *dC, double *dD,
+                       double *dz, double *ddelta_bias, double *dh0, double *mA, double *mB,
+                       double *mC, double *mD, double *mbias, int nthreads)
 {
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1)
         return -1;
     if (!A || !dA || (batch * dim > 0 && seqlen > 0 &&
                       (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)))
         return -1;
-    if ((D && !dD) || (z && !dz) || (delta_bias && !ddelta_bias))
+    if ((D && !dD) || (z && !dz) || (delta_bias && !ddelta_bias) || (h0 && !dh0))
         return -1;
     const int64_t N = dstate, L = seqlen;
     /* per-row partial sums over l, reduced over b afterwards in order */
     double *pA = calloc((size_t)(batch * dim * N + 1), sizeof(double));
     double *pD = calloc((size_t)(batch * dim + 1), sizeof(double));
     double *pbias = calloc((size_t)(batch * dim + 1), sizeof(double));
-    if (!pA || !pD || !pbias) {
-        free(pA), free(pD), free(pbias);
+    double *qA = calloc((size_t)(batch * dim * N + 1), sizeof(double)); /* the same, of |terms| */
+    double *qD = calloc((size_t)(batch * dim + 1), sizeof(double));
+    double *qbias = calloc((size_t)(batch * dim + 1), sizeof(double));
+    if (!pA || !pD || !pbias || !qA || !qD || !qbias) {
+        free(pA), free(pD), free(pbias), free(qA), free(qD), free(qbias);
         return -1;
     }
     if (batch > 0 && L > 0) {
         memset(dB, 0, sizeof(double) * (size_t)(batch * N * L));
         memset(dC, 0, sizeof(double) * (size_t)(batch * N * L));
+        if (mB)
+            memset(mB, 0, sizeof(double) * (size_t)(batch * N * L));
+        if (mC)
+            memset(mC, 0, sizeof(double) * (size_t)(batch * N * L));
     }
     int bad = 0;
 #ifdef _OPENMP
@@ -91,9 +110,9 @@ int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dsta
         }
         for (int64_t d = 0; d < dim; ++d) {
             const int64_t row = b * dim + d;
-            /* forward, keeping every state */
+            /* forward, keeping every state (h[0..N-1]: the state before step 0) */
             for (int64_t n = 0; n < N; ++n)
-                h[n] = 0.0;
+                h[n] = h0 ? h0[row * N + n] : 0.0;
             for (int64_t l = 0; l < L; ++l) {
                 const int64_t idx = row * L + l;
                 const int keep = !(reset && reset[b * L + l]); /* 0 at a sequence start */
@@ -127,7 +146,7 @@ int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dsta
                 }
                 double dui = D ? g * D[d] : 0.0;
                 if (D)
-                    pD[row] += g * u[idx];
+                    pD[row] += g * u[idx], qD[row] += fabs(g * u[idx]);
                 double ddl = 0.0;
                 for (int64_t n = 0; n < N; ++n) {
                     const int64_t bn = (b * N + n) * L + l;
@@ -135,10 +154,15 @@ int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dsta
                     const double lam = g * C[bn] + carry[n];
                     dC[bn] += g * h[(l + 1) * N + n];
                     dB[bn] += lam * dl[l] * u[idx];
+                    if (mC)
+                        mC[bn] += fabs(g * h[(l + 1) * N + n]);
+                    if (mB)
+                        mB[bn] += fabs(lam * dl[l] * u[idx]);
                     dui += lam * dl[l] * B[bn];
                     const double da = keep ? lam * h[l * N + n] : 0.0;
                     ddl += lam * B[bn] * u[idx] + da * a * A[d * N + n];
                     pA[row * N + n] += da * a * dl[l];
+                    qA[row * N + n] += fabs(da * a * dl[l]);
                     carry[n] = keep ? a * lam : 0.0;
                 }
                 du[idx] = dui;
@@ -146,27 +170,53 @@ int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dsta
                                                  : ddl * dl[l];
                 ddelta[idx] = dx;
                 pbias[row] += dx;
+                qbias[row] += fabs(dx);
             }
+            if (h0) /* the adjoint passed on past step 0 (zero after a start at step 0) */
+                for (int64_t n = 0; n < N; ++n)
+                    dh0[row * N + n] = L > 0 ? carry[n] : 0.0;
         }
         free(h), free(dl), free(xs), free(s), free(carry);
     }
     for (int64_t d = 0; d < dim; ++d) {
         for (int64_t n = 0; n < N; ++n) {
-            double acc = 0.0;
+            double acc = 0.0, mag = 0.0;
             for (int64_t b = 0; b < batch; ++b)
-                acc += pA[(b * dim + d) * N + n];
+                acc += pA[(b * dim + d) * N + n], mag += qA[(b * dim + d) * N + n];
             dA[d * N + n] = acc;
+            if (mA)
+                mA[d * N + n] = mag;
         }
-        double accD = 0.0, accb = 0.0;
-        for (int64_t b = 0; b < batch; ++b)
+        double accD = 0.0, accb = 0.0, magD = 0.0, magb = 0.0;
+        for (int64_t b = 0; b < batch; ++b) {
             accD += pD[b * dim + d], accb += pbias[b * dim + d];
+            magD += qD[b * dim + d], magb += qbias[b * dim + d];
+        }
         if (D)
             dD[d] = accD;
         if (delta_bias)
             ddelta_bias[d] = accb;
+        if (D && mD)
+            mD[d] = magD;
+        if (delta_bias && mbias)
+            mbias[d] = magb;
     }
-    free(pA), free(pD), free(pbias);
+    free(pA), free(pD), free(pbias), free(qA), free(qD), free(qbias);
     return bad ? -1 : 0;
+}
+
+/* With sequence starts, from a zero state, no |terms| sums. */
+int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                        const double *u, const double *delta, const double *A,
+                        const double *B, const double *C, const double *D,
+                        const double *z, const double *delta_bias, int delta_softplus,
+                        const uint8_t *reset, const double *dy, double *du, double *ddelta,
+                        double *dA, double *dB, double *dC, double *dD, double *dz,
+                        double *ddelta_bias, int nthreads)
+{
+    return ss_oracle_bwd_full(batch, dim, seqlen, dstate, u, delta, A, B, C, D, z, delta_bias,
+                              delta_softplus, reset, NULL, dy, du, ddelta, dA, dB, dC, dD, dz,
+                              ddelta_bias, NULL, NULL, NULL, NULL, NULL, NULL, nthreads);
 }
 
 /* The walkthrough's form: no sequence starts. */

@@ -126,5 +126,74 @@ def pin_bwd_sequence_starts(grad, scan):
                     f"starts case {k} d/d{name}: analytic {an!r} vs finite difference {fd!r}"
 
 
+def pin_bwd_initial_state(grad, scan):
+    """From a given state before step 0: the gradient with respect to that
+    state, and every other gradient, against central differences of the
+    forward from the same state; every element of a tiny problem, directions
+    for a mid-sized one, with and without sequence starts (a start at step 0
+    cuts the given state off: its gradient is zero there)."""
+    rng = np.random.default_rng(59)
+    cases = [((2, 3, 10, 4), None), ((2, 2, 5, 3), None), ((2, 2, 6, 3), {0: [0, 3], 1: [2]})]
+    for k, ((Bt, Dm, L, N), starts) in enumerate(cases):
+        p = _problem(rng, Bt, Dm, L, N)
+        p["h0"] = rng.standard_normal((Bt, Dm, N))
+        dy = rng.standard_normal((Bt, Dm, L))
+        reset = None
+        if starts is not None:
+            reset = np.zeros((Bt, L), dtype=np.uint8)
+            for b, ls in starts.items():
+                reset[b, ls] = 1
+
+        def F(q):
+            y = scan(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                     delta_bias=q["delta_bias"], delta_softplus=True, initial_state=q["h0"], reset=reset)
+            return float((np.asarray(y) * dy).sum())
+
+        g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+                 delta_bias=p["delta_bias"], delta_softplus=True, reset=reset, initial_state=p["h0"])
+        for name, gname in NAMES + [("h0", "dinitial_state")]:
+            dirs = ([rng.standard_normal(p[name].shape)] if k == 0 else
+                    [np.eye(p[name].size)[i].reshape(p[name].shape) for i in range(p[name].size)])
+            for v in dirs:
+                eps = 1e-6
+                fd = (F(dict(p, **{name: p[name] + eps * v})) - F(dict(p, **{name: p[name] - eps * v}))) / (2 * eps)
+                an = float((g[gname] * v).sum())
+                assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), \
+                    f"initial-state case {k} d/d{name}: analytic {an!r} vs finite difference {fd!r}"
+        if starts is not None:
+            assert not g["dinitial_state"][0].any(), "a start at step 0 must cut the given state off"
+
+
+def pin_bwd_term_magnitudes(grad, scan):
+    """The sums of |terms| that scale the tolerance of the summed gradients:
+    with one row and one step every sum has one term, so each equals the
+    gradient's absolute value; in general each is at least that; and the
+    sums over channels of dB and dC equal the sums of |dB|, |dC| of the
+    single-channel problems (each channel adds one term per element)."""
+    rng = np.random.default_rng(61)
+    p = _problem(rng, 1, 1, 1, 3)
+    dy = rng.standard_normal((1, 1, 1))
+    g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+             delta_bias=p["delta_bias"], delta_softplus=True, magnitudes=True)
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert np.array_equal(g["mag_" + k], np.abs(g[k])), f"one term: mag_{k} != |{k}|"
+    p = _problem(rng, 2, 4, 9, 3)
+    dy = rng.standard_normal((2, 4, 9))
+    g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+             delta_bias=p["delta_bias"], delta_softplus=True, magnitudes=True)
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert (g["mag_" + k] >= np.abs(g[k]) * (1 - 1e-12)).all(), f"mag_{k} below |{k}|"
+    for k in ("dB", "dC"):
+        acc = np.zeros_like(g[k])
+        for d in range(4):
+            q = {n: (None if v is None else (v[:, d:d + 1] if v.ndim == 3 and v.shape[1] == 4 and n not in ("B", "C")
+                                             else v[d:d + 1] if n in ("A", "D", "delta_bias") else v))
+                 for n, v in p.items()}
+            gd = grad(q["u"], q["delta"], q["A"], q["B"], q["C"], dy[:, d:d + 1], D=q["D"], z=q["z"],
+                      delta_bias=q["delta_bias"], delta_softplus=True)
+            acc += np.abs(gd[k])
+        assert np.allclose(g["mag_" + k], acc, rtol=1e-12, atol=0), f"mag_{k} != sum over channels of |{k}|"
+
+
 ALL_PINS = [pin_bwd_directional, pin_bwd_every_element, pin_bwd_softplus_linear_region,
-            pin_bwd_sequence_starts]
+            pin_bwd_sequence_starts, pin_bwd_initial_state, pin_bwd_term_magnitudes]
