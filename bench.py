@@ -16,8 +16,11 @@ host-buffer entry point ss_fwd_hostio: pinned host inputs copied in, the
 forward, y copied back, per step.  The roofline of the scan kernel is its
 exp count against the SFU rate (16 ex2 per clock per SM at the maximum SM
 clock); its HBM side (compulsory bytes over measured copy bandwidth) is
-reported beside it.  ``--impl reference`` times the fp64 CPU oracle on the
-host cores instead (a bounded sample of rows per step).
+reported beside it.  ``per_config`` adds, in the same line, the forward of
+every other configuration at full size (device time with L2 flushed per step,
+fewer steps each, clocks sampled over the warm-ups and timed steps).
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
+bounded sample of rows per step).
 """
 import argparse
 import json
@@ -294,16 +297,16 @@ def bench_ours(args, w, world, rank, local):
                        delta_bias=d["delta_bias"], delta_softplus=wr.delta_softplus,
                        last_state=last, stream=stream, workspace=ws)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        launch()
-    torch.cuda.synchronize(dev)
-
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
+    # Clocks are sampled over the whole forward leg: warm-ups and timed steps.
+    with ClockSampler(local, period_s=0.001) as clocks:
+        for _ in range(args.warmup):
+            flush.zero_()
+            launch()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        torch.cuda.synchronize(dev)
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
@@ -393,15 +396,82 @@ def bench_ours(args, w, world, rank, local):
         "kernel_ms": {"min": min(kernel_ms), "median": statistics.median(kernel_ms),
                       "max": max(kernel_ms)},
     }
+    clk = line["clocks"]
+    if clk.get("sm_mhz"):
+        line["clocks"]["ms_x_median_sm_mhz"] = my_ms * clk["sm_mhz"]
     line["decode"] = bench_decode(wr, d, out_dtype, stream, world)
     if not args.no_bwd:
         line["backward"] = bench_backward(args, wr, d, host, out_dtype, flush, stream, sfu_peak, world)
+    if not args.no_per_config:
+        # Every other configuration at full size, forward only, fewer steps
+        # each (the headline value stays the workload above).
+        per = {}
+        for name in W.WORKLOADS:
+            if name == w.name:
+                continue
+            per[name] = bench_forward_config(rank_workload(W.WORKLOADS[name], rank), dev, stream, flush,
+                                             steps=max(3, min(args.steps, 10)), warmup=3,
+                                             sfu_peak=sfu_peak, hbm_peak=hbm_peak)
+        line["per_config"] = per
     del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_sample(w, host)
         line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     return line if rank == 0 else None
+
+
+def bench_forward_config(w: W.Workload, dev, stream, flush, steps: int, warmup: int, sfu_peak: float,
+                         hbm_peak: float):
+    """Device time of one full forward of workload ``w`` (every kernel the
+    heuristic launches for it, with the workspace that enables the
+    sequence-segmented shape), L2 flushed before each step, clocks sampled
+    over warm-ups and timed steps.  Used for the configurations beside the
+    headline one."""
+    host = W.make_inputs(w)
+    names_in = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    d = {k: (host[k].to(dev) if host[k] is not None else None) for k in names_in}
+    del host
+    out_dtype = w.out_dtype or w.dtype
+    y = torch.empty(d["u"].shape, dtype=out_dtype, device=dev)
+    last = (torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+            if w.return_last_state else None)
+    ws = selscan.workspace_for(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, out_dtype, device=dev)
+
+    def launch():
+        selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
+                       delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus,
+                       last_state=last, stream=stream, workspace=ws)
+
+    ts = []
+    with ClockSampler(dev.index) as clocks:
+        for _ in range(warmup):
+            flush.zero_()
+            launch()
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            launch()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+    ms = sum(ts) / len(ts)
+    nbytes = algorithmic_bytes(w)
+    shape = selscan.ss_fwd_heuristic(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, out_dtype,
+                                     workspace_bytes=ws.numel() if ws is not None else 0)
+    clk = clocks.summary()
+    out = {"ms": ms, "ms_min": min(ts), "ms_max": max(ts), "steps": steps, "warmup": warmup,
+           "updates_per_s": w.updates / (ms * 1e-3),
+           "sfu_frac": w.updates / sfu_peak / (ms * 1e-3),
+           "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak,
+           "algorithmic_bytes": nbytes, "launch": shape,
+           "gpu_launches_per_step": 2 if shape["segments"] > 1 else 1, "clocks": clk}
+    if clk.get("sm_mhz"):
+        out["ms_x_median_sm_mhz"] = ms * clk["sm_mhz"]
+    del d, y, last, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_decode(w, d, out_dtype, stream, world, calls=200):
@@ -512,6 +582,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the forward of the other configurations")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per launch of the scan kernel from an ncu capture")
     args = ap.parse_args(argv)
