@@ -38,7 +38,7 @@ def _load(path=None):
         if hasattr(lib, "ss_oracle_bwd"):  # (a planted-mistake build of the forward alone has none)
             lib.ss_oracle_bwd_full.restype = ctypes.c_int
             lib.ss_oracle_bwd_full.argtypes = [i64, i64, i64, i64] + [P] * 8 + [ctypes.c_int] + \
-                [P] * 17 + [ctypes.c_int]
+                [P] * 18 + [ctypes.c_int]
             lib.ss_oracle_bwd_reset.restype = ctypes.c_int
             lib.ss_oracle_bwd_reset.argtypes = [i64, i64, i64, i64] + [P] * 8 + [ctypes.c_int] + \
                 [P] * 10 + [ctypes.c_int]
@@ -129,12 +129,14 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
                        delta_softplus=False, nthreads=0, lib=None, reset=None, initial_state=None,
-                       magnitudes=False):
-    """Gradients of sum(dy * y) for the forward of ``selective_scan``
-    (``reset`` and ``initial_state`` as there), in float64, as a dict: du,
-    ddelta, dz (batch, dim, L); dA (dim, N); dB, dC (batch, N, L); dD,
-    ddelta_bias (dim,); dinitial_state (batch, dim, N) when an initial state
-    is given.  The entries of absent optional operands are None.
+                       dlast_state=None, magnitudes=False):
+    """Gradients of sum(dy * y) (plus sum(dlast_state * last state) when
+    ``dlast_state`` (batch, dim, N) is given) for the forward of
+    ``selective_scan`` (``reset`` and ``initial_state`` as there), in
+    float64, as a dict: du, ddelta, dz (batch, dim, L); dA (dim, N); dB, dC
+    (batch, N, L); dD, ddelta_bias (dim,); dinitial_state (batch, dim, N) when
+    an initial state is given.  The entries of absent optional operands are
+    None.
     ``magnitudes``: also ``mag_<name>`` for each gradient that is a sum over
     rows or steps (dA, dB, dC, dD, ddelta_bias): the sum of the absolute
     values of its terms, which scales the tolerance of a finite-precision sum
@@ -160,7 +162,10 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     h0 = _f64(initial_state)
     if h0 is not None and h0.shape != (batch, dim, N):
         raise ValueError("bad initial_state shape")
-    if h0 is None and not magnitudes:
+    dlast = _f64(dlast_state)
+    if dlast is not None and dlast.shape != (batch, dim, N):
+        raise ValueError("bad dlast_state shape")
+    if h0 is None and dlast is None and not magnitudes:
         rc = _load(lib).ss_oracle_bwd_reset(batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
                                             _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
                                             1 if delta_softplus else 0, _ptr(rs), _ptr(dy), _ptr(g["du"]),
@@ -178,7 +183,8 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
                  "mag_ddelta_bias": np.zeros(dim) if delta_bias is not None else None}
         rc = _load(lib).ss_oracle_bwd_full(
             batch, dim, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-            _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(rs), _ptr(h0), _ptr(dy), _ptr(g["du"]),
+            _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(rs), _ptr(h0), _ptr(dlast), _ptr(dy),
+            _ptr(g["du"]),
             _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]),
             _ptr(g["ddelta_bias"]), _ptr(g.get("dinitial_state")), _ptr(m.get("mag_dA")),
             _ptr(m.get("mag_dB")), _ptr(m.get("mag_dC")), _ptr(m.get("mag_dD")),

@@ -32,6 +32,10 @@
  * With a given state h0 before step 0 (the initial state of ss_oracle.c),
  * h_(-1) = h0 in the loop above and its gradient is the adjoint carried past
  * step 0:  dh0_n = a_0n lam_0n  (0 when a sequence starts at step 0).
+ * With a gradient dlast of the loss with respect to the last state h_(L-1)
+ * (the loss is then sum(dy * y) + sum(dlast * h_(L-1)), as when the last
+ * state feeds the next piece of a sequence), the adjoint past the end is
+ * dlast instead of zero: lam_(L-1)n = g_(L-1) C_n,L-1 + dlast_n.
  *
  * Optionally, for every gradient that is a sum over rows or steps (dA, dB,
  * dC, dD, ddelta_bias), the sum of the absolute values of its terms (the
@@ -52,14 +56,16 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 /* Returns 0 on success, -1 on a bad argument or allocation failure.
  * Required: u, delta, A, B, C, dy, du, ddelta, dA, dB, dC.  dD is required
  * when D is given, dz when z is, ddelta_bias when delta_bias is, dh0 when h0
- * is.  h0 (batch, dim, N): the state before step 0 (NULL: zero).  mA, mB, mC,
- * mD, mbias: NULL, or the sums of |terms| of dA, dB, dC, dD, ddelta_bias
- * (shapes of those). */
+ * is.  h0 (batch, dim, N): the state before step 0 (NULL: zero).  dlast
+ * (batch, dim, N): the gradient with respect to the last state (NULL: zero).
+ * mA, mB, mC, mD, mbias: NULL, or the sums of |terms| of dA, dB, dC, dD,
+ * ddelta_bias (shapes of those). */
 int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                        const double *u, const double *delta, const double *A,
                        const double *B, const double *C, const double *D,
                        const double *z, const double *delta_bias, int delta_softplus,
-                       const uint8_t *reset, const double *h0, const double *dy, double *du,
+                       const uint8_t *reset, const double *h0, const double *dlast,
+                       const double *dy, double *du,
                        double *ddelta, double *dA, double *dB, double *dC, double *dD,
                        double *dz, double *ddelta_bias, double *dh0, double *mA, double *mB,
                        double *mC, double *mD, double *mbias, int nthreads)
@@ -133,8 +139,8 @@ int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
                 s[l] = acc;
             }
             /* reverse sweep with the adjoint state */
-            for (int64_t n = 0; n < N; ++n)
-                carry[n] = 0.0; /* a_(l+1) lam_(l+1), zero past the end */
+            for (int64_t n = 0; n < N; ++n) /* a_(l+1) lam_(l+1); past the end: dlast */
+                carry[n] = dlast ? dlast[row * N + n] : 0.0;
             for (int64_t l = L - 1; l >= 0; --l) {
                 const int64_t idx = row * L + l;
                 const int keep = !(reset && reset[b * L + l]);
@@ -174,7 +180,7 @@ int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
             }
             if (h0) /* the adjoint passed on past step 0 (zero after a start at step 0) */
                 for (int64_t n = 0; n < N; ++n)
-                    dh0[row * N + n] = L > 0 ? carry[n] : 0.0;
+                    dh0[row * N + n] = L > 0 ? carry[n] : (dlast ? dlast[row * N + n] : 0.0);
         }
         free(h), free(dl), free(xs), free(s), free(carry);
     }
@@ -215,7 +221,7 @@ int ss_oracle_bwd_reset(int64_t batch, int64_t dim, int64_t seqlen, int64_t dsta
                         double *ddelta_bias, int nthreads)
 {
     return ss_oracle_bwd_full(batch, dim, seqlen, dstate, u, delta, A, B, C, D, z, delta_bias,
-                              delta_softplus, reset, NULL, dy, du, ddelta, dA, dB, dC, dD, dz,
+                              delta_softplus, reset, NULL, NULL, dy, du, ddelta, dA, dB, dC, dD, dz,
                               ddelta_bias, NULL, NULL, NULL, NULL, NULL, NULL, nthreads);
 }
 

@@ -195,5 +195,61 @@ def pin_bwd_term_magnitudes(grad, scan):
         assert np.allclose(g["mag_" + k], acc, rtol=1e-12, atol=0), f"mag_{k} != sum over channels of |{k}|"
 
 
+def pin_bwd_last_state_gradient(grad, scan):
+    """A gradient on the last state (the loss sum(dy * y) + sum(dlast * h_L),
+    as when the state feeds the next piece of a sequence): every gradient,
+    with and without an initial state and starts, against central differences
+    of that loss; and a piece's gradient wrt its initial state fed back as the
+    previous piece's dlast reproduces the whole sequence's gradients."""
+    rng = np.random.default_rng(67)
+    for k, (Bt, Dm, L, N, with_h0, starts) in enumerate([(2, 2, 7, 3, False, None), (2, 2, 6, 3, True, {0: [2], 1: [0]})]):
+        p = _problem(rng, Bt, Dm, L, N)
+        p["h0"] = rng.standard_normal((Bt, Dm, N)) if with_h0 else None
+        dy = rng.standard_normal((Bt, Dm, L))
+        dlast = rng.standard_normal((Bt, Dm, N))
+        reset = None
+        if starts is not None:
+            reset = np.zeros((Bt, L), dtype=np.uint8)
+            for b, ls in starts.items():
+                reset[b, ls] = 1
+
+        def F(q):
+            y, last = scan(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"], delta_bias=q["delta_bias"],
+                           delta_softplus=True, initial_state=q["h0"], reset=reset, return_last_state=True)
+            return float((np.asarray(y) * dy).sum() + (np.asarray(last) * dlast).sum())
+
+        g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
+                 delta_softplus=True, reset=reset, initial_state=p["h0"], dlast_state=dlast)
+        names = NAMES + ([("h0", "dinitial_state")] if with_h0 else [])
+        for name, gname in names:
+            for i in range(p[name].size):
+                v = np.eye(p[name].size)[i].reshape(p[name].shape)
+                eps = 1e-6
+                fd = (F(dict(p, **{name: p[name] + eps * v})) - F(dict(p, **{name: p[name] - eps * v}))) / (2 * eps)
+                an = float((g[gname] * v).sum())
+                assert abs(fd - an) <= 1e-7 * (1.0 + abs(fd)), \
+                    f"dlast case {k} d/d{name}: analytic {an!r} vs finite difference {fd!r}"
+    # two pieces: [0, 5) then [5, 11), the second starting from the first's last state
+    p = _problem(rng, 2, 3, 11, 4)
+    dy = rng.standard_normal((2, 3, 11))
+    whole = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
+                 delta_softplus=True)
+    cut = 5
+    sl = lambda t, a, b: t[..., a:b]  # noqa: E731
+    _, h1 = scan(sl(p["u"], 0, cut), sl(p["delta"], 0, cut), p["A"], sl(p["B"], 0, cut), sl(p["C"], 0, cut), D=p["D"],
+                 z=sl(p["z"], 0, cut), delta_bias=p["delta_bias"], delta_softplus=True, return_last_state=True)
+    g2 = grad(sl(p["u"], cut, 11), sl(p["delta"], cut, 11), p["A"], sl(p["B"], cut, 11), sl(p["C"], cut, 11),
+              sl(dy, cut, 11), D=p["D"], z=sl(p["z"], cut, 11), delta_bias=p["delta_bias"], delta_softplus=True,
+              initial_state=h1)
+    g1 = grad(sl(p["u"], 0, cut), sl(p["delta"], 0, cut), p["A"], sl(p["B"], 0, cut), sl(p["C"], 0, cut),
+              sl(dy, 0, cut), D=p["D"], z=sl(p["z"], 0, cut), delta_bias=p["delta_bias"], delta_softplus=True,
+              dlast_state=g2["dinitial_state"])
+    for k in ("du", "ddelta", "dz", "dB", "dC"):
+        assert np.allclose(np.concatenate([g1[k], g2[k]], axis=-1), whole[k], rtol=1e-12, atol=1e-13), f"pieces: {k}"
+    for k in ("dA", "dD", "ddelta_bias"):
+        assert np.allclose(g1[k] + g2[k], whole[k], rtol=1e-12, atol=1e-13), f"pieces: {k}"
+
+
 ALL_PINS = [pin_bwd_directional, pin_bwd_every_element, pin_bwd_softplus_linear_region,
-            pin_bwd_sequence_starts, pin_bwd_initial_state, pin_bwd_term_magnitudes]
+            pin_bwd_sequence_starts, pin_bwd_initial_state, pin_bwd_term_magnitudes,
+            pin_bwd_last_state_gradient]

@@ -49,9 +49,10 @@ MUTANTS = {
     "du_missing_skip": ("double dui = D ? g * D[d] : 0.0;", "double dui = 0.0;"),
     "exp_mode_grad": (": ddl * dl[l];", ": ddl;"),
     "initial_state_ignored": ("h[n] = h0 ? h0[row * N + n] : 0.0;", "h[n] = 0.0;"),
-    "initial_state_grad_without_decay": ("dh0[row * N + n] = L > 0 ? carry[n] : 0.0;",
-                                         "dh0[row * N + n] = L > 0 ? carry[n] / exp(dl[0] * A[d * N + n]) : 0.0;"),
+    "initial_state_grad_without_decay": ("dh0[row * N + n] = L > 0 ? carry[n] :",
+                                         "dh0[row * N + n] = L > 0 ? carry[n] / exp(dl[0] * A[d * N + n]) :"),
     "magnitude_of_sum": ("mB[bn] += fabs(lam * dl[l] * u[idx]);", "mB[bn] += lam * dl[l] * u[idx];"),
+    "last_state_gradient_ignored": ("carry[n] = dlast ? dlast[row * N + n] : 0.0;", "carry[n] = 0.0;"),
 }
 
 
