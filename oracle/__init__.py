@@ -127,6 +127,28 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     return (y, last) if return_last_state else y
 
 
+def delta_from_projection(delta_r, W_dt):
+    """delta[b, d, l] = sum_r W_dt[d, r] delta_r[b, r, l]: the dt_proj linear
+    map of the mamba-minimal block ("Mamba-minimal项目解析", 核心组件解析 §5,
+    ``ssm``: x_dbl = x_proj(x), split into delta (dt_rank features), B, C;
+    delta = softplus(dt_proj(delta))), without its bias (the scan adds the
+    bias as delta_bias before the softplus).  delta_r (batch, dt_rank, L),
+    W_dt (dim, dt_rank); widened exactly to float64, one float64 matmul."""
+    r, w = _f64(delta_r), _f64(W_dt)
+    if r.ndim != 3 or w.ndim != 2 or r.shape[1] != w.shape[1]:
+        raise ValueError("delta_r (batch, dt_rank, L) and W_dt (dim, dt_rank)")
+    return np.ascontiguousarray(np.matmul(w[None, :, :], r))
+
+
+def selective_scan_dtproj(u, delta_r, W_dt, A, B, C, D=None, z=None, delta_bias=None,
+                          delta_softplus=True, return_last_state=False, nthreads=0):
+    """The forward with delta produced by the dt_proj map from its low-rank
+    input: ``selective_scan(u, W_dt delta_r, ...)`` (see delta_from_projection)."""
+    return selective_scan(u, delta_from_projection(delta_r, W_dt), A, B, C, D=D, z=z, delta_bias=delta_bias,
+                          delta_softplus=delta_softplus, return_last_state=return_last_state,
+                          nthreads=nthreads)
+
+
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
                        delta_softplus=False, nthreads=0, lib=None, reset=None, initial_state=None,
                        dlast_state=None, magnitudes=False):
