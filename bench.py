@@ -402,6 +402,9 @@ def bench_ours(args, w, world, rank, local):
     line["decode"] = bench_decode(wr, d, out_dtype, stream, world)
     if not args.no_bwd:
         line["backward"] = bench_backward(args, wr, d, host, out_dtype, flush, stream, sfu_peak, world)
+    if w.dtype == torch.bfloat16 and not args.no_per_config:
+        line["fused_dtproj"] = bench_dtproj(wr, dev, stream, flush, steps=max(3, min(args.steps, 20)), warmup=3,
+                                            sfu_peak=sfu_peak, unfused_ms=statistics.median(kernel_ms))
     if not args.no_per_config:
         # Every other configuration at full size, forward only, fewer steps
         # each (the headline value stays the workload above).
@@ -472,6 +475,43 @@ def bench_forward_config(w: W.Workload, dev, stream, flush, steps: int, warmup: 
     del d, y, last, ws
     torch.cuda.empty_cache()
     return out
+
+
+def bench_dtproj(w: W.Workload, dev, stream, flush, steps: int, warmup: int, sfu_peak: float, unfused_ms: float):
+    """Device time of the forward with delta produced inside the scan from its
+    low-rank input (ss_fwd_dtproj: delta = W_dt delta_r on the tensor cores,
+    dt_rank = ceil(d_model / 16) with d_model = dim / 2), beside the unfused
+    forward's time on the same layer."""
+    R = W.dt_rank_auto(w.dim // 2)
+    host = W.make_dtproj_inputs(w, R)
+    names_in = ("u", "delta_r", "W_dt", "A", "B", "C", "D", "z", "delta_bias")
+    d = {k: (host[k].to(dev) if host[k] is not None else None) for k in names_in}
+    y = torch.empty(d["u"].shape, dtype=w.dtype, device=dev)
+
+    def launch():
+        selscan.ss_fwd_dtproj(d["u"], d["delta_r"], d["W_dt"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
+                              delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, stream=stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        launch()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        launch()
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.median(ts)
+    status = selscan.ss_device_status()
+    del d, y
+    return {"ms": ms, "dt_rank": R, "updates_per_s": w.updates / (ms * 1e-3),
+            "sfu_frac": w.updates / sfu_peak / (ms * 1e-3), "unfused_ms": unfused_ms,
+            "vs_unfused": unfused_ms / ms, "steps": steps, "device_status": status,
+            "note": "delta = W_dt delta_r (tcgen05 bf16 MMA into tensor memory, one 64-step stage ahead of "
+                    "the scan) instead of reading delta; delta_r (B, dt_rank, L) and W_dt (D, dt_rank) bf16"}
 
 
 def bench_decode(w, d, out_dtype, stream, world, calls=200):

@@ -117,6 +117,11 @@ ss_status ss_fwd(const ss_desc *desc, const void *u, const void *delta, const fl
  *   split_states = 1: the lanes (1, 2, 4 or 8, at most half the state bucket
  *     4/8/16/32/64 that holds dstate) split the row's states and each runs
  *     every step;
+ *   split_states = 2: as 1, with B and C reaching the lanes through tensor
+ *     memory (a tcgen05 MMA with a 0/1 selection matrix broadcasts each
+ *     lane's B/C values into its TMEM lane).  bf16 inputs; 2 lanes holding
+ *     4 or 8 states each, or 4 or 8 lanes holding 2 or 4 states each; no
+ *     sequence starts; warps_per_block 0 or 4;
  *   one lane: the row's sequential recurrence in one lane, either way.
  * warps_per_block in {1,2,4,8}.
  * segments (states split or one lane only): 1 runs each row's whole sequence
@@ -238,9 +243,32 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
                         ss_stream_t stream);
 
 /*
+ * The forward with delta produced inside the scan by the dt_proj map of the
+ * mamba-minimal block (Mamba-minimal项目解析, 核心组件解析 §5 ssm: x_dbl = x_proj(x)
+ * splits into delta (dt_rank features), B and C, and delta =
+ * softplus(dt_proj(delta))): delta[b, d, l] = sum_r W_dt[d, r] delta_r[b, r, l],
+ * then the scan of ss_fwd_ws with delta_bias as dt_proj's bias.  The product
+ * runs on the tensor cores (tcgen05, bf16 operands, fp32 accumulation in
+ * tensor memory) one 64-step stage ahead of the scan, so delta never goes
+ * through device memory.
+ *   dt_rank   1..64 (the features of delta_r)
+ *   delta_r   device, (B, dt_rank, L) bf16, l contiguous (the layout of B and C)
+ *   W_dt      device, (D, dt_rank) bf16 (dt_proj's weight)
+ * desc->in_dtype must be SS_BF16 (SS_ERR_UNSUPPORTED_DTYPE otherwise); the
+ * launch is the direct kernel with 2 or 4 lanes per row (the heuristic's
+ * when it is one of those); no sequence starts and no initial state.  Other
+ * arguments, workspace and errors as ss_fwd_ws; SS_ERR_BAD_SHAPE for a
+ * dt_rank outside 1..64.
+ */
+ss_status ss_fwd_dtproj(const ss_desc *desc, int dt_rank, const void *u, const void *delta_r,
+                        const void *W_dt, const float *A, const void *B, const void *C, const float *D,
+                        const void *z, const float *delta_bias, int delta_softplus, void *y,
+                        float *last_state, void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
+/*
  * Bytes of the device scratch array built into the library for
- * ss_fwd_noalloc (8 MiB per device; 4.7 MB covers a 4 x 1024-channel,
- * 16-state layer over 100000 steps).
+ * ss_fwd_noalloc (8 MiB per device; a 4 x 1024-channel, 16-state layer over
+ * 100000 steps needs 4,456,448 bytes = 4.25 MiB in its default launch shape).
  */
 #define SS_NOALLOC_SCRATCH_BYTES (8u << 20)
 
@@ -258,7 +286,10 @@ ss_status ss_fwd_hostio(const ss_desc *desc, const void *h_u, const void *h_delt
  *     NULL) says how much it needs); other errors as ss_fwd_ws.
  *   - The first call on each device (the device current at the call) looks
  *     up the array's device address with cudaGetSymbolAddress and caches it;
- *     make that first call before any stream capture on that device.
+ *     make that first call before any stream capture on that device.  The
+ *     cached address belongs to that device context: after cudaDeviceReset
+ *     on the device it is stale, so do not call ss_fwd_noalloc on that
+ *     device again in the same process.
  *   - All calls on one device share the one array: calls whose work overlaps
  *     on the GPU (other streams, other host threads) race on it and give
  *     wrong results.  Calls queued in order on one stream are safe.
@@ -324,7 +355,36 @@ ss_status ss_bwd_reset(const ss_desc *desc, const void *u, const void *delta, co
                        float *dD, void *dz, float *ddelta_bias, void *workspace,
                        size_t workspace_bytes, ss_stream_t stream);
 
-/* Bytes of workspace ss_bwd and ss_bwd_reset need for `desc` (0 for an invalid descriptor). */
+/*
+ * The backward of the forward from a given state (ss_fwd_state, or
+ * ss_fwd_reset with sequence starts), for training a long sequence piece by
+ * piece: each piece runs from the last state of the piece before, and the
+ * gradient flows back through those states.  The loss is sum(dy * y) plus,
+ * when d_last_state is given, sum(d_last_state * h_(L-1)) (the last state
+ * feeding the next piece).  The pages train the forward through autograd
+ * (Mamba代码实战 §6) and give no initial-state interface; this is the chain rule
+ * of the §3.2 loop started from h_(-1) = initial_state:
+ *   reset           device (B, L) bytes, or NULL: as ss_bwd_reset
+ *   initial_state   device (B, D, N) float32, or NULL (zero)
+ *   d_last_state    device (B, D, N) float32, or NULL (zero): the gradient
+ *                   with respect to the state after step L-1
+ *   d_initial_state device (B, D, N) float32 output, or NULL (not written):
+ *                   the gradient with respect to the state before step 0,
+ *                   a_0 * lam_0 (zero where a sequence starts at step 0;
+ *                   d_last_state when L = 0)
+ * Other arguments, workspace (ss_bwd_workspace_bytes) and errors as ss_bwd.
+ * A piece's d_initial_state passed as the previous piece's d_last_state
+ * gives, piece by piece, the gradients of the whole sequence.
+ */
+ss_status ss_bwd_state(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const uint8_t *reset,
+                       const float *initial_state, const float *d_last_state, const void *dy, void *du,
+                       void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz,
+                       float *ddelta_bias, float *d_initial_state, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream);
+
+/* Bytes of workspace ss_bwd, ss_bwd_reset and ss_bwd_state need for `desc` (0 for an invalid descriptor). */
 size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 
 /*
@@ -354,6 +414,18 @@ const char *ss_status_string(ss_status status);
 
 /* SS_VERSION of the built library. */
 int ss_version(void);
+
+/*
+ * The current device's status word, then cleared (no counterpart on the
+ * pages).  A kernel that waits on other warps of its block (the
+ * tensor-memory-fed forward, split_states = 2) bounds every wait to about a
+ * second; if one runs out it records SS_DEVICE_TIMEOUT here, stops, frees
+ * its tensor memory and returns, so the context stays usable.  *code = 0
+ * when nothing was recorded.  Synchronous (copies from the device);
+ * SS_ERR_CUDA when the word cannot be read.
+ */
+#define SS_DEVICE_TIMEOUT 1
+ss_status ss_device_status(int *code);
 
 #ifdef __cplusplus
 }

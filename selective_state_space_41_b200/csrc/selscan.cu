@@ -13,10 +13,16 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <mutex>
+
 #include "selscan.h"
 #include "ss_bwd_launch.h"
 #include "ss_step_kernel.cuh"
 #include "ss_launch.h"
+
+// The device status word: a kernel whose bounded wait ran out writes a
+// nonzero code here (read and cleared by ss_device_status).
+static __device__ int g_ss_device_status;
 
 namespace {
 
@@ -24,6 +30,42 @@ using selscan::FwdParams;
 
 constexpr int kMaxState = 64;
 constexpr int kMaxDevices = 64;
+
+// Device address of g_ss_device_status on the current device (looked up once
+// per device), or null when the runtime cannot give it (then the kernels
+// record nothing).
+int *device_status_ptr() {
+    static std::mutex mu;
+    static int *addr[kMaxDevices];
+    static bool tried[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!tried[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_ss_device_status) == cudaSuccess) addr[dev] = static_cast<int *>(p);
+        else (void)cudaGetLastError();
+        tried[dev] = true;
+    }
+    return addr[dev];
+}
+
+// TMEM-fed direct kernel (split_states = 2): bf16 inputs, a state split and
+// bucket it is built for.
+bool tmem_ok(const ss_desc *desc, int lanes) {
+    return desc->in_dtype == SS_BF16 && selscan::tmem_supported(selscan::state_bucket((int)desc->dstate), lanes);
+}
+size_t tmem_smem(int nmax, int lanes) {
+    switch (nmax * 16 + lanes) {
+        case 8 * 16 + 2: return selscan::tmem_smem_bytes<8, 2>();
+        case 8 * 16 + 4: return selscan::tmem_smem_bytes<8, 4>();
+        case 16 * 16 + 2: return selscan::tmem_smem_bytes<16, 2>();
+        case 16 * 16 + 4: return selscan::tmem_smem_bytes<16, 4>();
+        case 16 * 16 + 8: return selscan::tmem_smem_bytes<16, 8>();
+        case 32 * 16 + 8: return selscan::tmem_smem_bytes<32, 8>();
+        default: return 0;
+    }
+}
 
 size_t dtype_size(ss_dtype t) { return t == SS_BF16 ? 2 : 4; }
 
@@ -77,6 +119,7 @@ int sm_count() {
 // bucket as fp32, plus a raw copy in the input dtype (see the kernel).
 size_t smem_for(const ss_desc *desc, int lanes, int split, int warps) {
     const int nmax = selscan::state_bucket((int)desc->dstate);
+    if (split == 2) return tmem_smem(nmax, lanes);
     if (lanes == 1 || split) return selscan::direct_smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
     return selscan::smem_bytes(dtype_size(desc->in_dtype), nmax, lanes, warps);
 }
@@ -172,7 +215,7 @@ ss_status resolve(const ss_desc *desc, int64_t rows, const ss_launch_config *cfg
     if (cfg) {
         const int lanes = cfg->lanes_per_row, warps = cfg->warps_per_block, split = cfg->split_states;
         if (lanes != 0 && (lanes < 1 || lanes > 32 || (lanes & (lanes - 1)) != 0)) return SS_ERR_BAD_CONFIG;
-        if (split != 0 && split != 1) return SS_ERR_BAD_CONFIG;
+        if (split != 0 && split != 1 && split != 2) return SS_ERR_BAD_CONFIG;
         if (warps != 0 && warps != 1 && warps != 2 && warps != 4 && warps != 8) return SS_ERR_BAD_CONFIG;
         if (cfg->segments < 0) return SS_ERR_BAD_CONFIG;
         if (lanes != 0) {
@@ -195,6 +238,11 @@ ss_status resolve(const ss_desc *desc, int64_t rows, const ss_launch_config *cfg
         return SS_ERR_BAD_CONFIG;
     if (pl.nseg > 1 && !direct) return SS_ERR_BAD_CONFIG;  // segments run in the direct kernel
     if (direct_only && !direct) return SS_ERR_BAD_CONFIG;  // sequence starts: direct kernel only
+    if (pl.split == 2) {  // TMEM-fed: bf16, a supported split, 4 compute warps, no sequence starts
+        if (!tmem_ok(desc, pl.lanes) || direct_only) return SS_ERR_BAD_CONFIG;
+        if (cfg && cfg->warps_per_block != 0 && cfg->warps_per_block != 4) return SS_ERR_BAD_CONFIG;
+        pl.warps = 4;
+    }
     if (pl.nseg < 1) pl.nseg = 1;
     if (pl.nseg == 1) pl.seg_len = desc->seqlen;
     *out = pl;
@@ -224,52 +272,71 @@ cudaError_t launch_bf16_f32(int n, int lanes, int split, dim3 grid, dim3 block, 
     SS_PICK_BUCKET(launch_bf16_f32)
 }
 
-template <typename Tin, typename Tout>
-void launch_fixup_t(int nmax, dim3 grid, cudaStream_t s, const FwdParams &p) {
-    switch (nmax) {
-        case 4: selscan::ss_fwd_fixup_kernel<Tin, Tout, 4><<<grid, 256, 0, s>>>(p); break;
-        case 8: selscan::ss_fwd_fixup_kernel<Tin, Tout, 8><<<grid, 256, 0, s>>>(p); break;
-        case 16: selscan::ss_fwd_fixup_kernel<Tin, Tout, 16><<<grid, 256, 0, s>>>(p); break;
-        case 32: selscan::ss_fwd_fixup_kernel<Tin, Tout, 32><<<grid, 256, 0, s>>>(p); break;
-        default: selscan::ss_fwd_fixup_kernel<Tin, Tout, 64><<<grid, 256, 0, s>>>(p); break;
-    }
-}
-
+// The fix-up after a segmented direct kernel: the carry fold (one warp per
+// row), then the correction of y (one warp per (row, segment >= 1)).
 cudaError_t launch_fixup(const ss_desc *desc, int64_t rows, int nseg, cudaStream_t s, const FwdParams &p) {
     const int nmax = selscan::state_bucket((int)desc->dstate);
-    const int64_t threads = rows * nseg * (nmax / 4);  // 4 states per thread
-    const dim3 grid((unsigned)((threads + 255) / 256));
-    if (desc->in_dtype == SS_F32)
-        launch_fixup_t<float, float>(nmax, grid, s, p);
-    else if (desc->out_dtype == SS_BF16)
-        launch_fixup_t<__nv_bfloat16, __nv_bfloat16>(nmax, grid, s, p);
+    const dim3 fold_grid((unsigned)((rows + 7) / 8));
+    if (nmax > 32)
+        selscan::ss_fwd_carry_kernel<64><<<fold_grid, 256, 0, s>>>(p);
     else
-        launch_fixup_t<__nv_bfloat16, float>(nmax, grid, s, p);
+        selscan::ss_fwd_carry_kernel<32><<<fold_grid, 256, 0, s>>>(p);
+    const int64_t tasks = rows * (nseg - 1);
+    const dim3 grid((unsigned)((tasks + selscan::kFixupWarps - 1) / selscan::kFixupWarps));
+    const dim3 block(selscan::kFixupWarps * 32);
+    if (desc->in_dtype == SS_F32)
+        selscan::ss_fwd_fixup_kernel<float, float><<<grid, block, 0, s>>>(p);
+    else if (desc->out_dtype == SS_BF16)
+        selscan::ss_fwd_fixup_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, block, 0, s>>>(p);
+    else
+        selscan::ss_fwd_fixup_kernel<__nv_bfloat16, float><<<grid, block, 0, s>>>(p);
     return cudaGetLastError();
+}
+
+// The dt_proj form (delta_r given): bf16, the direct kernel with 4 warps and
+// 2 or 4 lanes per row (double-buffered stages); the heuristic's state split
+// and segments when they fit, else 4 (or 2) lanes and one pass.
+bool dt_plan(const ss_desc *desc, Plan *pl) {
+    const int bucket = selscan::state_bucket((int)desc->dstate);
+    auto fits = [&](int g) { return g <= bucket / 2 && selscan::direct_double_buffer(bucket, g); };
+    if (!((pl->split == 1 || pl->lanes == 1) && (pl->lanes == 2 || pl->lanes == 4) && fits(pl->lanes))) {
+        pl->lanes = fits(4) ? 4 : fits(2) ? 2 : 0;
+        pl->nseg = 1;
+        pl->seg_len = desc->seqlen;
+    }
+    pl->split = 1;
+    pl->warps = 4;
+    return pl->lanes != 0;
 }
 
 ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D, const void *z,
                    const float *delta_bias, int delta_softplus, const float *initial_state,
                    const uint8_t *reset, void *y, float *last_state, const ss_launch_config *cfg,
-                   void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+                   void *workspace, size_t workspace_bytes, ss_stream_t stream,
+                   const void *delta_r = nullptr, const void *W_dt = nullptr, int dt_rank = 0) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
     if (!workspace) workspace_bytes = 0;
+    const bool dt = dt_rank != 0;  // the dt_proj form (ss_fwd_dtproj)
+    if (dt && desc->in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED_DTYPE;
+    if (dt && (dt_rank < 1 || dt_rank > selscan::kMaxDtRank)) return SS_ERR_BAD_SHAPE;
     Plan pl;
     st = resolve(desc, sz.rows, cfg, workspace_bytes, &pl, reset != nullptr);
     if (st != SS_OK) return st;
+    if (dt && !dt_plan(desc, &pl)) return SS_ERR_BAD_CONFIG;
     if (sz.rows == 0) return SS_OK;  // no rows: nothing to read or write
     const bool need_seq = desc->seqlen > 0;
     if (!A) return SS_ERR_NULL_POINTER;
-    if (need_seq && (!u || !delta || !B || !C || !y)) return SS_ERR_NULL_POINTER;
+    if (need_seq && (!u || (!dt && !delta) || (dt && (!delta_r || !W_dt)) || !B || !C || !y))
+        return SS_ERR_NULL_POINTER;
     if (!need_seq && !last_state) return SS_OK;  // nothing to write
     if (!need_seq) pl.nseg = 1, pl.seg_len = 0;
     if (initial_state && !aligned(initial_state, 4)) return SS_ERR_MISALIGNED;
 
     const size_t ein = dtype_size(desc->in_dtype), eout = dtype_size(desc->out_dtype);
-    const void *in_ptrs[] = {u, delta, B, C, z};
+    const void *in_ptrs[] = {u, delta, B, C, z, delta_r, W_dt};
     for (const void *q : in_ptrs)
         if (q && !aligned(q, ein)) return SS_ERR_MISALIGNED;
     if ((y && !aligned(y, eout)) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
@@ -281,13 +348,17 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
 
     // 16-byte vector path: every row of every streamed tensor starts aligned.
     bool vec = (desc->seqlen * (int64_t)ein) % 16 == 0 && (desc->seqlen * (int64_t)eout) % 16 == 0;
-    for (const void *q : in_ptrs)
+    for (const void *q : {u, delta, B, C, z, delta_r})
         if (q && !aligned(q, 16)) vec = false;
     if (y && !aligned(y, 16)) vec = false;
 
-    const size_t smem = smem_for(desc, pl.lanes, pl.split, pl.warps);
+    size_t smem = smem_for(desc, pl.lanes, pl.split, pl.warps);
+    if (dt) {  // + the dt_proj operands; at least 47 KB so that at most 4 blocks (4 x 128 TMEM columns) share an SM
+        smem += selscan::direct_dt_extra_bytes((dt_rank + 15) / 16 * 16);
+        if (smem < 47 * 1024) smem = 47 * 1024;
+    }
     if (smem > selscan::kMaxSmemBytes) return SS_ERR_BAD_CONFIG;
-    const int64_t rows_per_block = (int64_t)pl.warps * (32 / pl.lanes);
+    const int64_t rows_per_block = (int64_t)pl.warps * (32 / pl.lanes);  // compute warps
     const int64_t dtiles = (desc->dim + rows_per_block - 1) / rows_per_block;
     const int64_t blocks = dtiles * desc->batch * pl.nseg;
     if (blocks > INT_MAX || sz.rows * pl.nseg > INT_MAX) return SS_ERR_BAD_SHAPE;
@@ -316,6 +387,10 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.nseg = pl.nseg;
     p.ws_hend = pl.nseg > 1 ? static_cast<float *>(workspace) : nullptr;
     p.ws_dsum = pl.nseg > 1 ? p.ws_hend + (size_t)pl.nseg * sz.rows * desc->dstate : nullptr;
+    p.status = (pl.split == 2 || dt) ? device_status_ptr() : nullptr;
+    p.delta_r = delta_r;
+    p.W_dt = W_dt;
+    p.dt_rank = dt_rank;
 
     const dim3 grid((unsigned)blocks), block((unsigned)(pl.warps * 32));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -334,9 +409,20 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
 // ---------------------------------------------------------------- backward
 constexpr int kBwdWarps = selscan::kBwdThreads / 32;
 
+// The backward runs the batch in groups of `group` entries, one launch of
+// the adjoint kernel (and of the dB/dC sum) per group, so that the
+// checkpoints and the dB/dC block partials, which grow with B*D*L*N, are
+// held for one group at a time: the workspace of a group stays within
+// kBwdGroupBytes (whole batch entries, at least one; groups of equal size up
+// to the last).  The per-row partials of dA, dD and ddelta_bias are kept for
+// every row and summed once at the end, in batch order, so the grouping
+// changes no result bit.
+constexpr size_t kBwdGroupBytes = (size_t)7 << 30;
+
 struct BwdLayout {
     int lanes, rows;        // lanes per row, rows per block
     int64_t dtiles, nsub;
+    int64_t group;          // batch entries per launch
     size_t off_ckpt, off_dbc, off_dA, off_dD, off_dbias, total;  // workspace byte offsets
 };
 
@@ -350,9 +436,20 @@ BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz) {
     lo.dtiles = (desc->dim + lo.rows - 1) / lo.rows;
     lo.nsub = (desc->seqlen + selscan::kBwdSub - 1) / selscan::kBwdSub;
     const size_t N = (size_t)desc->dstate, rows = (size_t)sz.rows, L = (size_t)desc->seqlen;
+    // bytes one batch entry adds to the checkpoints and the block partials
+    const size_t per_entry = (size_t)desc->dim * (size_t)lo.nsub * N * 4 + (size_t)lo.dtiles * 2 * N * L * 4;
+    int64_t group = desc->batch;
+    if (per_entry > 0 && desc->batch > 0) {
+        const int64_t fit = (int64_t)(kBwdGroupBytes / per_entry);
+        const int64_t cap = fit < 1 ? 1 : fit;
+        const int64_t ngroups = (desc->batch + cap - 1) / cap;
+        group = (desc->batch + ngroups - 1) / ngroups;
+    }
+    lo.group = group;
+    const size_t grows = (size_t)group * (size_t)desc->dim;
     lo.off_ckpt = 0;
-    lo.off_dbc = align256(lo.off_ckpt + rows * (size_t)lo.nsub * N * 4);
-    lo.off_dA = align256(lo.off_dbc + (size_t)lo.dtiles * (size_t)desc->batch * 2 * N * L * 4);
+    lo.off_dbc = align256(lo.off_ckpt + grows * (size_t)lo.nsub * N * 4);
+    lo.off_dA = align256(lo.off_dbc + (size_t)lo.dtiles * (size_t)group * 2 * N * L * 4);
     lo.off_dD = align256(lo.off_dA + rows * N * 4);
     lo.off_dbias = align256(lo.off_dD + rows * 4);
     lo.total = align256(lo.off_dbias + rows * 4);
@@ -412,6 +509,15 @@ ss_status ss_fwd_state(const ss_desc *desc, const void *u, const void *delta, co
                        size_t workspace_bytes, ss_stream_t stream) {
     return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, nullptr,
                     y, last_state, config, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_fwd_dtproj(const ss_desc *desc, int dt_rank, const void *u, const void *delta_r,
+                        const void *W_dt, const float *A, const void *B, const void *C, const float *D,
+                        const void *z, const float *delta_bias, int delta_softplus, void *y,
+                        float *last_state, void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+    if (dt_rank == 0) return SS_ERR_BAD_SHAPE;
+    return fwd_impl(desc, u, nullptr, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y, last_state,
+                    nullptr, workspace, workspace_bytes, stream, delta_r, W_dt, dt_rank);
 }
 
 ss_status ss_fwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
@@ -602,8 +708,9 @@ namespace {
 
 ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
                    const void *C, const float *D, const void *z, const float *delta_bias,
-                   int delta_softplus, const uint8_t *reset, const void *dy, void *du, void *ddelta,
-                   float *dA, float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                   int delta_softplus, const uint8_t *reset, const float *init_state,
+                   const float *dlast, const void *dy, void *du, void *ddelta, float *dA, float *dB,
+                   float *dC, float *dD, void *dz, float *ddelta_bias, float *d_init_state,
                    void *workspace, size_t workspace_bytes, ss_stream_t stream) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
@@ -616,14 +723,14 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     const void *in_ptrs[] = {u, delta, B, C, z, du, ddelta, dz};
     for (const void *q : in_ptrs)
         if (q && !aligned(q, ein)) return SS_ERR_MISALIGNED;
-    const void *f_ptrs[] = {A, D, delta_bias, dA, dB, dC, dD, ddelta_bias};
+    const void *f_ptrs[] = {A, D, delta_bias, dA, dB, dC, dD, ddelta_bias, init_state, dlast, d_init_state};
     for (const void *q : f_ptrs)
         if (q && !aligned(q, 4)) return SS_ERR_MISALIGNED;
     if (dy && !aligned(dy, eout)) return SS_ERR_MISALIGNED;
     const BwdLayout lo = bwd_layout(desc, sz);
     if (!workspace || workspace_bytes < lo.total) return SS_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return SS_ERR_MISALIGNED;
-    const int64_t blocks = lo.dtiles * desc->batch;
+    const int64_t blocks = lo.dtiles * lo.group;
     if (blocks > INT_MAX) return SS_ERR_BAD_SHAPE;
 
     char *ws = static_cast<char *>(workspace);
@@ -647,6 +754,9 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.nsub = lo.nsub;
     p.reset = reset;
     p.reset_vec = reset && desc->seqlen % selscan::kBwdSub == 0 && aligned(reset, selscan::kBwdSub);
+    p.init_state = init_state;
+    p.dlast = dlast;
+    p.d_init_state = d_init_state;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int nmax = selscan::state_bucket(p.dstate), n = nmax;
@@ -656,12 +766,41 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
             desc->in_dtype == SS_F32 ? (SS_PICK_BWD(bwd_f32_f32))
             : desc->out_dtype == SS_BF16 ? (SS_PICK_BWD(bwd_bf16_bf16))
                                          : (SS_PICK_BWD(bwd_bf16_f32));
-        if (fn(dim3((unsigned)blocks), dim3(kBwdWarps * 32), smem, s, p) != cudaSuccess) return SS_ERR_CUDA;
-        const int64_t bc = desc->batch * 2 * desc->dstate * desc->seqlen;
-        if (bc > 0) {
-            const int64_t gb = (bc + 255) / 256;
-            selscan::ss_bwd_reduce_bc_kernel<<<(unsigned)(gb < 4 * 148 * 8 ? gb : 4 * 148 * 8), 256, 0, s>>>(p, dB, dC);
-            if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+        // One launch per batch group: every pointer indexed by batch entry
+        // starts at the group's first entry; checkpoints and block partials
+        // are reused, the per-row partials go to the group's rows.
+        const int64_t DL = desc->dim * desc->seqlen, NL = desc->dstate * desc->seqlen;
+        const int64_t DN = desc->dim * desc->dstate;
+        for (int64_t b0 = 0; b0 < desc->batch; b0 += lo.group) {
+            const int64_t gb = desc->batch - b0 < lo.group ? desc->batch - b0 : lo.group;
+            selscan::BwdParams q = p;
+            auto adv = [](const void *ptr, int64_t elems, size_t es) -> const void * {
+                return ptr ? static_cast<const char *>(ptr) + elems * (int64_t)es : nullptr;
+            };
+            auto advm = [](void *ptr, int64_t elems, size_t es) -> void * {
+                return ptr ? static_cast<char *>(ptr) + elems * (int64_t)es : nullptr;
+            };
+            q.batch = gb;
+            q.u = adv(u, b0 * DL, ein), q.delta = adv(delta, b0 * DL, ein), q.z = adv(z, b0 * DL, ein);
+            q.dy = adv(dy, b0 * DL, eout);
+            q.B = adv(B, b0 * NL, ein), q.C = adv(C, b0 * NL, ein);
+            q.du = advm(du, b0 * DL, ein), q.ddelta = advm(ddelta, b0 * DL, ein), q.dz = advm(dz, b0 * DL, ein);
+            q.ws_dA = p.ws_dA + b0 * DN;
+            q.ws_dD = p.ws_dD + b0 * desc->dim;
+            q.ws_dbias = p.ws_dbias + b0 * desc->dim;
+            q.reset = reset ? reset + b0 * desc->seqlen : nullptr;
+            q.init_state = init_state ? init_state + b0 * DN : nullptr;
+            q.dlast = dlast ? dlast + b0 * DN : nullptr;
+            q.d_init_state = d_init_state ? d_init_state + b0 * DN : nullptr;
+            if (fn(dim3((unsigned)(lo.dtiles * gb)), dim3(kBwdWarps * 32), smem, s, q) != cudaSuccess)
+                return SS_ERR_CUDA;
+            const int64_t bc = gb * 2 * NL;
+            if (bc > 0) {
+                const int64_t nb = (bc + 255) / 256;
+                selscan::ss_bwd_reduce_bc_kernel<<<(unsigned)(nb < 4 * 148 * 8 ? nb : 4 * 148 * 8), 256, 0, s>>>(
+                    q, dB + b0 * NL, dC + b0 * NL);
+                if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+            }
         }
     }
     const int64_t rr = desc->dim * (desc->dstate + 2);
@@ -683,8 +822,8 @@ ss_status ss_bwd(const ss_desc *desc, const void *u, const void *delta, const fl
                  int delta_softplus, const void *dy, void *du, void *ddelta, float *dA, float *dB,
                  float *dC, float *dD, void *dz, float *ddelta_bias, void *workspace,
                  size_t workspace_bytes, ss_stream_t stream) {
-    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, dy, du, ddelta,
-                    dA, dB, dC, dD, dz, ddelta_bias, workspace, workspace_bytes, stream);
+    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, nullptr, dy,
+                    du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, nullptr, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_bwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
@@ -694,8 +833,20 @@ ss_status ss_bwd_reset(const ss_desc *desc, const void *u, const void *delta, co
                        float *dD, void *dz, float *ddelta_bias, void *workspace,
                        size_t workspace_bytes, ss_stream_t stream) {
     if (!reset && desc && desc->batch > 0 && desc->dim > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
-    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, reset, dy, du, ddelta,
-                    dA, dB, dC, dD, dz, ddelta_bias, workspace, workspace_bytes, stream);
+    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, reset, nullptr, nullptr, dy,
+                    du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, nullptr, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_bwd_state(const ss_desc *desc, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, const uint8_t *reset,
+                       const float *initial_state, const float *d_last_state, const void *dy, void *du,
+                       void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz,
+                       float *ddelta_bias, float *d_initial_state, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream) {
+    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, reset, initial_state,
+                    d_last_state, dy, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, d_initial_state, workspace,
+                    workspace_bytes, stream);
 }
 
 ss_status ss_step(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
@@ -753,5 +904,19 @@ const char *ss_status_string(ss_status status) {
 }
 
 int ss_version(void) { return SS_VERSION; }
+
+ss_status ss_device_status(int *code) {
+    if (!code) return SS_ERR_NULL_POINTER;
+    *code = 0;
+    if (!device_status_ptr()) return SS_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_ss_device_status, sizeof(int)) != cudaSuccess) return SS_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_ss_device_status, &zero, sizeof(int)) != cudaSuccess) return SS_ERR_CUDA;
+    }
+    *code = v;
+    return SS_OK;
+}
 
 }  // extern "C"

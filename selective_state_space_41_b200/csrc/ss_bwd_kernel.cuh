@@ -28,6 +28,12 @@
 // entering a start is zero), h_(l-1) has no part in h_l at a start l: both
 // passes zero the state entering it, and the adjoint passes nothing from l to
 // l-1 and has no h_(l-1) term there (ddelta', dA).
+// From a given state (p.init_state, the forward of ss_fwd_state): phase A
+// starts from it, and the adjoint carried past step 0, a_0 lam_0, is the
+// gradient with respect to it (p.d_init_state).  With a gradient on the last
+// state (p.dlast: the loss also has sum(dlast h_(L-1)), as when the state
+// feeds the next piece of a sequence) the adjoint starts from dlast instead
+// of zero past the end.
 #pragma once
 
 #include <type_traits>
@@ -53,6 +59,9 @@ struct BwdParams {
     int64_t nsub;                             // sub-chunks per row
     const uint8_t *reset;                     // (batch, seqlen) sequence starts, or null
     int reset_vec;                            // every 8-step group of reset is 8-byte aligned
+    const float *init_state;                  // (batch, dim, dstate) state before step 0, or null (zero)
+    const float *dlast;                       // (batch, dim, dstate) gradient wrt the last state, or null
+    float *d_init_state;                      // (batch, dim, dstate) gradient wrt the state before step 0, or null
 };
 
 constexpr int kBwdSub = 8;                    // steps per sub-chunk
@@ -279,7 +288,14 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     // ---------------------------------------------------------------- phase A
     float2 h[kPL];
 #pragma unroll
-    for (int qq = 0; qq < kPL; ++qq) h[qq] = make_float2(0.f, 0.f);
+    for (int qq = 0; qq < kPL; ++qq) {  // the state before step 0 (mirrored rows: the true row's)
+        const int n = 2 * (q0 + qq);
+        h[qq] = make_float2(0.f, 0.f);
+        if (p.init_state != nullptr) {
+            if (n < N) h[qq].x = p.init_state[row * N + n];
+            if (n + 1 < N) h[qq].y = p.init_state[row * N + n + 1];
+        }
+    }
     uint32_t wu[kInWords], wd[kInWords];  // raw owned inputs of the next sub-chunk
     if (L > 0) {
         load_own(u_row, j0, wu);
@@ -363,9 +379,16 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     }
 
     // ---------------------------------------------------------------- phase B
-    float2 carry[kPL], dA_acc[kPL];
+    float2 carry[kPL], dA_acc[kPL];  // carry: a_(l+1) lam_(l+1); past the end, dlast (or zero)
 #pragma unroll
-    for (int qq = 0; qq < kPL; ++qq) carry[qq] = make_float2(0.f, 0.f), dA_acc[qq] = make_float2(0.f, 0.f);
+    for (int qq = 0; qq < kPL; ++qq) {
+        const int n = 2 * (q0 + qq);
+        carry[qq] = make_float2(0.f, 0.f), dA_acc[qq] = make_float2(0.f, 0.f);
+        if (p.dlast != nullptr && row_ok) {  // mirrored rows carry nothing (they add to dB, dC)
+            if (n < N) carry[qq].x = p.dlast[row * N + n];
+            if (n + 1 < N) carry[qq].y = p.dlast[row * N + n + 1];
+        }
+    }
     float dD_acc = 0.f, dbias_acc = 0.f;
     const int64_t nstages = (L + kBwdStage - 1) / kBwdStage;
     // Prefetched for the next sub-chunk (backwards): its checkpoint and raw owned inputs.
@@ -550,6 +573,15 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         }
     }
 
+    // The adjoint carried past step 0 is the gradient wrt the state before it.
+    if (p.d_init_state != nullptr && row_ok) {
+#pragma unroll
+        for (int qq = 0; qq < kPL; ++qq) {
+            const int n = 2 * (q0 + qq);
+            if (n < N) p.d_init_state[row * N + n] = carry[qq].x;
+            if (n + 1 < N) p.d_init_state[row * N + n + 1] = carry[qq].y;
+        }
+    }
     // Per-row partials of dA, dD and dbias.
     if (row_ok) {
 #pragma unroll

@@ -38,6 +38,8 @@
 
 #include <type_traits>
 
+#include "ss_tcgen05.cuh"
+
 namespace selscan {
 
 constexpr size_t kMaxSmemBytes = 227 * 1024;  // opt-in dynamic shared memory per block (sm_100)
@@ -67,6 +69,14 @@ struct FwdParams {
     int64_t seg_len;
     int nseg;
     float *ws_hend, *ws_dsum;
+    // Device status word (or null): a kernel whose bounded wait ran out
+    // writes a nonzero code here (the kernels that use tensor memory).
+    int *status;
+    // The dt_proj form of delta (delta null, direct kernel, bf16):
+    // delta[b, d, l] = sum_r W_dt[d, r] delta_r[b, r, l], delta_r (batch,
+    // dt_rank, L) and W_dt (dim, dt_rank) in the input dtype.
+    const void *delta_r, *W_dt;
+    int dt_rank;
 };
 
 // ------------------------------------------------------------ element I/O
@@ -157,12 +167,6 @@ __device__ __forceinline__ float sfu_exp2(float x) {
     return r;
 }
 
-// log2(x) on the SFU (MUFU.LG2).
-__device__ __forceinline__ float sfu_log2(float x) {
-    float r;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
 
 // 1/x on the SFU (MUFU.RCP).
 __device__ __forceinline__ float sfu_rcp(float x) {
@@ -171,24 +175,36 @@ __device__ __forceinline__ float sfu_rcp(float x) {
     return r;
 }
 
-constexpr float kLn2 = 0.6931471805599453f;
+
+// log1p(t) / t for t in [0, 1]: the degree-7 polynomial through that
+// function's values at the 8 Chebyshev nodes of [0, 1] (Chebyshev
+// interpolation, within a small factor of the minimax error: 2.2e-7 relative
+// with exact coefficients, 2.8e-7 with these fp32 ones evaluated in fp32 by
+// Horner's rule), the coefficients as immediates of the FMAs.
+__device__ __forceinline__ float log1p_over_t(float t) {
+    float q = fmaf(-0.00837115291506052f, t, 0.04349390044808388f);
+    q = fmaf(q, t, -0.1068500280380249f);
+    q = fmaf(q, t, 0.1768747717142105f);
+    q = fmaf(q, t, -0.24474774301052094f);
+    q = fmaf(q, t, 0.3327192962169647f);
+    q = fmaf(q, t, -0.49997174739837646f);
+    return fmaf(q, t, 0.9999997615814209f);
+}
 
 // delta' of §2.2: torch's softplus (beta 1, linear above 20) or exp.
 // kFast (bf16 inputs, whose values carry 2^-9 relative rounding):
-//   softplus(x) = ln2 * log2(1 + e), e = 2^(x log2 e), on the SFU; when
-//   e < 1/32 the rounding of 1 + e would dominate, so log1p(e) is taken from
-//   its series e - e^2/2 + e^3/3 - e^4/4 (relative error below e^4/5 < 2e-7).
-//   Relative error of delta' stays below about 1e-5.
+//   softplus(x) = max(x, 0) + log1p(t), t = exp(-|x|) = 2^(-|x| log2 e) in
+//   (0, 1] on the SFU (one MUFU op), log1p(t) = t P(t) with the polynomial
+//   above on the FMA pipe.  Above 20, t P(t) < 2.1e-9 is below half an ulp
+//   of x, so the sum is exactly x: torch's linear region.  Relative error
+//   below 2e-6 (the fp32 rounding of the exp argument dominates at large |x|).
 // Otherwise (fp32 inputs): libm-accurate log1pf(expf(x)) and expf(x).
 template <bool kFast>
 __device__ __forceinline__ float delta_transform(float x, bool softplus) {
     if constexpr (kFast) {
-        const float e = sfu_exp2(x * kLog2e);
-        if (!softplus) return e;
-        const float series = e * fmaf(-e, fmaf(-e, fmaf(-e, 0.25f, 1.f / 3.f), 0.5f), 1.f);
-        const float viaLog = sfu_log2(1.f + e) * kLn2;
-        const float sp = e < 0.03125f ? series : viaLog;
-        return x > 20.f ? x : sp;
+        if (!softplus) return sfu_exp2(x * kLog2e);
+        const float t = sfu_exp2(-fabsf(x) * kLog2e);
+        return fmaxf(x, 0.f) + t * log1p_over_t(t);
     } else {
         if (softplus) return x > 20.f ? x : log1pf(expf(x));
         return expf(x);
@@ -724,6 +740,20 @@ __host__ __device__ constexpr size_t direct_smem_bytes(size_t in_size, int nmax,
            (g > 1 ? sizeof(float) * (size_t)warps * ((32 / g) * gather_stride(g) + 32 * reduce_stride(g)) : 0);
 }
 
+// The dt_proj form (kDt): delta of the block's rows is one tensor-core
+// product per 64-step stage, delta[rows, steps] = W_dt[rows, :] x delta_r[:, steps]
+// (bf16 operands, fp32 accumulation in tensor memory), read by each lane for
+// its own steps.  Extra shared memory after the slabs (rpad: dt_rank rounded
+// up to 16): the A operand (W_dt rows of the 128 TMEM lanes, K-major, rpad/8
+// K halves of 128 x 16 bytes), three B operand buffers (delta_r of a stage
+// transposed, rpad/8 K halves of 64 x 16 bytes each), two mbarriers and the
+// TMEM address; plus 1 KB of alignment slack.
+__host__ __device__ constexpr size_t direct_dt_extra_bytes(int rpad) {
+    return 1024 + (size_t)rpad * 256 + 3 * (size_t)rpad * 128 + 64;
+}
+// Largest dt_rank of the dt_proj form.
+constexpr int kMaxDtRank = 64;
+
 // kW consecutive floats to / from shared memory as one access (kW in {1, 2, 4}).
 template <int kW>
 __device__ __forceinline__ void st_vec(float *p, const float *v) {
@@ -778,8 +808,9 @@ struct DirectOccupancy {
 #endif
 
 // kReset: the instance that reads p.reset (sequence starts inside the rows);
-// the other one has no code for it.
-template <typename Tin, typename Tout, int kNmax, int kG, bool kReset = false>
+// the other one has no code for it.  kDt: the instance whose delta is the
+// dt_proj product (p.delta_r, p.W_dt; 4 warps, bf16, 2 or 4 lanes per row).
+template <typename Tin, typename Tout, int kNmax, int kG, bool kReset = false, bool kDt = false>
 __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParams p) {
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                        // state pairs per lane
@@ -797,6 +828,8 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     constexpr int kAccs = kPL >= 4 ? 2 : 1;                 // y accumulators per step
     constexpr bool kFast = sizeof(Tin) == 2;
     constexpr bool kA2InRegs = kNmax / kG <= 32;
+    static_assert(!kDt || (sizeof(Tin) == 2 && (kG == 2 || kG == 4) && !kReset && direct_double_buffer(kNmax, kG)),
+                  "dt_proj form: bf16, 2 or 4 lanes per row, double-buffered stages, no sequence starts");
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
@@ -843,7 +876,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
                           static_cast<const Tin *>(p.C) + b * N * L};
     // This lane's first owned step of each stream (advanced per sub-chunk).
     const Tin *u_own = static_cast<const Tin *>(p.u) + row * L + c_begin + g * kOwn;
-    const Tin *d_own = static_cast<const Tin *>(p.delta) + row * L + c_begin + g * kOwn;
+    const Tin *d_own = kDt ? nullptr : static_cast<const Tin *>(p.delta) + row * L + c_begin + g * kOwn;
     const Tin *z_own = has_z ? static_cast<const Tin *>(p.z) + row * L + c_begin + g * kOwn : nullptr;
     Tout *const y_row = static_cast<Tout *>(p.y) + row * L;
     Tout *y_own = y_row + c_begin + g * kOwn;
@@ -961,8 +994,106 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     };
     load_starts(c_begin + g * kOwn);
     load_own_checked(u_own, c_begin + g * kOwn, wu);
-    load_own_checked(d_own, c_begin + g * kOwn, wd);
+    if constexpr (!kDt) load_own_checked(d_own, c_begin + g * kOwn, wd);
+    else
+#pragma unroll
+        for (int j = 0; j < kOwnWords; ++j) wd[j] = 0u;
     if (has_z) load_own_checked(z_own, c_begin + g * kOwn, wz);
+
+    // dt_proj form: the operands in shared memory, the TMEM accumulator, and
+    // the first stage's product.  Stage k's delta sits in TMEM columns
+    // [64 (k & 1), 64 (k & 1) + 64), column e holding step e of the stage in
+    // the lane of the thread whose row it is.  A tcgen05.ld reads the same
+    // columns for every thread of a warp (its address is warp-uniform), so
+    // each thread loads the sub-chunk's kDirectSub columns and keeps its own
+    // kOwn of them.  The product of stage k + 1 is issued at the start of
+    // stage k (by thread 0), its B operand built at the start of stage k - 1
+    // from delta_r loaded one stage before that.
+    uint8_t *dt_A = nullptr, *dt_B = nullptr;
+    uint64_t *dt_full = nullptr;
+    uint32_t dt_taddr = 0, dt_col = 0;
+    const int dt_R = kDt ? p.dt_rank : 0, dt_rpad = (dt_R + 15) / 16 * 16;
+    const int64_t dt_nst = (Lend - c_begin + kDirectStage - 1) / kDirectStage;  // stages of this block
+    bool dt_ok = true;
+    uint4 dt_raw[kDt ? kMaxDtRank * 8 / 128 : 1];  // this thread's 16-byte chunks of delta_r of a coming stage
+    const Tin *dt_src = kDt ? static_cast<const Tin *>(p.delta_r) + b * dt_R * L : nullptr;
+    auto dt_load_raw = [&](int64_t k) {  // delta_r[b, r, stage k]: chunks (r, 8 steps)
+#pragma unroll
+        for (int q = 0; q < kMaxDtRank * 8 / 128; ++q) {
+            const int c = tid + 128 * q, rr = c / 8, j = c % 8;
+            const int64_t l0 = c_begin + k * kDirectStage + 8 * j;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (rr < dt_R) {
+                const Tin *src = dt_src + (int64_t)rr * L + l0;
+                if (vec && l0 + 8 <= Lend) {
+                    v = __ldg(reinterpret_cast<const uint4 *>(src));
+                } else {
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (l0 + i < Lend) w[i >> 1] |= Io<Tin>::bits(src, i) << (16 * (i & 1));
+                    v = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            dt_raw[q] = v;
+        }
+    };
+    auto dt_build = [&](int64_t k) {  // B operand of stage k from dt_raw (transposed: N = steps, K = rank)
+        uint8_t *Bb = dt_B + (size_t)(k % 3) * dt_rpad * 128;
+#pragma unroll
+        for (int q = 0; q < kMaxDtRank * 8 / 128; ++q) {
+            const int c = tid + 128 * q, rr = c / 8, j = c % 8;
+            if (rr < dt_R) {
+                const uint32_t w[4] = {dt_raw[q].x, dt_raw[q].y, dt_raw[q].z, dt_raw[q].w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int n = 8 * j + i;  // step of the stage = column of the product
+                    *reinterpret_cast<uint16_t *>(Bb + (rr / 8) * 1024 + n * 16 + (rr % 8) * 2) =
+                        (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
+                }
+            }
+        }
+    };
+    auto dt_issue = [&](int64_t k) {  // D[(k & 1)] = A x B(k), K = dt_rpad in steps of 16
+        const uint32_t a0 = tc_smem_addr(dt_A), b0 = tc_smem_addr(dt_B + (size_t)(k % 3) * dt_rpad * 128);
+        for (int j = 0; j < dt_rpad / 16; ++j)
+            tc::mma_bf16_acc(dt_taddr + (uint32_t)((k & 1) * kDirectStage), tc::sdesc(a0 + j * 4096, 2048, 128),
+                             tc::sdesc(b0 + j * 2048, 1024, 128), tc::idesc_bf16(128, kDirectStage), j > 0);
+        tc::commit(&dt_full[k & 1]);
+    };
+    if constexpr (kDt) {
+        const size_t slab_end = reinterpret_cast<size_t>(reinterpret_cast<float *>(RB1 + 2 * kNmax * kDirectStage) +
+                                                         (nthreads / 32) * (kRowsPerWarp * kGatherStride + 32 * kRS));
+        dt_A = reinterpret_cast<uint8_t *>((slab_end + 1023) / 1024 * 1024);
+        dt_B = dt_A + (size_t)dt_rpad * 256;
+        dt_full = reinterpret_cast<uint64_t *>(dt_B + (size_t)3 * dt_rpad * 128);
+        uint32_t *dt_slot = reinterpret_cast<uint32_t *>(dt_full + 2);
+        for (int i = tid; i < 3 * dt_rpad * 128 / 16; i += nthreads)
+            reinterpret_cast<uint4 *>(dt_B)[i] = make_uint4(0u, 0u, 0u, 0u);
+        const int64_t d0 = (bt % p.dtiles) * rows;
+        const unsigned short *W16 = static_cast<const unsigned short *>(p.W_dt);
+        for (int i = tid; i < 128 * dt_rpad; i += nthreads) {  // lane m's row: W_dt of its channel
+            const int m = i / dt_rpad, k = i % dt_rpad;
+            const int64_t dm = d0 + m / kG < p.dim ? d0 + m / kG : p.dim - 1;
+            *reinterpret_cast<uint16_t *>(dt_A + (k / 8) * 2048 + m * 16 + (k % 8) * 2) =
+                k < dt_R ? W16[dm * dt_R + k] : (uint16_t)0;
+        }
+        if (tid == 0) {
+            tc::mbar_init(&dt_full[0], 1), tc::mbar_init(&dt_full[1], 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        if (warp == 0) tc::alloc(dt_slot, 128);
+        __syncthreads();  // B buffers zeroed before the builds write into them
+        if (dt_nst > 0) dt_load_raw(0), dt_build(0);
+        if (dt_nst > 1) dt_load_raw(1), dt_build(1);
+        if (dt_nst > 2) dt_load_raw(2);
+        tc::fence_async_smem();
+        tc::fence_before();
+        __syncthreads();
+        tc::fence_after();
+        dt_taddr = *dt_slot;
+        if (tid == 0 && dt_nst > 0) dt_issue(0);
+    }
     // Stage k's B/C sit in F[k & 1]; the raw copies of stage k + 1 are in
     // flight (into RB[(k + 1) & 1]) while stage k is computed.  The first
     // stage is converted here.
@@ -989,16 +1120,32 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 #pragma unroll
         for (int j = 0; j < kOwnWords; ++j) cu[j] = wu[j], cd[j] = wd[j], cz[j] = wz[j];
         const int64_t s_next = l0 + kDirectSub + g * kOwn;   // next owned step
-        u_own += kDirectSub, d_own += kDirectSub;
+        u_own += kDirectSub;
+        if constexpr (!kDt) d_own += kDirectSub;
         if (has_z) z_own += kDirectSub;
         if (kOwnBytes >= 4 && !kChecked && m + 1 < kSubs) {  // next sub-chunk lies in this full stage
             ld_words<kOwnBytes>(u_own, wu);
-            ld_words<kOwnBytes>(d_own, wd);
+            if constexpr (!kDt) ld_words<kOwnBytes>(d_own, wd);
             if (has_z) ld_words<kOwnBytes>(z_own, wz);
         } else if (l0 + kDirectSub < Lend) {
             load_own_checked(u_own, s_next, wu);
-            load_own_checked(d_own, s_next, wd);
+            if constexpr (!kDt) load_own_checked(d_own, s_next, wd);
             if (has_z) load_own_checked(z_own, s_next, wz);
+        }
+        // dt_proj form: this lane's delta of its own steps, from tensor memory.
+        uint32_t dtv[kDt ? kOwn : 1];
+        if constexpr (kDt) {
+            static_assert(kOwn == 4 && (kDirectSub == 8 || kDirectSub == 16), "4 own steps of 8 or 16");
+            uint32_t all[kDirectSub];
+            tc::ld_sync(dt_col + (uint32_t)(m * kDirectSub), all);
+#pragma unroll
+            for (int i = 0; i < kOwn; ++i) dtv[i] = all[i];
+#pragma unroll
+            for (int gg = 1; gg < kG; ++gg)
+                if (g == gg) {
+#pragma unroll
+                    for (int i = 0; i < kOwn; ++i) dtv[i] = all[gg * kOwn + i];
+                }
         }
         // Bit i: a sequence starts at step l0 + i (the state entering it is
         // zero).  Each lane reads its owned steps; the row's lanes (and so the
@@ -1020,7 +1167,8 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 #pragma unroll
         for (int i = 0; i < kOwn; ++i) {
             uo[i] = Io<Tin>::widen(cu, i);
-            dl_own[i] = delta_transform<kFast>(Io<Tin>::widen(cd, i) + bias, softplus);
+            const float dx = kDt ? __uint_as_float(dtv[kDt ? i : 0]) : Io<Tin>::widen(cd, i);
+            dl_own[i] = delta_transform<kFast>(dx + bias, softplus);
             if constexpr (kChecked) {
                 if (l0 + g * kOwn + i >= Lend) dl_own[i] = 0.f;
             }
@@ -1148,10 +1296,25 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
             const bool odd = stage & 1;
             F = odd ? F1 : F0;
             if (cn < Lend && stage_fast(cn)) cp_async_wait_all();  // the next stage's copies (the only group in flight)
+            if constexpr (kDt) tc::fence_before();  // last stage's TMEM reads before the next product
             __syncthreads();  // F of this stage is complete; the next stage's raw copies have landed; the
                               // other F (last stage's) and this stage's RB (converted before) are free
             if (cn < Lend) fill_F(cn, stage_fast(cn), odd ? RB0 : RB1, odd ? F0 : F1);
             if (cnn < Lend && stage_fast(cnn)) issue_copies(cnn, odd ? RB1 : RB0);
+            if constexpr (kDt) {
+                if (tid == 0 && stage + 1 < dt_nst) {
+                    tc::fence_after();
+                    dt_issue(stage + 1);  // its B operand was built and fenced before this barrier
+                }
+                if (stage + 2 < dt_nst) dt_build(stage + 2);
+                if (stage + 3 < dt_nst) dt_load_raw(stage + 3);
+                tc::fence_async_smem();
+                // This stage's product (issued a stage ago) is complete before its reads.
+                if (!tc::mbar_wait(&dt_full[stage & 1], (uint32_t)((stage >> 1) & 1))) dt_ok = false;
+                __syncwarp();
+                tc::fence_after();
+                dt_col = dt_taddr + ((uint32_t)(32 * warp) << 16) + (uint32_t)((stage & 1) * kDirectStage);
+            }
         } else {
             if (fast) cp_async_wait_all();
             __syncthreads();  // RB holds this stage; every warp is done with F
@@ -1171,6 +1334,12 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         }
     }
 
+    if constexpr (kDt) {  // every product was waited for; every TMEM read is done before the free
+        tc::fence_before();
+        __syncthreads();
+        if (warp == 0) tc::dealloc(dt_taddr, 128);
+        if (!dt_ok && lane == 0 && p.status) atomicExch(p.status, kDeviceTimeout);
+    }
     if (p.nseg > 1) {  // segment record for the fix-up kernel
         const int64_t rec = seg * (p.batch * p.dim) + row;
         if constexpr (kG > 1) {
@@ -1196,72 +1365,125 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     }
 }
 
-// ------------------------------------------------------------ fix-up kernel
+// ------------------------------------------------------------ fix-up kernels
 // After the direct kernel ran every sequence segment from a zero state, the
 // true state entering segment s > 0 is the carry of segments 0..s-1:
 //   h_in(s) = P(s-1) h_in(s-1) + h_end(s-1),   P(j)_n = 2^(A_n log2e sum_j delta'),
 // and its share of y at step l of segment s is
 //   (sum_n C[b,n,l] 2^(A_n log2e S_l) h_in(s)_n) silu(z_l),   S_l = delta' summed
 // over the segment up to and including l (linearity of the recurrence in h).
-// One thread per (row, segment) adds that share to y step by step; it stops
-// once every state's exponent A_n log2e S_l is below -127, where ex2.ftz
-// returns exactly 0, so the remaining shares are exactly zero, or at the
-// segment's first sequence start (p.reset), where the carried state is
-// dropped; a segment holding a start passes no state on (P = 0, recorded as
-// a delta' sum of -1).  Thread (row, segment 0) instead writes the last
-// state h_in(nseg) when asked.
-// Threads: kT = kNmax/4 per (row, segment), 4 states each; they share the
-// step loop (each computes the same delta' sums, so they stop together) and
-// add their shares of the correction by shuffles within their group.
-template <typename Tin, typename Tout, int kNmax>
-__global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
-    constexpr bool kFast = sizeof(Tin) == 2;
-    constexpr int kT = kNmax / 4 < 1 ? 1 : kNmax / 4;  // threads per (row, segment)
-    constexpr int kS = kNmax / kT;                       // states per thread
+// A segment holding a sequence start (p.reset) passes no state on (P = 0,
+// recorded as a delta' sum of -1), and the carried state's share ends at its
+// first start.
+//
+// Two kernels.  ss_fwd_carry_kernel folds the segments of one row in order
+// (one warp per row, states over lanes) and overwrites the record h_end(j)
+// with h_in(j + 1), so that segment s finds its incoming state in record
+// s - 1; it writes last_state = h_in(nseg) when asked.
+// ss_fwd_fixup_kernel then adds the share of y: one warp per (row, segment
+// s > 0), the steps over lanes, kFixupSteps per lane per chunk (lane i takes
+// steps c + 32 k + i, so each load is one coalesced run), S by warp scans,
+// states looped with h_in and A_n log2e in shared memory.  A warp stops
+// after the chunk in which every state's exponent A_n log2e S passed -127
+// (from there ex2.ftz returns exactly 0, so the remaining shares are exactly
+// zero, and steps past that point are not rewritten) or that held a start.
+// With bf16 output y is rounded twice: once by the direct kernel (its
+// zero-state value) and once here after the share is added in fp32; the
+// result is within 1.5 bf16 ulp of the single rounding of the exact sum.
+// The dt_proj form (p.delta null) recomputes delta = W_dt delta_r for the
+// steps it corrects, in fp32 from the exact bf16 products (the direct kernel
+// sums the same products on the tensor cores, in its own order).
+template <int kNmax>
+__global__ void __launch_bounds__(256) ss_fwd_carry_kernel(const FwdParams p) {
+    constexpr int kPer = kNmax > 32 ? 2 : 1;  // states per lane
+    constexpr int kBatchJ = 4;                // segment records loaded ahead
     const int64_t rows_total = p.batch * p.dim;
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t grp = t / kT;                          // (row, segment) of this thread's group
-    const int q = (int)(t % kT);
-    if (grp >= rows_total * p.nseg) return;              // whole groups leave together
-    const int64_t row = grp % rows_total;
-    const int s = (int)(grp / rows_total);
-    const int64_t b = row / p.dim, d = row % p.dim;
-    const int N = p.dstate;
-    const int64_t L = p.seqlen;
-    if (s == 0 && p.last_state == nullptr) return;
+    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const unsigned mask = (kT >= 32 ? 0xffffffffu : ((1u << kT) - 1u) << (lane / kT * kT));
-
-    // Registers: this thread's 4 states of the bucket (states past N stay 0).
-    float A2[kS], h[kS];
-    float A2max = __int_as_float(0xff800000u);  // -inf, over all N states: the group stops together
-    for (int n = 0; n < N; ++n) A2max = fmaxf(A2max, p.A[d * N + n] * kLog2e);
+    if (row >= rows_total) return;  // whole warps leave together
+    const int64_t d = row % p.dim;
+    const int N = p.dstate;
+    float A2[kPer], h[kPer];
 #pragma unroll
-    for (int k = 0; k < kS; ++k) {
-        const int n = q * kS + k;
+    for (int k = 0; k < kPer; ++k) {
+        const int n = lane + 32 * k;
         A2[k] = n < N ? p.A[d * N + n] * kLog2e : 0.f;
         h[k] = 0.f;
     }
-    const int upto = s == 0 ? p.nseg : s;  // segments folded into the carry
-    for (int j = 0; j < upto; ++j) {
-        const int64_t rec = j * rows_total + row;
-        const float ds = p.ws_dsum[rec];
+    for (int j0 = 0; j0 < p.nseg; j0 += kBatchJ) {
+        float ds[kBatchJ], he[kBatchJ][kPer];
 #pragma unroll
-        for (int k = 0; k < kS; ++k) {
-            const int n = q * kS + k;
-            if (n < N) h[k] = fmaf(ds < 0.f ? 0.f : sfu_exp2(A2[k] * ds), h[k], p.ws_hend[rec * N + n]);
+        for (int jj = 0; jj < kBatchJ; ++jj) {
+            const int64_t rec = (int64_t)(j0 + jj) * rows_total + row;
+            const bool ok = j0 + jj < p.nseg;
+            ds[jj] = ok ? p.ws_dsum[rec] : 0.f;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int n = lane + 32 * k;
+                he[jj][k] = ok && n < N ? p.ws_hend[rec * N + n] : 0.f;
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kBatchJ; ++jj) {
+            const int j = j0 + jj;
+            if (j >= p.nseg) break;
+            const int64_t rec = (int64_t)j * rows_total + row;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int n = lane + 32 * k;
+                h[k] = fmaf(ds[jj] < 0.f ? 0.f : sfu_exp2(A2[k] * ds[jj]), h[k], he[jj][k]);
+                if (n < N && j + 1 < p.nseg) p.ws_hend[rec * N + n] = h[k];
+            }
         }
     }
-    if (s == 0) {
+    if (p.last_state != nullptr) {
 #pragma unroll
-        for (int k = 0; k < kS; ++k) {
-            const int n = q * kS + k;
+        for (int k = 0; k < kPer; ++k) {
+            const int n = lane + 32 * k;
             if (n < N) p.last_state[row * N + n] = h[k];
         }
-        return;
     }
+}
 
-    const Tin *dl_row = static_cast<const Tin *>(p.delta) + row * L;
+constexpr int kFixupWarps = 8;
+constexpr int kMaxDstate = 64;  // the largest state size the library takes
+constexpr int kFixupSteps = 4;  // steps per lane per chunk (128-step chunks)
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kFixupWarps * 32) ss_fwd_fixup_kernel(const FwdParams p) {
+    constexpr bool kFast = sizeof(Tin) == 2;
+    constexpr int kK = kFixupSteps;
+    __shared__ float sh_h[kFixupWarps][kMaxDstate], sh_A2[kFixupWarps][kMaxDstate];
+    __shared__ float sh_W[kFixupWarps][kMaxDtRank];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rows_total = p.batch * p.dim;
+    const int64_t task = (int64_t)blockIdx.x * kFixupWarps + warp;  // (row, segment s >= 1)
+    if (task >= rows_total * (p.nseg - 1)) return;                 // whole warps leave together
+    const int64_t row = task % rows_total;
+    const int s = 1 + (int)(task / rows_total);
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const int N = p.dstate;
+    const int64_t L = p.seqlen;
+    const bool dt = p.delta == nullptr;
+    const int R = p.dt_rank;
+
+    float A2max = __int_as_float(0xff800000u);  // -inf
+    const int64_t rec_in = ((int64_t)(s - 1) * rows_total + row) * N;
+    for (int n = lane; n < N; n += 32) {
+        const float a2 = p.A[d * N + n] * kLog2e;
+        sh_A2[warp][n] = a2;
+        sh_h[warp][n] = p.ws_hend[rec_in + n];
+        A2max = fmaxf(A2max, a2);
+    }
+    if (dt)
+        for (int r = lane; r < R; r += 32)
+            sh_W[warp][r] = static_cast<float>(static_cast<const Tin *>(p.W_dt)[d * R + r]);
+#pragma unroll
+    for (int off = 16; off >= 1; off /= 2) A2max = fmaxf(A2max, __shfl_xor_sync(0xffffffffu, A2max, off));
+    __syncwarp();
+
+    const Tin *dl_row = dt ? nullptr : static_cast<const Tin *>(p.delta) + row * L;
+    const Tin *dr_b = dt ? static_cast<const Tin *>(p.delta_r) + b * R * L : nullptr;
     const Tin *z_row = p.z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
     const Tin *C_b = static_cast<const Tin *>(p.C) + b * N * L;
     Tout *y_row = static_cast<Tout *>(p.y) + row * L;
@@ -1270,23 +1492,74 @@ __global__ void __launch_bounds__(256) ss_fwd_fixup_kernel(const FwdParams p) {
     const uint8_t *const reset_b = p.reset ? p.reset + b * L : nullptr;
     const int64_t c_begin = (int64_t)s * p.seg_len;
     const int64_t c_end = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
-    float S = 0.f;
-    for (int64_t l = c_begin; l < c_end; ++l) {
-        if (reset_b && reset_b[l] != 0) break;  // a new sequence: the carried state ends here
-        S += delta_transform<kFast>(static_cast<float>(dl_row[l]) + bias, softplus);
-        if (A2max * S < -127.f) break;  // every 2^(A2 S) is 0 from here on
-        float corr = 0.f;
+
+    float S0 = 0.f;  // delta' summed over the chunks before this one
+    for (int64_t c = c_begin; c < c_end; c += 32 * kK) {
+        float S[kK];
+        bool in[kK];
+        unsigned starts = 0;  // nonzero if a step of this chunk starts a sequence
+        int first_start = 32 * kK;
 #pragma unroll
-        for (int k = 0; k < kS; ++k) {
-            const int n = q * kS + k;
-            if (n < N) corr = fmaf(static_cast<float>(C_b[(int64_t)n * L + l]) * sfu_exp2(A2[k] * S), h[k], corr);
+        for (int k = 0; k < kK; ++k) {
+            const int64_t l = c + 32 * k + lane;
+            in[k] = l < c_end;
+            float x = 0.f;
+            if (in[k]) {
+                if (dt) {
+                    for (int r = 0; r < R; ++r) x = fmaf(sh_W[warp][r], static_cast<float>(dr_b[(int64_t)r * L + l]), x);
+                } else {
+                    x = static_cast<float>(dl_row[l]);
+                }
+            }
+            S[k] = in[k] ? delta_transform<kFast>(x + bias, softplus) : 0.f;
+            const unsigned m = __ballot_sync(0xffffffffu, in[k] && reset_b != nullptr && reset_b[l] != 0);
+            if (m != 0 && first_start == 32 * kK) first_start = 32 * k + __ffs(m) - 1;
+            starts |= m;
         }
+        // inclusive scan of delta' over the chunk's steps, in step order
 #pragma unroll
-        for (int off = kT / 2; off >= 1; off /= 2) corr += __shfl_xor_sync(mask, corr, off, kT);
-        if (q == 0) {
-            if (z_row) corr *= silu<kFast>(static_cast<float>(z_row[l]));
-            y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + corr);
+        for (int k = 0; k < kK; ++k) {
+#pragma unroll
+            for (int off = 1; off < 32; off *= 2) {
+                const float t = __shfl_up_sync(0xffffffffu, S[k], off);
+                if (lane >= off) S[k] += t;
+            }
+            S[k] += S0;
+            S0 = __shfl_sync(0xffffffffu, S[k], 31);
         }
+        bool live[kK];
+        bool any = false;
+#pragma unroll
+        for (int k = 0; k < kK; ++k) {
+            live[k] = in[k] && 32 * k + lane < first_start && !(A2max * S[k] < -127.f);
+            any |= live[k];
+        }
+        if (any) {
+            float corr[kK];
+#pragma unroll
+            for (int k = 0; k < kK; ++k) corr[k] = 0.f;
+#pragma unroll 4
+            for (int n = 0; n < N; ++n) {
+                const float a2 = sh_A2[warp][n], hn = sh_h[warp][n];
+#pragma unroll
+                for (int k = 0; k < kK; ++k) {
+                    if (live[k]) {
+                        const float cv = static_cast<float>(C_b[(int64_t)n * L + c + 32 * k + lane]);
+                        corr[k] = fmaf(cv * sfu_exp2(a2 * S[k]), hn, corr[k]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kK; ++k) {
+                if (live[k]) {
+                    const int64_t l = c + 32 * k + lane;
+                    float v = corr[k];
+                    if (z_row) v *= silu<kFast>(static_cast<float>(z_row[l]));
+                    y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + v);
+                }
+            }
+        }
+        if (starts != 0 || A2max * S0 < -127.f) break;
     }
 }
 

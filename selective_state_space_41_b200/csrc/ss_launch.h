@@ -6,12 +6,13 @@
 #include <cuda_runtime.h>
 
 #include "ss_fwd_kernel.cuh"
+#include "ss_fwd_tmem.cuh"
 
 namespace selscan {
 
 // lanes: lanes per row; split_states: the lanes split the row's states (direct
-// kernel, 1/2/4 lanes) rather than its steps (scan kernel, 2..32 lanes); one
-// lane is the direct kernel either way.
+// kernel, 1/2/4 lanes; 2: its TMEM-fed form, bf16 inputs) rather than its
+// steps (scan kernel, 2..32 lanes); one lane is the direct kernel either way.
 #define SS_DECLARE_LAUNCHER(NAME)                                                            \
     cudaError_t NAME(int lanes, int split_states, dim3 grid, dim3 block, size_t smem, cudaStream_t s, \
                      const FwdParams &p);

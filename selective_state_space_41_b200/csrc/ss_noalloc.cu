@@ -14,7 +14,9 @@
 // looked up once per device, under a lock, by the first call made with that
 // device current (so that first call should not be made while a stream is
 // being captured); later calls reuse the cached address and make no CUDA
-// runtime call beyond the launches of ss_fwd_ws.  Nothing in the array has to
+// runtime call beyond the launches of ss_fwd_ws.  The cache is not refreshed:
+// after cudaDeviceReset the cached address of that device is stale, and the
+// header tells callers not to use this entry on that device again.  Nothing in the array has to
 // start at zero: every word the kernels read in a call was first written by
 // the segment kernel of that same call (end states and delta' sums of each
 // segment), and the fix-up kernel starts its carried state at zero in

@@ -9,8 +9,8 @@ fails to load, every call raises.
 The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``,
 ``ss_fwd_reset``, ``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
-``ss_fwd_noalloc``, ``ss_step``, ``ss_bwd``, ``ss_bwd_reset``, ``ss_bwd_workspace_bytes``,
-``ss_status_string``, ``ss_version``); ``ss_fwd`` dispatches to the
+``ss_fwd_noalloc``, ``ss_fwd_dtproj``, ``ss_step``, ``ss_bwd``, ``ss_bwd_reset``, ``ss_bwd_state``, ``ss_bwd_workspace_bytes``,
+``ss_status_string``, ``ss_version``, ``ss_device_status``); ``ss_fwd`` dispatches to the
 workspace, config, initial-state and sequence-start forms by keyword, ``ss_fwd_hostio`` to
 the pipelined form when given streams.  ``selective_scan_fwd`` and
 ``selective_scan_bwd`` are the allocate-and-call convenience forms, with the
@@ -37,7 +37,8 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 # Names the header declares; the ABI test checks each is exported.
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
            "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc",
-           "ss_step", "ss_bwd", "ss_bwd_reset", "ss_bwd_workspace_bytes", "ss_status_string", "ss_version")
+           "ss_step", "ss_bwd", "ss_bwd_reset", "ss_bwd_state", "ss_bwd_workspace_bytes", "ss_status_string",
+           "ss_version", "ss_device_status", "ss_fwd_dtproj")
 
 
 class SelscanError(RuntimeError):
@@ -88,6 +89,8 @@ def lib():
         L.ss_fwd_heuristic.argtypes = [DP, SZ, CP]
         L.ss_fwd_hostio.restype = I
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
+        L.ss_fwd_dtproj.restype = I
+        L.ss_fwd_dtproj.argtypes = [DP, I] + [P] * 9 + [I, P, P, P, SZ, P]
         L.ss_fwd_noalloc.restype = I
         L.ss_fwd_noalloc.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
         L.ss_fwd_hostio_streams.restype = I
@@ -98,12 +101,16 @@ def lib():
         L.ss_bwd.argtypes = [DP] + [P] * 8 + [I] + [P] * 9 + [P, SZ, P]
         L.ss_bwd_reset.restype = I
         L.ss_bwd_reset.argtypes = [DP] + [P] * 8 + [I] + [P] * 10 + [P, SZ, P]
+        L.ss_bwd_state.restype = I
+        L.ss_bwd_state.argtypes = [DP] + [P] * 8 + [I] + [P] * 13 + [P, SZ, P]
         L.ss_bwd_workspace_bytes.restype = SZ
         L.ss_bwd_workspace_bytes.argtypes = [DP]
         L.ss_status_string.restype = ctypes.c_char_p
         L.ss_status_string.argtypes = [I]
         L.ss_version.restype = I
         L.ss_version.argtypes = []
+        L.ss_device_status.restype = I
+        L.ss_device_status.argtypes = [ctypes.POINTER(I)]
         _lib = L
     return _lib
 
@@ -114,6 +121,17 @@ def ss_status_string(status: int) -> str:
 
 def ss_version() -> int:
     return int(lib().ss_version())
+
+
+# SS_DEVICE_TIMEOUT: a kernel's bounded wait on other warps of its block ran out.
+SS_DEVICE_TIMEOUT = 1
+
+
+def ss_device_status() -> int:
+    """The current device's status word (0: nothing recorded), then cleared."""
+    code = ctypes.c_int(0)
+    _check(lib().ss_device_status(ctypes.byref(code)), "ss_device_status")
+    return int(code.value)
 
 
 def _ptr(t):
@@ -145,9 +163,11 @@ def _check(status, where):
 
 
 def _config(lanes_per_row, split_states, warps_per_block, segments):
+    """split_states: False/0 (lanes split steps), True/1 (lanes split states),
+    2 (lanes split states, B/C through tensor memory)."""
     if lanes_per_row is None and warps_per_block is None and segments is None:
         return None
-    return LaunchConfig(int(lanes_per_row or 0), 1 if split_states else 0, int(warps_per_block or 0),
+    return LaunchConfig(int(lanes_per_row or 0), int(split_states or 0), int(warps_per_block or 0),
                         int(segments or 0))
 
 
@@ -202,6 +222,26 @@ def ss_fwd(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus
         _check(lib().ss_fwd(*args, s), "ss_fwd")
 
 
+def ss_fwd_dtproj(u, delta_r, W_dt, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=True,
+                  last_state=None, stream=None, workspace=None):
+    """Queue the forward with delta = W_dt delta_r computed inside the scan
+    (the dt_proj map).  delta_r: (batch, dt_rank, L) bf16; W_dt: (dim, dt_rank)
+    bf16; other tensors as ``ss_fwd``."""
+    u, delta_r, W_dt, A, B, C, D, z, delta_bias = map(_contig, (u, delta_r, W_dt, A, B, C, D, z, delta_bias))
+    if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
+        raise ValueError("outputs must be contiguous")
+    batch, dim, L = u.shape
+    R = W_dt.shape[-1]
+    if tuple(delta_r.shape) != (batch, R, L) or tuple(W_dt.shape) != (dim, R):
+        raise ValueError("delta_r must be (batch, dt_rank, L) and W_dt (dim, dt_rank)")
+    desc = make_desc(batch, dim, L, A.shape[-1], u.dtype, y.dtype)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().ss_fwd_dtproj(ctypes.byref(desc), int(R), _ptr(u), _ptr(delta_r), _ptr(W_dt), _ptr(A), _ptr(B),
+                               _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(y),
+                               _ptr(last_state), _ptr(workspace), ws_bytes, _stream_handle(stream, u.device)),
+           "ss_fwd_dtproj")
+
+
 def ss_fwd_noalloc(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
                    last_state=None, stream=None):
     """Queue the forward with the library's static scratch array as the
@@ -240,12 +280,15 @@ def ss_bwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, 
 
 
 def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_softplus=False,
-           workspace=None, stream=None, reset=None):
+           workspace=None, stream=None, reset=None, initial_state=None, d_last_state=None):
     """Queue the backward: ``grads`` maps du, ddelta, dA, dB, dC and (when the
     operand is given) dD, dz, ddelta_bias to output tensors (du, ddelta, dz in
-    u's dtype; the others float32).  ``workspace``: a CUDA tensor of at least
+    u's dtype; the others float32), and optionally dinitial_state ((batch,
+    dim, N) float32).  ``workspace``: a CUDA tensor of at least
     ss_bwd_workspace_bytes() bytes (allocated here when None).  ``reset``: the
-    forward's (batch, L) mask of sequence starts (selects ``ss_bwd_reset``)."""
+    forward's (batch, L) mask of sequence starts (selects ``ss_bwd_reset``).
+    ``initial_state`` / ``d_last_state`` ((batch, dim, N) float32) or a
+    dinitial_state output select ``ss_bwd_state``."""
     u, delta, A, B, C, dy, D, z, delta_bias = map(_contig, (u, delta, A, B, C, dy, D, z, delta_bias))
     batch, dim, L = u.shape
     N = A.shape[-1]
@@ -263,14 +306,23 @@ def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_
             reset = reset.view(torch.uint8)
         if reset.dtype != torch.uint8 or tuple(reset.shape) != (batch, L) or not reset.is_contiguous():
             raise ValueError("reset must be a contiguous (batch, L) uint8 or bool tensor")
+    for t in (initial_state, d_last_state, grads.get("dinitial_state")):
+        if t is not None and not (t.is_contiguous() and tuple(t.shape) == (batch, dim, N) and t.dtype == torch.float32):
+            raise ValueError("states must be contiguous (batch, dim, N) float32 tensors")
+    if initial_state is not None or d_last_state is not None or grads.get("dinitial_state") is not None:
+        _check(lib().ss_bwd_state(*head, _ptr(reset), _ptr(initial_state), _ptr(d_last_state), *tail[:9],
+                                  g("dinitial_state"), *tail[9:]), "ss_bwd_state")
+    elif reset is not None:
         _check(lib().ss_bwd_reset(*head, _ptr(reset), *tail), "ss_bwd_reset")
     else:
         _check(lib().ss_bwd(*head, *tail), "ss_bwd")
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=False,
-                       stream=None, reset=None):
-    """Gradients of sum(dy * y) as a dict (see ss_bwd); allocates the outputs."""
+                       stream=None, reset=None, initial_state=None, d_last_state=None):
+    """Gradients of sum(dy * y) (+ sum(d_last_state * last state)) as a dict
+    (see ss_bwd); allocates the outputs; dinitial_state when an initial
+    state or a last-state gradient is given."""
     batch, dim, L = u.shape
     N = A.shape[-1]
     dev = u.device
@@ -282,8 +334,11 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, d
              "dD": torch.empty(dim, dtype=f32, device=dev) if D is not None else None,
              "dz": torch.empty_like(u) if z is not None else None,
              "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None}
+    if initial_state is not None or d_last_state is not None:
+        grads["dinitial_state"] = torch.empty((batch, dim, N), dtype=f32, device=dev)
     ss_bwd(u, delta, A, B, C, dy, grads, D=D, z=z, delta_bias=delta_bias,
-           delta_softplus=delta_softplus, stream=stream, reset=reset)
+           delta_softplus=delta_softplus, stream=stream, reset=reset, initial_state=initial_state,
+           d_last_state=d_last_state)
     return grads
 
 
@@ -310,7 +365,7 @@ def ss_fwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dt
     cfg = LaunchConfig()
     _check(lib().ss_fwd_heuristic(ctypes.byref(desc), int(workspace_bytes), ctypes.byref(cfg)),
            "ss_fwd_heuristic")
-    return {"lanes_per_row": cfg.lanes_per_row, "split_states": bool(cfg.split_states),
+    return {"lanes_per_row": cfg.lanes_per_row, "split_states": int(cfg.split_states),
             "warps_per_block": cfg.warps_per_block, "segments": cfg.segments}
 
 

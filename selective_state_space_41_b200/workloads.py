@@ -18,7 +18,13 @@ import torch
 from . import gen
 
 # Philox stream ids, one per operand.
-STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "delta_bias": 7}
+STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "delta_bias": 7, "delta_r": 11, "W_dt": 12}
+
+# dt_rank of the dt_proj form for a layer of model width d_model: the pages
+# give dt_rank = 'auto' without a rule ("Mamba-minimal项目解析", 1. ModelArgs);
+# read as mamba-minimal's ceil(d_model / 16) (48 for d_model 768).
+def dt_rank_auto(d_model: int) -> int:
+    return -(-d_model // 16)
 
 
 @dataclass(frozen=True)
@@ -124,4 +130,18 @@ def make_inputs(w: Workload, pin: bool = False, nthreads: int = 0) -> dict:
             if out[k] is not None:
                 out[k] = out[k].pin_memory()
     out["out_dtype"] = w.out_dtype or w.dtype
+    return out
+
+
+def make_dtproj_inputs(w: Workload, dt_rank: int, pin: bool = False) -> dict:
+    """make_inputs(w) plus the low-rank input of the dt_proj form: delta_r
+    (B, dt_rank, L) ~ N(0, 1) and W_dt (D, dt_rank) ~ U(-dt_rank^-1/2,
+    dt_rank^-1/2), both in the workload's dtype (delta = W_dt delta_r then has
+    standard deviation about 0.58); delta is left out (None)."""
+    out = make_inputs(w, pin=pin)
+    out["delta"] = None
+    bound = dt_rank ** -0.5
+    out["delta_r"] = gen.fill((w.batch, dt_rank, w.seqlen), w.dtype, w.seed, STREAM["delta_r"], gen.NORMAL,
+                              0.0, 1.0, pin)
+    out["W_dt"] = gen.fill((w.dim, dt_rank), w.dtype, w.seed, STREAM["W_dt"], gen.UNIFORM, -bound, bound, pin)
     return out

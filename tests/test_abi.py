@@ -29,6 +29,26 @@ def test_header_declares_the_binding_exports():
     assert sorted(selscan.EXPORTS) == declared_functions()
 
 
+def declared_arity():
+    """Number of parameters of each function prototype in the header."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for name, params in re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(ss_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_prototypes(lib):
+    """Every ctypes signature the binding sets has as many arguments as the
+    header's prototype (a wrong count fails only at call time, on a GPU)."""
+    arity = declared_arity()
+    assert sorted(arity) == declared_functions()
+    for name, n in arity.items():
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), f"{name} not exported"
@@ -156,6 +176,33 @@ def test_noalloc_rejections_before_any_launch(lib):
     assert "scratch" in selscan.ss_status_string(9)
 
 
+def test_noalloc_scratch_covers_the_genomic_layer(lib):
+    """The figure the header gives for the 4 x 1024 x 100000, 16-state bf16
+    layer is what ss_fwd_workspace_bytes reports for its default shape, and
+    it fits the static scratch array."""
+    d = _desc(batch=4, dim=1024, seqlen=100_000, dstate=16, in_dtype=1, out_dtype=1)
+    n = lib.ss_fwd_workspace_bytes(ctypes.byref(d), None)
+    assert n == 4_456_448
+    assert n <= selscan.NOALLOC_SCRATCH_BYTES
+
+
+def test_bwd_workspace_bounded_by_batch_groups(lib):
+    """The backward's workspace grows with one batch group, not the batch: the
+    16 x 4096 x 8192 layers stay under 8 GB at every state size, and a batch
+    whose entries each fit alone needs no more than the whole batch would."""
+    for n in (16, 32, 64):
+        d = _desc(batch=16, dim=4096, seqlen=8192, dstate=n, in_dtype=1, out_dtype=1)
+        assert 0 < lib.ss_bwd_workspace_bytes(ctypes.byref(d)) < 8_000_000_000, n
+    one = lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(batch=1, dim=4096, seqlen=8192, dstate=64,
+                                                        in_dtype=1, out_dtype=1)))
+    three = lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(batch=3, dim=4096, seqlen=8192, dstate=64,
+                                                          in_dtype=1, out_dtype=1)))
+    assert one < three < 3 * one
+    small = [lib.ss_bwd_workspace_bytes(ctypes.byref(_desc(batch=b, dim=1536, seqlen=2048, dstate=16,
+                                                           in_dtype=1, out_dtype=1))) for b in (1, 8)]
+    assert small[1] > 7 * small[0] - 8 * 4096   # small batches run whole: the workspace scales with B
+
+
 def test_state_entry_rejections(lib):
     """ss_fwd_state: a misaligned initial state or a bad config is rejected
     before any launch."""
@@ -200,11 +247,11 @@ def test_reset_mask_checked_by_the_binding():
 
 @pytest.mark.parametrize("shape,ws,want", [
     # (B, D, L, N), workspace bytes, (lanes_per_row, split_states, warps_per_block, segments)
-    ((8, 1536, 2048, 16), 0, (4, True, 4, 1)),          # mamba-130m-shaped layer: measured best 4s/4
-    ((4, 1024, 100000, 16), 1 << 30, (2, True, 4, 16)),  # 100k genomic, with workspace: 2s/4, 16 segments
-    ((16, 4096, 8192, 16), 0, (2, True, 4, 1)),          # wide layers: 2s/4 at 16, 32 and 64 states
-    ((16, 4096, 8192, 32), 0, (2, True, 4, 1)),
-    ((16, 4096, 8192, 64), 0, (2, True, 4, 1)),
+    ((8, 1536, 2048, 16), 0, (4, 1, 4, 1)),          # mamba-130m-shaped layer: measured best 4s/4
+    ((4, 1024, 100000, 16), 1 << 30, (2, 1, 4, 16)),  # 100k genomic, with workspace: 2s/4, 16 segments
+    ((16, 4096, 8192, 16), 0, (2, 1, 4, 1)),          # wide layers: 2s/4 at 16, 32 and 64 states
+    ((16, 4096, 8192, 32), 0, (2, 1, 4, 1)),
+    ((16, 4096, 8192, 64), 0, (2, 1, 4, 1)),
 ])
 def test_heuristic_picks_the_measured_shapes(shape, ws, want):
     """The launch heuristic (host logic, 148 SMs when no device answers)
@@ -220,7 +267,7 @@ def test_heuristic_genomic_without_workspace_and_its_workspace():
     with one, 16 segments need nseg x rows x (N + 1) floats."""
     import torch
     h = selscan.ss_fwd_heuristic(4, 1024, 100000, 16, torch.bfloat16)
-    assert h["split_states"] is False and h["segments"] == 1
+    assert h["split_states"] == 0 and h["segments"] == 1
     assert selscan.ss_fwd_workspace_bytes(4, 1024, 100000, 16, torch.bfloat16) == 16 * 4096 * 17 * 4
 
 

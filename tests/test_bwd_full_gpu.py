@@ -128,3 +128,35 @@ def test_bwd_wide_state_n64_batch_entry():
     """One batch entry (4096 channels x 8192 steps) of the 64-state wide layer."""
     w = W.with_shape(W.WORKLOADS["wide_state_b16_d4096_l8192_n64"], batch=1)
     _full_size_check(w, rows=[(0, 0), (0, 2049), (0, 4095)], channels=[0, 1234, 4095], batch_entry=0)
+
+
+def test_bwd_batch_groups_equal_per_entry_runs():
+    """A batch whose backward workspace exceeds one group's budget runs in
+    batch groups (here 3 entries of the 64-state wide layer: groups of 2 and
+    1).  Every per-entry gradient equals, bit for bit, the backward of that
+    entry alone, and dA, dD (summed over the batch in batch order) equal the
+    per-entry sums added in that order."""
+    w = W.with_shape(W.WORKLOADS["wide_state_b16_d4096_l8192_n64"], batch=3)
+    one = selscan.ss_bwd_workspace_bytes(1, w.dim, w.seqlen, w.dstate, w.dtype)
+    assert selscan.ss_bwd_workspace_bytes(3, w.dim, w.seqlen, w.dstate, w.dtype) < 3 * one
+    inp = W.make_inputs(w)
+    inp["dy"] = gen.fill(tuple(inp["u"].shape), w.dtype, w.seed, DY_STREAM)
+    dev = torch.device("cuda")
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+    def bwd(sl):
+        return selscan.selective_scan_bwd(sl(d["u"]), sl(d["delta"]), d["A"], sl(d["B"]), sl(d["C"]), sl(d["dy"]),
+                                          D=d["D"], z=sl(d["z"]), delta_bias=d["delta_bias"],
+                                          delta_softplus=w.delta_softplus)
+
+    whole = bwd(lambda t: t)
+    parts = [bwd(lambda t, b=b: t[b:b + 1].contiguous()) for b in range(3)]
+    torch.cuda.synchronize()
+    for k in ("du", "ddelta", "dz", "dB", "dC"):
+        for b in range(3):
+            assert torch.equal(whole[k][b:b + 1], parts[b][k]), f"{k} entry {b}"
+    for k in ("dA", "dD"):
+        s = parts[0][k].clone()
+        for b in (1, 2):
+            s = s + parts[b][k]
+        assert torch.equal(whole[k], s), k

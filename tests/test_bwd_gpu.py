@@ -201,3 +201,125 @@ def test_bwd_starts_mamba130m_one_batch():
     inp["dy"] = gen.fill((1, w.dim, w.seqlen), torch.bfloat16, 77, DY_STREAM)
     _check(inp, torch.bfloat16, "starts, mamba-130m-shaped batch entry",
            reset=_starts(1, w.seqlen, seed=77, fixed=range(0, w.seqlen, 512), p=0.002))
+
+
+# ---------------------------------------------------------------- initial state
+# (ss_bwd_state: the backward of ss_fwd_state's forward from a given state,
+# with an optional gradient on the last state, returning the gradient with
+# respect to the initial state; the oracle's form is pinned by finite
+# differences in tests/pins_bwd.py.)
+
+def _check_state(inp, dtype, what, reset=None, with_h0=True, with_dlast=True, seed=0):
+    batch, dim, L = inp["u"].shape
+    N = inp["A"].shape[1]
+    g = torch.Generator().manual_seed(seed)
+    h0 = torch.randn((batch, dim, N), generator=g) if with_h0 else None
+    dlast = torch.randn((batch, dim, N), generator=g) if with_dlast else None
+    d = to_dev(inp)
+    got = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], D=d.get("D"),
+                                     z=d.get("z"), delta_bias=d.get("delta_bias"),
+                                     delta_softplus=inp["delta_softplus"],
+                                     reset=None if reset is None else torch.as_tensor(reset).cuda(),
+                                     initial_state=None if h0 is None else h0.cuda(),
+                                     d_last_state=None if dlast is None else dlast.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"],
+                                    D=inp.get("D"), z=inp.get("z"), delta_bias=inp.get("delta_bias"),
+                                    delta_softplus=inp["delta_softplus"], reset=reset, magnitudes=True,
+                                    initial_state=h0 if h0 is not None else torch.zeros((batch, dim, N)),
+                                    dlast_state=dlast)
+    for k, want in ref.items():
+        if k.startswith("mag_") or want is None:
+            continue
+        if k == "dinitial_state" and h0 is None and dlast is None:
+            assert k not in got   # asked for only with a state or a last-state gradient
+            continue
+        gk = got[k].detach().to("cpu", torch.float64).numpy()
+        assert np.isfinite(gk).all(), f"{what}: {k} not finite"
+        if k in ELEM:
+            e = float(np.max(np.abs(gk - want) / (1.0 + np.abs(want))))
+            assert e <= TOL_ELEM[dtype], f"{what}: {k} max |err|/(1+|ref|) = {e:.3e}"
+        elif k == "dinitial_state":
+            # a sum over the row's steps of adjoint terms, each accurate to the
+            # fp32/SFU rounding of its factors: per element against 1 + |ref|
+            e = float(np.max(np.abs(gk - want) / (1.0 + np.abs(want))))
+            assert e <= TOL_ELEM[dtype], f"{what}: dinitial_state max |err|/(1+|ref|) = {e:.3e}"
+        else:
+            check_summed(k, gk, want, ref["mag_" + k], TOL_SUM[dtype], what)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N", [4, 16, 33, 64])
+def test_bwd_initial_state(dtype, N):
+    """From a given state with a last-state gradient: every bucket, ragged
+    length and channels, every operand."""
+    _check_state(_case(2, 45, 203, N, dtype, seed=N + 500, has_z=True), dtype, f"h0 N={N}", seed=N)
+
+
+@pytest.mark.parametrize("with_h0,with_dlast", [(True, False), (False, True), (False, False)])
+def test_bwd_initial_state_parts(with_h0, with_dlast):
+    """Only the initial state, only the last-state gradient (the
+    initial-state gradient of a zero start is returned), neither (plain
+    ss_bwd)."""
+    _check_state(_case(2, 33, 150, 16, torch.bfloat16, seed=31, has_z=True), torch.bfloat16,
+                 f"h0={with_h0} dlast={with_dlast}", with_h0=with_h0, with_dlast=with_dlast, seed=3)
+
+
+def test_bwd_initial_state_with_starts():
+    """With sequence starts, one at step 0 in batch entry 0 (its initial
+    state is cut off: zero gradient there)."""
+    reset = _starts(2, 203, seed=41, fixed=(7, 64, 100), p=0.02)
+    reset[0, 0] = 1
+    _check_state(_case(2, 40, 203, 16, torch.float32, seed=41, has_z=True), torch.float32, "h0 + starts",
+                 reset=reset, seed=41)
+
+
+def test_bwd_initial_state_empty_sequence():
+    """L = 0: the initial-state gradient is the last-state gradient."""
+    inp = _case(2, 5, 0, 16, torch.float32, seed=1)
+    d = to_dev(inp)
+    dlast = torch.randn((2, 5, 16), device="cuda")
+    got = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], D=d["D"],
+                                     delta_bias=d["delta_bias"], delta_softplus=True,
+                                     initial_state=torch.zeros_like(dlast), d_last_state=dlast)
+    torch.cuda.synchronize()
+    assert torch.equal(got["dinitial_state"], dlast)
+
+
+def test_bwd_in_pieces_equals_whole():
+    """A 1000-step sequence trained in two pieces (cut at a stage boundary,
+    640): forward piece 1 from h0, piece 2 from piece 1's last state; backward
+    of piece 2 from that state, then of piece 1 with piece 2's initial-state
+    gradient as its last-state gradient.  The per-step gradients agree with
+    the whole sequence's: per-step gradients to bf16 output rounding, the
+    state-carried and summed ones to fp32 rounding of the split sums."""
+    inp = _case(2, 48, 1000, 16, torch.bfloat16, seed=57, has_z=True)
+    d = to_dev(inp)
+    h0 = torch.randn((2, 48, 16), device="cuda")
+    kw = dict(D=d["D"], z=None, delta_bias=d["delta_bias"], delta_softplus=True)
+    whole = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], initial_state=h0,
+                                       **dict(kw, z=d["z"]))
+    cut = 640
+    sl = lambda t, a, b: t[..., a:b].contiguous()  # noqa: E731
+    y1 = torch.empty_like(sl(d["u"], 0, cut))
+    h1 = torch.empty_like(h0)
+    selscan.ss_fwd(sl(d["u"], 0, cut), sl(d["delta"], 0, cut), d["A"], sl(d["B"], 0, cut), sl(d["C"], 0, cut), y1,
+                   z=sl(d["z"], 0, cut), last_state=h1, initial_state=h0, lanes_per_row=4, split_states=1,
+                   warps_per_block=4, segments=1, **{k: v for k, v in kw.items() if k != "z"})
+    g2 = selscan.selective_scan_bwd(sl(d["u"], cut, 1000), sl(d["delta"], cut, 1000), d["A"], sl(d["B"], cut, 1000),
+                                    sl(d["C"], cut, 1000), sl(d["dy"], cut, 1000), initial_state=h1,
+                                    **dict(kw, z=sl(d["z"], cut, 1000)))
+    g1 = selscan.selective_scan_bwd(sl(d["u"], 0, cut), sl(d["delta"], 0, cut), d["A"], sl(d["B"], 0, cut),
+                                    sl(d["C"], 0, cut), sl(d["dy"], 0, cut), initial_state=h0,
+                                    d_last_state=g2["dinitial_state"], **dict(kw, z=sl(d["z"], 0, cut)))
+    torch.cuda.synchronize()
+    for k in ("du", "ddelta", "dz"):
+        joined = torch.cat([g1[k], g2[k]], dim=-1).double()
+        e = float(((joined - whole[k].double()).abs() / (1 + whole[k].double().abs())).max())
+        assert e <= 1e-2, f"pieces: {k} {e:.3e}"
+    for k in ("dB", "dC"):
+        joined = torch.cat([g1[k], g2[k]], dim=-1)
+        assert torch.allclose(joined, whole[k], rtol=1e-4, atol=1e-5 * float(whole[k].abs().max())), k
+    assert torch.allclose(g1["dinitial_state"], whole["dinitial_state"], rtol=1e-4, atol=1e-5)
+    for k in ("dA", "dD", "ddelta_bias"):
+        assert torch.allclose(g1[k] + g2[k], whole[k], rtol=1e-4, atol=1e-5 * float(whole[k].abs().max())), k

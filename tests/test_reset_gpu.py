@@ -122,7 +122,7 @@ def test_reset_heuristic_shapes():
     same with a workspace (sequence segments)."""
     inp = _case(1, 16, 9000, 16, torch.bfloat16, seed=17, has_z=False, bias_kind="none",
                 return_last_state=True)
-    assert selscan.ss_fwd_heuristic(1, 16, 9000, 16, torch.bfloat16)["split_states"] is False
+    assert selscan.ss_fwd_heuristic(1, 16, 9000, 16, torch.bfloat16)["split_states"] == 0
     reset = _mask(1, 9000, seed=17, starts=(0, 4096, 4097), p=0.001)
     d = to_dev(inp)
     y_ref, last_ref = _oracle(inp, reset)

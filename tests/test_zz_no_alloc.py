@@ -82,3 +82,40 @@ def test_no_alloc_matches_workspace_entry(w, segmented):
         assert torch.equal(y, y_ref), f"{w.name}: y differs on call {call + 1}"
         assert torch.equal(last, last_ref), f"{w.name}: last_state differs on call {call + 1}"
     assert not torch.equal(got[0][0], got[1][0])   # the two calls saw different inputs
+
+
+def test_no_alloc_against_oracle():
+    """A segmented no-alloc call checked directly against the fp64 oracle
+    (every output of a 2 x 64-channel, 9000-step, 16-state layer)."""
+    import oracle
+    from gpu_util import TOL, assert_parity
+    w = W.custom("noalloc_oracle_b2_d64_l9000_n16", 2, 64, 9000, 16, torch.bfloat16, 9105, has_z=True,
+                 D_kind="normal", bias_kind="uniform_dt", return_last_state=True)
+    assert selscan.ss_fwd_heuristic(2, 64, 9000, 16, torch.bfloat16,
+                                    workspace_bytes=selscan.NOALLOC_SCRATCH_BYTES)["segments"] > 1
+    inp = W.make_inputs(w)
+    y, last = _no_alloc(to_dev(inp), torch.bfloat16)
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                                            z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True,
+                                            return_last_state=True)
+    assert_parity(y, last, y_ref, last_ref, TOL[torch.bfloat16], w.name)
+
+
+def test_no_alloc_first_call_in_a_fresh_process():
+    """The first call on a device is the one that looks up the array's
+    address: run it in a new process (whatever ran before in this one), two
+    calls in a row, against ss_fwd_ws."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys, torch\n"
+        "sys.path.insert(0, %r); sys.path.insert(0, %r)\n"
+        "import test_zz_no_alloc as T\n"
+        "w, seg = T.CASES[0]\n"
+        "T.test_no_alloc_matches_workspace_entry(w, seg)\n"
+        "print('fresh ok')\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))), os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "fresh ok" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
