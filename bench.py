@@ -18,7 +18,8 @@ exp count against the SFU rate (16 ex2 per clock per SM at the maximum SM
 clock); its HBM side (compulsory bytes over measured copy bandwidth) is
 reported beside it.  ``per_config`` adds, in the same line, the forward of
 every other configuration at full size (device time with L2 flushed per step,
-fewer steps each, clocks sampled over the warm-ups and timed steps).
+fewer steps each, clocks sampled over the warm-ups and timed steps) and its
+backward (ss_bwd, all gradients, 3 timed steps).
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
 bounded sample of rows per step).
 """
@@ -412,9 +413,12 @@ def bench_ours(args, w, world, rank, local):
         for name in W.WORKLOADS:
             if name == w.name:
                 continue
-            per[name] = bench_forward_config(rank_workload(W.WORKLOADS[name], rank), dev, stream, flush,
-                                             steps=max(3, min(args.steps, 10)), warmup=3,
+            wn = rank_workload(W.WORKLOADS[name], rank)
+            per[name] = bench_forward_config(wn, dev, stream, flush, steps=max(3, min(args.steps, 10)), warmup=3,
                                              sfu_peak=sfu_peak, hbm_peak=hbm_peak)
+            if not args.no_bwd:
+                per[name]["backward"] = bench_backward_config(wn, dev, stream, flush, steps=3, warmup=3,
+                                                              sfu_peak=sfu_peak)
         line["per_config"] = per
     del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -469,7 +473,7 @@ def bench_forward_config(w: W.Workload, dev, stream, flush, steps: int, warmup: 
            "sfu_frac": w.updates / sfu_peak / (ms * 1e-3),
            "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak,
            "algorithmic_bytes": nbytes, "launch": shape,
-           "gpu_launches_per_step": 2 if shape["segments"] > 1 else 1, "clocks": clk}
+           "gpu_launches_per_step": 3 if shape["segments"] > 1 else 1, "clocks": clk}
     if clk.get("sm_mhz"):
         out["ms_x_median_sm_mhz"] = ms * clk["sm_mhz"]
     del d, y, last, ws
@@ -569,12 +573,10 @@ def bench_decode(w, d, out_dtype, stream, world, calls=200):
                     "us_per_step_python_calls: the same steps called one by one from Python"}
 
 
-def bench_backward(args, w, d, host, out_dtype, flush, stream, sfu_peak, world):
-    """Device time of ss_bwd (all gradients of sum(dy * y)) on the same inputs:
-    a forward-state pass plus the adjoint pass recomputing the states, about
-    two exps per state update (a seeded synthetic dy)."""
+def _time_backward(w, d, dy, out_dtype, flush, stream, steps, warmup):
+    """Device time (median ms) of ss_bwd (all gradients) on resident inputs,
+    L2 flushed before each step; the workspace size and the launch plan."""
     dev = d["u"].device
-    dy = gen.fill(tuple(host["u"].shape), out_dtype, w.seed, 9).to(dev)
     grads = {"du": torch.empty_like(d["u"]), "ddelta": torch.empty_like(d["u"]),
              "dA": torch.empty((w.dim, w.dstate), dtype=torch.float32, device=dev),
              "dB": torch.empty((w.batch, w.dstate, w.seqlen), dtype=torch.float32, device=dev),
@@ -591,10 +593,9 @@ def bench_backward(args, w, d, host, out_dtype, flush, stream, sfu_peak, world):
                        delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, workspace=ws,
                        stream=stream)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(warmup):
         flush.zero_()
         launch()
-    steps = max(3, min(args.steps, 30))
     ts = []
     for _ in range(steps):
         flush.zero_()
@@ -604,13 +605,51 @@ def bench_backward(args, w, d, host, out_dtype, flush, stream, sfu_peak, world):
         e1.record(stream)
         e1.synchronize()
         ts.append(e0.elapsed_time(e1))
-    ms = max_over_ranks(statistics.median(ts), world)
-    del ws
+    del ws, grads
+    plan = selscan.ss_bwd_heuristic(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, out_dtype)
+    return statistics.median(ts), nws, plan
+
+
+def _bwd_launches(w, plan):
+    """Kernel launches of one ss_bwd call: per batch group the adjoint kernel
+    and the dB/dC sum (plus, with sequence segments, the forward summary,
+    its carry fold, the adjoint summary and its fold), then the row sums."""
+    groups = -(-w.batch // plan["batch_group"])
+    return groups * (2 + (4 if plan["segments"] > 1 else 0)) + 1
+
+
+def bench_backward(args, w, d, host, out_dtype, flush, stream, sfu_peak, world):
+    """Device time of ss_bwd (all gradients of sum(dy * y)) on the same inputs:
+    a forward-state pass plus the adjoint pass recomputing the states, about
+    two exps per state update (a seeded synthetic dy)."""
+    dev = d["u"].device
+    dy = gen.fill(tuple(host["u"].shape), out_dtype, w.seed, 9).to(dev)
+    steps = max(3, min(args.steps, 30))
+    ms, nws, plan = _time_backward(w, d, dy, out_dtype, flush, stream, steps, max(3, args.warmup))
+    ms = max_over_ranks(ms, world)
     return {"ms_per_step": ms, "value": w.updates * world / (ms * 1e-3), "unit": "updates/s",
-            "steps": steps, "workspace_bytes": nws, "gpu_launches_per_step": 3,
+            "steps": steps, "workspace_bytes": nws, "plan": plan, "gpu_launches_per_step": _bwd_launches(w, plan),
             "ex2_per_update": 2, "sfu_frac": 2 * w.updates / sfu_peak / (ms * 1e-3),
             "note": "forward-state checkpoint pass + adjoint pass (recomputing the states) + "
                     "fixed-order reductions; L2 flushed before each step"}
+
+
+def bench_backward_config(w: W.Workload, dev, stream, flush, steps: int, warmup: int, sfu_peak: float):
+    """ss_bwd of workload ``w`` at full size (its own inputs and a seeded dy),
+    as bench_backward; with sequence segments the two summary passes add
+    about two exps per update to the two of the segmented adjoint kernel."""
+    host = W.make_inputs(w)
+    out_dtype = w.out_dtype or w.dtype
+    names_in = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    d = {k: (host[k].to(dev) if host[k] is not None else None) for k in names_in}
+    dy = gen.fill(tuple(host["u"].shape), out_dtype, w.seed, 9).to(dev)
+    del host
+    ms, nws, plan = _time_backward(w, d, dy, out_dtype, flush, stream, steps, warmup)
+    del d, dy
+    torch.cuda.empty_cache()
+    return {"ms": ms, "steps": steps, "warmup": warmup, "updates_per_s": w.updates / (ms * 1e-3),
+            "sfu_frac": 2 * w.updates / sfu_peak / (ms * 1e-3), "ex2_per_update_counted": 2,
+            "workspace_bytes": nws, "plan": plan, "gpu_launches_per_step": _bwd_launches(w, plan)}
 
 
 def main(argv=None):

@@ -388,6 +388,25 @@ ss_status ss_bwd_state(const ss_desc *desc, const void *u, const void *delta, co
 size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 
 /*
+ * The launch plan of the backward for `desc` (host only, no CUDA call but
+ * the device's SM count):
+ *   batch_group  host out: batch entries per launch.  The batch runs in
+ *                groups whose forward-state checkpoints and dB/dC block
+ *                partials fit 7 GiB, so the workspace stays bounded for
+ *                large layers; results do not depend on the grouping.
+ *   segments     host out: sequence segments per row (1: none).  When one
+ *                group's blocks cannot give each SM three, a long sequence
+ *                (at least 4096 steps) is cut into segments of at least 2048
+ *                steps, each run as extra rows from the true state entering
+ *                it and the true adjoint leaving it, which two summary passes
+ *                (a forward over each segment from a zero state, an adjoint
+ *                pass over each segment from a zero end) and their folds
+ *                across the segments provide.
+ * Errors as ss_bwd's descriptor checks; SS_ERR_NULL_POINTER for a NULL out.
+ */
+ss_status ss_bwd_heuristic(const ss_desc *desc, int64_t *batch_group, int *segments);
+
+/*
  * As ss_fwd_hostio, pipelined over `nstreams` caller-owned streams (1..16):
  * the batch is cut into `chunks` ranges of batch entries (0: min(batch,
  * 2 * nstreams)); range c has its inputs copied in, its forward run and its

@@ -423,8 +423,27 @@ struct BwdLayout {
     int lanes, rows;        // lanes per row, rows per block
     int64_t dtiles, nsub;
     int64_t group;          // batch entries per launch
-    size_t off_ckpt, off_dbc, off_dA, off_dD, off_dbias, total;  // workspace byte offsets
+    int nseg;               // sequence segments (1: none)
+    int64_t seg_len;
+    size_t off_ckpt, off_dbc, off_dA, off_dD, off_dbias;                  // workspace byte offsets
+    size_t off_hend, off_dsum, off_lam0, off_D, total;                    // segment records (nseg > 1)
 };
+
+// Sequence segments of the backward: when one batch group's blocks cannot
+// give every SM three (the genomic shape: 4 x 1024 rows, 128 blocks of 32
+// rows), the sequence is cut into segments of at least kMinSegSteps steps (a
+// multiple of 64) so that about six blocks per SM run, each segment of each
+// row from the true state entering it and the true adjoint entering its end
+// (see ss_bwd_kernel.cuh).
+int bwd_segments(const ss_desc *desc, int64_t blocks, int64_t *seg_len) {
+    const int64_t sms = sm_count();
+    *seg_len = desc->seqlen;
+    if (blocks <= 0 || blocks >= 3 * sms || desc->seqlen < 2 * kMinSegSteps) return 1;
+    int64_t want = (6 * sms + blocks - 1) / blocks;
+    if (want > desc->seqlen / kMinSegSteps) want = desc->seqlen / kMinSegSteps;
+    if (want < 2) return 1;
+    return segment(desc, (int)want, seg_len);
+}
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -446,13 +465,19 @@ BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz) {
         group = (desc->batch + ngroups - 1) / ngroups;
     }
     lo.group = group;
-    const size_t grows = (size_t)group * (size_t)desc->dim;
+    lo.nseg = bwd_segments(desc, lo.dtiles * group, &lo.seg_len);
+    const size_t grows = (size_t)group * (size_t)desc->dim, S = (size_t)lo.nseg;
     lo.off_ckpt = 0;
     lo.off_dbc = align256(lo.off_ckpt + grows * (size_t)lo.nsub * N * 4);
     lo.off_dA = align256(lo.off_dbc + (size_t)lo.dtiles * (size_t)group * 2 * N * L * 4);
-    lo.off_dD = align256(lo.off_dA + rows * N * 4);
-    lo.off_dbias = align256(lo.off_dD + rows * 4);
-    lo.total = align256(lo.off_dbias + rows * 4);
+    lo.off_dD = align256(lo.off_dA + S * rows * N * 4);
+    lo.off_dbias = align256(lo.off_dD + S * rows * 4);
+    lo.off_hend = align256(lo.off_dbias + S * rows * 4);
+    const size_t seg_rec = lo.nseg > 1 ? S * grows : 0;  // (segment, row) records of one group
+    lo.off_dsum = align256(lo.off_hend + seg_rec * N * 4);
+    lo.off_lam0 = align256(lo.off_dsum + seg_rec * 4);
+    lo.off_D = align256(lo.off_lam0 + seg_rec * N * 4);
+    lo.total = align256(lo.off_D + seg_rec * N * 4);
     return lo;
 }
 
@@ -702,9 +727,90 @@ size_t ss_bwd_workspace_bytes(const ss_desc *desc) {
     return bwd_layout(desc, sz).total;
 }
 
+ss_status ss_bwd_heuristic(const ss_desc *desc, int64_t *batch_group, int *segments) {
+    Sizes sz;
+    const ss_status st = check_desc(desc, &sz);
+    if (st != SS_OK) return st;
+    if (!batch_group || !segments) return SS_ERR_NULL_POINTER;
+    const BwdLayout lo = bwd_layout(desc, sz);
+    *batch_group = lo.group;
+    *segments = lo.nseg;
+    return SS_OK;
+}
+
 }  // extern "C"
 
 namespace {
+
+// The per-segment summaries and their folds for one batch group (q: the
+// group's backward parameters): the forward direct kernel in segment mode
+// without y (end states and delta' sums), the forward carry fold (true
+// entering states), the adjoint summaries and the backward fold (true
+// last-state gradients), into the workspace's segment records.
+template <typename Tin, typename Tout>
+cudaError_t launch_seg_adjoint(int nmax, dim3 grid, cudaStream_t s, const selscan::BwdParams &q, float *lam0) {
+    switch (nmax) {
+        case 4: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 4><<<grid, 128, 0, s>>>(q, lam0); break;
+        case 8: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 8><<<grid, 128, 0, s>>>(q, lam0); break;
+        case 16: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 16><<<grid, 128, 0, s>>>(q, lam0); break;
+        case 32: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 32><<<grid, 128, 0, s>>>(q, lam0); break;
+        default: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 64><<<grid, 128, 0, s>>>(q, lam0); break;
+    }
+    return cudaGetLastError();
+}
+
+ss_status bwd_segment_summaries(const ss_desc *desc, const BwdLayout &lo, const selscan::BwdParams &q, char *ws,
+                                cudaStream_t s) {
+    const int nmax = selscan::state_bucket(q.dstate), n = nmax;
+    const int64_t grows = q.batch * q.dim;
+    const size_t ein = dtype_size(desc->in_dtype);
+    float *hend = reinterpret_cast<float *>(ws + lo.off_hend);
+    float *dsum = reinterpret_cast<float *>(ws + lo.off_dsum);
+    float *lam0 = reinterpret_cast<float *>(ws + lo.off_lam0);
+    float *D = reinterpret_cast<float *>(ws + lo.off_D);
+
+    // Forward summaries: the direct kernel with 2 lanes per row (1 below 4
+    // states), segment mode, no y, no gate or skip (they do not touch the state).
+    FwdParams f{};
+    f.u = q.u, f.delta = q.delta, f.B = q.B, f.C = q.C, f.z = nullptr;
+    f.A = q.A, f.D = nullptr, f.delta_bias = q.delta_bias;
+    f.y = nullptr, f.last_state = nullptr, f.init_state = q.init_state, f.reset = q.reset;
+    f.batch = q.batch, f.dim = q.dim, f.seqlen = q.seqlen, f.dstate = q.dstate, f.softplus = q.softplus;
+    bool vec = (q.seqlen * (int64_t)ein) % 16 == 0;
+    for (const void *ptr : {q.u, q.delta, q.B, q.C})
+        if (ptr && !aligned(ptr, 16)) vec = false;
+    f.vec = vec ? 1 : 0;
+    const int lanes = nmax / 2 >= 2 ? 2 : 1, warps = 4;
+    const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
+    f.dtiles = (q.dim + rows_per_block - 1) / rows_per_block;
+    f.seg_len = q.seg_len, f.nseg = q.nseg;
+    f.ws_hend = hend, f.ws_dsum = dsum;
+    f.status = nullptr, f.delta_r = nullptr, f.W_dt = nullptr, f.dt_rank = 0;
+    const size_t smem = selscan::direct_smem_bytes(ein, nmax, lanes, warps);
+    const dim3 grid((unsigned)(f.dtiles * q.batch * q.nseg)), block((unsigned)(warps * 32));
+    const int split = lanes > 1 ? 1 : 0;
+    cudaError_t err;
+    if (desc->in_dtype == SS_F32) err = launch_f32_f32(n, lanes, split, grid, block, smem, s, f);
+    else if (desc->out_dtype == SS_BF16) err = launch_bf16_bf16(n, lanes, split, grid, block, smem, s, f);
+    else err = launch_bf16_f32(n, lanes, split, grid, block, smem, s, f);
+    if (err != cudaSuccess) return SS_ERR_CUDA;
+    const dim3 fold_grid((unsigned)((grows + 7) / 8));
+    if (nmax > 32) selscan::ss_fwd_carry_kernel<64><<<fold_grid, 256, 0, s>>>(f);
+    else selscan::ss_fwd_carry_kernel<32><<<fold_grid, 256, 0, s>>>(f);
+    if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+
+    // Adjoint summaries of segments 1.., then the backward fold.
+    const int per = nmax < 8 ? 1 : nmax / 8;  // threads per (segment, row)
+    const int64_t threads = grows * (q.nseg - 1) * per;
+    const dim3 agrid((unsigned)((threads + 127) / 128));
+    if (desc->in_dtype == SS_F32) err = launch_seg_adjoint<float, float>(nmax, agrid, s, q, lam0);
+    else if (desc->out_dtype == SS_BF16) err = launch_seg_adjoint<__nv_bfloat16, __nv_bfloat16>(nmax, agrid, s, q, lam0);
+    else err = launch_seg_adjoint<__nv_bfloat16, float>(nmax, agrid, s, q, lam0);
+    if (err != cudaSuccess) return SS_ERR_CUDA;
+    if (nmax > 32) selscan::ss_bwd_seg_fold_kernel<64><<<fold_grid, 256, 0, s>>>(q, lam0, dsum, D);
+    else selscan::ss_bwd_seg_fold_kernel<32><<<fold_grid, 256, 0, s>>>(q, lam0, dsum, D);
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
 
 ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
                    const void *C, const float *D, const void *z, const float *delta_bias,
@@ -730,8 +836,8 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     const BwdLayout lo = bwd_layout(desc, sz);
     if (!workspace || workspace_bytes < lo.total) return SS_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return SS_ERR_MISALIGNED;
-    const int64_t blocks = lo.dtiles * lo.group;
-    if (blocks > INT_MAX) return SS_ERR_BAD_SHAPE;
+    const int64_t blocks = lo.dtiles * lo.group * lo.nseg;
+    if (blocks > INT_MAX || sz.rows * lo.nseg * 8 > INT_MAX) return SS_ERR_BAD_SHAPE;
 
     char *ws = static_cast<char *>(workspace);
     selscan::BwdParams p;
@@ -757,6 +863,11 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.init_state = init_state;
     p.dlast = dlast;
     p.d_init_state = d_init_state;
+    p.seg_len = lo.nseg > 1 ? lo.seg_len : desc->seqlen;
+    p.nseg = lo.nseg;
+    p.rows_all = sz.rows;
+    p.seg_h = nullptr;
+    p.seg_dl = nullptr;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int nmax = selscan::state_bucket(p.dstate), n = nmax;
@@ -792,7 +903,13 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
             q.init_state = init_state ? init_state + b0 * DN : nullptr;
             q.dlast = dlast ? dlast + b0 * DN : nullptr;
             q.d_init_state = d_init_state ? d_init_state + b0 * DN : nullptr;
-            if (fn(dim3((unsigned)(lo.dtiles * gb)), dim3(kBwdWarps * 32), smem, s, q) != cudaSuccess)
+            if (lo.nseg > 1 && desc->seqlen > 0) {
+                const ss_status ss = bwd_segment_summaries(desc, lo, q, ws, s);
+                if (ss != SS_OK) return ss;
+                q.seg_h = reinterpret_cast<const float *>(ws + lo.off_hend);
+                q.seg_dl = reinterpret_cast<const float *>(ws + lo.off_D);
+            }
+            if (fn(dim3((unsigned)(lo.dtiles * gb * lo.nseg)), dim3(kBwdWarps * 32), smem, s, q) != cudaSuccess)
                 return SS_ERR_CUDA;
             const int64_t bc = gb * 2 * NL;
             if (bc > 0) {

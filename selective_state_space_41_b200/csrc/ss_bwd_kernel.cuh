@@ -62,6 +62,17 @@ struct BwdParams {
     const float *init_state;                  // (batch, dim, dstate) state before step 0, or null (zero)
     const float *dlast;                       // (batch, dim, dstate) gradient wrt the last state, or null
     float *d_init_state;                      // (batch, dim, dstate) gradient wrt the state before step 0, or null
+    // Sequence segments (nseg > 1): block (s, b, tile) runs steps
+    // [s seg_len, (s + 1) seg_len) from seg_h[s - 1] (the true state entering
+    // segment s, s >= 1) and with seg_dl[s] (the adjoint entering its last
+    // step from the right, s <= nseg - 2) as its last-state gradient; the
+    // per-row partials of dA, dD and dbias are kept per segment, at
+    // (s rows_all + row), rows_all the rows of the whole batch.
+    int64_t seg_len;
+    int nseg;
+    int64_t rows_all;
+    const float *seg_h;                       // (nseg, rows, dstate)
+    const float *seg_dl;                      // (nseg, rows, dstate)
 };
 
 constexpr int kBwdSub = 8;                    // steps per sub-chunk
@@ -135,13 +146,19 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     constexpr int RS = rows + 2;                      // floats per step in the block's dB/dC slab
     constexpr int GS = bwd_group_stride(rows, kG);    // floats per (dB or dC, state) group
     const int N = p.dstate;
-    const int64_t b = blockIdx.x / p.dtiles;
+    const int64_t blocks_per_seg = p.batch * p.dtiles;
+    const int seg = (int)(blockIdx.x / blocks_per_seg);
+    const int64_t b = (blockIdx.x % blocks_per_seg) / p.dtiles;
     const int64_t dtile = blockIdx.x % p.dtiles;
     const int64_t d_raw = dtile * rows + rib;
     const bool row_ok = d_raw < p.dim;
     const int64_t d = row_ok ? d_raw : p.dim - 1;     // mirrored rows contribute nothing (g = 0)
-    const int64_t L = p.seqlen;
+    const int64_t L = p.seqlen;                       // row length (stride)
     const int64_t row = b * p.dim + d;
+    // This block's steps: [c_begin, Lend) (the whole row unless segmented).
+    const int64_t c_begin = (int64_t)seg * p.seg_len;
+    const int64_t Lend = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
+    const int64_t rows_grp = p.batch * p.dim;         // rows of this launch
     const bool vec = p.vec != 0;
     const bool vrows = p.vec_rows != 0;
     const bool softplus = p.softplus != 0;
@@ -184,7 +201,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
 
     // B/C of a stage: raw copies into RB by cp.async (issued one stage ahead),
     // converted into F (fp32 float4 per step and state pair) at the stage's start.
-    auto stage_fast = [&](int64_t c0) { return vec && c0 >= 0 && c0 + kBwdStage <= L; };
+    auto stage_fast = [&](int64_t c0) { return vec && c0 >= c_begin && c0 + kBwdStage <= Lend; };
     auto issue_copies = [&](int64_t c0) {
         for (int u = tid; u < 2 * kNmax * kStageUnits; u += nthreads) {
             const int j = u % kStageUnits, rowid = u / kStageUnits;
@@ -224,7 +241,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     for (int m = 0; m < 8; ++m) {
                         const int64_t l = c0 + i0 + m;
                         uint32_t bits = 0u;
-                        if (l < L) bits = Io<Tin>::bits(src, l);
+                        if (l < Lend) bits = Io<Tin>::bits(src, l);
                         if constexpr (sizeof(Tin) == 2) bits <<= 16;
                         v[c][m] = __uint_as_float(bits);
                     }
@@ -237,21 +254,21 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         if (stage_fast(next)) issue_copies(next);
     };
     auto put = [&](Tin *dst, int64_t l, float v) {
-        if (l < L) dst[l] = static_cast<Tin>(v);
+        if (l < Lend) dst[l] = static_cast<Tin>(v);
     };
 
     // This lane's kOwn steps of a row stream from step `so` as raw words (0 past the end).
     auto load_own = [&](const auto *src, int64_t so, uint32_t *w) {
         using T = std::remove_cv_t<std::remove_pointer_t<decltype(src)>>;
         constexpr int kBytes = kOwn * (int)sizeof(T), kWords = (kBytes + 3) / 4;
-        if (kBytes >= 4 && vrows && so + kOwn <= L) {
+        if (kBytes >= 4 && vrows && so + kOwn <= Lend) {
             ld_words<kBytes>(src + so, w);
         } else {
 #pragma unroll
             for (int j = 0; j < kWords; ++j) w[j] = 0u;
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
-                if (so + i < L) {
+                if (so + i < Lend) {
                     const uint32_t bits = Io<T>::bits(src, so + i);
                     if constexpr (sizeof(T) == 2) w[i >> 1] |= bits << (16 * (i & 1));
                     else w[i] = bits;
@@ -265,13 +282,13 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     const uint8_t *const reset_b = kReset ? p.reset + b * L : nullptr;
     auto load_flags = [&](int64_t l0, uint2 &w) {
         if constexpr (kReset) {
-            if (p.reset_vec && l0 + kBwdSub <= L) {
+            if (p.reset_vec && l0 + kBwdSub <= Lend) {
                 w = __ldg(reinterpret_cast<const uint2 *>(reset_b + l0));
             } else {
                 w = make_uint2(0u, 0u);
 #pragma unroll
                 for (int i = 0; i < kBwdSub; ++i)
-                    if (l0 + i < L && reset_b[l0 + i] != 0) (i < 4 ? w.x : w.y) |= 1u << (8 * (i & 3));
+                    if (l0 + i < Lend && reset_b[l0 + i] != 0) (i < 4 ? w.x : w.y) |= 1u << (8 * (i & 3));
             }
         }
     };
@@ -291,21 +308,23 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     for (int qq = 0; qq < kPL; ++qq) {  // the state before step 0 (mirrored rows: the true row's)
         const int n = 2 * (q0 + qq);
         h[qq] = make_float2(0.f, 0.f);
-        if (p.init_state != nullptr) {
-            if (n < N) h[qq].x = p.init_state[row * N + n];
-            if (n + 1 < N) h[qq].y = p.init_state[row * N + n + 1];
+        // the given state enters segment 0; segment s >= 1 starts from the true carry
+        const float *h_src = seg == 0 ? p.init_state : p.seg_h + ((int64_t)(seg - 1) * rows_grp) * N;
+        if (h_src != nullptr) {
+            if (n < N) h[qq].x = h_src[row * N + n];
+            if (n + 1 < N) h[qq].y = h_src[row * N + n + 1];
         }
     }
     uint32_t wu[kInWords], wd[kInWords];  // raw owned inputs of the next sub-chunk
-    if (L > 0) {
-        load_own(u_row, j0, wu);
-        load_own(d_row, j0, wd);
-        load_flags(0, wfl);
-        if (stage_fast(0)) issue_copies(0);
+    if (Lend > c_begin) {
+        load_own(u_row, c_begin + j0, wu);
+        load_own(d_row, c_begin + j0, wd);
+        load_flags(c_begin, wfl);
+        if (stage_fast(c_begin)) issue_copies(c_begin);
     }
-    for (int64_t c0 = 0; c0 < L; c0 += kBwdStage) {
-        load_stage(c0, c0 + kBwdStage < L ? c0 + kBwdStage : -1);
-        const int nsub = (int)(((L - c0 < kBwdStage ? L - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
+    for (int64_t c0 = c_begin; c0 < Lend; c0 += kBwdStage) {
+        load_stage(c0, c0 + kBwdStage < Lend ? c0 + kBwdStage : -1);
+        const int nsub = (int)(((Lend - c0 < kBwdStage ? Lend - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
 #pragma unroll 1
         for (int m = 0; m < nsub; ++m) {
             const int64_t l0 = c0 + m * kBwdSub;
@@ -319,14 +338,14 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
 #pragma unroll
             for (int i = 0; i < kOwn; ++i) {
                 const int64_t l = l0 + j0 + i;
-                const float dl = l < L ? delta_transform<kFast>(Io<Tin>::widen(wd, i) + bias, softplus) : 0.f;
+                const float dl = l < Lend ? delta_transform<kFast>(Io<Tin>::widen(wd, i) + bias, softplus) : 0.f;
                 if (owner) {
                     gat[j0 + i] = dl;
                     gat[kBwdSub + j0 + i] = dl * Io<Tin>::widen(wu, i);
                 }
             }
             const uint32_t starts = kReset ? flag_bits(wfl) : 0u;
-            if (l0 + kBwdSub < L) {
+            if (l0 + kBwdSub < Lend) {
                 load_own(u_row, l0 + kBwdSub + j0, wu);
                 load_own(d_row, l0 + kBwdSub + j0, wd);
                 load_flags(l0 + kBwdSub, wfl);
@@ -384,13 +403,16 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
     for (int qq = 0; qq < kPL; ++qq) {
         const int n = 2 * (q0 + qq);
         carry[qq] = make_float2(0.f, 0.f), dA_acc[qq] = make_float2(0.f, 0.f);
-        if (p.dlast != nullptr && row_ok) {  // mirrored rows carry nothing (they add to dB, dC)
-            if (n < N) carry[qq].x = p.dlast[row * N + n];
-            if (n + 1 < N) carry[qq].y = p.dlast[row * N + n + 1];
+        // the last segment from the given last-state gradient, the others from
+        // the adjoint entering from the right; mirrored rows carry nothing
+        const float *c_src = seg == p.nseg - 1 ? p.dlast : p.seg_dl + ((int64_t)seg * rows_grp) * N;
+        if (c_src != nullptr && row_ok) {
+            if (n < N) carry[qq].x = c_src[row * N + n];
+            if (n + 1 < N) carry[qq].y = c_src[row * N + n + 1];
         }
     }
     float dD_acc = 0.f, dbias_acc = 0.f;
-    const int64_t nstages = (L + kBwdStage - 1) / kBwdStage;
+    const int64_t nstages = (Lend - c_begin + kBwdStage - 1) / kBwdStage;
     // Prefetched for the next sub-chunk (backwards): its checkpoint and raw owned inputs.
     float2 h0n[kPL];
     uint32_t wz[kInWords], wdy[kDyWords];
@@ -407,15 +429,15 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         load_own(dy_row, l0 + j0, wdy);
         load_flags(l0, wfl);
     };
-    if (L > 0) prefetch(((L - 1) / kBwdSub) * kBwdSub);
+    if (Lend > c_begin) prefetch(((Lend - 1) / kBwdSub) * kBwdSub);
     for (int64_t st = nstages - 1; st >= 0; --st) {
-        const int64_t c0 = st * kBwdStage;
+        const int64_t c0 = c_begin + st * kBwdStage;
         if (st == nstages - 1) {  // F still holds the last stage from phase A
             if (stage_fast(c0 - kBwdStage)) issue_copies(c0 - kBwdStage);
         } else {
             load_stage(c0, c0 - kBwdStage);
         }
-        const int nsub = (int)(((L - c0 < kBwdStage ? L - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
+        const int nsub = (int)(((Lend - c0 < kBwdStage ? Lend - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
 #pragma unroll 1
         for (int m = nsub - 1; m >= 0; --m) {
             const int64_t l0 = c0 + m * kBwdSub;
@@ -426,7 +448,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 const int64_t l = l0 + j0 + i;
                 o_u[i] = Io<Tin>::widen(wu, i);
                 o_x[i] = Io<Tin>::widen(wd, i) + bias;
-                o_dl[i] = l < L ? delta_transform<kFast>(o_x[i], softplus) : 0.f;
+                o_dl[i] = l < Lend ? delta_transform<kFast>(o_x[i], softplus) : 0.f;
                 o_dy[i] = row_ok ? Io<Tout>::widen(wdy, i) : 0.f;
                 o_z[i] = has_z ? Io<Tin>::widen(wz, i) : 0.f;
                 o_sg[i] = has_z ? sigmoid_of<kFast>(o_z[i]) : 1.f;
@@ -441,7 +463,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
 #pragma unroll
             for (int qq = 0; qq < kPL; ++qq) h0[qq] = h0n[qq];
             const uint32_t starts = kReset ? flag_bits(wfl) : 0u;
-            if (l0 > 0) prefetch(l0 - kBwdSub);
+            if (l0 > c_begin) prefetch(l0 - kBwdSub);
             __syncwarp();
             float dl[kBwdSub], du[kBwdSub], gg[kBwdSub];
 #pragma unroll
@@ -544,7 +566,7 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 s = fmaf(Dd, o_u[i], s);
                 const float ddl = fmaf(o_u[i], LB, LHA);
                 const float dx = softplus ? (o_x[i] > 20.f ? ddl : ddl * sigmoid_of<kFast>(o_x[i])) : ddl * o_dl[i];
-                if (owner && row_ok && l < L) {
+                if (owner && row_ok && l < Lend) {
                     put(du_row, l, fmaf(o_g[i], Dd, o_dl[i] * LB));
                     put(dd_row, l, dx);
                     if (has_z) put(dz_row, l, o_dy[i] * s * o_sg[i] * fmaf(o_z[i], 1.f - o_sg[i], 1.f));
@@ -567,14 +589,14 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                     if (q + 1 < rows / 2) t2 = __fadd2_rn(t2, src[q + 1]);
                 }
                 s2 = __fadd2_rn(s2, t2);
-                if (l0 + out_i[k] < L) out_dst[k][l0] = s2.x + s2.y;
+                if (l0 + out_i[k] < Lend) out_dst[k][l0] = s2.x + s2.y;
             }
             __syncthreads();  // the slabs are free for the next sub-chunk
         }
     }
 
     // The adjoint carried past step 0 is the gradient wrt the state before it.
-    if (p.d_init_state != nullptr && row_ok) {
+    if (p.d_init_state != nullptr && row_ok && seg == 0) {
 #pragma unroll
         for (int qq = 0; qq < kPL; ++qq) {
             const int n = 2 * (q0 + qq);
@@ -582,13 +604,14 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
             if (n + 1 < N) p.d_init_state[row * N + n + 1] = carry[qq].y;
         }
     }
-    // Per-row partials of dA, dD and dbias.
+    // Per-row partials of dA, dD and dbias (per segment).
+    const int64_t prow = (int64_t)seg * p.rows_all + row;
     if (row_ok) {
 #pragma unroll
         for (int qq = 0; qq < kPL; ++qq) {
             const int n = 2 * (q0 + qq);
-            if (n < N) p.ws_dA[row * N + n] = dA_acc[qq].x;
-            if (n + 1 < N) p.ws_dA[row * N + n + 1] = dA_acc[qq].y;
+            if (n < N) p.ws_dA[prow * N + n] = dA_acc[qq].x;
+            if (n + 1 < N) p.ws_dA[prow * N + n + 1] = dA_acc[qq].y;
         }
     }
     if constexpr (kG > 1) {
@@ -599,8 +622,187 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         }
     }
     if (row_ok && g == 0) {
-        p.ws_dD[row] = dD_acc;
-        p.ws_dbias[row] = dbias_acc;
+        p.ws_dD[prow] = dD_acc;
+        p.ws_dbias[prow] = dbias_acc;
+    }
+}
+
+// ------------------------------------------------------ sequence segments
+// For few rows and a long sequence the backward runs each row's sequence as
+// nseg segments, as extra rows.  Segment s needs the true state entering it
+// and the adjoint entering its last step from the right; both come from
+// per-segment summaries, folded across the segments in order:
+//  - forward: h_end(s), the state at the end of s from a zero state, and
+//    P(s) = 2^(A log2e sum_s delta') (0 if s holds a sequence start), written
+//    by the forward direct kernel in its segment mode without y; the fold
+//    h_in(s) = P(s-1) h_in(s-1) + h_end(s-1) is the forward's carry kernel;
+//  - backward: lam0(s), the adjoint carried past the first step of s when the
+//    adjoint past its last step is zero (the recurrence lam_l = g_l C_l +
+//    a_(l+1) lam_(l+1) does not involve the state); the fold
+//    D(nseg-1) = dlast (or 0), D(s-1) = lam0(s) + P(s) D(s) gives segment
+//    s's last-state gradient D(s).
+// ss_bwd_seg_adjoint_kernel computes lam0(s) for s >= 1: one thread per
+// (segment, row, group of up to 8 states), the steps backwards 8 at a time
+// (vector loads when the rows are 16-byte aligned), exps on the SFU.
+template <typename Tin, typename Tout, int kNmax>
+__global__ void __launch_bounds__(128) ss_bwd_seg_adjoint_kernel(const BwdParams p, float *lam0) {
+    constexpr bool kFast = sizeof(Tin) == 2;
+    constexpr int kS = kNmax < 8 ? kNmax : 8;          // states per thread
+    constexpr int kT = kNmax / kS;                      // threads per (segment, row)
+    constexpr int kP = kS / 2 > 0 ? kS / 2 : 1;         // state pairs per thread
+    const int64_t rows = p.batch * p.dim;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int q = (int)(t % kT);
+    const int64_t rs = t / kT;
+    if (rs >= rows * (p.nseg - 1)) return;
+    const int64_t row = rs % rows;
+    const int s = 1 + (int)(rs / rows);
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const int N = p.dstate;
+    const int64_t L = p.seqlen;
+    const int64_t c_begin = (int64_t)s * p.seg_len;
+    const int64_t Lend = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
+    const bool softplus = p.softplus != 0;
+    const bool has_z = p.z != nullptr;
+    const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
+    float2 A2[kP], carry[kP];
+#pragma unroll
+    for (int k = 0; k < kP; ++k) {
+        const int n = q * kS + 2 * k;
+        A2[k] = make_float2(n < N ? p.A[d * N + n] * kLog2e : 0.f, n + 1 < N ? p.A[d * N + n + 1] * kLog2e : 0.f);
+        carry[k] = make_float2(0.f, 0.f);
+    }
+    const Tin *d_row = static_cast<const Tin *>(p.delta) + row * L;
+    const Tin *z_row = has_z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
+    const Tout *dy_row = static_cast<const Tout *>(p.dy) + row * L;
+    const Tin *C_b = static_cast<const Tin *>(p.C) + b * N * L;
+    const uint8_t *reset_b = p.reset ? p.reset + b * L : nullptr;
+    const bool vrows = p.vec_rows != 0, vbc = p.vec != 0;
+    // Groups of 8 steps [l0, l0 + 8), the last one first (c_begin is a
+    // multiple of 64, so every group starts on a multiple of 8).
+    for (int64_t l0 = ((Lend - 1) / 8) * 8; l0 >= c_begin; l0 -= 8) {
+        const bool full = l0 + 8 <= Lend;
+        float dl[8], g[8];
+        uint32_t starts = 0u;
+        {
+            uint32_t wd[4], wz[4];
+            if constexpr (sizeof(Tin) == 2) {
+                if (full && vrows) {
+                    ld_words<16>(d_row + l0, wd);
+                    if (has_z) ld_words<16>(z_row + l0, wz);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) wd[i] = 0u, wz[i] = 0u;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (l0 + i < Lend) {
+                            wd[i >> 1] |= Io<Tin>::bits(d_row, l0 + i) << (16 * (i & 1));
+                            if (has_z) wz[i >> 1] |= Io<Tin>::bits(z_row, l0 + i) << (16 * (i & 1));
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const bool in = l0 + i < Lend;
+                float x, zv = 0.f;
+                if constexpr (sizeof(Tin) == 2) {
+                    x = Io<Tin>::widen(wd, i);
+                    if (has_z) zv = Io<Tin>::widen(wz, i);
+                } else {
+                    x = in ? d_row[l0 + i] : 0.f;
+                    if (has_z) zv = in ? z_row[l0 + i] : 0.f;
+                }
+                const float dyv = in ? static_cast<float>(dy_row[l0 + i]) : 0.f;
+                dl[i] = in ? delta_transform<kFast>(x + bias, softplus) : 0.f;
+                g[i] = has_z ? dyv * zv * sigmoid_of<kFast>(zv) : dyv;
+                if (reset_b != nullptr && in && reset_b[l0 + i] != 0) starts |= 1u << i;
+            }
+        }
+        // C of the group's steps for this thread's states.
+        float2 c[8][kP];
+#pragma unroll
+        for (int k = 0; k < kP; ++k) {
+            const int n = q * kS + 2 * k;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int nn = n + h2;
+                float v[8];
+                bool vload = false;
+                if constexpr (sizeof(Tin) == 2) vload = nn < N && full && vbc;
+                if (nn >= N) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+                } else if (vload) {
+                    if constexpr (sizeof(Tin) == 2) {
+                        uint32_t w[4];
+                        ld_words<16>(C_b + (int64_t)nn * L + l0, w);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[i] = Io<Tin>::widen(w, i);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        v[i] = l0 + i < Lend ? static_cast<float>(C_b[(int64_t)nn * L + l0 + i]) : 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (h2 == 0) c[i][k].x = v[i];
+                    else c[i][k].y = v[i];
+                }
+            }
+        }
+        // lam_l = g_l C_l + carry; carry = a_l lam_l (nothing past a start).
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            const float2 d2 = make_float2(dl[i], dl[i]), g2 = make_float2(g[i], g[i]);
+            const bool st = (starts >> i) & 1u;
+#pragma unroll
+            for (int k = 0; k < kP; ++k) {
+                const float2 lam = __ffma2_rn(g2, c[i][k], carry[k]);
+                const float2 tt = __fmul2_rn(d2, A2[k]);
+                carry[k] = st ? make_float2(0.f, 0.f) : __fmul2_rn(make_float2(sfu_exp2(tt.x), sfu_exp2(tt.y)), lam);
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kP; ++k) {
+        const int n = q * kS + 2 * k;
+        if (n < N) lam0[((int64_t)s * rows + row) * N + n] = carry[k].x;
+        if (n + 1 < N) lam0[((int64_t)s * rows + row) * N + n + 1] = carry[k].y;
+    }
+}
+
+// The backward fold: D(nseg-1) = dlast (or 0); D(s-1) = lam0(s) + P(s) D(s),
+// P(s) = 2^(A log2e dsum(s)), 0 where dsum(s) < 0 (a start in s).  One warp
+// per row, states over lanes; D(s) written for s <= nseg - 2.
+template <int kNmax>
+__global__ void __launch_bounds__(256) ss_bwd_seg_fold_kernel(const BwdParams p, const float *lam0,
+                                                              const float *dsum, float *D) {
+    constexpr int kPer = kNmax > 32 ? 2 : 1;
+    const int64_t rows = p.batch * p.dim;
+    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int64_t d = row % p.dim;
+    const int N = p.dstate;
+    float A2[kPer], v[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int n = lane + 32 * k;
+        A2[k] = n < N ? p.A[d * N + n] * kLog2e : 0.f;
+        v[k] = n < N && p.dlast != nullptr ? p.dlast[row * N + n] : 0.f;
+    }
+    for (int s = p.nseg - 1; s >= 1; --s) {
+        const float ds = dsum[(int64_t)s * rows + row];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int n = lane + 32 * k;
+            if (n < N) {
+                v[k] = fmaf(ds < 0.f ? 0.f : sfu_exp2(A2[k] * ds), v[k], lam0[((int64_t)s * rows + row) * N + n]);
+                D[((int64_t)(s - 1) * rows + row) * N + n] = v[k];
+            }
+        }
     }
 }
 
@@ -617,7 +819,8 @@ static __global__ void __launch_bounds__(256) ss_bwd_reduce_bc_kernel(const BwdP
     }
 }
 
-// dA, dD, dbias = the per-row partials summed over the batch, in batch order.
+// dA, dD, dbias = the per-row partials summed over the segments and the
+// batch, in (segment, batch) order.
 static __global__ void __launch_bounds__(256) ss_bwd_reduce_rows_kernel(const BwdParams p, float *dA, float *dD,
                                                                   float *dbias) {
     const int64_t N = p.dstate;
@@ -626,7 +829,8 @@ static __global__ void __launch_bounds__(256) ss_bwd_reduce_rows_kernel(const Bw
          e += (int64_t)gridDim.x * blockDim.x) {
         if (e < p.dim * N) {
             float s = 0.f;
-            for (int64_t b = 0; b < p.batch; ++b) s += p.ws_dA[b * p.dim * N + e];
+            for (int sg = 0; sg < p.nseg; ++sg)
+                for (int64_t b = 0; b < p.batch; ++b) s += p.ws_dA[((int64_t)sg * p.rows_all + b * p.dim) * N + e];
             dA[e] = s;
         } else {
             const int64_t j = e - p.dim * N, d = j % p.dim;
@@ -635,7 +839,8 @@ static __global__ void __launch_bounds__(256) ss_bwd_reduce_rows_kernel(const Bw
             if (out == nullptr) continue;
             const float *src = is_bias ? p.ws_dbias : p.ws_dD;
             float s = 0.f;
-            for (int64_t b = 0; b < p.batch; ++b) s += src[b * p.dim + d];
+            for (int sg = 0; sg < p.nseg; ++sg)
+                for (int64_t b = 0; b < p.batch; ++b) s += src[(int64_t)sg * p.rows_all + b * p.dim + d];
             out[d] = s;
         }
     }

@@ -851,6 +851,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     const bool vec = p.vec != 0;
     const bool softplus = p.softplus != 0;
     const bool has_z = p.z != nullptr;
+    const bool want_y = p.y != nullptr;
     // This block's steps: [c_begin, Lend) (the whole row unless segmented).
     const int64_t c_begin = seg * p.seg_len;
     const int64_t Lend = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
@@ -1247,7 +1248,12 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
         } else {
             steps(std::false_type{});
         }
-        // Totals of the owned steps.
+        // Totals of the owned steps (none without y: the backward's segment
+        // summary runs this kernel for its segment records only).
+        if (!want_y) {
+            y_own += kDirectSub;
+            return;
+        }
         float yv[kOwn];
         if constexpr (kG == 1) {
 #pragma unroll

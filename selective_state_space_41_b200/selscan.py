@@ -10,6 +10,7 @@ The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``,
 ``ss_fwd_reset``, ``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
 ``ss_fwd_noalloc``, ``ss_fwd_dtproj``, ``ss_step``, ``ss_bwd``, ``ss_bwd_reset``, ``ss_bwd_state``, ``ss_bwd_workspace_bytes``,
+``ss_bwd_heuristic``,
 ``ss_status_string``, ``ss_version``, ``ss_device_status``); ``ss_fwd`` dispatches to the
 workspace, config, initial-state and sequence-start forms by keyword, ``ss_fwd_hostio`` to
 the pipelined form when given streams.  ``selective_scan_fwd`` and
@@ -38,7 +39,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
            "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc",
            "ss_step", "ss_bwd", "ss_bwd_reset", "ss_bwd_state", "ss_bwd_workspace_bytes", "ss_status_string",
-           "ss_version", "ss_device_status", "ss_fwd_dtproj")
+           "ss_version", "ss_device_status", "ss_fwd_dtproj", "ss_bwd_heuristic")
 
 
 class SelscanError(RuntimeError):
@@ -105,6 +106,8 @@ def lib():
         L.ss_bwd_state.argtypes = [DP] + [P] * 8 + [I] + [P] * 13 + [P, SZ, P]
         L.ss_bwd_workspace_bytes.restype = SZ
         L.ss_bwd_workspace_bytes.argtypes = [DP]
+        L.ss_bwd_heuristic.restype = I
+        L.ss_bwd_heuristic.argtypes = [DP, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(I)]
         L.ss_status_string.restype = ctypes.c_char_p
         L.ss_status_string.argtypes = [I]
         L.ss_version.restype = I
@@ -277,6 +280,14 @@ def ss_step(u, delta, A, B, C, state, y, D=None, z=None, delta_bias=None, delta_
 def ss_bwd_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None) -> int:
     desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
     return int(lib().ss_bwd_workspace_bytes(ctypes.byref(desc)))
+
+
+def ss_bwd_heuristic(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None) -> dict:
+    """The backward's launch plan: batch entries per launch and sequence segments."""
+    desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
+    group, segs = ctypes.c_int64(0), ctypes.c_int(0)
+    _check(lib().ss_bwd_heuristic(ctypes.byref(desc), ctypes.byref(group), ctypes.byref(segs)), "ss_bwd_heuristic")
+    return {"batch_group": int(group.value), "segments": int(segs.value)}
 
 
 def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_softplus=False,
