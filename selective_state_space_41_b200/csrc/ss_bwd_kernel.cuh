@@ -645,11 +645,13 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
 // (segment, row, group of up to 8 states), the steps backwards 8 at a time
 // (vector loads when the rows are 16-byte aligned), exps on the SFU.
 template <typename Tin, typename Tout, int kNmax>
-__global__ void __launch_bounds__(128) ss_bwd_seg_adjoint_kernel(const BwdParams p, float *lam0) {
+__global__ void __launch_bounds__(128, 3) ss_bwd_seg_adjoint_kernel(const BwdParams p, float *lam0) {
     constexpr bool kFast = sizeof(Tin) == 2;
     constexpr int kS = kNmax < 8 ? kNmax : 8;          // states per thread
     constexpr int kT = kNmax / kS;                      // threads per (segment, row)
     constexpr int kP = kS / 2 > 0 ? kS / 2 : 1;         // state pairs per thread
+    constexpr int kWin = 8 * (int)sizeof(Tin) / 4;      // words of 8 steps of an input row
+    constexpr int kWout = 8 * (int)sizeof(Tout) / 4;    // words of 8 steps of dy
     const int64_t rows = p.batch * p.dim;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int q = (int)(t % kT);
@@ -678,88 +680,85 @@ __global__ void __launch_bounds__(128) ss_bwd_seg_adjoint_kernel(const BwdParams
     const Tin *C_b = static_cast<const Tin *>(p.C) + b * N * L;
     const uint8_t *reset_b = p.reset ? p.reset + b * L : nullptr;
     const bool vrows = p.vec_rows != 0, vbc = p.vec != 0;
-    // Groups of 8 steps [l0, l0 + 8), the last one first (c_begin is a
-    // multiple of 64, so every group starts on a multiple of 8).
-    for (int64_t l0 = ((Lend - 1) / 8) * 8; l0 >= c_begin; l0 -= 8) {
-        const bool full = l0 + 8 <= Lend;
-        float dl[8], g[8];
-        uint32_t starts = 0u;
-        {
-            uint32_t wd[4], wz[4];
-            if constexpr (sizeof(Tin) == 2) {
-                if (full && vrows) {
-                    ld_words<16>(d_row + l0, wd);
-                    if (has_z) ld_words<16>(z_row + l0, wz);
-                } else {
+
+    // The raw words of a group of 8 steps [l0, l0 + 8): delta, z, dy, this
+    // thread's C rows, start flags (zero past the segment's end).  The group
+    // before (in time) is loaded while this one is computed.
+    struct Raw {
+        uint32_t d[kWin], z[kWin], dy[kWout], c[2 * kP][kWin];
+        uint32_t st;
+    };
+    auto load_row = [&](const auto *src, int64_t l0, bool vec_ok, uint32_t *w, auto words) {
+        using T = std::remove_cv_t<std::remove_pointer_t<decltype(src)>>;
+        constexpr int kW = decltype(words)::value;
+        if (vec_ok && l0 + 8 <= Lend) {
+            ld_words<8 * (int)sizeof(T)>(src + l0, w);
+        } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) wd[i] = 0u, wz[i] = 0u;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (l0 + i < Lend) {
-                            wd[i >> 1] |= Io<Tin>::bits(d_row, l0 + i) << (16 * (i & 1));
-                            if (has_z) wz[i >> 1] |= Io<Tin>::bits(z_row, l0 + i) << (16 * (i & 1));
-                        }
-                    }
-                }
-            }
+            for (int k = 0; k < kW; ++k) w[k] = 0u;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const bool in = l0 + i < Lend;
-                float x, zv = 0.f;
-                if constexpr (sizeof(Tin) == 2) {
-                    x = Io<Tin>::widen(wd, i);
-                    if (has_z) zv = Io<Tin>::widen(wz, i);
-                } else {
-                    x = in ? d_row[l0 + i] : 0.f;
-                    if (has_z) zv = in ? z_row[l0 + i] : 0.f;
+                if (l0 + i < Lend) {
+                    const uint32_t bits = Io<T>::bits(src, l0 + i);
+                    if constexpr (sizeof(T) == 2) w[i >> 1] |= bits << (16 * (i & 1));
+                    else w[i] = bits;
                 }
-                const float dyv = in ? static_cast<float>(dy_row[l0 + i]) : 0.f;
-                dl[i] = in ? delta_transform<kFast>(x + bias, softplus) : 0.f;
-                g[i] = has_z ? dyv * zv * sigmoid_of<kFast>(zv) : dyv;
-                if (reset_b != nullptr && in && reset_b[l0 + i] != 0) starts |= 1u << i;
             }
         }
-        // C of the group's steps for this thread's states.
-        float2 c[8][kP];
+    };
+    auto load_group = [&](int64_t l0, Raw &r) {
+        load_row(d_row, l0, vrows, r.d, std::integral_constant<int, kWin>{});
+        if (has_z) load_row(z_row, l0, vrows, r.z, std::integral_constant<int, kWin>{});
+        load_row(dy_row, l0, vrows, r.dy, std::integral_constant<int, kWout>{});
 #pragma unroll
-        for (int k = 0; k < kP; ++k) {
-            const int n = q * kS + 2 * k;
+        for (int k = 0; k < 2 * kP; ++k) {
+            const int n = q * kS + k;
+            if (n < N) {
+                load_row(C_b + (int64_t)n * L, l0, vbc, r.c[k], std::integral_constant<int, kWin>{});
+            } else {
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int nn = n + h2;
-                float v[8];
-                bool vload = false;
-                if constexpr (sizeof(Tin) == 2) vload = nn < N && full && vbc;
-                if (nn >= N) {
+                for (int w = 0; w < kWin; ++w) r.c[k][w] = 0u;
+            }
+        }
+        r.st = 0u;
+        if (reset_b != nullptr) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] = 0.f;
-                } else if (vload) {
-                    if constexpr (sizeof(Tin) == 2) {
-                        uint32_t w[4];
-                        ld_words<16>(C_b + (int64_t)nn * L + l0, w);
+            for (int i = 0; i < 8; ++i)
+                if (l0 + i < Lend && reset_b[l0 + i] != 0) r.st |= 1u << i;
+        }
+    };
+
+    // Groups of 8 steps, the last one first (c_begin is a multiple of 64, so
+    // every group starts on a multiple of 8).
+    int64_t l0 = ((Lend - 1) / 8) * 8;
+    Raw nxt;
+    load_group(l0, nxt);
+    for (; l0 >= c_begin; l0 -= 8) {
+        const Raw cur = nxt;
+        if (l0 - 8 >= c_begin) load_group(l0 - 8, nxt);
+        float dl[8], g[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) v[i] = Io<Tin>::widen(w, i);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        v[i] = l0 + i < Lend ? static_cast<float>(C_b[(int64_t)nn * L + l0 + i]) : 0.f;
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (h2 == 0) c[i][k].x = v[i];
-                    else c[i][k].y = v[i];
-                }
+        for (int i = 0; i < 8; ++i) {
+            const bool in = l0 + i < Lend;
+            const float x = Io<Tin>::widen(cur.d, i) + bias;
+            const float dyv = Io<Tout>::widen(cur.dy, i);
+            dl[i] = in ? delta_transform<kFast>(x, softplus) : 0.f;
+            if (has_z) {
+                const float zv = Io<Tin>::widen(cur.z, i);
+                g[i] = dyv * zv * sigmoid_of<kFast>(zv);
+            } else {
+                g[i] = dyv;
             }
         }
         // lam_l = g_l C_l + carry; carry = a_l lam_l (nothing past a start).
 #pragma unroll
         for (int i = 7; i >= 0; --i) {
             const float2 d2 = make_float2(dl[i], dl[i]), g2 = make_float2(g[i], g[i]);
-            const bool st = (starts >> i) & 1u;
+            const bool st = (cur.st >> i) & 1u;
 #pragma unroll
             for (int k = 0; k < kP; ++k) {
-                const float2 lam = __ffma2_rn(g2, c[i][k], carry[k]);
+                const float2 cv = make_float2(Io<Tin>::widen(cur.c[2 * k], i), Io<Tin>::widen(cur.c[2 * k + 1], i));
+                const float2 lam = __ffma2_rn(g2, cv, carry[k]);
                 const float2 tt = __fmul2_rn(d2, A2[k]);
                 carry[k] = st ? make_float2(0.f, 0.f) : __fmul2_rn(make_float2(sfu_exp2(tt.x), sfu_exp2(tt.y)), lam);
             }

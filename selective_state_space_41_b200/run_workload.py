@@ -2,20 +2,21 @@
 
     python -m selective_state_space_41_b200.run_workload NAME [--batch B]
         [--repeat K] [--lanes G] [--split S] [--warps W] [--segments P]
-        [--dt-rank R]
+        [--dt-rank R] [--backward]
 
 Draws the workload's seeded inputs (optionally only its first B batch
 entries, to keep a capture small), moves them to ``cuda:0`` and calls
 ``ss_fwd`` (or ``ss_fwd_dtproj`` with ``--dt-rank``) K times in the launch
 shape given, zeros meaning the heuristic's choice.  A workspace is passed
-when the shape uses sequence segments.  Prints ``ok`` after a final
-synchronize.
+when the shape uses sequence segments.  ``--backward`` calls ``ss_bwd`` (all
+gradients, a seeded dy, its own plan) K times instead.  Prints ``ok`` after
+a final synchronize.
 """
 import argparse
 
 import torch
 
-from . import selscan, workloads as W
+from . import gen, selscan, workloads as W
 
 
 def main(argv=None):
@@ -28,6 +29,7 @@ def main(argv=None):
     ap.add_argument("--warps", type=int, default=0)
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--dt-rank", type=int, default=0)
+    ap.add_argument("--backward", action="store_true")
     a = ap.parse_args(argv)
     w = W.WORKLOADS[a.name]
     if a.batch:
@@ -40,7 +42,12 @@ def main(argv=None):
     if a.lanes or a.split or a.warps or a.segments:
         cfg = dict(lanes_per_row=a.lanes, split_states=a.split, warps_per_block=a.warps, segments=a.segments)
     kw = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, last_state=last)
-    if a.dt_rank:
+    if a.backward:
+        dy = gen.fill(tuple(inp["u"].shape), w.out_dtype or w.dtype, w.seed, 9).cuda()
+        for _ in range(a.repeat):
+            selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], dy, D=d["D"], z=d["z"],
+                                       delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus)
+    elif a.dt_rank:
         ws = selscan.workspace_for(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, y.dtype)
         for _ in range(a.repeat):
             selscan.ss_fwd_dtproj(d["u"], d["delta_r"], d["W_dt"], d["A"], d["B"], d["C"], y, workspace=ws, **kw)
