@@ -245,6 +245,41 @@ def test_reset_mask_checked_by_the_binding():
                            workspace=torch.zeros(16, dtype=torch.uint8), stream=s0, reset=bad)
 
 
+@pytest.mark.parametrize("shape,want", [
+    # (B, D, L, N), (batch entries per launch, sequence segments) on 148 SMs
+    ((8, 1536, 2048, 16), (8, 1)),        # mamba-130m-shaped layer: 384 blocks, whole batch
+    ((4, 1024, 100000, 16), (4, 7)),      # genomic: 128 blocks -> 7 segments of 14 336 steps
+    ((16, 4096, 8192, 16), (16, 1)),      # wide layers: groups within 7 GiB of workspace
+    ((16, 4096, 8192, 32), (6, 1)),
+    ((16, 4096, 8192, 64), (2, 1)),
+    ((1, 8, 9000, 16), (1, 4)),           # few rows: segments capped at L / 2048
+    ((1, 8, 4095, 16), (1, 1)),           # too short to cut
+])
+def test_bwd_plan(shape, want):
+    """The backward's plan for the measured layers and the segment limits."""
+    plan = selscan.ss_bwd_heuristic(*shape, selscan.SS_BF16)
+    assert (plan["batch_group"], plan["segments"]) == want
+
+
+def test_bwd_plan_rejections(lib):
+    g, s = ctypes.c_int64(0), ctypes.c_int(0)
+    assert lib.ss_bwd_heuristic(None, ctypes.byref(g), ctypes.byref(s)) == 1
+    assert lib.ss_bwd_heuristic(ctypes.byref(_desc(dstate=65)), ctypes.byref(g), ctypes.byref(s)) == 4
+    assert lib.ss_bwd_heuristic(ctypes.byref(_desc()), None, ctypes.byref(s)) == 1
+
+
+def test_bwd_segment_records_in_the_workspace(lib):
+    """A segmented plan adds its per-segment records (end states, delta'
+    sums, adjoint summaries and their fold: (3 N + 1) floats per segment and
+    row, plus per-segment row partials) to the unsegmented layout."""
+    d = _desc(batch=1, dim=8, seqlen=9000, dstate=16, in_dtype=1, out_dtype=1)
+    n = lib.ss_bwd_workspace_bytes(ctypes.byref(d))
+    rows, N, segs, nsub = 8, 16, 4, (9000 + 7) // 8
+    base = rows * nsub * N * 4 + 1 * 2 * N * 9000 * 4   # checkpoints + one tile's dB/dC partials
+    extra = segs * rows * (3 * N + 1) * 4 + segs * rows * (N + 2) * 4
+    assert base + extra <= n <= base + extra + 16 * 256  # 256-byte alignment of each region
+
+
 @pytest.mark.parametrize("shape,ws,want", [
     # (B, D, L, N), workspace bytes, (lanes_per_row, split_states, warps_per_block, segments)
     ((8, 1536, 2048, 16), 0, (4, 1, 4, 1)),          # mamba-130m-shaped layer: measured best 4s/4
