@@ -1394,8 +1394,10 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 // (from there ex2.ftz returns exactly 0, so the remaining shares are exactly
 // zero, and steps past that point are not rewritten) or that held a start.
 // With bf16 output y is rounded twice: once by the direct kernel (its
-// zero-state value) and once here after the share is added in fp32; the
-// result is within 1.5 bf16 ulp of the single rounding of the exact sum.
+// zero-state value y0) and once here after the share is added in fp32, so
+// the result differs from the exact sum by up to half a bf16 ulp of y0 plus
+// half a bf16 ulp of the result (2^-9 |y0| + 2^-9 |y| at most), more than one
+// rounding only where the share cancels much of y0.
 // The dt_proj form (p.delta null) recomputes delta = W_dt delta_r for the
 // steps it corrects, in fp32 from the exact bf16 products (the direct kernel
 // sums the same products on the tensor cores, in its own order).

@@ -205,6 +205,23 @@ def test_segments_long_memory():
     assert_parity(y, last, y_ref, last_ref, TOL[torch.float32], "fast decay")
 
 
+def test_segments_bf16_carry_dominated():
+    """bf16 output where, after the first segment, y is mostly the carried
+    state's share: u large over the first 1000 steps and 1/64 of it after,
+    slow decay (delta' ~ 1e-3), no skip term.  The fix-up adds a share that is
+    large against the segment kernel's own (rounded) value, so y is rounded
+    twice where that matters; the 1e-2 (1 + |y|) bound still holds."""
+    inp = _case(2, 6, 4000, 16, torch.bfloat16, seed=29, has_z=True, D_kind="none", return_last_state=True)
+    u = inp["u"].float()
+    u[..., 1000:] *= 1.0 / 64
+    inp["u"] = u.to(torch.bfloat16)
+    inp["delta"] = (inp["delta"].float() * 0.1 - 7.0).to(torch.bfloat16)
+    for segs in (3, 4):
+        y, last = run_gpu(inp, lanes=2, split=True, warps=1, segments=segs)
+        y_ref, last_ref = run_oracle(inp)
+        assert_parity(y, last, y_ref, last_ref, TOL[torch.bfloat16], f"carry-dominated, {segs} segments")
+
+
 def test_heuristic_segments_genomic_shape():
     """The genomic shape segments when given a workspace, and not without one."""
     h_ws = selscan.ss_fwd_heuristic(4, 1024, 100000, 16, torch.bfloat16, workspace_bytes=1 << 30)
