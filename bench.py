@@ -216,8 +216,11 @@ def cpu_oracle_sample(w: W.Workload, inp: dict = None, target_s: float = 10.0):
     per_row = run_rows(probe) / probe
     want = target_s / max(per_row, 1e-12)
     if want >= total:
-        reps = int(min(50, max(1, round(want / total))))
-        dt = sum(run_rows(total) for _ in range(reps))
+        # one whole pass, then as many more as fill target_s at its measured rate
+        # (the probe's few rows overstate the per-row time)
+        dt = run_rows(total)
+        reps = 1 + int(min(49, max(0, round((target_s - dt) / max(dt, 1e-9)))))
+        dt += sum(run_rows(total) for _ in range(reps - 1))
         updates = reps * w.updates
         desc = (f"the whole workload ({total} rows x {w.seqlen} steps x N={w.dstate}), "
                 f"{reps} pass(es): {updates:.3e} updates in {dt:.2f} s")
