@@ -384,6 +384,48 @@ ss_status ss_bwd_state(const ss_desc *desc, const void *u, const void *delta, co
                        float *ddelta_bias, float *d_initial_state, void *workspace,
                        size_t workspace_bytes, ss_stream_t stream);
 
+/*
+ * The forward that also writes the checkpoints its backward needs (for
+ * training: the backward, ss_bwd_ckpt, then skips its own forward pass over
+ * the sequence, about one exp per state update fewer).  Arguments as
+ * ss_fwd_reset (initial_state and reset may be NULL), launch shape from the
+ * heuristic given the workspace, plus:
+ *   ckpt    device, (B, D, ceil(L/8), N) float32 output: the state entering
+ *           every step l = 8k, i.e. after step l-1 (before a sequence start
+ *           at l zeroes it; the initial state at k = 0).  With sequence
+ *           segments the fix-up completes the checkpoints of segments >= 1.
+ * The checkpoints come from the direct kernel: where the heuristic would pick
+ * the scan kernel (few rows, no workspace) the direct kernel's widest state
+ * split runs instead.  y and last_state are bitwise those of ss_fwd_reset in
+ * the same launch shape.  SS_ERR_NULL_POINTER when ckpt is NULL and there is
+ * work; other errors as ss_fwd_reset.
+ */
+ss_status ss_fwd_ckpt(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                      const void *C, const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                      const float *initial_state, const uint8_t *reset, void *y, float *last_state, float *ckpt,
+                      void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
+/*
+ * ss_bwd_state from the forward's checkpoints (ss_fwd_ckpt of the same
+ * inputs, initial state and starts) instead of its own checkpointing pass.
+ *   ckpt          device, (B, D, ceil(L/8), N) float32, read only
+ *   d_last_state, d_initial_state, reset: as ss_bwd_state (the initial state
+ *                 itself is in the checkpoints)
+ *   workspace     ss_bwd_ckpt_workspace_bytes(desc) bytes (no checkpoint
+ *                 region; ss_bwd_workspace_bytes is enough too)
+ * The gradients equal ss_bwd_state's up to the fp32 order of the segment
+ * summaries (bitwise without sequence segments, where the checkpoints are the
+ * same values).  SS_ERR_NULL_POINTER when ckpt is NULL and there is work.
+ */
+ss_status ss_bwd_ckpt(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                      const void *C, const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                      const uint8_t *reset, const float *ckpt, const float *d_last_state, const void *dy, void *du,
+                      void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                      float *d_initial_state, void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
+/* Bytes of workspace ss_bwd_ckpt needs for `desc` (0 for an invalid descriptor). */
+size_t ss_bwd_ckpt_workspace_bytes(const ss_desc *desc);
+
 /* Bytes of workspace ss_bwd, ss_bwd_reset and ss_bwd_state need for `desc` (0 for an invalid descriptor). */
 size_t ss_bwd_workspace_bytes(const ss_desc *desc);
 

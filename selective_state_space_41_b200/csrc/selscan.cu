@@ -314,7 +314,8 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
                    const float *delta_bias, int delta_softplus, const float *initial_state,
                    const uint8_t *reset, void *y, float *last_state, const ss_launch_config *cfg,
                    void *workspace, size_t workspace_bytes, ss_stream_t stream,
-                   const void *delta_r = nullptr, const void *W_dt = nullptr, int dt_rank = 0) {
+                   const void *delta_r = nullptr, const void *W_dt = nullptr, int dt_rank = 0,
+                   float *ckpt = nullptr) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
@@ -323,9 +324,12 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     if (dt && desc->in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED_DTYPE;
     if (dt && (dt_rank < 1 || dt_rank > selscan::kMaxDtRank)) return SS_ERR_BAD_SHAPE;
     Plan pl;
-    st = resolve(desc, sz.rows, cfg, workspace_bytes, &pl, reset != nullptr);
+    // sequence starts and checkpoints are read / written by the direct kernel only
+    st = resolve(desc, sz.rows, cfg, workspace_bytes, &pl, reset != nullptr || ckpt != nullptr);
     if (st != SS_OK) return st;
     if (dt && !dt_plan(desc, &pl)) return SS_ERR_BAD_CONFIG;
+    if (ckpt != nullptr && (pl.split == 2 || dt)) return SS_ERR_BAD_CONFIG;  // the shared-memory direct kernel
+    if (ckpt != nullptr && !aligned(ckpt, 4)) return SS_ERR_MISALIGNED;
     if (sz.rows == 0) return SS_OK;  // no rows: nothing to read or write
     const bool need_seq = desc->seqlen > 0;
     if (!A) return SS_ERR_NULL_POINTER;
@@ -391,6 +395,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.delta_r = delta_r;
     p.W_dt = W_dt;
     p.dt_rank = dt_rank;
+    p.ckpt = ckpt;
 
     const dim3 grid((unsigned)blocks), block((unsigned)(pl.warps * 32));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -447,7 +452,9 @@ int bwd_segments(const ss_desc *desc, int64_t blocks, int64_t *seg_len) {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz) {
+// ckpt_given: the forward's checkpoints come from the caller (ss_bwd_ckpt),
+// so the workspace holds none; the plan is the same.
+BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz, bool ckpt_given = false) {
     BwdLayout lo{};
     const int nmax = selscan::state_bucket((int)desc->dstate);
     lo.lanes = selscan::bwd_lanes(nmax);
@@ -468,7 +475,7 @@ BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz) {
     lo.nseg = bwd_segments(desc, lo.dtiles * group, &lo.seg_len);
     const size_t grows = (size_t)group * (size_t)desc->dim, S = (size_t)lo.nseg;
     lo.off_ckpt = 0;
-    lo.off_dbc = align256(lo.off_ckpt + grows * (size_t)lo.nsub * N * 4);
+    lo.off_dbc = align256(lo.off_ckpt + (ckpt_given ? 0 : grows * (size_t)lo.nsub * N * 4));
     lo.off_dA = align256(lo.off_dbc + (size_t)lo.dtiles * (size_t)group * 2 * N * L * 4);
     lo.off_dD = align256(lo.off_dA + S * rows * N * 4);
     lo.off_dbias = align256(lo.off_dD + S * rows * 4);
@@ -543,6 +550,15 @@ ss_status ss_fwd_dtproj(const ss_desc *desc, int dt_rank, const void *u, const v
     if (dt_rank == 0) return SS_ERR_BAD_SHAPE;
     return fwd_impl(desc, u, nullptr, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y, last_state,
                     nullptr, workspace, workspace_bytes, stream, delta_r, W_dt, dt_rank);
+}
+
+ss_status ss_fwd_ckpt(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                      const void *C, const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                      const float *initial_state, const uint8_t *reset, void *y, float *last_state, float *ckpt,
+                      void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+    if (!ckpt && desc && desc->batch > 0 && desc->dim > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
+    return fwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, reset, y, last_state,
+                    nullptr, workspace, workspace_bytes, stream, nullptr, nullptr, 0, ckpt);
 }
 
 ss_status ss_fwd_reset(const ss_desc *desc, const void *u, const void *delta, const float *A,
@@ -748,13 +764,14 @@ namespace {
 // entering states), the adjoint summaries and the backward fold (true
 // last-state gradients), into the workspace's segment records.
 template <typename Tin, typename Tout>
-cudaError_t launch_seg_adjoint(int nmax, dim3 grid, cudaStream_t s, const selscan::BwdParams &q, float *lam0) {
+cudaError_t launch_seg_adjoint(int nmax, dim3 grid, cudaStream_t s, const selscan::BwdParams &q, float *lam0,
+                               float *dsum) {
     switch (nmax) {
-        case 4: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 4><<<grid, 128, 0, s>>>(q, lam0); break;
-        case 8: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 8><<<grid, 128, 0, s>>>(q, lam0); break;
-        case 16: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 16><<<grid, 128, 0, s>>>(q, lam0); break;
-        case 32: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 32><<<grid, 128, 0, s>>>(q, lam0); break;
-        default: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 64><<<grid, 128, 0, s>>>(q, lam0); break;
+        case 4: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 4><<<grid, 128, 0, s>>>(q, lam0, dsum); break;
+        case 8: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 8><<<grid, 128, 0, s>>>(q, lam0, dsum); break;
+        case 16: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 16><<<grid, 128, 0, s>>>(q, lam0, dsum); break;
+        case 32: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 32><<<grid, 128, 0, s>>>(q, lam0, dsum); break;
+        default: selscan::ss_bwd_seg_adjoint_kernel<Tin, Tout, 64><<<grid, 128, 0, s>>>(q, lam0, dsum); break;
     }
     return cudaGetLastError();
 }
@@ -769,43 +786,48 @@ ss_status bwd_segment_summaries(const ss_desc *desc, const BwdLayout &lo, const 
     float *lam0 = reinterpret_cast<float *>(ws + lo.off_lam0);
     float *D = reinterpret_cast<float *>(ws + lo.off_D);
 
-    // Forward summaries: the direct kernel with 2 lanes per row (1 below 4
-    // states), segment mode, no y, no gate or skip (they do not touch the state).
-    FwdParams f{};
-    f.u = q.u, f.delta = q.delta, f.B = q.B, f.C = q.C, f.z = nullptr;
-    f.A = q.A, f.D = nullptr, f.delta_bias = q.delta_bias;
-    f.y = nullptr, f.last_state = nullptr, f.init_state = q.init_state, f.reset = q.reset;
-    f.batch = q.batch, f.dim = q.dim, f.seqlen = q.seqlen, f.dstate = q.dstate, f.softplus = q.softplus;
-    bool vec = (q.seqlen * (int64_t)ein) % 16 == 0;
-    for (const void *ptr : {q.u, q.delta, q.B, q.C})
-        if (ptr && !aligned(ptr, 16)) vec = false;
-    f.vec = vec ? 1 : 0;
-    const int lanes = nmax / 2 >= 2 ? 2 : 1, warps = 4;
-    const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
-    f.dtiles = (q.dim + rows_per_block - 1) / rows_per_block;
-    f.seg_len = q.seg_len, f.nseg = q.nseg;
-    f.ws_hend = hend, f.ws_dsum = dsum;
-    f.status = nullptr, f.delta_r = nullptr, f.W_dt = nullptr, f.dt_rank = 0;
-    const size_t smem = selscan::direct_smem_bytes(ein, nmax, lanes, warps);
-    const dim3 grid((unsigned)(f.dtiles * q.batch * q.nseg)), block((unsigned)(warps * 32));
-    const int split = lanes > 1 ? 1 : 0;
+    // Forward summaries (only when the adjoint kernel runs its own phase A:
+    // the forward's checkpoints already hold the true states): the direct
+    // kernel with 2 lanes per row (1 below 4 states), segment mode, no y, no
+    // gate or skip (they do not touch the state).
     cudaError_t err;
-    if (desc->in_dtype == SS_F32) err = launch_f32_f32(n, lanes, split, grid, block, smem, s, f);
-    else if (desc->out_dtype == SS_BF16) err = launch_bf16_bf16(n, lanes, split, grid, block, smem, s, f);
-    else err = launch_bf16_f32(n, lanes, split, grid, block, smem, s, f);
-    if (err != cudaSuccess) return SS_ERR_CUDA;
     const dim3 fold_grid((unsigned)((grows + 7) / 8));
-    if (nmax > 32) selscan::ss_fwd_carry_kernel<64><<<fold_grid, 256, 0, s>>>(f);
-    else selscan::ss_fwd_carry_kernel<32><<<fold_grid, 256, 0, s>>>(f);
-    if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    if (!q.ckpt_given) {
+        FwdParams f{};
+        f.u = q.u, f.delta = q.delta, f.B = q.B, f.C = q.C, f.z = nullptr;
+        f.A = q.A, f.D = nullptr, f.delta_bias = q.delta_bias;
+        f.y = nullptr, f.last_state = nullptr, f.init_state = q.init_state, f.reset = q.reset;
+        f.batch = q.batch, f.dim = q.dim, f.seqlen = q.seqlen, f.dstate = q.dstate, f.softplus = q.softplus;
+        bool vec = (q.seqlen * (int64_t)ein) % 16 == 0;
+        for (const void *ptr : {q.u, q.delta, q.B, q.C})
+            if (ptr && !aligned(ptr, 16)) vec = false;
+        f.vec = vec ? 1 : 0;
+        const int lanes = nmax / 2 >= 2 ? 2 : 1, warps = 4;
+        const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
+        f.dtiles = (q.dim + rows_per_block - 1) / rows_per_block;
+        f.seg_len = q.seg_len, f.nseg = q.nseg;
+        f.ws_hend = hend, f.ws_dsum = dsum;
+        f.status = nullptr, f.delta_r = nullptr, f.W_dt = nullptr, f.dt_rank = 0;
+        const size_t smem = selscan::direct_smem_bytes(ein, nmax, lanes, warps);
+        const dim3 grid((unsigned)(f.dtiles * q.batch * q.nseg)), block((unsigned)(warps * 32));
+        const int split = lanes > 1 ? 1 : 0;
+        if (desc->in_dtype == SS_F32) err = launch_f32_f32(n, lanes, split, grid, block, smem, s, f);
+        else if (desc->out_dtype == SS_BF16) err = launch_bf16_bf16(n, lanes, split, grid, block, smem, s, f);
+        else err = launch_bf16_f32(n, lanes, split, grid, block, smem, s, f);
+        if (err != cudaSuccess) return SS_ERR_CUDA;
+        if (nmax > 32) selscan::ss_fwd_carry_kernel<64><<<fold_grid, 256, 0, s>>>(f);
+        else selscan::ss_fwd_carry_kernel<32><<<fold_grid, 256, 0, s>>>(f);
+        if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    }
 
     // Adjoint summaries of segments 1.., then the backward fold.
     const int per = nmax < 8 ? 1 : nmax / 8;  // threads per (segment, row)
     const int64_t threads = grows * (q.nseg - 1) * per;
     const dim3 agrid((unsigned)((threads + 127) / 128));
-    if (desc->in_dtype == SS_F32) err = launch_seg_adjoint<float, float>(nmax, agrid, s, q, lam0);
-    else if (desc->out_dtype == SS_BF16) err = launch_seg_adjoint<__nv_bfloat16, __nv_bfloat16>(nmax, agrid, s, q, lam0);
-    else err = launch_seg_adjoint<__nv_bfloat16, float>(nmax, agrid, s, q, lam0);
+    if (desc->in_dtype == SS_F32) err = launch_seg_adjoint<float, float>(nmax, agrid, s, q, lam0, dsum);
+    else if (desc->out_dtype == SS_BF16)
+        err = launch_seg_adjoint<__nv_bfloat16, __nv_bfloat16>(nmax, agrid, s, q, lam0, dsum);
+    else err = launch_seg_adjoint<__nv_bfloat16, float>(nmax, agrid, s, q, lam0, dsum);
     if (err != cudaSuccess) return SS_ERR_CUDA;
     if (nmax > 32) selscan::ss_bwd_seg_fold_kernel<64><<<fold_grid, 256, 0, s>>>(q, lam0, dsum, D);
     else selscan::ss_bwd_seg_fold_kernel<32><<<fold_grid, 256, 0, s>>>(q, lam0, dsum, D);
@@ -817,7 +839,8 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
                    int delta_softplus, const uint8_t *reset, const float *init_state,
                    const float *dlast, const void *dy, void *du, void *ddelta, float *dA, float *dB,
                    float *dC, float *dD, void *dz, float *ddelta_bias, float *d_init_state,
-                   void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+                   void *workspace, size_t workspace_bytes, ss_stream_t stream,
+                   const float *fwd_ckpt = nullptr) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
@@ -829,11 +852,11 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     const void *in_ptrs[] = {u, delta, B, C, z, du, ddelta, dz};
     for (const void *q : in_ptrs)
         if (q && !aligned(q, ein)) return SS_ERR_MISALIGNED;
-    const void *f_ptrs[] = {A, D, delta_bias, dA, dB, dC, dD, ddelta_bias, init_state, dlast, d_init_state};
+    const void *f_ptrs[] = {A, D, delta_bias, dA, dB, dC, dD, ddelta_bias, init_state, dlast, d_init_state, fwd_ckpt};
     for (const void *q : f_ptrs)
         if (q && !aligned(q, 4)) return SS_ERR_MISALIGNED;
     if (dy && !aligned(dy, eout)) return SS_ERR_MISALIGNED;
-    const BwdLayout lo = bwd_layout(desc, sz);
+    const BwdLayout lo = bwd_layout(desc, sz, fwd_ckpt != nullptr);
     if (!workspace || workspace_bytes < lo.total) return SS_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return SS_ERR_MISALIGNED;
     const int64_t blocks = lo.dtiles * lo.group * lo.nseg;
@@ -868,6 +891,8 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.rows_all = sz.rows;
     p.seg_h = nullptr;
     p.seg_dl = nullptr;
+    p.ckpt_given = fwd_ckpt != nullptr ? 1 : 0;
+    if (fwd_ckpt != nullptr) p.ckpt = const_cast<float *>(fwd_ckpt);  // read only in that mode
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int nmax = selscan::state_bucket(p.dstate), n = nmax;
@@ -903,6 +928,7 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
             q.init_state = init_state ? init_state + b0 * DN : nullptr;
             q.dlast = dlast ? dlast + b0 * DN : nullptr;
             q.d_init_state = d_init_state ? d_init_state + b0 * DN : nullptr;
+            if (fwd_ckpt != nullptr) q.ckpt = p.ckpt + b0 * desc->dim * lo.nsub * desc->dstate;
             if (lo.nseg > 1 && desc->seqlen > 0) {
                 const ss_status ss = bwd_segment_summaries(desc, lo, q, ws, s);
                 if (ss != SS_OK) return ss;
@@ -952,6 +978,23 @@ ss_status ss_bwd_reset(const ss_desc *desc, const void *u, const void *delta, co
     if (!reset && desc && desc->batch > 0 && desc->dim > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
     return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, reset, nullptr, nullptr, dy,
                     du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, nullptr, workspace, workspace_bytes, stream);
+}
+
+ss_status ss_bwd_ckpt(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
+                      const void *C, const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                      const uint8_t *reset, const float *ckpt, const float *d_last_state, const void *dy, void *du,
+                      void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+                      float *d_initial_state, void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+    if (!ckpt && desc && desc->batch > 0 && desc->dim > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
+    return bwd_impl(desc, u, delta, A, B, C, D, z, delta_bias, delta_softplus, reset, nullptr, d_last_state, dy, du,
+                    ddelta, dA, dB, dC, dD, dz, ddelta_bias, d_initial_state, workspace, workspace_bytes, stream,
+                    ckpt);
+}
+
+size_t ss_bwd_ckpt_workspace_bytes(const ss_desc *desc) {
+    Sizes sz;
+    if (check_desc(desc, &sz) != SS_OK) return 0;
+    return bwd_layout(desc, sz, true).total;
 }
 
 ss_status ss_bwd_state(const ss_desc *desc, const void *u, const void *delta, const float *A,

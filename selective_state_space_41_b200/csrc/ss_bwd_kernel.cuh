@@ -73,6 +73,9 @@ struct BwdParams {
     int64_t rows_all;
     const float *seg_h;                       // (nseg, rows, dstate)
     const float *seg_dl;                      // (nseg, rows, dstate)
+    // Nonzero: ckpt holds the forward's checkpoints (written by the forward
+    // with checkpoints, ss_fwd_ckpt) and phase A is skipped.
+    int ckpt_given;
 };
 
 constexpr int kBwdSub = 8;                    // steps per sub-chunk
@@ -316,13 +319,14 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         }
     }
     uint32_t wu[kInWords], wd[kInWords];  // raw owned inputs of the next sub-chunk
-    if (Lend > c_begin) {
+    // With the forward's checkpoints given (p.ckpt_given) there is no phase A.
+    if (Lend > c_begin && !p.ckpt_given) {
         load_own(u_row, c_begin + j0, wu);
         load_own(d_row, c_begin + j0, wd);
         load_flags(c_begin, wfl);
         if (stage_fast(c_begin)) issue_copies(c_begin);
     }
-    for (int64_t c0 = c_begin; c0 < Lend; c0 += kBwdStage) {
+    for (int64_t c0 = c_begin; c0 < Lend && !p.ckpt_given; c0 += kBwdStage) {
         load_stage(c0, c0 + kBwdStage < Lend ? c0 + kBwdStage : -1);
         const int nsub = (int)(((Lend - c0 < kBwdStage ? Lend - c0 : kBwdStage) + kBwdSub - 1) / kBwdSub);
 #pragma unroll 1
@@ -430,9 +434,13 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         load_flags(l0, wfl);
     };
     if (Lend > c_begin) prefetch(((Lend - 1) / kBwdSub) * kBwdSub);
+    if (p.ckpt_given && nstages > 0) {  // no phase A: start the last stage's copies here
+        const int64_t c_last = c_begin + (nstages - 1) * kBwdStage;
+        if (stage_fast(c_last)) issue_copies(c_last);
+    }
     for (int64_t st = nstages - 1; st >= 0; --st) {
         const int64_t c0 = c_begin + st * kBwdStage;
-        if (st == nstages - 1) {  // F still holds the last stage from phase A
+        if (st == nstages - 1 && !p.ckpt_given) {  // F still holds the last stage from phase A
             if (stage_fast(c0 - kBwdStage)) issue_copies(c0 - kBwdStage);
         } else {
             load_stage(c0, c0 - kBwdStage);
@@ -643,9 +651,11 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
 //    s's last-state gradient D(s).
 // ss_bwd_seg_adjoint_kernel computes lam0(s) for s >= 1: one thread per
 // (segment, row, group of up to 8 states), the steps backwards 8 at a time
-// (vector loads when the rows are 16-byte aligned), exps on the SFU.
+// (vector loads when the rows are 16-byte aligned), exps on the SFU; it also
+// records each segment's delta' sum (-1 with a start) for the fold, so the
+// fold needs no forward pass when the forward's checkpoints are given.
 template <typename Tin, typename Tout, int kNmax>
-__global__ void __launch_bounds__(128, 3) ss_bwd_seg_adjoint_kernel(const BwdParams p, float *lam0) {
+__global__ void __launch_bounds__(128, 3) ss_bwd_seg_adjoint_kernel(const BwdParams p, float *lam0, float *dsum) {
     constexpr bool kFast = sizeof(Tin) == 2;
     constexpr int kS = kNmax < 8 ? kNmax : 8;          // states per thread
     constexpr int kT = kNmax / kS;                      // threads per (segment, row)
@@ -733,8 +743,11 @@ __global__ void __launch_bounds__(128, 3) ss_bwd_seg_adjoint_kernel(const BwdPar
     int64_t l0 = ((Lend - 1) / 8) * 8;
     Raw nxt;
     load_group(l0, nxt);
+    float dl_sum = 0.f;      // delta' over the segment (its decay product's exponent)
+    uint32_t any_start = 0u;  // a sequence start inside the segment
     for (; l0 >= c_begin; l0 -= 8) {
         const Raw cur = nxt;
+        any_start |= cur.st;
         if (l0 - 8 >= c_begin) load_group(l0 - 8, nxt);
         float dl[8], g[8];
 #pragma unroll
@@ -743,6 +756,7 @@ __global__ void __launch_bounds__(128, 3) ss_bwd_seg_adjoint_kernel(const BwdPar
             const float x = Io<Tin>::widen(cur.d, i) + bias;
             const float dyv = Io<Tout>::widen(cur.dy, i);
             dl[i] = in ? delta_transform<kFast>(x, softplus) : 0.f;
+            dl_sum += dl[i];
             if (has_z) {
                 const float zv = Io<Tin>::widen(cur.z, i);
                 g[i] = dyv * zv * sigmoid_of<kFast>(zv);
@@ -770,6 +784,8 @@ __global__ void __launch_bounds__(128, 3) ss_bwd_seg_adjoint_kernel(const BwdPar
         if (n < N) lam0[((int64_t)s * rows + row) * N + n] = carry[k].x;
         if (n + 1 < N) lam0[((int64_t)s * rows + row) * N + n + 1] = carry[k].y;
     }
+    // the segment's record for the backward fold (-1: it passes nothing on)
+    if (q == 0) dsum[(int64_t)s * rows + row] = any_start != 0u ? -1.f : dl_sum;
 }
 
 // The backward fold: D(nseg-1) = dlast (or 0); D(s-1) = lam0(s) + P(s) D(s),

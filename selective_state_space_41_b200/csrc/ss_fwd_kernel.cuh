@@ -77,7 +77,16 @@ struct FwdParams {
     // dt_rank, L) and W_dt (dim, dt_rank) in the input dtype.
     const void *delta_r, *W_dt;
     int dt_rank;
+    // Checkpoints for the backward (direct kernel; or null): the state
+    // entering every step l = 8k, (batch, dim, ceil(L / 8), dstate) fp32 —
+    // the state after step l - 1, before any sequence start at l zeroes it.
+    // With sequence segments the fix-up adds the carried state's share to
+    // the checkpoints of segments >= 1, as to y.
+    float *ckpt;
 };
+
+// Steps between two checkpoints of the state (the backward's sub-chunk).
+constexpr int kCkptStride = 8;
 
 // ------------------------------------------------------------ element I/O
 template <typename T>
@@ -852,6 +861,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     const bool softplus = p.softplus != 0;
     const bool has_z = p.z != nullptr;
     const bool want_y = p.y != nullptr;
+    static_assert(direct_sub(kG) % kCkptStride == 0, "checkpoints at sub-chunk steps");
     // This block's steps: [c_begin, Lend) (the whole row unless segmented).
     const int64_t c_begin = seg * p.seg_len;
     const int64_t Lend = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
@@ -883,6 +893,13 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     Tout *y_own = y_row + c_begin + g * kOwn;
 
     const int q0 = g * kPL;                                 // this lane's first state pair
+    // This row's checkpoints (null when none are asked for, or a mirrored row).
+    float *const ckpt_row = (p.ckpt != nullptr && row_ok)
+                                ? p.ckpt + row * ((L + kCkptStride - 1) / kCkptStride) * N : nullptr;
+    // Vector stores of the checkpoints: whole groups of 4 states in the row
+    // (N a multiple of 4) and a 16-byte-aligned buffer; a lane's pairs start on
+    // an even pair when it holds 2 or more (else one 8-byte pair).
+    const bool ckpt_vec = N % 4 == 0 && (reinterpret_cast<uintptr_t>(p.ckpt) & 15u) == 0 && (kPL % 2 == 0 || kPL == 1);
     const float *A_d = p.A + d * N;
     float2 A2[kA2InRegs ? kPL : 1], h[kPL];
 #pragma unroll
@@ -1212,6 +1229,28 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
             constexpr bool kStarts = decltype(with_starts)::value;
 #pragma unroll
             for (int i = 0; i < kDirectSub; ++i) {
+                if (i % kCkptStride == 0 && ckpt_row != nullptr && l0 + i < Lend) {
+                    float *dst = ckpt_row + ((l0 + i) / kCkptStride) * N;
+                    if (ckpt_vec) {  // this lane's states as 16- (or 8-) byte streaming stores
+#pragma unroll
+                        for (int qq = 0; qq < kPL; qq += 2) {
+                            const int n = 2 * (q0 + qq);
+                            if (n >= N) continue;
+                            if (qq + 1 < kPL)
+                                __stcs(reinterpret_cast<float4 *>(dst + n),
+                                       make_float4(h[qq].x, h[qq].y, h[qq + 1].x, h[qq + 1].y));
+                            else
+                                __stcs(reinterpret_cast<float2 *>(dst + n), h[qq]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int qq = 0; qq < kPL; ++qq) {
+                            const int n = 2 * (q0 + qq);
+                            if (n < N) dst[n] = h[qq].x;
+                            if (n + 1 < N) dst[n + 1] = h[qq].y;
+                        }
+                    }
+                }
                 const float2 d2 = make_float2(dl[i], dl[i]), u2 = make_float2(du[i], du[i]);
                 float2 acc[kAccs];
 #pragma unroll
@@ -1500,6 +1539,7 @@ __global__ void __launch_bounds__(kFixupWarps * 32) ss_fwd_fixup_kernel(const Fw
     const uint8_t *const reset_b = p.reset ? p.reset + b * L : nullptr;
     const int64_t c_begin = (int64_t)s * p.seg_len;
     const int64_t c_end = c_begin + p.seg_len < L ? c_begin + p.seg_len : L;
+    float *const ckpt_b = p.ckpt != nullptr ? p.ckpt + row * ((L + kCkptStride - 1) / kCkptStride) * N : nullptr;
 
     float S0 = 0.f;  // delta' summed over the chunks before this one
     for (int64_t c = c_begin; c < c_end; c += 32 * kK) {
@@ -1524,6 +1564,9 @@ __global__ void __launch_bounds__(kFixupWarps * 32) ss_fwd_fixup_kernel(const Fw
             if (m != 0 && first_start == 32 * kK) first_start = 32 * k + __ffs(m) - 1;
             starts |= m;
         }
+        float own[kK];  // this lane's delta' of each of its steps
+#pragma unroll
+        for (int k = 0; k < kK; ++k) own[k] = S[k];
         // inclusive scan of delta' over the chunk's steps, in step order
 #pragma unroll
         for (int k = 0; k < kK; ++k) {
@@ -1564,6 +1607,20 @@ __global__ void __launch_bounds__(kFixupWarps * 32) ss_fwd_fixup_kernel(const Fw
                     float v = corr[k];
                     if (z_row) v *= silu<kFast>(static_cast<float>(z_row[l]));
                     y_row[l] = static_cast<Tout>(static_cast<float>(y_row[l]) + v);
+                }
+            }
+        }
+        // Checkpoints (the state entering steps l = 8k, after step l - 1):
+        // the carried share 2^(A log2e S_(l-1)) h_in, up to and including the
+        // segment's first start (a start zeroes the state only after it).
+        if (ckpt_b != nullptr) {
+#pragma unroll
+            for (int k = 0; k < kK; ++k) {
+                const int64_t l = c + 32 * k + lane;
+                const float Sx = S[k] - own[k];
+                if (in[k] && l % kCkptStride == 0 && 32 * k + lane <= first_start && !(A2max * Sx < -127.f)) {
+                    float *ck = ckpt_b + (l / kCkptStride) * N;
+                    for (int n = 0; n < N; ++n) ck[n] = fmaf(sfu_exp2(sh_A2[warp][n] * Sx), sh_h[warp][n], ck[n]);
                 }
             }
         }

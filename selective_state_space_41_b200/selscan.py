@@ -10,7 +10,7 @@ The Python names match the C entry points (``ss_fwd``, ``ss_fwd_ws``,
 ``ss_fwd_workspace_bytes``, ``ss_fwd_with_config``, ``ss_fwd_state``,
 ``ss_fwd_reset``, ``ss_fwd_heuristic``, ``ss_fwd_hostio``, ``ss_fwd_hostio_streams``,
 ``ss_fwd_noalloc``, ``ss_fwd_dtproj``, ``ss_step``, ``ss_bwd``, ``ss_bwd_reset``, ``ss_bwd_state``, ``ss_bwd_workspace_bytes``,
-``ss_bwd_heuristic``,
+``ss_bwd_heuristic``, ``ss_fwd_ckpt``, ``ss_bwd_ckpt``, ``ss_bwd_ckpt_workspace_bytes``,
 ``ss_status_string``, ``ss_version``, ``ss_device_status``); ``ss_fwd`` dispatches to the
 workspace, config, initial-state and sequence-start forms by keyword, ``ss_fwd_hostio`` to
 the pipelined form when given streams.  ``selective_scan_fwd`` and
@@ -39,7 +39,8 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config", "ss_fwd_state",
            "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc",
            "ss_step", "ss_bwd", "ss_bwd_reset", "ss_bwd_state", "ss_bwd_workspace_bytes", "ss_status_string",
-           "ss_version", "ss_device_status", "ss_fwd_dtproj", "ss_bwd_heuristic")
+           "ss_version", "ss_device_status", "ss_fwd_dtproj", "ss_bwd_heuristic", "ss_fwd_ckpt", "ss_bwd_ckpt",
+           "ss_bwd_ckpt_workspace_bytes")
 
 
 class SelscanError(RuntimeError):
@@ -106,6 +107,12 @@ def lib():
         L.ss_bwd_state.argtypes = [DP] + [P] * 8 + [I] + [P] * 13 + [P, SZ, P]
         L.ss_bwd_workspace_bytes.restype = SZ
         L.ss_bwd_workspace_bytes.argtypes = [DP]
+        L.ss_fwd_ckpt.restype = I
+        L.ss_fwd_ckpt.argtypes = [DP] + [P] * 8 + [I] + [P] * 5 + [P, SZ, P]
+        L.ss_bwd_ckpt.restype = I
+        L.ss_bwd_ckpt.argtypes = [DP] + [P] * 8 + [I] + [P] * 13 + [P, SZ, P]
+        L.ss_bwd_ckpt_workspace_bytes.restype = SZ
+        L.ss_bwd_ckpt_workspace_bytes.argtypes = [DP]
         L.ss_bwd_heuristic.restype = I
         L.ss_bwd_heuristic.argtypes = [DP, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(I)]
         L.ss_status_string.restype = ctypes.c_char_p
@@ -329,8 +336,62 @@ def ss_bwd(u, delta, A, B, C, dy, grads, D=None, z=None, delta_bias=None, delta_
         _check(lib().ss_bwd(*head, *tail), "ss_bwd")
 
 
+def ckpt_shape(batch, dim, seqlen, dstate):
+    """Shape of the forward's checkpoints: (batch, dim, ceil(seqlen / 8), dstate)."""
+    return (batch, dim, (seqlen + 7) // 8, dstate)
+
+
+def ss_fwd_ckpt(u, delta, A, B, C, y, ckpt, D=None, z=None, delta_bias=None, delta_softplus=False,
+                last_state=None, initial_state=None, reset=None, stream=None, workspace=None):
+    """Queue the forward that also writes the backward's checkpoints into
+    ``ckpt`` (float32, ckpt_shape(...)); other arguments as ``ss_fwd``
+    (``workspace``: a CUDA tensor enabling sequence segments, or None)."""
+    u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    if tuple(ckpt.shape) != ckpt_shape(batch, dim, L, N) or ckpt.dtype != torch.float32 or not ckpt.is_contiguous():
+        raise ValueError("ckpt must be a contiguous float32 tensor of ckpt_shape(batch, dim, L, N)")
+    if reset is not None and reset.dtype == torch.bool:
+        reset = reset.view(torch.uint8)
+    desc = make_desc(batch, dim, L, N, u.dtype, y.dtype)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().ss_fwd_ckpt(ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                             _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(initial_state), _ptr(reset), _ptr(y),
+                             _ptr(last_state), _ptr(ckpt), _ptr(workspace), ws_bytes,
+                             _stream_handle(stream, u.device)), "ss_fwd_ckpt")
+
+
+def ss_bwd_ckpt_workspace_bytes(batch, dim, seqlen, dstate, in_dtype=torch.bfloat16, out_dtype=None) -> int:
+    desc = make_desc(batch, dim, seqlen, dstate, in_dtype, out_dtype)
+    return int(lib().ss_bwd_ckpt_workspace_bytes(ctypes.byref(desc)))
+
+
+def ss_bwd_ckpt(u, delta, A, B, C, dy, ckpt, grads, D=None, z=None, delta_bias=None, delta_softplus=False,
+                reset=None, d_last_state=None, workspace=None, stream=None):
+    """Queue the backward from the forward's checkpoints (``ss_fwd_ckpt``):
+    ``grads`` as ``ss_bwd`` (with an optional dinitial_state output)."""
+    u, delta, A, B, C, dy, D, z, delta_bias = map(_contig, (u, delta, A, B, C, dy, D, z, delta_bias))
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    if tuple(ckpt.shape) != ckpt_shape(batch, dim, L, N) or ckpt.dtype != torch.float32 or not ckpt.is_contiguous():
+        raise ValueError("ckpt must be a contiguous float32 tensor of ckpt_shape(batch, dim, L, N)")
+    if reset is not None and reset.dtype == torch.bool:
+        reset = reset.view(torch.uint8)
+    desc = make_desc(batch, dim, L, N, u.dtype, dy.dtype)
+    if workspace is None:
+        n = ss_bwd_ckpt_workspace_bytes(batch, dim, L, N, u.dtype, dy.dtype)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=u.device)
+    g = lambda k: _ptr(grads.get(k))  # noqa: E731
+    _check(lib().ss_bwd_ckpt(ctypes.byref(desc), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                             _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(reset), _ptr(ckpt),
+                             _ptr(d_last_state), _ptr(dy), g("du"), g("ddelta"), g("dA"), g("dB"), g("dC"), g("dD"),
+                             g("dz"), g("ddelta_bias"), g("dinitial_state"), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream_handle(stream, u.device)),
+           "ss_bwd_ckpt")
+
+
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=False,
-                       stream=None, reset=None, initial_state=None, d_last_state=None):
+                       stream=None, reset=None, initial_state=None, d_last_state=None, ckpt=None):
     """Gradients of sum(dy * y) (+ sum(d_last_state * last state)) as a dict
     (see ss_bwd); allocates the outputs; dinitial_state when an initial
     state or a last-state gradient is given."""
@@ -347,6 +408,10 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, d
              "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None}
     if initial_state is not None or d_last_state is not None:
         grads["dinitial_state"] = torch.empty((batch, dim, N), dtype=f32, device=dev)
+    if ckpt is not None:  # from the forward's checkpoints (ss_fwd_ckpt); they hold the initial state
+        ss_bwd_ckpt(u, delta, A, B, C, dy, ckpt, grads, D=D, z=z, delta_bias=delta_bias,
+                    delta_softplus=delta_softplus, reset=reset, d_last_state=d_last_state, stream=stream)
+        return grads
     ss_bwd(u, delta, A, B, C, dy, grads, D=D, z=z, delta_bias=delta_bias,
            delta_softplus=delta_softplus, stream=stream, reset=reset, initial_state=initial_state,
            d_last_state=d_last_state)
