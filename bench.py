@@ -19,7 +19,10 @@ clock); its HBM side (compulsory bytes over measured copy bandwidth) is
 reported beside it.  ``per_config`` adds, in the same line, the forward of
 every other configuration at full size (device time with L2 flushed per step,
 fewer steps each, clocks sampled over the warm-ups and timed steps) and its
-backward (ss_bwd, all gradients, 3 timed steps).
+backward (ss_bwd, all gradients, 3 timed steps).  ``train_step`` (headline
+layer and each configuration) times forward + backward both ways: ss_fwd +
+ss_bwd, and ss_fwd_ckpt + ss_bwd_ckpt (the forward keeps the checkpoints the
+backward would otherwise recompute).
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
 bounded sample of rows per step).
 """
@@ -406,6 +409,10 @@ def bench_ours(args, w, world, rank, local):
     line["decode"] = bench_decode(wr, d, out_dtype, stream, world)
     if not args.no_bwd:
         line["backward"] = bench_backward(args, wr, d, host, out_dtype, flush, stream, sfu_peak, world)
+        dy = gen.fill(tuple(host["u"].shape), out_dtype, wr.seed, 9).to(dev)
+        line["train_step"] = _time_train_step(wr, d, dy, out_dtype, flush, stream, steps=max(3, min(args.steps, 20)),
+                                              warmup=3)
+        del dy
     if w.dtype == torch.bfloat16 and not args.no_per_config:
         line["fused_dtproj"] = bench_dtproj(wr, dev, stream, flush, steps=max(3, min(args.steps, 20)), warmup=3,
                                             sfu_peak=sfu_peak, unfused_ms=statistics.median(kernel_ms))
@@ -613,6 +620,61 @@ def _time_backward(w, d, dy, out_dtype, flush, stream, steps, warmup):
     return statistics.median(ts), nws, plan
 
 
+def _time_train_step(w, d, dy, out_dtype, flush, stream, steps, warmup):
+    """A training step's device time (median ms over ``steps``, L2 flushed
+    before each) two ways: the forward (ss_fwd, with the workspace that
+    enables sequence segments) then ss_bwd, which runs its own forward pass
+    for its checkpoints; and ss_fwd_ckpt, which writes them, then ss_bwd_ckpt,
+    which reads them.  Each half is timed alone too."""
+    dev = d["u"].device
+    B, D, L, N = w.batch, w.dim, w.seqlen, w.dstate
+    f32 = torch.float32
+    y = torch.empty((B, D, L), dtype=out_dtype, device=dev)
+    ck = torch.empty(selscan.ckpt_shape(B, D, L, N), dtype=f32, device=dev)
+    wsf = selscan.workspace_for(B, D, L, N, w.dtype, out_dtype, device=dev)
+    grads = {"du": torch.empty_like(d["u"]), "ddelta": torch.empty_like(d["u"]),
+             "dA": torch.empty((D, N), dtype=f32, device=dev), "dB": torch.empty((B, N, L), dtype=f32, device=dev),
+             "dC": torch.empty((B, N, L), dtype=f32, device=dev),
+             "dD": torch.empty(D, dtype=f32, device=dev) if d["D"] is not None else None,
+             "dz": torch.empty_like(d["u"]) if d["z"] is not None else None,
+             "ddelta_bias": torch.empty(D, dtype=f32, device=dev) if d["delta_bias"] is not None else None}
+    wsb = torch.empty(selscan.ss_bwd_workspace_bytes(B, D, L, N, w.dtype, out_dtype), dtype=torch.uint8, device=dev)
+    kw = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, stream=stream)
+    legs = {
+        "fwd": lambda: selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, workspace=wsf, **kw),
+        "bwd": lambda: selscan.ss_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], dy, grads, workspace=wsb, **kw),
+        "fwd_ckpt": lambda: selscan.ss_fwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"], y, ck, workspace=wsf,
+                                                **kw),
+        "bwd_ckpt": lambda: selscan.ss_bwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"], dy, ck, grads,
+                                                workspace=wsb, **kw),
+    }
+    runs = {"step": ("fwd", "bwd"), "step_ckpt": ("fwd_ckpt", "bwd_ckpt"), "fwd": ("fwd",), "bwd": ("bwd",),
+            "fwd_ckpt": ("fwd_ckpt",), "bwd_ckpt": ("bwd_ckpt",)}
+    out = {}
+    for name, parts in runs.items():
+        for _ in range(warmup):
+            flush.zero_()
+            for leg in parts:
+                legs[leg]()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for leg in parts:
+                legs[leg]()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        out[name + "_ms"] = statistics.median(ts)
+    del y, ck, wsf, wsb, grads
+    out["step_speedup"] = out["step_ms"] / out["step_ckpt_ms"]
+    out["steps"] = steps
+    out["note"] = ("training step = forward + backward: ss_fwd + ss_bwd (the backward's own checkpointing pass) "
+                   "against ss_fwd_ckpt + ss_bwd_ckpt (checkpoints written by the forward); L2 flushed per step")
+    return out
+
+
 def _bwd_launches(w, plan):
     """Kernel launches of one ss_bwd call: per batch group the adjoint kernel
     and the dB/dC sum (plus, with sequence segments, the forward summary,
@@ -648,11 +710,13 @@ def bench_backward_config(w: W.Workload, dev, stream, flush, steps: int, warmup:
     dy = gen.fill(tuple(host["u"].shape), out_dtype, w.seed, 9).to(dev)
     del host
     ms, nws, plan = _time_backward(w, d, dy, out_dtype, flush, stream, steps, warmup)
+    train = _time_train_step(w, d, dy, out_dtype, flush, stream, steps, warmup)
     del d, dy
     torch.cuda.empty_cache()
     return {"ms": ms, "steps": steps, "warmup": warmup, "updates_per_s": w.updates / (ms * 1e-3),
             "sfu_frac": 2 * w.updates / sfu_peak / (ms * 1e-3), "ex2_per_update_counted": 2,
-            "workspace_bytes": nws, "plan": plan, "gpu_launches_per_step": _bwd_launches(w, plan)}
+            "workspace_bytes": nws, "plan": plan, "gpu_launches_per_step": _bwd_launches(w, plan),
+            "train_step": train}
 
 
 def main(argv=None):

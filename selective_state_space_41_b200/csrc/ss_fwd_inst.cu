@@ -56,6 +56,16 @@ cudaError_t launch_direct(dim3 grid, dim3 block, size_t smem, cudaStream_t s, co
                 return cudaErrorInvalidValue;
             }
         }
+        if (p.ckpt) {  // the instances that write the backward's checkpoints
+            if (p.reset) {
+                static bool opted_in_ck_reset[kMaxDevices];
+                return launch_kernel(ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kG, true, false, true>,
+                                     grid, block, smem, s, p, opted_in_ck_reset);
+            }
+            static bool opted_in_ck[kMaxDevices];
+            return launch_kernel(ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kG, false, false, true>,
+                                 grid, block, smem, s, p, opted_in_ck);
+        }
         if (p.reset) {  // the instance that reads the sequence starts
             static bool opted_in_reset[kMaxDevices];
             return launch_kernel(ss_fwd_direct_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kG, true>,

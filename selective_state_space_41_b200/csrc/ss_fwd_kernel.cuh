@@ -819,7 +819,9 @@ struct DirectOccupancy {
 // kReset: the instance that reads p.reset (sequence starts inside the rows);
 // the other one has no code for it.  kDt: the instance whose delta is the
 // dt_proj product (p.delta_r, p.W_dt; 4 warps, bf16, 2 or 4 lanes per row).
-template <typename Tin, typename Tout, int kNmax, int kG, bool kReset = false, bool kDt = false>
+// kCkpt: the instance that writes the checkpoints p.ckpt (the others have no
+// code for them: the stores cost registers and time in the step loop).
+template <typename Tin, typename Tout, int kNmax, int kG, bool kReset = false, bool kDt = false, bool kCkpt = false>
 __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParams p) {
     constexpr int kPairs = kNmax / 2;
     constexpr int kPL = kPairs / kG;                        // state pairs per lane
@@ -894,7 +896,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
 
     const int q0 = g * kPL;                                 // this lane's first state pair
     // This row's checkpoints (null when none are asked for, or a mirrored row).
-    float *const ckpt_row = (p.ckpt != nullptr && row_ok)
+    float *const ckpt_row = (kCkpt && row_ok)
                                 ? p.ckpt + row * ((L + kCkptStride - 1) / kCkptStride) * N : nullptr;
     // Vector stores of the checkpoints: whole groups of 4 states in the row
     // (N a multiple of 4) and a 16-byte-aligned buffer; a lane's pairs start on
@@ -1229,7 +1231,7 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
             constexpr bool kStarts = decltype(with_starts)::value;
 #pragma unroll
             for (int i = 0; i < kDirectSub; ++i) {
-                if (i % kCkptStride == 0 && ckpt_row != nullptr && l0 + i < Lend) {
+                if (kCkpt && i % kCkptStride == 0 && ckpt_row != nullptr && l0 + i < Lend) {
                     float *dst = ckpt_row + ((l0 + i) / kCkptStride) * N;
                     if (ckpt_vec) {  // this lane's states as 16- (or 8-) byte streaming stores
 #pragma unroll
