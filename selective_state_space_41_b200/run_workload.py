@@ -2,15 +2,16 @@
 
     python -m selective_state_space_41_b200.run_workload NAME [--batch B]
         [--repeat K] [--lanes G] [--split S] [--warps W] [--segments P]
-        [--dt-rank R] [--backward]
+        [--dt-rank R] [--backward] [--backward-ckpt]
 
 Draws the workload's seeded inputs (optionally only its first B batch
 entries, to keep a capture small), moves them to ``cuda:0`` and calls
 ``ss_fwd`` (or ``ss_fwd_dtproj`` with ``--dt-rank``) K times in the launch
 shape given, zeros meaning the heuristic's choice.  A workspace is passed
 when the shape uses sequence segments.  ``--backward`` calls ``ss_bwd`` (all
-gradients, a seeded dy, its own plan) K times instead.  Prints ``ok`` after
-a final synchronize.
+gradients, a seeded dy, its own plan) K times instead; ``--backward-ckpt``
+calls ``ss_fwd_ckpt`` once, then ``ss_bwd_ckpt`` from its checkpoints K
+times.  Prints ``ok`` after a final synchronize.
 """
 import argparse
 
@@ -30,6 +31,7 @@ def main(argv=None):
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--dt-rank", type=int, default=0)
     ap.add_argument("--backward", action="store_true")
+    ap.add_argument("--backward-ckpt", action="store_true")
     a = ap.parse_args(argv)
     w = W.WORKLOADS[a.name]
     if a.batch:
@@ -42,7 +44,15 @@ def main(argv=None):
     if a.lanes or a.split or a.warps or a.segments:
         cfg = dict(lanes_per_row=a.lanes, split_states=a.split, warps_per_block=a.warps, segments=a.segments)
     kw = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, last_state=last)
-    if a.backward:
+    if a.backward_ckpt:
+        dy = gen.fill(tuple(inp["u"].shape), w.out_dtype or w.dtype, w.seed, 9).cuda()
+        ck = torch.empty(selscan.ckpt_shape(w.batch, w.dim, w.seqlen, w.dstate), device="cuda")
+        ws = selscan.workspace_for(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, y.dtype)
+        selscan.ss_fwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"], y, ck, workspace=ws, **kw)
+        for _ in range(a.repeat):
+            selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], dy, D=d["D"], z=d["z"],
+                                       delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, ckpt=ck)
+    elif a.backward:
         dy = gen.fill(tuple(inp["u"].shape), w.out_dtype or w.dtype, w.seed, 9).cuda()
         for _ in range(a.repeat):
             selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], dy, D=d["D"], z=d["z"],

@@ -306,6 +306,28 @@ def test_heuristic_genomic_without_workspace_and_its_workspace():
     assert selscan.ss_fwd_workspace_bytes(4, 1024, 100000, 16, torch.bfloat16) == 16 * 4096 * 17 * 4
 
 
+def test_ckpt_entry_rejections(lib):
+    """The checkpoint entries reject before any launch (fake pointers): no
+    checkpoint buffer, a misaligned one; the backward from checkpoints needs
+    no checkpoint region in its workspace."""
+    P = FAKE
+    d = _desc(seqlen=64, dstate=16)
+    fwd_head = (ctypes.byref(d), P, P, P, P, P, None, None, None, 1, None, None, P, None)
+    assert lib.ss_fwd_ckpt(*fwd_head, None, None, 0, None) == 1
+    assert lib.ss_fwd_ckpt(*fwd_head, ODD, None, 0, None) == 5
+    grads = (P, P, P, P, P, None, None, None)
+    bwd_head = (ctypes.byref(d), P, P, P, P, P, None, None, None, 1, None)
+    assert lib.ss_bwd_ckpt(*bwd_head, None, None, P, *grads, None, None, 0, None) == 1
+    assert lib.ss_bwd_ckpt(*bwd_head, ODD, None, P, *grads, None, None, 0, None) == 5
+    assert lib.ss_bwd_ckpt(*bwd_head, P, None, P, *grads, None, None, 0, None) == 8   # no workspace
+    for shape in ((8, 1536, 2048, 16), (4, 1024, 100000, 16), (1, 8, 9000, 64)):
+        big = _desc(batch=shape[0], dim=shape[1], seqlen=shape[2], dstate=shape[3], in_dtype=1, out_dtype=1)
+        full = lib.ss_bwd_workspace_bytes(ctypes.byref(big))
+        ck = lib.ss_bwd_ckpt_workspace_bytes(ctypes.byref(big))
+        rows, nsub = shape[0] * shape[1], -(-shape[2] // 8)
+        assert 0 < ck < full and full - ck >= rows * nsub * shape[3] * 4 - 256, shape
+
+
 def test_bwd_rejections(lib):
     """ss_bwd rejects before any launch (the pointers are fake): no
     descriptor, more than 64 states, a missing gradient output, no workspace.
