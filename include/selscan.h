@@ -413,9 +413,11 @@ ss_status ss_fwd_ckpt(const ss_desc *desc, const void *u, const void *delta, con
  *                 itself is in the checkpoints)
  *   workspace     ss_bwd_ckpt_workspace_bytes(desc) bytes (no checkpoint
  *                 region; ss_bwd_workspace_bytes is enough too)
- * The gradients equal ss_bwd_state's up to the fp32 order of the segment
- * summaries (bitwise without sequence segments, where the checkpoints are the
- * same values).  SS_ERR_NULL_POINTER when ckpt is NULL and there is work.
+ * The gradients equal ss_bwd_state's bit for bit when neither the forward
+ * nor the backward cuts the sequence into segments (the checkpoints are then
+ * the values the backward's own pass computes); with segments they differ
+ * only in the fp32 rounding of the segment carries.  SS_ERR_NULL_POINTER when
+ * ckpt is NULL and there is work.
  */
 ss_status ss_bwd_ckpt(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,
                       const void *C, const float *D, const void *z, const float *delta_bias, int delta_softplus,

@@ -1,7 +1,10 @@
 // Selective-scan forward kernels for sm_100a: the scan kernel (lanes split a
 // row's steps; described here), the direct kernel (lanes split a row's
-// states; used whenever the rows fill the GPU) and the fix-up kernel of
-// sequence segments, each with its own description further down.
+// states; used whenever the rows fill the GPU; its instances also read
+// sequence starts, take delta from the dt_proj product on the tensor cores,
+// or write the backward's checkpoints) and the two fix-up kernels of sequence
+// segments (the carry fold and the correction of y), each with its own
+// description further down.
 //
 // Computes, per row (b, d) of the (batch, dim) grid and per state n, the
 // recurrence of the selective_scan_ref walkthrough ("Mamba代码实战：手把手教你用
