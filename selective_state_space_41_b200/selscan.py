@@ -497,3 +497,40 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
            last_state=last, stream=stream, workspace=ws, initial_state=initial_state, reset=reset)
     return (y, last) if return_last_state else y
+
+
+class SelectiveScanFn(torch.autograd.Function):
+    """The scan as a torch autograd Function: the forward is ``ss_fwd_ckpt``
+    (keeping the backward's checkpoints for the saved context), the backward
+    ``ss_bwd_ckpt`` (all gradients, no second forward pass).  Gradients come
+    back in the dtypes of their inputs (dB, dC are summed in fp32 and then
+    cast for bf16 B, C)."""
+
+    @staticmethod
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus):
+        u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
+        batch, dim, L = u.shape
+        N = A.shape[-1]
+        y = torch.empty_like(u)
+        ck = torch.empty(ckpt_shape(batch, dim, L, N), dtype=torch.float32, device=u.device)
+        ws = workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=u.device)
+        ss_fwd_ckpt(u, delta, A, B, C, y, ck, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                    workspace=ws)
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, ck)
+        ctx.delta_softplus = bool(delta_softplus)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        u, delta, A, B, C, D, z, delta_bias, ck = ctx.saved_tensors
+        g = selective_scan_bwd(u, delta, A, B, C, dy.contiguous(), D=D, z=z, delta_bias=delta_bias,
+                               delta_softplus=ctx.delta_softplus, ckpt=ck)
+        return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype), g["dD"], g["dz"],
+                g["ddelta_bias"], None)
+
+
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False):
+    """y of the selective scan (argument order of the walkthrough's
+    selective_scan_ref), differentiable through torch autograd; see
+    SelectiveScanFn."""
+    return SelectiveScanFn.apply(u, delta, A, B, C, D, z, delta_bias, delta_softplus)

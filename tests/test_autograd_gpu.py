@@ -1,0 +1,70 @@
+"""selective_scan_fn, the scan as a torch autograd Function over the training
+path (ss_fwd_ckpt forward, ss_bwd_ckpt backward): its gradients through
+torch.autograd against the fp64 backward oracle (fp32 inputs, tolerances of
+test_bwd_gpu.py) and, for bf16 inputs, bit for bit against the direct
+backward call cast to the inputs' dtypes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from test_bwd_gpu import ELEM, TOL_ELEM, TOL_SUM, _case, check_summed
+from selective_state_space_41_b200 import selscan
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+NAMES = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+GRAD = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD", "z": "dz",
+        "delta_bias": "ddelta_bias"}
+
+
+def _leaves(inp):
+    return {k: (inp[k].cuda().requires_grad_(True) if inp.get(k) is not None else None) for k in NAMES}
+
+
+def _autograd(inp):
+    t = _leaves(inp)
+    y = selscan.selective_scan_fn(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"],
+                                  delta_bias=t["delta_bias"], delta_softplus=inp["delta_softplus"])
+    (y.float() * inp["dy"].cuda().float()).sum().backward()
+    torch.cuda.synchronize()
+    return y, {GRAD[k]: (v.grad if v is not None else None) for k, v in t.items()}
+
+
+@pytest.mark.parametrize("has_z,D_kind,bias_kind", [(True, "normal", "normal"), (False, "none", "none")])
+def test_autograd_against_oracle(has_z, D_kind, bias_kind):
+    inp = _case(2, 24, 300, 16, torch.float32, seed=951, has_z=has_z, D_kind=D_kind, bias_kind=bias_kind)
+    y, got = _autograd(inp)
+    y_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"], z=inp["z"],
+                                  delta_bias=inp["delta_bias"], delta_softplus=inp["delta_softplus"])
+    assert float(np.max(np.abs(y.detach().double().cpu().numpy() - y_ref) / (1 + np.abs(y_ref)))) <= 1e-5
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"], D=inp["D"],
+                                    z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=inp["delta_softplus"],
+                                    magnitudes=True)
+    for k, want in ref.items():
+        if k.startswith("mag_"):
+            continue
+        if want is None:
+            assert got[k] is None, k
+            continue
+        g = got[k].double().cpu().numpy()
+        if k in ELEM:
+            e = float(np.max(np.abs(g - want) / (1.0 + np.abs(want))))
+            assert e <= TOL_ELEM[torch.float32], f"{k}: {e:.3e}"
+        else:
+            check_summed(k, g, want, ref["mag_" + k], TOL_SUM[torch.float32], "autograd")
+
+
+def test_autograd_bf16_matches_the_direct_backward():
+    inp = _case(2, 40, 512, 16, torch.bfloat16, seed=953, has_z=True, bias_kind="uniform_dt")
+    _, got = _autograd(inp)
+    d = {k: (inp[k].cuda() if inp.get(k) is not None else None) for k in NAMES}
+    want = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], inp["dy"].cuda(), D=d["D"],
+                                      z=d["z"], delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"])
+    torch.cuda.synchronize()
+    for k, g in got.items():
+        w = want[k]
+        if k in ("dB", "dC"):
+            w = w.to(torch.bfloat16)
+        assert g.dtype == w.dtype and torch.equal(g, w), k
