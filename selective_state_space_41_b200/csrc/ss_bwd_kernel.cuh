@@ -507,14 +507,29 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
                 sp[i] = acc.x + acc.y;
             }
             // The adjoint over the sub-chunk, last step first.
+            // B/C of each step are read two steps ahead: the compiler cannot
+            // move a shared-memory load above the dB/dC stores of the steps in
+            // between, so without this every read would wait its full latency.
             float lb[kBwdSub], lha[kBwdSub];
+            float4 bc_next[kPL], bc_next2[kPL];
+#pragma unroll
+            for (int qq = 0; qq < kPL; ++qq) bc_next[qq] = Fm[(kBwdSub - 1) * kPairs + qq];
+#pragma unroll
+            for (int qq = 0; qq < kPL; ++qq) bc_next2[qq] = Fm[(kBwdSub - 2) * kPairs + qq];
 #pragma unroll
             for (int i = kBwdSub - 1; i >= 0; --i) {
                 const float2 g2 = make_float2(gg[i], gg[i]), u2 = make_float2(du[i], du[i]);
                 float2 sLB = make_float2(0.f, 0.f), sLHA = make_float2(0.f, 0.f);
+                float4 bc_cur[kPL];
 #pragma unroll
                 for (int qq = 0; qq < kPL; ++qq) {
-                    const float4 bc = Fm[i * kPairs + qq];
+                    bc_cur[qq] = bc_next[qq];
+                    bc_next[qq] = bc_next2[qq];
+                    if (i > 1) bc_next2[qq] = Fm[(i - 2) * kPairs + qq];
+                }
+#pragma unroll
+                for (int qq = 0; qq < kPL; ++qq) {
+                    const float4 bc = bc_cur[qq];
                     const float2 lam = __ffma2_rn(g2, make_float2(bc.z, bc.w), carry[qq]);
                     const float2 dCp = __fmul2_rn(g2, hs[i][qq]);
                     const float2 dBp = __fmul2_rn(lam, u2);
