@@ -502,30 +502,43 @@ def bench_dtproj(w: W.Workload, dev, stream, flush, steps: int, warmup: int, sfu
     d = {k: (host[k].to(dev) if host[k] is not None else None) for k in names_in}
     y = torch.empty(d["u"].shape, dtype=w.dtype, device=dev)
 
+    # x_proj's output as one tensor: feature rows delta_r, B, C (ss_fwd_xdbl reads them in place)
+    x_dbl = torch.cat([d["delta_r"], d["B"], d["C"]], dim=1).contiguous()
+
     def launch():
         selscan.ss_fwd_dtproj(d["u"], d["delta_r"], d["W_dt"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
                               delta_bias=d["delta_bias"], delta_softplus=w.delta_softplus, stream=stream)
 
-    for _ in range(warmup):
-        flush.zero_()
-        launch()
-    ts = []
-    for _ in range(steps):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        launch()
-        e1.record(stream)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    ms = statistics.median(ts)
+    def launch_xdbl():
+        selscan.ss_fwd_xdbl(d["u"], x_dbl, d["W_dt"], d["A"], y, D=d["D"], z=d["z"], delta_bias=d["delta_bias"],
+                            delta_softplus=w.delta_softplus, stream=stream)
+
+    def timed(fn):
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    ms = timed(launch)
+    xdbl_ms = timed(launch_xdbl)
     status = selscan.ss_device_status()
-    del d, y
+    del d, y, x_dbl
     return {"ms": ms, "dt_rank": R, "updates_per_s": w.updates / (ms * 1e-3),
             "sfu_frac": w.updates / sfu_peak / (ms * 1e-3), "unfused_ms": unfused_ms,
-            "vs_unfused": unfused_ms / ms, "steps": steps, "device_status": status,
+            "vs_unfused": unfused_ms / ms, "xdbl_ms": xdbl_ms, "steps": steps, "device_status": status,
             "note": "delta = W_dt delta_r (tcgen05 bf16 MMA into tensor memory, one 64-step stage ahead of "
-                    "the scan) instead of reading delta; delta_r (B, dt_rank, L) and W_dt (D, dt_rank) bf16"}
+                    "the scan) instead of reading delta; delta_r (B, dt_rank, L) and W_dt (D, dt_rank) bf16; "
+                    "xdbl_ms: the same with delta_r, B and C read in place from one (B, dt_rank + 2 N, L) "
+                    "x_proj output (ss_fwd_xdbl)"}
 
 
 def bench_decode(w, d, out_dtype, stream, world, calls=200):

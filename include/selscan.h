@@ -266,6 +266,22 @@ ss_status ss_fwd_dtproj(const ss_desc *desc, int dt_rank, const void *u, const v
                         float *last_state, void *workspace, size_t workspace_bytes, ss_stream_t stream);
 
 /*
+ * ss_fwd_dtproj reading the x_proj output as it is (Mamba-minimal项目解析,
+ * 核心组件解析 §5 ssm: x_dbl = x_proj(x), split into delta (dt_rank
+ * features), B and C): delta_r, B and C are the row ranges [0, R),
+ * [R, R + N) and [R + N, R + 2N) of each batch entry of one tensor, so the
+ * split makes no copies.
+ *   x_dbl   device, (B, dt_rank + 2 N, L) bf16, l contiguous (the layout of B
+ *           and C of ss_fwd, with dt_rank + 2 N feature rows per batch entry)
+ * Every other argument, the launch, workspace and errors as ss_fwd_dtproj
+ * (B and C come from x_dbl); results equal ss_fwd_dtproj's on the three
+ * ranges copied out, bit for bit.
+ */
+ss_status ss_fwd_xdbl(const ss_desc *desc, int dt_rank, const void *u, const void *x_dbl, const void *W_dt,
+                      const float *A, const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                      void *y, float *last_state, void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
+/*
  * Bytes of the device scratch array built into the library for
  * ss_fwd_noalloc (8 MiB per device; a 4 x 1024-channel, 16-state layer over
  * 100000 steps needs 4,456,448 bytes = 4.25 MiB in its default launch shape).

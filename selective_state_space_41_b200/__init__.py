@@ -11,14 +11,14 @@ generator.
 from .selscan import (SS_BF16, SS_F32, SelscanError, lib, selective_scan_bwd, selective_scan_fwd,  # noqa: F401
                       ss_bwd, ss_bwd_workspace_bytes, ss_fwd, ss_step,
                       ss_fwd_heuristic, ss_fwd_hostio, ss_fwd_noalloc, ss_fwd_workspace_bytes,
-                      ss_status_string, ss_fwd_dtproj, ss_bwd_heuristic, ss_device_status,
+                      ss_status_string, ss_fwd_dtproj, ss_fwd_xdbl, ss_bwd_heuristic, ss_device_status,
                       ss_fwd_ckpt, ss_bwd_ckpt, ss_bwd_ckpt_workspace_bytes, ckpt_shape,
                       SelectiveScanFn, selective_scan_fn,
                       ss_version, workspace_for)
 
 __all__ = ["selective_scan_fwd", "selective_scan_bwd", "ss_bwd", "ss_bwd_workspace_bytes", "ss_fwd", "ss_step", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_noalloc",
            "ss_fwd_workspace_bytes", "workspace_for", "ss_status_string", "ss_version",
-           "ss_fwd_dtproj", "ss_bwd_heuristic", "ss_device_status",
+           "ss_fwd_dtproj", "ss_fwd_xdbl", "ss_bwd_heuristic", "ss_device_status",
            "ss_fwd_ckpt", "ss_bwd_ckpt", "ss_bwd_ckpt_workspace_bytes", "ckpt_shape",
            "SelectiveScanFn", "selective_scan_fn",
            "SelscanError", "SS_F32", "SS_BF16", "lib"]

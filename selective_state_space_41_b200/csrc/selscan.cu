@@ -315,7 +315,7 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
                    const uint8_t *reset, void *y, float *last_state, const ss_launch_config *cfg,
                    void *workspace, size_t workspace_bytes, ss_stream_t stream,
                    const void *delta_r = nullptr, const void *W_dt = nullptr, int dt_rank = 0,
-                   float *ckpt = nullptr) {
+                   float *ckpt = nullptr, int64_t bc_bstride = 0, int64_t dtr_bstride = 0) {
     Sizes sz;
     ss_status st = check_desc(desc, &sz);
     if (st != SS_OK) return st;
@@ -396,6 +396,8 @@ ss_status fwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
     p.W_dt = W_dt;
     p.dt_rank = dt_rank;
     p.ckpt = ckpt;
+    p.bc_bstride = bc_bstride;
+    p.dtr_bstride = dtr_bstride;
 
     const dim3 grid((unsigned)blocks), block((unsigned)(pl.warps * 32));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -550,6 +552,26 @@ ss_status ss_fwd_dtproj(const ss_desc *desc, int dt_rank, const void *u, const v
     if (dt_rank == 0) return SS_ERR_BAD_SHAPE;
     return fwd_impl(desc, u, nullptr, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y, last_state,
                     nullptr, workspace, workspace_bytes, stream, delta_r, W_dt, dt_rank);
+}
+
+ss_status ss_fwd_xdbl(const ss_desc *desc, int dt_rank, const void *u, const void *x_dbl, const void *W_dt,
+                      const float *A, const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                      void *y, float *last_state, void *workspace, size_t workspace_bytes, ss_stream_t stream) {
+    Sizes sz;
+    const ss_status st = check_desc(desc, &sz);
+    if (st != SS_OK) return st;
+    if (dt_rank < 1 || dt_rank > selscan::kMaxDtRank) return SS_ERR_BAD_SHAPE;
+    if (desc->in_dtype != SS_BF16) return SS_ERR_UNSUPPORTED_DTYPE;
+    if (!x_dbl && sz.rows > 0 && desc->seqlen > 0) return SS_ERR_NULL_POINTER;
+    // delta_r, B and C are the row ranges [0, R), [R, R + N), [R + N, R + 2N)
+    // of each batch entry's (R + 2N, L) block.
+    const int64_t L = desc->seqlen, N = desc->dstate, feats = dt_rank + 2 * N;
+    const size_t e = dtype_size(desc->in_dtype);
+    const char *xb = static_cast<const char *>(x_dbl);
+    const void *B = xb ? xb + (size_t)dt_rank * (size_t)L * e : nullptr;
+    const void *C = xb ? xb + (size_t)(dt_rank + N) * (size_t)L * e : nullptr;
+    return fwd_impl(desc, u, nullptr, A, B, C, D, z, delta_bias, delta_softplus, nullptr, nullptr, y, last_state,
+                    nullptr, workspace, workspace_bytes, stream, x_dbl, W_dt, dt_rank, nullptr, feats * L, feats * L);
 }
 
 ss_status ss_fwd_ckpt(const ss_desc *desc, const void *u, const void *delta, const float *A, const void *B,

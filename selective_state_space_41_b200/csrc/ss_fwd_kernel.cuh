@@ -80,6 +80,11 @@ struct FwdParams {
     // dt_rank, L) and W_dt (dim, dt_rank) in the input dtype.
     const void *delta_r, *W_dt;
     int dt_rank;
+    // Elements between consecutive batch entries of B and C, and of delta_r
+    // (direct kernel and fix-up); 0: contiguous, N L and dt_rank L.  The
+    // x_proj output form passes B, C and delta_r as row ranges of one
+    // (batch, dt_rank + 2 N, L) tensor, so all three step by its batch stride.
+    int64_t bc_bstride = 0, dtr_bstride = 0;
     // Checkpoints for the backward (direct kernel; or null): the state
     // entering every step l = 8k, (batch, dim, ceil(L / 8), dstate) fp32 —
     // the state after step l - 1, before any sequence start at l zeroes it.
@@ -888,8 +893,9 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     float *gat = slab + r * kGatherStride;                  // this row: 8 delta', 8 delta' u
     float *red = slab + kRowsPerWarp * kGatherStride;       // per lane: 8 partial sums of y
 
-    const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * N * L,
-                          static_cast<const Tin *>(p.C) + b * N * L};
+    const int64_t bc_bstride = p.bc_bstride ? p.bc_bstride : N * L;
+    const Tin *Bsrc[2] = {static_cast<const Tin *>(p.B) + b * bc_bstride,
+                          static_cast<const Tin *>(p.C) + b * bc_bstride};
     // This lane's first owned step of each stream (advanced per sub-chunk).
     const Tin *u_own = static_cast<const Tin *>(p.u) + row * L + c_begin + g * kOwn;
     const Tin *d_own = kDt ? nullptr : static_cast<const Tin *>(p.delta) + row * L + c_begin + g * kOwn;
@@ -1039,7 +1045,8 @@ __global__ void SS_DIRECT_BOUNDS(kNmax / kG) ss_fwd_direct_kernel(const FwdParam
     const int64_t dt_nst = (Lend - c_begin + kDirectStage - 1) / kDirectStage;  // stages of this block
     bool dt_ok = true;
     uint4 dt_raw[kDt ? kMaxDtRank * 8 / 128 : 1];  // this thread's 16-byte chunks of delta_r of a coming stage
-    const Tin *dt_src = kDt ? static_cast<const Tin *>(p.delta_r) + b * dt_R * L : nullptr;
+    const Tin *dt_src = kDt ? static_cast<const Tin *>(p.delta_r) + b * (p.dtr_bstride ? p.dtr_bstride : dt_R * L)
+                            : nullptr;
     auto dt_load_raw = [&](int64_t k) {  // delta_r[b, r, stage k]: chunks (r, 8 steps)
 #pragma unroll
         for (int q = 0; q < kMaxDtRank * 8 / 128; ++q) {
@@ -1535,9 +1542,9 @@ __global__ void __launch_bounds__(kFixupWarps * 32) ss_fwd_fixup_kernel(const Fw
     __syncwarp();
 
     const Tin *dl_row = dt ? nullptr : static_cast<const Tin *>(p.delta) + row * L;
-    const Tin *dr_b = dt ? static_cast<const Tin *>(p.delta_r) + b * R * L : nullptr;
+    const Tin *dr_b = dt ? static_cast<const Tin *>(p.delta_r) + b * (p.dtr_bstride ? p.dtr_bstride : R * L) : nullptr;
     const Tin *z_row = p.z ? static_cast<const Tin *>(p.z) + row * L : nullptr;
-    const Tin *C_b = static_cast<const Tin *>(p.C) + b * N * L;
+    const Tin *C_b = static_cast<const Tin *>(p.C) + b * (p.bc_bstride ? p.bc_bstride : N * L);
     Tout *y_row = static_cast<Tout *>(p.y) + row * L;
     const float bias = p.delta_bias ? p.delta_bias[d] : 0.f;
     const bool softplus = p.softplus != 0;

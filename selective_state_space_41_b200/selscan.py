@@ -40,7 +40,7 @@ EXPORTS = ("ss_fwd", "ss_fwd_ws", "ss_fwd_workspace_bytes", "ss_fwd_with_config"
            "ss_fwd_reset", "ss_fwd_heuristic", "ss_fwd_hostio", "ss_fwd_hostio_streams", "ss_fwd_noalloc",
            "ss_step", "ss_bwd", "ss_bwd_reset", "ss_bwd_state", "ss_bwd_workspace_bytes", "ss_status_string",
            "ss_version", "ss_device_status", "ss_fwd_dtproj", "ss_bwd_heuristic", "ss_fwd_ckpt", "ss_bwd_ckpt",
-           "ss_bwd_ckpt_workspace_bytes")
+           "ss_bwd_ckpt_workspace_bytes", "ss_fwd_xdbl")
 
 
 class SelscanError(RuntimeError):
@@ -93,6 +93,8 @@ def lib():
         L.ss_fwd_hostio.argtypes = [DP] + [P] * 8 + [I] + [P] * 12 + [P, SZ, P]
         L.ss_fwd_dtproj.restype = I
         L.ss_fwd_dtproj.argtypes = [DP, I] + [P] * 9 + [I, P, P, P, SZ, P]
+        L.ss_fwd_xdbl.restype = I
+        L.ss_fwd_xdbl.argtypes = [DP, I] + [P] * 7 + [I, P, P, P, SZ, P]
         L.ss_fwd_noalloc.restype = I
         L.ss_fwd_noalloc.argtypes = [DP, P, P, P, P, P, P, P, P, I, P, P, P]
         L.ss_fwd_hostio_streams.restype = I
@@ -250,6 +252,27 @@ def ss_fwd_dtproj(u, delta_r, W_dt, A, B, C, y, D=None, z=None, delta_bias=None,
                                _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(y),
                                _ptr(last_state), _ptr(workspace), ws_bytes, _stream_handle(stream, u.device)),
            "ss_fwd_dtproj")
+
+
+def ss_fwd_xdbl(u, x_dbl, W_dt, A, y, D=None, z=None, delta_bias=None, delta_softplus=True, last_state=None,
+                stream=None, workspace=None):
+    """Queue ss_fwd_dtproj with delta_r, B and C read from the x_proj output
+    ``x_dbl`` ((batch, dt_rank + 2 N, L) bf16: feature rows [0, R) delta_r,
+    [R, R + N) B, [R + N, R + 2N) C; no copies); W_dt: (dim, dt_rank) bf16,
+    N = A.shape[1]; other tensors as ``ss_fwd``."""
+    u, x_dbl, W_dt, A, D, z, delta_bias = map(_contig, (u, x_dbl, W_dt, A, D, z, delta_bias))
+    if not (y.is_contiguous() and (last_state is None or last_state.is_contiguous())):
+        raise ValueError("outputs must be contiguous")
+    batch, dim, L = u.shape
+    N, R = A.shape[-1], W_dt.shape[-1]
+    if tuple(x_dbl.shape) != (batch, R + 2 * N, L) or tuple(W_dt.shape) != (dim, R):
+        raise ValueError("x_dbl must be (batch, dt_rank + 2 N, L) and W_dt (dim, dt_rank)")
+    desc = make_desc(batch, dim, L, N, u.dtype, y.dtype)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().ss_fwd_xdbl(ctypes.byref(desc), int(R), _ptr(u), _ptr(x_dbl), _ptr(W_dt), _ptr(A), _ptr(D),
+                             _ptr(z), _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(y), _ptr(last_state),
+                             _ptr(workspace), ws_bytes, _stream_handle(stream, u.device)),
+           "ss_fwd_xdbl")
 
 
 def ss_fwd_noalloc(u, delta, A, B, C, y, D=None, z=None, delta_bias=None, delta_softplus=False,
@@ -502,9 +525,10 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
 class SelectiveScanFn(torch.autograd.Function):
     """The scan as a torch autograd Function: the forward is ``ss_fwd_ckpt``
     (keeping the backward's checkpoints for the saved context), the backward
-    ``ss_bwd_ckpt`` (all gradients, no second forward pass).  Gradients come
-    back in the dtypes of their inputs (dB, dC are summed in fp32 and then
-    cast for bf16 B, C)."""
+    ``ss_bwd_ckpt`` (all gradients, no second forward pass).  When no input
+    needs a gradient the forward is plain ``ss_fwd`` and nothing is saved.
+    Gradients come back in the dtypes of their inputs (dB, dC are summed in
+    fp32 and then cast for bf16 B, C)."""
 
     @staticmethod
     def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus):
@@ -512,8 +536,12 @@ class SelectiveScanFn(torch.autograd.Function):
         batch, dim, L = u.shape
         N = A.shape[-1]
         y = torch.empty_like(u)
-        ck = torch.empty(ckpt_shape(batch, dim, L, N), dtype=torch.float32, device=u.device)
         ws = workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=u.device)
+        if not any(ctx.needs_input_grad):
+            ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                   workspace=ws)
+            return y
+        ck = torch.empty(ckpt_shape(batch, dim, L, N), dtype=torch.float32, device=u.device)
         ss_fwd_ckpt(u, delta, A, B, C, y, ck, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
                     workspace=ws)
         ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, ck)

@@ -328,6 +328,19 @@ def test_ckpt_entry_rejections(lib):
         assert 0 < ck < full and full - ck >= rows * nsub * shape[3] * 4 - 256, shape
 
 
+def test_xdbl_entry_rejections(lib):
+    """ss_fwd_xdbl rejects before any launch (fake pointers): dt_rank outside
+    1..64, fp32 inputs, no x_dbl."""
+    P = FAKE
+    d = _desc(seqlen=64, dstate=16, in_dtype=1, out_dtype=1)
+    tail = (P, P, P, P, None, None, None, 1, P, None, None, 0, None)   # u, x_dbl, W_dt, A, D, z, bias, sp, y, ...
+    assert lib.ss_fwd_xdbl(ctypes.byref(d), 0, *tail) == 2
+    assert lib.ss_fwd_xdbl(ctypes.byref(d), 65, *tail) == 2
+    assert lib.ss_fwd_xdbl(ctypes.byref(_desc(seqlen=64, dstate=16)), 48, *tail) == 3
+    assert lib.ss_fwd_xdbl(ctypes.byref(d), 48, P, None, P, P, None, None, None, 1, P, None, None, 0, None) == 1
+    assert lib.ss_fwd_xdbl(None, 48, *tail) == 1
+
+
 def test_bwd_rejections(lib):
     """ss_bwd rejects before any launch (the pointers are fake): no
     descriptor, more than 64 states, a missing gradient output, no workspace.

@@ -68,3 +68,15 @@ def test_autograd_bf16_matches_the_direct_backward():
         if k in ("dB", "dC"):
             w = w.to(torch.bfloat16)
         assert g.dtype == w.dtype and torch.equal(g, w), k
+
+
+def test_no_grad_forward_is_the_plain_forward():
+    """Without inputs that need gradients the Function runs ss_fwd (no
+    checkpoints): y is selective_scan_fwd's, bit for bit."""
+    inp = _case(2, 40, 512, 16, torch.bfloat16, seed=955, has_z=True)
+    d = {k: (inp[k].cuda() if inp.get(k) is not None else None) for k in NAMES}
+    kw = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"])
+    y = selscan.selective_scan_fn(d["u"], d["delta"], d["A"], d["B"], d["C"], **kw)
+    want = selscan.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], **kw)
+    torch.cuda.synchronize()
+    assert not y.requires_grad and torch.equal(y.view(torch.int16), want.view(torch.int16))

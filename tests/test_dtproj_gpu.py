@@ -122,3 +122,63 @@ def test_dtproj_rejections():
     with pytest.raises(selscan.SelscanError):   # dt_rank above 64
         selscan.ss_fwd_dtproj(d["u"], big, torch.zeros((8, 65), dtype=BF16, device="cuda"), d["A"], d["B"],
                               d["C"], y)
+
+
+# ---------------------------------------------------------------- x_dbl form
+def _xdbl(inp):
+    """x_proj's output as one (batch, dt_rank + 2 N, L) tensor: feature rows
+    delta_r, then B, then C."""
+    return torch.cat([inp["delta_r"], inp["B"], inp["C"]], dim=1).contiguous()
+
+
+def _run_xdbl(inp, x_dbl, out_dtype=None, workspace=False):
+    d = to_dev(inp)
+    batch, dim, L = d["u"].shape
+    N = d["A"].shape[1]
+    y = torch.full((batch, dim, L), float("nan"), dtype=out_dtype or BF16, device="cuda")
+    last = torch.full((batch, dim, N), float("nan"), device="cuda") if inp["return_last_state"] else None
+    ws = selscan.workspace_for(batch, dim, L, N, BF16, y.dtype) if workspace else None
+    selscan.ss_fwd_xdbl(d["u"], x_dbl.cuda(), d["W_dt"], d["A"], y, D=d["D"], z=d["z"],
+                        delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"], last_state=last,
+                        workspace=ws)
+    torch.cuda.synchronize()
+    return y, last
+
+
+@pytest.mark.parametrize("R,N,L", [(48, 16, 300), (7, 33, 203), (64, 64, 129), (16, 4, 1000), (1, 8, 65)])
+def test_xdbl_against_oracle_and_dtproj(R, N, L):
+    """delta_r, B and C read in place from x_dbl: the oracle fed the three
+    row ranges of the same tensor (the x_proj split), and ss_fwd_dtproj on
+    contiguous copies of them bit for bit."""
+    inp = _case(3, 40, L, N, R, seed=700 + R + N, has_z=True, bias_kind="uniform_dt", return_last_state=True)
+    x = _xdbl(inp)
+    y, last = _run_xdbl(inp, x)
+    split = dict(inp, delta_r=x[:, :R], B=x[:, R:R + N], C=x[:, R + N:])
+    y_ref, last_ref = _oracle(split)
+    assert_parity(y, last, y_ref, last_ref, TOL[BF16], f"x_dbl R={R} N={N} L={L}")
+    y2, last2 = _run(inp)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16)) and torch.equal(last, last2)
+
+
+def test_xdbl_segments_and_f32_output():
+    """Few rows over a long sequence (sequence segments: the fix-up reads C
+    and delta_r from x_dbl too), fp32 output."""
+    inp = _case(1, 64, 9000, 16, 48, seed=777, has_z=True, return_last_state=True)
+    assert selscan.ss_fwd_heuristic(1, 64, 9000, 16, BF16, workspace_bytes=1 << 26)["segments"] > 1
+    x = _xdbl(inp)
+    y, last = _run_xdbl(inp, x, out_dtype=torch.float32, workspace=True)
+    y_ref, last_ref = _oracle(inp)
+    assert_parity(y, last, y_ref, last_ref, 1e-4, "x_dbl segments")
+    y2, last2 = _run(inp, out_dtype=torch.float32, workspace=True)
+    assert torch.equal(y, y2) and torch.equal(last, last2)
+
+
+def test_xdbl_rejections():
+    inp = _case(1, 8, 64, 16, 48, seed=3)
+    d = to_dev(inp)
+    y = torch.empty_like(d["u"])
+    x = _xdbl(inp).cuda()
+    with pytest.raises(ValueError):   # feature rows do not match dt_rank + 2 N
+        selscan.ss_fwd_xdbl(d["u"], x[:, :-1], d["W_dt"], d["A"], y)
+    with pytest.raises(selscan.SelscanError):   # fp32 inputs
+        selscan.ss_fwd_xdbl(d["u"].float(), x.float(), d["W_dt"].float(), d["A"], y.float())
