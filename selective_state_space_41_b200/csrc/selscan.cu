@@ -960,8 +960,10 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
             if (fn(dim3((unsigned)(lo.dtiles * gb * lo.nseg)), dim3(kBwdWarps * 32), smem, s, q) != cudaSuccess)
                 return SS_ERR_CUDA;
             const int64_t bc = gb * 2 * NL;
-            if (bc > 0) {
-                const int64_t nb = (bc + 255) / 256;
+            if (bc > 0) {  // one thread per four outputs when the kernel can read float4 rows
+                const bool v4 = NL % 4 == 0 && aligned(q.ws_dBC, 16) && aligned(dB + b0 * NL, 16) &&
+                                aligned(dC + b0 * NL, 16);
+                const int64_t nb = ((v4 ? bc / 4 : bc) + 255) / 256;
                 selscan::ss_bwd_reduce_bc_kernel<<<(unsigned)(nb < 4 * 148 * 8 ? nb : 4 * 148 * 8), 256, 0, s>>>(
                     q, dB + b0 * NL, dC + b0 * NL);
                 if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;

@@ -836,10 +836,40 @@ __global__ void __launch_bounds__(256) ss_bwd_seg_fold_kernel(const BwdParams p,
     }
 }
 
-// dB, dC = the block partials summed over the row tiles, in tile order.
+// dB, dC = the block partials summed over the row tiles, in tile order.  With
+// whole float4 rows (N L a multiple of 4, 16-byte aligned buffers) a thread
+// sums four consecutive outputs and keeps eight tiles' loads in flight (each
+// output still adds its tiles in order, so the bits do not change; the plain
+// form ran at 2 TB/s, waiting on one load at a time).
 static __global__ void __launch_bounds__(256) ss_bwd_reduce_bc_kernel(const BwdParams p, float *dB, float *dC) {
     const int64_t per = (int64_t)p.dstate * p.seqlen;
     const int64_t total = p.batch * 2 * per;
+    const bool vec4 = per % 4 == 0 && ((reinterpret_cast<uintptr_t>(p.ws_dBC) | reinterpret_cast<uintptr_t>(dB) |
+                                        reinterpret_cast<uintptr_t>(dC)) & 15u) == 0;
+    if (vec4) {  // four consecutive outputs per thread, eight tiles' loads in flight
+        const int64_t per4 = per / 4, tstride = p.batch * 2 * per4;
+        const float4 *src = reinterpret_cast<const float4 *>(p.ws_dBC);
+        for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total / 4;
+             e += (int64_t)gridDim.x * blockDim.x) {
+            const int64_t b = e / (2 * per4), which = (e / per4) % 2, q = e % per4;
+            const float4 *t0 = src + (b * 2 + which) * per4 + q;
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+            int64_t t = 0;
+            for (; t + 8 <= p.dtiles; t += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = __ldcs(t0 + (t + k) * tstride);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) s.x += v[k].x, s.y += v[k].y, s.z += v[k].z, s.w += v[k].w;
+            }
+            for (; t < p.dtiles; ++t) {
+                const float4 v = __ldcs(t0 + t * tstride);
+                s.x += v.x, s.y += v.y, s.z += v.z, s.w += v.w;
+            }
+            reinterpret_cast<float4 *>(which ? dC : dB)[b * per4 + q] = s;
+        }
+        return;
+    }
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t b = e / (2 * per), which = (e / per) % 2, nl = e % per;
