@@ -549,6 +549,7 @@ class SelectiveScanFn(torch.autograd.Function):
         return y
 
     @staticmethod
+    @torch.autograd.function.once_differentiable
     def backward(ctx, dy):
         u, delta, A, B, C, D, z, delta_bias, ck = ctx.saved_tensors
         g = selective_scan_bwd(u, delta, A, B, C, dy.contiguous(), D=D, z=z, delta_bias=delta_bias,
