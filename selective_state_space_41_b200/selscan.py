@@ -527,39 +527,64 @@ class SelectiveScanFn(torch.autograd.Function):
     (keeping the backward's checkpoints for the saved context), the backward
     ``ss_bwd_ckpt`` (all gradients, no second forward pass).  When no input
     needs a gradient the forward is plain ``ss_fwd`` and nothing is saved.
-    Gradients come back in the dtypes of their inputs (dB, dC are summed in
-    fp32 and then cast for bf16 B, C)."""
+    Optional: a float32 (batch, dim, N) state before step 0 (differentiable),
+    a (batch, L) mask of sequence starts, and the last state as a second
+    output (differentiable: a loss on it, as when it feeds the next piece of
+    a sequence, reaches every input).  Gradients come back in the dtypes of
+    their inputs (dB, dC are summed in fp32 and then cast for bf16 B, C)."""
 
     @staticmethod
-    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus):
-        u, delta, A, B, C, D, z, delta_bias = map(_contig, (u, delta, A, B, C, D, z, delta_bias))
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, initial_state, reset, delta_softplus, return_last_state):
+        u, delta, A, B, C, D, z, delta_bias, initial_state, reset = map(
+            _contig, (u, delta, A, B, C, D, z, delta_bias, initial_state, reset))
         batch, dim, L = u.shape
         N = A.shape[-1]
         y = torch.empty_like(u)
+        last = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device) if return_last_state else None
         ws = workspace_for(batch, dim, L, N, u.dtype, y.dtype, device=u.device)
+        kw = dict(D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus, last_state=last,
+                  initial_state=initial_state, reset=reset, workspace=ws)
         if not any(ctx.needs_input_grad):
-            ss_fwd(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
-                   workspace=ws)
-            return y
+            ss_fwd(u, delta, A, B, C, y, **kw)
+            return (y, last) if return_last_state else y
         ck = torch.empty(ckpt_shape(batch, dim, L, N), dtype=torch.float32, device=u.device)
-        ss_fwd_ckpt(u, delta, A, B, C, y, ck, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
-                    workspace=ws)
-        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, ck)
+        ss_fwd_ckpt(u, delta, A, B, C, y, ck, **kw)
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, reset, ck)
         ctx.delta_softplus = bool(delta_softplus)
-        return y
+        ctx.has_h0 = initial_state is not None
+        ctx.return_last_state = bool(return_last_state)
+        return (y, last) if return_last_state else y
 
     @staticmethod
     @torch.autograd.function.once_differentiable
-    def backward(ctx, dy):
-        u, delta, A, B, C, D, z, delta_bias, ck = ctx.saved_tensors
-        g = selective_scan_bwd(u, delta, A, B, C, dy.contiguous(), D=D, z=z, delta_bias=delta_bias,
-                               delta_softplus=ctx.delta_softplus, ckpt=ck)
+    def backward(ctx, dy, dlast=None):
+        u, delta, A, B, C, D, z, delta_bias, reset, ck = ctx.saved_tensors
+        batch, dim, L = u.shape
+        N = A.shape[-1]
+        f32, dev = torch.float32, u.device
+        g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+             "dA": torch.empty((dim, N), dtype=f32, device=dev),
+             "dB": torch.empty((batch, N, L), dtype=f32, device=dev),
+             "dC": torch.empty((batch, N, L), dtype=f32, device=dev),
+             "dD": torch.empty(dim, dtype=f32, device=dev) if D is not None else None,
+             "dz": torch.empty_like(u) if z is not None else None,
+             "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None,
+             "dinitial_state": (torch.empty((batch, dim, N), dtype=f32, device=dev)
+                                if ctx.has_h0 and ctx.needs_input_grad[8] else None)}
+        ss_bwd_ckpt(u, delta, A, B, C, dy.contiguous(), ck, g, D=D, z=z, delta_bias=delta_bias,
+                    delta_softplus=ctx.delta_softplus, reset=reset,
+                    d_last_state=dlast.contiguous() if dlast is not None else None)
         return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype), g["dD"], g["dz"],
-                g["ddelta_bias"], None)
+                g["ddelta_bias"], g["dinitial_state"], None, None, None)
 
 
-def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False):
-    """y of the selective scan (argument order of the walkthrough's
-    selective_scan_ref), differentiable through torch autograd; see
-    SelectiveScanFn."""
-    return SelectiveScanFn.apply(u, delta, A, B, C, D, z, delta_bias, delta_softplus)
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+                      initial_state=None, reset=None, return_last_state=False):
+    """y (and, with return_last_state, the float32 last state) of the
+    selective scan (argument order of the walkthrough's selective_scan_ref,
+    plus an optional initial state and mask of sequence starts),
+    differentiable through torch autograd; see SelectiveScanFn."""
+    if reset is not None and reset.dtype == torch.bool:
+        reset = reset.view(torch.uint8)
+    return SelectiveScanFn.apply(u, delta, A, B, C, D, z, delta_bias, initial_state, reset, delta_softplus,
+                                 return_last_state)
