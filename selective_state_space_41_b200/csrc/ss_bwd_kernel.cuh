@@ -114,7 +114,10 @@ __device__ __forceinline__ float sigmoid_of(float x) {
 
 // Three 128-thread blocks per SM (at most 168 registers a thread): with the
 // 4-warp blocks of the mamba-130m-shaped layer (384 blocks) that is one wave
-// on 148 SMs; measured 1.35 ms there against 1.77 ms at 255 registers.
+// on 148 SMs.  Measured there on an earlier form of the kernel: 1.35 ms
+// against 1.77 ms at 255 registers (two blocks per SM); four blocks at 128
+// registers (the dB/dC slab summed in two halves to fit) spill 260 bytes and
+// take 1.68 ms against 1.01 ms from the forward's checkpoints.
 #ifndef SS_BWD_MIN_BLOCKS
 #define SS_BWD_MIN_BLOCKS 3
 #endif
