@@ -398,7 +398,7 @@ def bench_ours(args, w, world, rank, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms,
                 "api": "ss_fwd_hostio_streams (pinned host buffers, batch ranges pipelined over 3 streams)"},
-        "gpu_launches": args.steps * (2 if shape["segments"] > 1 else 1),
+        "gpu_launches": args.steps * (3 if shape["segments"] > 1 else 1),  # segments: + carry fold + fix-up
         "clocks": clocks.summary(),
         "kernel_ms": {"min": min(kernel_ms), "median": statistics.median(kernel_ms),
                       "max": max(kernel_ms)},
