@@ -10,11 +10,11 @@ namespace selscan {
 
 namespace {
 
-template <bool kReset>
+template <bool kReset, bool kZ = true>
 cudaError_t launch(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const BwdParams &p) {
     constexpr int kMaxDevices = 64;
     static bool opted_in[kMaxDevices];
-    auto kernel = ss_bwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kReset>;
+    auto kernel = ss_bwd_kernel<SS_INST_TIN, SS_INST_TOUT, SS_INST_NMAX, kReset, kZ>;
     if (smem > 48 * 1024) {  // above the default a kernel opts in to more dynamic shared memory, once per device
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
@@ -31,9 +31,11 @@ cudaError_t launch(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const Bwd
 
 }  // namespace
 
-// The instance that reads sequence starts when p.reset is given.
+// The instance that reads sequence starts when p.reset is given; without
+// them, the one without the gate's sums when there is no z.
 cudaError_t SS_INST_NAME(dim3 grid, dim3 block, size_t smem, cudaStream_t s, const BwdParams &p) {
-    return p.reset ? launch<true>(grid, block, smem, s, p) : launch<false>(grid, block, smem, s, p);
+    if (p.reset) return launch<true>(grid, block, smem, s, p);
+    return p.z ? launch<false>(grid, block, smem, s, p) : launch<false, false>(grid, block, smem, s, p);
 }
 
 }  // namespace selscan
