@@ -413,15 +413,12 @@ def ss_bwd_ckpt(u, delta, A, B, C, dy, ckpt, grads, D=None, z=None, delta_bias=N
            "ss_bwd_ckpt")
 
 
-def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=False,
-                       stream=None, reset=None, initial_state=None, d_last_state=None, ckpt=None):
-    """Gradients of sum(dy * y) (+ sum(d_last_state * last state)) as a dict
-    (see ss_bwd); allocates the outputs; dinitial_state when an initial
-    state or a last-state gradient is given."""
+def _grad_outputs(u, A, D, z, delta_bias, with_initial_state):
+    """Output tensors of the backward: du, ddelta, dz in u's dtype; dA, dB,
+    dC, dD, ddelta_bias (and dinitial_state) float32; None for absent operands."""
     batch, dim, L = u.shape
     N = A.shape[-1]
-    dev = u.device
-    f32 = torch.float32
+    dev, f32 = u.device, torch.float32
     grads = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
              "dA": torch.empty((dim, N), dtype=f32, device=dev),
              "dB": torch.empty((batch, N, L), dtype=f32, device=dev),
@@ -429,8 +426,17 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, d
              "dD": torch.empty(dim, dtype=f32, device=dev) if D is not None else None,
              "dz": torch.empty_like(u) if z is not None else None,
              "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None}
-    if initial_state is not None or d_last_state is not None:
+    if with_initial_state:
         grads["dinitial_state"] = torch.empty((batch, dim, N), dtype=f32, device=dev)
+    return grads
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=False,
+                       stream=None, reset=None, initial_state=None, d_last_state=None, ckpt=None):
+    """Gradients of sum(dy * y) (+ sum(d_last_state * last state)) as a dict
+    (see ss_bwd); allocates the outputs; dinitial_state when an initial
+    state or a last-state gradient is given."""
+    grads = _grad_outputs(u, A, D, z, delta_bias, initial_state is not None or d_last_state is not None)
     if ckpt is not None:  # from the forward's checkpoints (ss_fwd_ckpt); they hold the initial state
         ss_bwd_ckpt(u, delta, A, B, C, dy, ckpt, grads, D=D, z=z, delta_bias=delta_bias,
                     delta_softplus=delta_softplus, reset=reset, d_last_state=d_last_state, stream=stream)
@@ -559,23 +565,12 @@ class SelectiveScanFn(torch.autograd.Function):
     @torch.autograd.function.once_differentiable
     def backward(ctx, dy, dlast=None):
         u, delta, A, B, C, D, z, delta_bias, reset, ck = ctx.saved_tensors
-        batch, dim, L = u.shape
-        N = A.shape[-1]
-        f32, dev = torch.float32, u.device
-        g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
-             "dA": torch.empty((dim, N), dtype=f32, device=dev),
-             "dB": torch.empty((batch, N, L), dtype=f32, device=dev),
-             "dC": torch.empty((batch, N, L), dtype=f32, device=dev),
-             "dD": torch.empty(dim, dtype=f32, device=dev) if D is not None else None,
-             "dz": torch.empty_like(u) if z is not None else None,
-             "ddelta_bias": torch.empty(dim, dtype=f32, device=dev) if delta_bias is not None else None,
-             "dinitial_state": (torch.empty((batch, dim, N), dtype=f32, device=dev)
-                                if ctx.has_h0 and ctx.needs_input_grad[8] else None)}
+        g = _grad_outputs(u, A, D, z, delta_bias, ctx.has_h0 and ctx.needs_input_grad[8])
         ss_bwd_ckpt(u, delta, A, B, C, dy.contiguous(), ck, g, D=D, z=z, delta_bias=delta_bias,
                     delta_softplus=ctx.delta_softplus, reset=reset,
                     d_last_state=dlast.contiguous() if dlast is not None else None)
         return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype), g["dD"], g["dz"],
-                g["ddelta_bias"], g["dinitial_state"], None, None, None)
+                g["ddelta_bias"], g.get("dinitial_state"), None, None, None)
 
 
 def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
