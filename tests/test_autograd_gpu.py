@@ -154,3 +154,26 @@ def test_autograd_starts_and_state_against_oracle():
     torch.cuda.synchronize()
     for k, v in direct.items():
         assert (v is None and got.get(k) is None) or torch.equal(v, got[k]), k
+
+
+def test_autograd_empty_batch_and_sequence():
+    """No batch entries: empty outputs and gradients; an empty sequence
+    with a returned last state: the last state is the initial one and its
+    gradient reaches the initial state unchanged."""
+    inp = _case(0, 8, 32, 16, torch.float32, seed=961)
+    t = _leaves(inp)
+    y = selscan.selective_scan_fn(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"],
+                                  delta_bias=t["delta_bias"], delta_softplus=True)
+    y.sum().backward()
+    torch.cuda.synchronize()
+    assert y.shape == (0, 8, 32) and t["u"].grad.shape == (0, 8, 32) and float(t["A"].grad.abs().sum()) == 0.0
+    inp = _case(2, 8, 0, 16, torch.float32, seed=962)
+    t = _leaves(inp)
+    h0 = torch.randn((2, 8, 16), generator=torch.Generator().manual_seed(962)).cuda().requires_grad_(True)
+    y, last = selscan.selective_scan_fn(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"],
+                                        delta_bias=t["delta_bias"], delta_softplus=True, initial_state=h0,
+                                        return_last_state=True)
+    g = torch.randn_like(last)
+    (last * g).sum().backward()
+    torch.cuda.synchronize()
+    assert torch.equal(last.detach(), h0.detach()) and torch.equal(h0.grad, g)

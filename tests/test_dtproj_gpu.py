@@ -182,3 +182,28 @@ def test_xdbl_rejections():
         selscan.ss_fwd_xdbl(d["u"], x[:, :-1], d["W_dt"], d["A"], y)
     with pytest.raises(selscan.SelscanError):   # fp32 inputs
         selscan.ss_fwd_xdbl(d["u"].float(), x.float(), d["W_dt"].float(), d["A"], y.float())
+
+
+@pytest.mark.parametrize("form", ["dtproj", "xdbl"])
+def test_empty_sequence_and_no_rows(form):
+    """L = 0 writes a zero last state (no initial state is taken here); no
+    batch entries is a no-op; both for delta_r/B/C passed apart and in place."""
+    inp = _case(2, 24, 0, 16, 48, seed=31, return_last_state=True)
+    d = to_dev(inp)
+    last = torch.full((2, 24, 16), 7.0, device="cuda")
+    y = torch.empty((2, 24, 0), dtype=BF16, device="cuda")
+    if form == "dtproj":
+        selscan.ss_fwd_dtproj(d["u"], d["delta_r"], d["W_dt"], d["A"], d["B"], d["C"], y, last_state=last)
+    else:
+        selscan.ss_fwd_xdbl(d["u"], _xdbl(inp).cuda(), d["W_dt"], d["A"], y, last_state=last)
+    torch.cuda.synchronize()
+    assert torch.all(last == 0)
+    inp = _case(0, 24, 64, 16, 48, seed=32)
+    d = to_dev(inp)
+    y = torch.empty((0, 24, 64), dtype=BF16, device="cuda")
+    if form == "dtproj":
+        selscan.ss_fwd_dtproj(d["u"], d["delta_r"], d["W_dt"], d["A"], d["B"], d["C"], y)
+    else:
+        selscan.ss_fwd_xdbl(d["u"], _xdbl(inp).cuda(), d["W_dt"], d["A"], y)
+    torch.cuda.synchronize()
+    assert selscan.ss_device_status() == 0
