@@ -432,6 +432,7 @@ struct BwdLayout {
     int64_t group;          // batch entries per launch
     int nseg;               // sequence segments (1: none)
     int64_t seg_len;
+    int fsum_k;             // forward-summary segments per segment (1 or 2)
     size_t off_ckpt, off_dbc, off_dA, off_dD, off_dbias;                  // workspace byte offsets
     size_t off_hend, off_dsum, off_lam0, off_D, total;                    // segment records (nseg > 1)
 };
@@ -475,6 +476,12 @@ BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz, bool ckpt_given = fal
     }
     lo.group = group;
     lo.nseg = bwd_segments(desc, lo.dtiles * group, &lo.seg_len);
+    // The forward summary (run only without the forward's checkpoints) is the
+    // direct kernel with 64-row blocks, half the adjoint kernel's row tiles:
+    // over the adjoint's segments it would fill under one wave of the GPU
+    // (the genomic layer: 448 blocks), so it cuts each segment in two where
+    // the halves stay whole 64-step stages.
+    lo.fsum_k = (lo.nseg > 1 && !ckpt_given && lo.seg_len % 128 == 0) ? 2 : 1;
     const size_t grows = (size_t)group * (size_t)desc->dim, S = (size_t)lo.nseg;
     lo.off_ckpt = 0;
     lo.off_dbc = align256(lo.off_ckpt + (ckpt_given ? 0 : grows * (size_t)lo.nsub * N * 4));
@@ -483,8 +490,9 @@ BwdLayout bwd_layout(const ss_desc *desc, const Sizes &sz, bool ckpt_given = fal
     lo.off_dbias = align256(lo.off_dD + S * rows * 4);
     lo.off_hend = align256(lo.off_dbias + S * rows * 4);
     const size_t seg_rec = lo.nseg > 1 ? S * grows : 0;  // (segment, row) records of one group
-    lo.off_dsum = align256(lo.off_hend + seg_rec * N * 4);
-    lo.off_lam0 = align256(lo.off_dsum + seg_rec * 4);
+    const size_t fsum_rec = seg_rec * (size_t)lo.fsum_k;  // the forward summary's records
+    lo.off_dsum = align256(lo.off_hend + fsum_rec * N * 4);
+    lo.off_lam0 = align256(lo.off_dsum + fsum_rec * 4);
     lo.off_D = align256(lo.off_lam0 + seg_rec * N * 4);
     lo.total = align256(lo.off_D + seg_rec * N * 4);
     return lo;
@@ -827,11 +835,11 @@ ss_status bwd_segment_summaries(const ss_desc *desc, const BwdLayout &lo, const 
         const int lanes = nmax / 2 >= 2 ? 2 : 1, warps = 4;
         const int64_t rows_per_block = (int64_t)warps * (32 / lanes);
         f.dtiles = (q.dim + rows_per_block - 1) / rows_per_block;
-        f.seg_len = q.seg_len, f.nseg = q.nseg;
+        f.seg_len = q.seg_len / lo.fsum_k, f.nseg = q.nseg * lo.fsum_k;
         f.ws_hend = hend, f.ws_dsum = dsum;
         f.status = nullptr, f.delta_r = nullptr, f.W_dt = nullptr, f.dt_rank = 0;
         const size_t smem = selscan::direct_smem_bytes(ein, nmax, lanes, warps);
-        const dim3 grid((unsigned)(f.dtiles * q.batch * q.nseg)), block((unsigned)(warps * 32));
+        const dim3 grid((unsigned)(f.dtiles * q.batch * f.nseg)), block((unsigned)(warps * 32));
         const int split = lanes > 1 ? 1 : 0;
         if (desc->in_dtype == SS_F32) err = launch_f32_f32(n, lanes, split, grid, block, smem, s, f);
         else if (desc->out_dtype == SS_BF16) err = launch_bf16_bf16(n, lanes, split, grid, block, smem, s, f);
@@ -955,6 +963,7 @@ ss_status bwd_impl(const ss_desc *desc, const void *u, const void *delta, const 
                 const ss_status ss = bwd_segment_summaries(desc, lo, q, ws, s);
                 if (ss != SS_OK) return ss;
                 q.seg_h = reinterpret_cast<const float *>(ws + lo.off_hend);
+                q.seg_h_k = lo.fsum_k;
                 q.seg_dl = reinterpret_cast<const float *>(ws + lo.off_D);
             }
             if (fn(dim3((unsigned)(lo.dtiles * gb * lo.nseg)), dim3(kBwdWarps * 32), smem, s, q) != cudaSuccess)

@@ -71,7 +71,10 @@ struct BwdParams {
     int64_t seg_len;
     int nseg;
     int64_t rows_all;
-    const float *seg_h;                       // (nseg, rows, dstate)
+    const float *seg_h;                       // (nseg * seg_h_k, rows, dstate)
+    // The entering state of segment s is seg_h[seg_h_k s - 1]: the forward
+    // summary may cut each segment into seg_h_k pieces (more blocks).
+    int seg_h_k = 1;
     const float *seg_dl;                      // (nseg, rows, dstate)
     // Nonzero: ckpt holds the forward's checkpoints (written by the forward
     // with checkpoints, ss_fwd_ckpt) and phase A is skipped.
@@ -319,7 +322,8 @@ __global__ void __launch_bounds__(128, SS_BWD_MIN_BLOCKS) ss_bwd_kernel(const Bw
         const int n = 2 * (q0 + qq);
         h[qq] = make_float2(0.f, 0.f);
         // the given state enters segment 0; segment s >= 1 starts from the true carry
-        const float *h_src = seg == 0 ? p.init_state : p.seg_h + ((int64_t)(seg - 1) * rows_grp) * N;
+        const float *h_src =
+            seg == 0 ? p.init_state : p.seg_h + ((int64_t)p.seg_h_k * seg - 1) * rows_grp * N;
         if (h_src != nullptr) {
             if (n < N) h[qq].x = h_src[row * N + n];
             if (n + 1 < N) h[qq].y = h_src[row * N + n + 1];
