@@ -269,14 +269,16 @@ def test_bwd_plan_rejections(lib):
 
 
 def test_bwd_segment_records_in_the_workspace(lib):
-    """A segmented plan adds its per-segment records (end states, delta'
-    sums, adjoint summaries and their fold: (3 N + 1) floats per segment and
-    row, plus per-segment row partials) to the unsegmented layout."""
+    """A segmented plan adds its per-segment records to the unsegmented
+    layout: the forward summary's end states and delta' sums ((N + 1) floats
+    per piece and row; 4 segments of 2304 steps, each cut into four 576-step
+    pieces), the adjoint summaries and their fold (2 N floats per segment and
+    row), and per-segment row partials (N + 2)."""
     d = _desc(batch=1, dim=8, seqlen=9000, dstate=16, in_dtype=1, out_dtype=1)
     n = lib.ss_bwd_workspace_bytes(ctypes.byref(d))
-    rows, N, segs, nsub = 8, 16, 4, (9000 + 7) // 8
+    rows, N, segs, pieces, nsub = 8, 16, 4, 4, (9000 + 7) // 8
     base = rows * nsub * N * 4 + 1 * 2 * N * 9000 * 4   # checkpoints + one tile's dB/dC partials
-    extra = segs * rows * (3 * N + 1) * 4 + segs * rows * (N + 2) * 4
+    extra = segs * pieces * rows * (N + 1) * 4 + segs * rows * 2 * N * 4 + segs * rows * (N + 2) * 4
     assert base + extra <= n <= base + extra + 16 * 256  # 256-byte alignment of each region
 
 
