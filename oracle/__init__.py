@@ -161,8 +161,9 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     None.
     ``magnitudes``: also ``mag_<name>`` for each gradient that is a sum over
     rows or steps (dA, dB, dC, dD, ddelta_bias): the sum of the absolute
-    values of its terms, which scales the tolerance of a finite-precision sum
-    element by element."""
+    values of its terms, the state and the adjoint in each taken at the
+    magnitudes of their recursions (see ss_oracle_bwd.c), which scales the
+    tolerance of a finite-precision sum element by element."""
     u, delta, A, B, C, dy = (_f64(t) for t in (u, delta, A, B, C, dy))
     D, z, delta_bias = _f64(D), _f64(z), _f64(delta_bias)
     batch, dim, L = u.shape

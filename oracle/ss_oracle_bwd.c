@@ -38,9 +38,17 @@
  * dlast instead of zero: lam_(L-1)n = g_(L-1) C_n,L-1 + dlast_n.
  *
  * Optionally, for every gradient that is a sum over rows or steps (dA, dB,
- * dC, dD, ddelta_bias), the sum of the absolute values of its terms (the
- * same terms, each taken with |.|).  These scale the tolerance of a finite
- * precision sum per element; they are not gradients.
+ * dC, dD, ddelta_bias), the sum of the absolute values of its terms.  The
+ * state and the adjoint in a term are themselves sums built by their
+ * recursions, whose terms can cancel; a finite-precision value of either
+ * carries an error of the order of the sum of the absolute values of its own
+ * terms.  So each term is taken with h and lam replaced by those magnitudes,
+ *   hm_ln = |a_ln| hm_(l-1)n + |d_l B_nl u_l|,   lam_m_ln = |g_l C_nl| + |a_(l+1)n| lam_m_(l+1)n
+ * (hm before step 0 = |h0|, lam_m past the end = |dlast|, both cut at a
+ * sequence start like h and lam), and the other factors with |.|; a step's
+ * ddelta term with the magnitudes of its terms over the states.  These scale
+ * the tolerance of a finite-precision sum per element; they are not
+ * gradients, and the gradients above do not depend on them.
  */
 #include <math.h>
 #include <stdint.h>
@@ -109,16 +117,20 @@ int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
         double *xs = malloc(sizeof(double) * (size_t)(L + 1));
         double *s = malloc(sizeof(double) * (size_t)(L + 1));
         double *carry = malloc(sizeof(double) * (size_t)N);
-        if (!h || !dl || !xs || !s || !carry) {
+        double *hm = malloc(sizeof(double) * (size_t)((L + 1) * N)); /* magnitudes of h */
+        double *cm = malloc(sizeof(double) * (size_t)N);              /* magnitudes of carry */
+        if (!h || !dl || !xs || !s || !carry || !hm || !cm) {
             bad |= 1;
-            free(h), free(dl), free(xs), free(s), free(carry);
+            free(h), free(dl), free(xs), free(s), free(carry), free(hm), free(cm);
             continue;
         }
         for (int64_t d = 0; d < dim; ++d) {
             const int64_t row = b * dim + d;
             /* forward, keeping every state (h[0..N-1]: the state before step 0) */
-            for (int64_t n = 0; n < N; ++n)
+            for (int64_t n = 0; n < N; ++n) {
                 h[n] = h0 ? h0[row * N + n] : 0.0;
+                hm[n] = fabs(h[n]);
+            }
             for (int64_t l = 0; l < L; ++l) {
                 const int64_t idx = row * L + l;
                 const int keep = !(reset && reset[b * L + l]); /* 0 at a sequence start */
@@ -132,6 +144,7 @@ int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
                     const int64_t bn = (b * N + n) * L + l;
                     const double a = exp(dl[l] * A[d * N + n]);
                     h[(l + 1) * N + n] = a * (keep ? h[l * N + n] : 0.0) + dl[l] * B[bn] * u[idx];
+                    hm[(l + 1) * N + n] = fabs(a) * (keep ? hm[l * N + n] : 0.0) + fabs(dl[l] * B[bn] * u[idx]);
                     acc += C[bn] * h[(l + 1) * N + n];
                 }
                 if (D)
@@ -139,8 +152,10 @@ int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
                 s[l] = acc;
             }
             /* reverse sweep with the adjoint state */
-            for (int64_t n = 0; n < N; ++n) /* a_(l+1) lam_(l+1); past the end: dlast */
+            for (int64_t n = 0; n < N; ++n) { /* a_(l+1) lam_(l+1); past the end: dlast */
                 carry[n] = dlast ? dlast[row * N + n] : 0.0;
+                cm[n] = fabs(carry[n]);
+            }
             for (int64_t l = L - 1; l >= 0; --l) {
                 const int64_t idx = row * L + l;
                 const int keep = !(reset && reset[b * L + l]);
@@ -153,36 +168,41 @@ int ss_oracle_bwd_full(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstat
                 double dui = D ? g * D[d] : 0.0;
                 if (D)
                     pD[row] += g * u[idx], qD[row] += fabs(g * u[idx]);
-                double ddl = 0.0;
+                double ddl = 0.0, ddl_m = 0.0;
                 for (int64_t n = 0; n < N; ++n) {
                     const int64_t bn = (b * N + n) * L + l;
                     const double a = exp(dl[l] * A[d * N + n]);
                     const double lam = g * C[bn] + carry[n];
+                    const double lam_m = fabs(g * C[bn]) + cm[n];
                     dC[bn] += g * h[(l + 1) * N + n];
                     dB[bn] += lam * dl[l] * u[idx];
                     if (mC)
-                        mC[bn] += fabs(g * h[(l + 1) * N + n]);
+                        mC[bn] += fabs(g) * hm[(l + 1) * N + n];
                     if (mB)
-                        mB[bn] += fabs(lam * dl[l] * u[idx]);
+                        mB[bn] += lam_m * fabs(dl[l] * u[idx]);
                     dui += lam * dl[l] * B[bn];
                     const double da = keep ? lam * h[l * N + n] : 0.0;
+                    const double da_m = keep ? lam_m * hm[l * N + n] : 0.0;
                     ddl += lam * B[bn] * u[idx] + da * a * A[d * N + n];
+                    ddl_m += lam_m * fabs(B[bn] * u[idx]) + da_m * fabs(a * A[d * N + n]);
                     pA[row * N + n] += da * a * dl[l];
-                    qA[row * N + n] += fabs(da * a * dl[l]);
+                    qA[row * N + n] += da_m * fabs(a * dl[l]);
                     carry[n] = keep ? a * lam : 0.0;
+                    cm[n] = keep ? fabs(a) * lam_m : 0.0;
                 }
                 du[idx] = dui;
                 const double dx = delta_softplus ? ddl * (xs[l] > 20.0 ? 1.0 : sigmoid(xs[l]))
                                                  : ddl * dl[l];
+                const double fx = delta_softplus ? (xs[l] > 20.0 ? 1.0 : sigmoid(xs[l])) : dl[l];
                 ddelta[idx] = dx;
                 pbias[row] += dx;
-                qbias[row] += fabs(dx);
+                qbias[row] += ddl_m * fabs(fx);
             }
             if (h0) /* the adjoint passed on past step 0 (zero after a start at step 0) */
                 for (int64_t n = 0; n < N; ++n)
                     dh0[row * N + n] = L > 0 ? carry[n] : (dlast ? dlast[row * N + n] : 0.0);
         }
-        free(h), free(dl), free(xs), free(s), free(carry);
+        free(h), free(dl), free(xs), free(s), free(carry), free(hm), free(cm);
     }
     for (int64_t d = 0; d < dim; ++d) {
         for (int64_t n = 0; n < N; ++n) {

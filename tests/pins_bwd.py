@@ -165,18 +165,30 @@ def pin_bwd_initial_state(grad, scan):
 
 
 def pin_bwd_term_magnitudes(grad, scan):
-    """The sums of |terms| that scale the tolerance of the summed gradients:
-    with one row and one step every sum has one term, so each equals the
-    gradient's absolute value; in general each is at least that; and the
-    sums over channels of dB and dC equal the sums of |dB|, |dC| of the
-    single-channel problems (each channel adds one term per element)."""
+    """The sums of |terms| that scale the tolerance of the summed gradients,
+    each term taken with the state and the adjoint replaced by the
+    magnitudes of their own recursions: with one row and one step (no
+    initial state) neither has a recursion, so every sum over rows and steps
+    has one term and equals the gradient's absolute value, except
+    ddelta_bias, whose one step still sums over the states (|g C_n B_n u|
+    sigmoid(x) summed over n); in general each is at least |gradient|; the
+    sums over channels of dB and dC are the single-channel problems' sums
+    added up (each channel adds its own terms); and where the adjoint
+    cancels (two steps, lam_0 = g_0 C_0 + a_1 g_1 C_1 close to zero) the
+    dB term is the closed form (|g_0 C_0| + a_1 |g_1 C_1|) |d_0 u_0|, far
+    above |dB|."""
     rng = np.random.default_rng(61)
     p = _problem(rng, 1, 1, 1, 3)
     dy = rng.standard_normal((1, 1, 1))
     g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
              delta_bias=p["delta_bias"], delta_softplus=True, magnitudes=True)
-    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
-        assert np.array_equal(g["mag_" + k], np.abs(g[k])), f"one term: mag_{k} != |{k}|"
+    for k in ("dA", "dB", "dC", "dD"):  # (the products are associated differently: to rounding)
+        assert np.allclose(g["mag_" + k], np.abs(g[k]), rtol=1e-14, atol=0), f"one term: mag_{k} != |{k}|"
+    x = p["delta"][0, 0, 0] + p["delta_bias"][0]
+    sig = lambda v: 1.0 / (1.0 + np.exp(-v))  # noqa: E731
+    gg = dy[0, 0, 0] * p["z"][0, 0, 0] * sig(p["z"][0, 0, 0])
+    want = sum(abs(gg * p["C"][0, n, 0] * p["B"][0, n, 0] * p["u"][0, 0, 0]) for n in range(3)) * sig(x)
+    assert np.isclose(g["mag_ddelta_bias"][0], want, rtol=1e-12, atol=0), "one step: mag_ddelta_bias"
     p = _problem(rng, 2, 4, 9, 3)
     dy = rng.standard_normal((2, 4, 9))
     g = grad(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
@@ -190,9 +202,21 @@ def pin_bwd_term_magnitudes(grad, scan):
                                              else v[d:d + 1] if n in ("A", "D", "delta_bias") else v))
                  for n, v in p.items()}
             gd = grad(q["u"], q["delta"], q["A"], q["B"], q["C"], dy[:, d:d + 1], D=q["D"], z=q["z"],
-                      delta_bias=q["delta_bias"], delta_softplus=True)
-            acc += np.abs(gd[k])
-        assert np.allclose(g["mag_" + k], acc, rtol=1e-12, atol=0), f"mag_{k} != sum over channels of |{k}|"
+                      delta_bias=q["delta_bias"], delta_softplus=True, magnitudes=True)
+            acc += gd["mag_" + k]
+        assert np.allclose(g["mag_" + k], acc, rtol=1e-12, atol=0), f"mag_{k} != sum over channels"
+    # cancelling adjoint: one channel, one state, two steps, no gate or skip
+    u = np.array([[[0.7, -1.3]]]); delta = np.array([[[0.4, -0.2]]]); A = np.array([[-0.9]])
+    B = np.array([[[1.1, 0.6]]]); C1 = 0.8
+    sp = lambda v: np.log1p(np.exp(v))  # noqa: E731
+    a1 = np.exp(sp(delta[0, 0, 1]) * A[0, 0])
+    dy = np.array([[[1.0, 0.5]]])
+    C0 = -a1 * dy[0, 0, 1] * C1 / dy[0, 0, 0] * (1 + 1e-6)   # g_0 C_0 = -a_1 g_1 C_1 (1 + 1e-6)
+    C = np.array([[[C0, C1]]])
+    g = grad(u, delta, A, B, C, dy, delta_softplus=True, magnitudes=True)
+    want = (abs(dy[0, 0, 0] * C0) + a1 * abs(dy[0, 0, 1] * C1)) * abs(sp(delta[0, 0, 0]) * u[0, 0, 0])
+    assert np.isclose(g["mag_dB"][0, 0, 0], want, rtol=1e-12, atol=0), "cancelling adjoint: mag_dB"
+    assert g["mag_dB"][0, 0, 0] > 1e5 * abs(g["dB"][0, 0, 0]), "cancelling adjoint: mag_dB must stay large"
 
 
 def pin_bwd_last_state_gradient(grad, scan):

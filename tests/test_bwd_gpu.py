@@ -10,8 +10,11 @@ Tolerances (the pages state none for gradients; derived from the arithmetic):
     element's terms (from the oracle), tol 1e-4 for fp32 inputs, 1e-3 for
     bf16: each term carries a relative error of the order of the fp32 and
     SFU rounding of its factors, and the fp32 sum adds rounding of the order
-    of eps times the partial sums, both bounded by a multiple of S.  The
-    floor 1e-6 max S only matters for elements whose terms all vanish.
+    of eps times the partial sums, both bounded by a multiple of S.  The state
+    and the adjoint inside a term are sums built by their recursions, whose
+    terms can cancel, so S takes them at the magnitudes of those recursions
+    (the sums of their own terms' absolute values).  The floor 1e-6 max S only
+    matters for elements whose terms all vanish.
 """
 import numpy as np
 import pytest

@@ -1,0 +1,104 @@
+"""Seeded random cases: each seed draws a shape (batch, channels, length,
+states), the input dtype and the optional parts (z gate, D skip, delta bias,
+softplus or exp mode, sequence starts, an initial state, a last-state
+gradient), then checks the forward (ss_fwd with the workspace its shape can
+use) and the backward (ss_bwd) through the C ABI against the fp64 oracle,
+under the tolerances of test_parity_gpu.py and test_bwd_gpu.py.  The draws
+are fixed by the seed, so a failure names a reproducible case."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import TOL, assert_parity, to_dev
+from test_bwd_gpu import ELEM, TOL_ELEM, TOL_SUM, check_summed
+from selective_state_space_41_b200 import gen, selscan, workloads as W
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+SEEDS = range(24)
+
+
+def _draw(seed):
+    rng = np.random.default_rng(1000 + seed)
+    batch = int(rng.integers(1, 4))
+    dim = int(rng.integers(1, 49))
+    L = int(rng.integers(1, 601))
+    N = int(rng.choice([1, 3, 4, 8, 9, 16, 17, 32, 33, 64]))
+    dtype = torch.bfloat16 if rng.random() < 0.5 else torch.float32
+    softplus = bool(rng.random() < 0.75)
+    kw = dict(has_z=bool(rng.random() < 0.5), D_kind=str(rng.choice(["normal", "ones", "none"])),
+              bias_kind=str(rng.choice(["normal", "zeros", "uniform_dt", "none"])) if softplus else "none",
+              delta_softplus=softplus, return_last_state=True)
+    inp = W.make_inputs(W.custom(f"fuzz{seed}", batch, dim, L, N, dtype, 5000 + seed, **kw))
+    if not softplus:  # exp mode: keep delta' = exp(delta) in a moderate range
+        inp["delta"] = (inp["delta"].float() * 0.5).to(dtype)
+    reset = None
+    if rng.random() < 0.4:
+        reset = (rng.random((batch, L)) < 0.02).astype(np.uint8)
+        reset[:, int(rng.integers(0, L))] = 1
+    h0 = torch.from_numpy(rng.standard_normal((batch, dim, N)).astype(np.float32)) if rng.random() < 0.4 else None
+    dlast = torch.from_numpy(rng.standard_normal((batch, dim, N)).astype(np.float32)) if rng.random() < 0.4 else None
+    inp["dy"] = gen.fill((batch, dim, L), dtype, 5000 + seed, 9)
+    return inp, reset, h0, dlast
+
+
+def _case_name(inp, reset, h0, dlast):
+    b, d, L = inp["u"].shape
+    return (f"{b}x{d}x{L} N={inp['A'].shape[1]} {str(inp['u'].dtype)[6:]} z={inp['z'] is not None} "
+            f"D={inp['D'] is not None} bias={inp['delta_bias'] is not None} softplus={inp['delta_softplus']} "
+            f"starts={reset is not None} h0={h0 is not None} dlast={dlast is not None}")
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_fuzz_forward(seed):
+    inp, reset, h0, _ = _draw(seed)
+    what = _case_name(inp, reset, h0, None)
+    d = to_dev(inp)
+    b, dim, L = d["u"].shape
+    N = d["A"].shape[1]
+    y = torch.full((b, dim, L), float("nan"), dtype=d["u"].dtype, device="cuda")
+    last = torch.full((b, dim, N), float("nan"), device="cuda")
+    ws = selscan.workspace_for(b, dim, L, N, d["u"].dtype, y.dtype)
+    selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"], delta_bias=d["delta_bias"],
+                   delta_softplus=inp["delta_softplus"], last_state=last, workspace=ws,
+                   initial_state=None if h0 is None else h0.cuda(),
+                   reset=None if reset is None else torch.as_tensor(reset).cuda())
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                                            z=inp["z"], delta_bias=inp["delta_bias"],
+                                            delta_softplus=inp["delta_softplus"], return_last_state=True,
+                                            initial_state=h0, reset=reset)
+    assert_parity(y, last, y_ref, last_ref, TOL[inp["u"].dtype], what)
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_fuzz_backward(seed):
+    inp, reset, h0, dlast = _draw(seed)
+    what = _case_name(inp, reset, h0, dlast)
+    dtype = inp["u"].dtype
+    d = to_dev(inp)
+    got = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], D=d["D"], z=d["z"],
+                                     delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"],
+                                     reset=None if reset is None else torch.as_tensor(reset).cuda(),
+                                     initial_state=None if h0 is None else h0.cuda(),
+                                     d_last_state=None if dlast is None else dlast.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"], D=inp["D"],
+                                    z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=inp["delta_softplus"],
+                                    magnitudes=True, reset=reset, initial_state=h0, dlast_state=dlast)
+    for k, want in ref.items():
+        if k.startswith("mag_") or want is None:
+            continue
+        if k == "dinitial_state" and "dinitial_state" not in got:
+            continue
+        g = got[k].detach().to("cpu", torch.float64).numpy()
+        assert np.isfinite(g).all(), f"{what}: {k} not finite"
+        if want.size == 0:
+            continue
+        if k in ELEM or k == "dinitial_state":
+            e = float(np.max(np.abs(g - want) / (1.0 + np.abs(want))))
+            assert e <= TOL_ELEM[dtype], f"{what}: {k} max |err|/(1+|ref|) = {e:.3e}"
+        else:
+            check_summed(k, g, want, ref["mag_" + k], TOL_SUM[dtype], what)

@@ -51,7 +51,9 @@ MUTANTS = {
     "initial_state_ignored": ("h[n] = h0 ? h0[row * N + n] : 0.0;", "h[n] = 0.0;"),
     "initial_state_grad_without_decay": ("dh0[row * N + n] = L > 0 ? carry[n] :",
                                          "dh0[row * N + n] = L > 0 ? carry[n] / exp(dl[0] * A[d * N + n]) :"),
-    "magnitude_of_sum": ("mB[bn] += fabs(lam * dl[l] * u[idx]);", "mB[bn] += lam * dl[l] * u[idx];"),
+    "magnitude_of_sum": ("mB[bn] += lam_m * fabs(dl[l] * u[idx]);", "mB[bn] += lam * dl[l] * u[idx];"),
+    "magnitude_without_recursion": ("const double lam_m = fabs(g * C[bn]) + cm[n];",
+                                    "const double lam_m = fabs(g * C[bn] + carry[n]);"),
     "last_state_gradient_ignored": ("carry[n] = dlast ? dlast[row * N + n] : 0.0;", "carry[n] = 0.0;"),
 }
 
