@@ -1,10 +1,15 @@
 """Seeded random cases: each seed draws a shape (batch, channels, length,
-states), the input dtype and the optional parts (z gate, D skip, delta bias,
-softplus or exp mode, sequence starts, an initial state, a last-state
-gradient), then checks the forward (ss_fwd with the workspace its shape can
-use) and the backward (ss_bwd) through the C ABI against the fp64 oracle,
-under the tolerances of test_parity_gpu.py and test_bwd_gpu.py.  The draws
-are fixed by the seed, so a failure names a reproducible case."""
+states), the input dtype (bf16 sometimes with fp32 output) and the optional
+parts (z gate, D skip, delta bias, softplus or exp mode, sequence starts, an
+initial state, a last-state gradient), then checks the forward (ss_fwd with
+the workspace its shape can use) and the backward both ways (ss_bwd with its
+own checkpointing pass; ss_fwd_ckpt then the backward from its checkpoints)
+through the C ABI against the fp64 oracle, under the tolerances of
+test_parity_gpu.py and test_bwd_gpu.py.  The draws are fixed by the seed, so
+a failure names a reproducible case; SS_FUZZ_SEEDS sets how many seeds run
+(48 by default; 300 passed when the training path was added)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -17,7 +22,7 @@ from selective_state_space_41_b200 import gen, selscan, workloads as W
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
-SEEDS = range(24)
+SEEDS = range(int(os.environ.get("SS_FUZZ_SEEDS", "48")))
 
 
 def _draw(seed):
@@ -31,7 +36,9 @@ def _draw(seed):
     kw = dict(has_z=bool(rng.random() < 0.5), D_kind=str(rng.choice(["normal", "ones", "none"])),
               bias_kind=str(rng.choice(["normal", "zeros", "uniform_dt", "none"])) if softplus else "none",
               delta_softplus=softplus, return_last_state=True)
+    out_dtype = torch.float32 if dtype == torch.bfloat16 and rng.random() < 0.25 else None
     inp = W.make_inputs(W.custom(f"fuzz{seed}", batch, dim, L, N, dtype, 5000 + seed, **kw))
+    inp["out_dtype"] = out_dtype
     if not softplus:  # exp mode: keep delta' = exp(delta) in a moderate range
         inp["delta"] = (inp["delta"].float() * 0.5).to(dtype)
     reset = None
@@ -40,7 +47,7 @@ def _draw(seed):
         reset[:, int(rng.integers(0, L))] = 1
     h0 = torch.from_numpy(rng.standard_normal((batch, dim, N)).astype(np.float32)) if rng.random() < 0.4 else None
     dlast = torch.from_numpy(rng.standard_normal((batch, dim, N)).astype(np.float32)) if rng.random() < 0.4 else None
-    inp["dy"] = gen.fill((batch, dim, L), dtype, 5000 + seed, 9)
+    inp["dy"] = gen.fill((batch, dim, L), out_dtype or dtype, 5000 + seed, 9)
     return inp, reset, h0, dlast
 
 
@@ -48,7 +55,8 @@ def _case_name(inp, reset, h0, dlast):
     b, d, L = inp["u"].shape
     return (f"{b}x{d}x{L} N={inp['A'].shape[1]} {str(inp['u'].dtype)[6:]} z={inp['z'] is not None} "
             f"D={inp['D'] is not None} bias={inp['delta_bias'] is not None} softplus={inp['delta_softplus']} "
-            f"starts={reset is not None} h0={h0 is not None} dlast={dlast is not None}")
+            f"starts={reset is not None} h0={h0 is not None} dlast={dlast is not None} "
+            f"out={'f32' if inp.get('out_dtype') else 'in'}")
 
 
 @pytest.mark.parametrize("seed", SEEDS)
@@ -58,7 +66,7 @@ def test_fuzz_forward(seed):
     d = to_dev(inp)
     b, dim, L = d["u"].shape
     N = d["A"].shape[1]
-    y = torch.full((b, dim, L), float("nan"), dtype=d["u"].dtype, device="cuda")
+    y = torch.full((b, dim, L), float("nan"), dtype=inp["out_dtype"] or d["u"].dtype, device="cuda")
     last = torch.full((b, dim, N), float("nan"), device="cuda")
     ws = selscan.workspace_for(b, dim, L, N, d["u"].dtype, y.dtype)
     selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"], delta_bias=d["delta_bias"],
@@ -70,19 +78,32 @@ def test_fuzz_forward(seed):
                                             z=inp["z"], delta_bias=inp["delta_bias"],
                                             delta_softplus=inp["delta_softplus"], return_last_state=True,
                                             initial_state=h0, reset=reset)
-    assert_parity(y, last, y_ref, last_ref, TOL[inp["u"].dtype], what)
+    assert_parity(y, last, y_ref, last_ref, 1e-4 if inp["out_dtype"] else TOL[inp["u"].dtype], what)
 
 
+@pytest.mark.parametrize("path", ["own_pass", "checkpoints"])
 @pytest.mark.parametrize("seed", SEEDS)
-def test_fuzz_backward(seed):
+def test_fuzz_backward(seed, path):
+    """ss_bwd (its own checkpointing pass), or the training path: the
+    forward that writes the checkpoints, then the backward from them."""
     inp, reset, h0, dlast = _draw(seed)
-    what = _case_name(inp, reset, h0, dlast)
+    what = _case_name(inp, reset, h0, dlast) + " " + path
     dtype = inp["u"].dtype
     d = to_dev(inp)
+    rs = None if reset is None else torch.as_tensor(reset).cuda()
+    hd = None if h0 is None else h0.cuda()
+    ck = None
+    if path == "checkpoints":
+        b, dim, L = d["u"].shape
+        N = d["A"].shape[1]
+        y = torch.empty((b, dim, L), dtype=inp["out_dtype"] or dtype, device="cuda")
+        ck = torch.empty(selscan.ckpt_shape(b, dim, L, N), device="cuda")
+        selscan.ss_fwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"], y, ck, D=d["D"], z=d["z"],
+                            delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"], initial_state=hd,
+                            reset=rs, workspace=selscan.workspace_for(b, dim, L, N, dtype, y.dtype))
     got = selscan.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["dy"], D=d["D"], z=d["z"],
                                      delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"],
-                                     reset=None if reset is None else torch.as_tensor(reset).cuda(),
-                                     initial_state=None if h0 is None else h0.cuda(),
+                                     reset=rs, initial_state=hd, ckpt=ck,
                                      d_last_state=None if dlast is None else dlast.cuda())
     torch.cuda.synchronize()
     ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"], D=inp["D"],
