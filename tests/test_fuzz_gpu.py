@@ -123,3 +123,47 @@ def test_fuzz_backward(seed, path):
             assert e <= TOL_ELEM[dtype], f"{what}: {k} max |err|/(1+|ref|) = {e:.3e}"
         else:
             check_summed(k, g, want, ref["mag_" + k], TOL_SUM[dtype], what)
+
+
+# ---------------------------------------------------------------- launch shapes
+# (lanes per row, split_states) pairs the forward takes: one lane per row
+# (scan kernel when split_states is 0), the state split over 2/4/8 lanes in
+# shared memory (1) or fed through tensor memory (2).
+_SHAPES = [(1, 0), (2, 0), (4, 0), (8, 0), (16, 0), (32, 0), (1, 1), (2, 1), (4, 1), (8, 1), (2, 2), (4, 2), (8, 2)]
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_fuzz_launch_shapes(seed):
+    """A random shape in a random launch shape the library accepts (lanes,
+    state split, warps per block, sequence segments), with the optional
+    parts drawn as above (no sequence starts or initial state: not every
+    launch shape reads them)."""
+    inp, _, _, _ = _draw(seed)
+    rng = np.random.default_rng(7000 + seed)
+    d = to_dev(inp)
+    b, dim, L = d["u"].shape
+    N = d["A"].shape[1]
+    y = torch.full((b, dim, L), float("nan"), dtype=inp["out_dtype"] or d["u"].dtype, device="cuda")
+    last = torch.full((b, dim, N), float("nan"), device="cuda")
+    for attempt in range(64):
+        lanes, split = _SHAPES[int(rng.integers(0, len(_SHAPES)))]
+        cfg = dict(lanes_per_row=lanes, split_states=split, warps_per_block=int(rng.choice([1, 2, 4, 8])),
+                   segments=int(rng.integers(1, 9)) if split == 1 or lanes == 1 else 1)
+        try:
+            ws = selscan.workspace_for(b, dim, L, N, d["u"].dtype, y.dtype, **cfg)
+            selscan.ss_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
+                           delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"], last_state=last,
+                           workspace=ws, **cfg)
+            break
+        except selscan.SelscanError as e:
+            if e.status != 7:  # only SS_ERR_BAD_CONFIG means "another shape"
+                raise
+    else:
+        pytest.skip("no accepted launch shape drawn")
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                                            z=inp["z"], delta_bias=inp["delta_bias"],
+                                            delta_softplus=inp["delta_softplus"], return_last_state=True)
+    assert_parity(y, last, y_ref, last_ref, 1e-4 if inp["out_dtype"] else TOL[inp["u"].dtype],
+                  _case_name(inp, None, None, None) + f" {cfg}")
+    assert selscan.ss_device_status() == 0
