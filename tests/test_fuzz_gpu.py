@@ -5,9 +5,12 @@ initial state, a last-state gradient), then checks the forward (ss_fwd with
 the workspace its shape can use) and the backward both ways (ss_bwd with its
 own checkpointing pass; ss_fwd_ckpt then the backward from its checkpoints)
 through the C ABI against the fp64 oracle, under the tolerances of
-test_parity_gpu.py and test_bwd_gpu.py.  The draws are fixed by the seed, so
-a failure names a reproducible case; SS_FUZZ_SEEDS sets how many seeds run
-(48 by default; 300 passed when the training path was added)."""
+test_parity_gpu.py and test_bwd_gpu.py.  Further families draw a random
+accepted launch shape, a few decoding steps from a random state, the dt_proj
+form with a random rank (apart and in place from x_dbl, bit for bit equal),
+and the host-buffer forward over random streams and batch ranges.  The draws
+are fixed by the seed, so a failure names a reproducible case; SS_FUZZ_SEEDS
+sets how many seeds run (48 by default; 300 of each family passed)."""
 import os
 
 import numpy as np
@@ -167,3 +170,99 @@ def test_fuzz_launch_shapes(seed):
     assert_parity(y, last, y_ref, last_ref, 1e-4 if inp["out_dtype"] else TOL[inp["u"].dtype],
                   _case_name(inp, None, None, None) + f" {cfg}")
     assert selscan.ss_device_status() == 0
+
+
+# ---------------------------------------------------------------- other entries
+@pytest.mark.parametrize("seed", SEEDS)
+def test_fuzz_decode_steps(seed):
+    """ss_step, a few steps with the state updated in place from a random
+    initial state, against the oracle's run from that state."""
+    inp, _, h0, _ = _draw(seed)
+    rng = np.random.default_rng(8000 + seed)
+    b, dim, L = inp["u"].shape
+    steps = min(int(rng.integers(1, 9)), L)
+    N = inp["A"].shape[1]
+    sl = {k: (inp[k][..., :steps].contiguous() if k in ("u", "delta", "z", "B", "C") and inp[k] is not None
+              else inp[k]) for k in ("u", "delta", "z", "B", "C", "A", "D", "delta_bias")}
+    h0 = h0 if h0 is not None else torch.from_numpy(rng.standard_normal((b, dim, N)).astype(np.float32))
+    d = to_dev(sl)
+    state = h0.cuda().clone()
+    out_dtype = inp["out_dtype"] or inp["u"].dtype
+    ys = []
+    for t in range(steps):
+        y = torch.empty((b, dim), dtype=out_dtype, device="cuda")
+        col = lambda k: None if d[k] is None else d[k][..., t].contiguous()  # noqa: E731
+        selscan.ss_step(col("u"), col("delta"), d["A"], col("B"), col("C"), state, y, D=d["D"], z=col("z"),
+                        delta_bias=d["delta_bias"], delta_softplus=inp["delta_softplus"])
+        ys.append(y)
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle.selective_scan(sl["u"], sl["delta"], sl["A"], sl["B"], sl["C"], D=sl["D"], z=sl["z"],
+                                            delta_bias=sl["delta_bias"], delta_softplus=inp["delta_softplus"],
+                                            return_last_state=True, initial_state=h0)
+    assert_parity(torch.stack(ys, dim=-1), state, y_ref, last_ref,
+                  1e-4 if inp["out_dtype"] else TOL[inp["u"].dtype], _case_name(inp, None, h0, None) + f" {steps} steps")
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_fuzz_dtproj_and_xdbl(seed):
+    """The dt_proj form with a random rank, delta_r/B/C passed apart and
+    read in place from one x_dbl tensor (bf16 only): against the oracle fed
+    W_dt delta_r, and the two entries bit for bit."""
+    rng = np.random.default_rng(9000 + seed)
+    batch, dim, L = int(rng.integers(1, 4)), int(rng.integers(1, 49)), int(rng.integers(1, 601))
+    N = int(rng.choice([1, 4, 8, 9, 16, 17, 32, 64]))
+    R = int(rng.integers(1, 65))
+    kw = dict(has_z=bool(rng.random() < 0.5), D_kind=str(rng.choice(["normal", "ones", "none"])),
+              bias_kind=str(rng.choice(["normal", "uniform_dt", "none"])), return_last_state=True)
+    w = W.custom(f"fuzzdt{seed}", batch, dim, L, N, torch.bfloat16, 9500 + seed, **kw)
+    inp = W.make_dtproj_inputs(w, R)
+    out_dtype = torch.float32 if rng.random() < 0.25 else torch.bfloat16
+    d = to_dev(inp)
+    ws = selscan.workspace_for(batch, dim, L, N, torch.bfloat16, out_dtype) if rng.random() < 0.5 else None
+    y = torch.empty((batch, dim, L), dtype=out_dtype, device="cuda")
+    last = torch.empty((batch, dim, N), device="cuda")
+    selscan.ss_fwd_dtproj(d["u"], d["delta_r"], d["W_dt"], d["A"], d["B"], d["C"], y, D=d["D"], z=d["z"],
+                          delta_bias=d["delta_bias"], delta_softplus=True, last_state=last, workspace=ws)
+    x = torch.cat([d["delta_r"], d["B"], d["C"]], dim=1).contiguous()
+    y2, last2 = torch.empty_like(y), torch.empty_like(last)
+    selscan.ss_fwd_xdbl(d["u"], x, d["W_dt"], d["A"], y2, D=d["D"], z=d["z"], delta_bias=d["delta_bias"],
+                        delta_softplus=True, last_state=last2, workspace=ws)
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle.selective_scan_dtproj(inp["u"], inp["delta_r"], inp["W_dt"], inp["A"], inp["B"],
+                                                   inp["C"], D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                                                   delta_softplus=True, return_last_state=True)
+    what = f"{batch}x{dim}x{L} N={N} R={R} out={out_dtype} ws={ws is not None}"
+    assert_parity(y, last, y_ref, last_ref, 1e-4 if out_dtype == torch.float32 else TOL[torch.bfloat16], what)
+    assert torch.equal(y.view(torch.int16) if out_dtype == torch.bfloat16 else y,
+                       y2.view(torch.int16) if out_dtype == torch.bfloat16 else y2) and torch.equal(last, last2), what
+    assert selscan.ss_device_status() == 0
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_fuzz_host_buffers(seed):
+    """The host-buffer forward pipelined over a random number of streams and
+    batch ranges, against the oracle."""
+    inp, _, _, _ = _draw(seed)
+    rng = np.random.default_rng(9900 + seed)
+    b, dim, L = inp["u"].shape
+    N = inp["A"].shape[1]
+    names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    host = {k: (inp[k].pin_memory() if inp[k] is not None else None) for k in names}
+    out_dtype = inp["out_dtype"] or inp["u"].dtype
+    host["y"] = torch.empty((b, dim, L), dtype=out_dtype).pin_memory()
+    host["last_state"] = torch.empty((b, dim, N)).pin_memory()
+    dev = {k: (torch.empty_like(inp[k], device="cuda") if inp[k] is not None else None) for k in names}
+    dev["y"] = torch.empty((b, dim, L), dtype=out_dtype, device="cuda")
+    dev["last_state"] = torch.empty((b, dim, N), device="cuda")
+    nst = int(rng.integers(1, 5))
+    streams = [torch.cuda.current_stream()] + [torch.cuda.Stream() for _ in range(nst - 1)]
+    ws = torch.empty(nst * max(selscan.ss_fwd_workspace_bytes(b, dim, L, N, inp["u"].dtype, out_dtype), 1) + 4096,
+                     dtype=torch.uint8, device="cuda")
+    selscan.ss_fwd_hostio(host, dev, delta_softplus=inp["delta_softplus"], workspace=ws, streams=streams,
+                          chunks=int(rng.integers(0, 2 * b + 1)))
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                                            z=inp["z"], delta_bias=inp["delta_bias"],
+                                            delta_softplus=inp["delta_softplus"], return_last_state=True)
+    assert_parity(host["y"], host["last_state"], y_ref, last_ref, 1e-4 if inp["out_dtype"] else TOL[inp["u"].dtype],
+                  _case_name(inp, None, None, None) + f" streams={nst}")
