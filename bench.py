@@ -188,6 +188,40 @@ def rank_workload(w: W.Workload, rank: int) -> W.Workload:
     return W.with_shape(w, seed=w.seed + 1000003 * rank)
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def cpu_oracle_one_core(w: W.Workload, inp: dict, target_s: float = 2.0):
+    """The oracle on one thread over the first rows of the workload (about
+    ``target_s`` seconds).  Returns (updates/s, description)."""
+    import oracle
+
+    def run(nrows):
+        sl = lambda t: None if t is None else t[0:1, :nrows]  # noqa: E731
+        pd = lambda t: None if t is None else t[:nrows]  # noqa: E731
+        t0 = time.perf_counter()
+        oracle.selective_scan(sl(inp["u"]), sl(inp["delta"]), inp["A"][:nrows], inp["B"][0:1], inp["C"][0:1],
+                              D=pd(inp["D"]), z=sl(inp["z"]), delta_bias=pd(inp["delta_bias"]),
+                              delta_softplus=w.delta_softplus, return_last_state=w.return_last_state, nthreads=1)
+        return time.perf_counter() - t0
+
+    per_row = run(1)
+    rows = int(max(1, min(w.dim, target_s / max(per_row, 1e-9))))
+    dt = run(rows)
+    updates = rows * w.seqlen * w.dstate
+    return updates / dt, f"the first {rows} (b, d) rows, all {w.seqlen} steps, N={w.dstate}, 1 thread"
+
+
 def cpu_oracle_sample(w: W.Workload, inp: dict = None, target_s: float = 10.0):
     """The oracle, as it stands, on all host cores over a bounded sample of the
     same workload (about ``target_s`` seconds): the whole workload, repeated,
@@ -433,8 +467,10 @@ def bench_ours(args, w, world, rank, local):
     del flush
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_sample(w, host)
+        v1, sample1 = cpu_oracle_one_core(w, host)
         line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample, "cpu_model": cpu_model(),
+                                "one_core": {"value": v1, "unit": "updates/s", "sample": sample1}}
     return line if rank == 0 else None
 
 
